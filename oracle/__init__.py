@@ -1,0 +1,108 @@
+"""fp64 CPU oracle for the gated delta rule -- TEST INFRASTRUCTURE ONLY.
+
+Only tests/, __graft_entry__.smoke() and the CPU-baseline leg of bench.py may
+import this package.  It shares no code with the CUDA library and the product
+path never reaches it.
+
+The arithmetic lives in gdr_oracle.c (plain sequential recurrences in double
+precision, one token at a time).  This module only marshals numpy float64
+arrays into that library.  Parity of each function is pinned by the
+tests/test_oracle_*.py files.
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from .build import build
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        path = build()
+        lib = ctypes.CDLL(path)
+        dp = ctypes.POINTER(ctypes.c_double)
+        i = ctypes.c_int
+        lib.oracle_gdr_fwd.argtypes = [i, i, i, i, i] + [dp] * 8
+        lib.oracle_gdr_step.argtypes = [i, i, i, i] + [dp] * 7
+        lib.oracle_gdr_bwd.argtypes = [i, i, i, i, i] + [dp] * 14
+        lib.oracle_gdr2_fwd.argtypes = [i, i, i, i, i] + [dp] * 9
+        lib.oracle_num_threads.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _in(x):
+    if x is None:
+        return None
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _p(x):
+    if x is None:
+        return None
+    return x.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def num_threads() -> int:
+    """Host threads the oracle's OpenMP loops use."""
+    return int(_load().oracle_num_threads())
+
+
+def gdr_fwd(q, k, v, log_alpha, beta, S0=None):
+    """Sequential gated delta rule forward.  Shapes: q,k [B,T,H,dk],
+    v [B,T,H,dv], log_alpha/beta [B,T,H], S0 [B,H,dv,dk] or None.
+    Returns (o [B,T,H,dv], S_T [B,H,dv,dk]) as float64."""
+    q, k, v, la, be, S0 = map(_in, (q, k, v, log_alpha, beta, S0))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    o = np.zeros((B, T, H, dv))
+    ST = np.zeros((B, H, dv, dk))
+    _load().oracle_gdr_fwd(B, T, H, dk, dv, _p(q), _p(k), _p(v), _p(la), _p(be),
+                           _p(S0), _p(o), _p(ST))
+    return o, ST
+
+
+def gdr_step(q, k, v, log_alpha, beta, S):
+    """One decode token.  q,k [B,H,dk], v [B,H,dv], log_alpha/beta [B,H],
+    S [B,H,dv,dk].  Returns (o [B,H,dv], S_new) without modifying S."""
+    q, k, v, la, be = map(_in, (q, k, v, log_alpha, beta))
+    S = np.array(S, dtype=np.float64, copy=True, order="C")
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    o = np.zeros((B, H, dv))
+    _load().oracle_gdr_step(B, H, dk, dv, _p(q), _p(k), _p(v), _p(la), _p(be),
+                            _p(S), _p(o))
+    return o, S
+
+
+def gdr_bwd(q, k, v, log_alpha, beta, S0, dO, dS_T=None):
+    """Hand-derived reverse mode of gdr_fwd.  Returns a dict with dq, dk, dv,
+    dlog_alpha, dbeta, dS0 (float64)."""
+    q, k, v, la, be, S0, dO, dST = map(_in, (q, k, v, log_alpha, beta, S0, dO, dS_T))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    out = dict(dq=np.zeros_like(q), dk=np.zeros_like(k), dv=np.zeros_like(v),
+               dlog_alpha=np.zeros_like(la), dbeta=np.zeros_like(be),
+               dS0=np.zeros((B, H, dv, dk)))
+    _load().oracle_gdr_bwd(B, T, H, dk, dv, _p(q), _p(k), _p(v), _p(la), _p(be),
+                           _p(S0), _p(dO), _p(dST), _p(out["dq"]), _p(out["dk"]),
+                           _p(out["dv"]), _p(out["dlog_alpha"]), _p(out["dbeta"]),
+                           _p(out["dS0"]))
+    return out
+
+
+def gdr2_fwd(q, k, v, log_alpha, b, w, S0=None):
+    """Gated Delta Rule-2 forward.  log_alpha, b [B,T,H,dk]; w [B,T,H,dv].
+    Returns (o, S_T) as float64."""
+    q, k, v, la, bb, ww, S0 = map(_in, (q, k, v, log_alpha, b, w, S0))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    o = np.zeros((B, T, H, dv))
+    ST = np.zeros((B, H, dv, dk))
+    _load().oracle_gdr2_fwd(B, T, H, dk, dv, _p(q), _p(k), _p(v), _p(la), _p(bb),
+                            _p(ww), _p(S0), _p(o), _p(ST))
+    return o, ST

@@ -1,0 +1,136 @@
+"""Pin of the chunkwise (UT transform / WY) reading that the CUDA kernels
+implement, against the sequential oracle (CPU only, fp64).
+
+The chunkwise equations are printed in the Gated DeltaNet review
+(meaningful96.github.io/nr/GDN), section 3.7, partly garbled: the arrow
+decorations are undefined, W is never defined and the intra-chunk mask has
+lost its decay.  The reading taken (derived by substituting the ansatz
+S_r = gamma_r S + sum_{i<=r} (gamma_r/gamma_i) u_i k_i^T into the rule of
+section 3.4) is, per chunk of C tokens with g_r = sum_{s<=r} log alpha_s,
+gamma_r = exp(g_r):
+
+    A     = strictLower(diag(beta) (Gamma * K K^T)),  Gamma_ri = gamma_r/gamma_i
+    T     = (I + A)^-1
+    U^g   = T diag(beta) V
+    W     = T diag(beta*gamma) K
+    U     = U^g - W S^T
+    O     = diag(gamma) Q S^T + (Q K^T * L) U,        L_ri = gamma_r/gamma_i, i <= r
+    S'    = gamma_C S + U^T diag(gamma_C/gamma) K
+
+and for Gated DeltaNet-2 ("Gated DeltaNet-2: Decoupling Erase and Write in
+Linear Attention", agihunt.info/papers/2605.22791: the channel decay is
+absorbed into an asymmetric rank-1 erase factor, WY triangular solve at
+chunk 64), with E = exp(per-channel cumulative log alpha):
+
+    A  = strictLower((K*B*E)(K/E)^T),  U = (I + A)^-1 ((W*V) - (K*B*E) S^T)
+    O  = (Q*E) S^T + (((Q*E)(K/E)^T) * M_incl) U
+    S' = S Diag(E_C) + U^T (K * E_C/E)
+
+If this reading were wrong (a missing decay on the mask, gamma on the wrong
+side of T, a wrong transpose) the comparison below would fail by O(1).
+The result must not depend on C; C = 1 is the recurrence itself.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from pins_common import rand_inputs, rel_err
+
+
+def chunkwise_gdr(q, k, v, la, be, S0, C):
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    o = np.zeros((B, T, H, dv))
+    ST = np.zeros((B, H, dv, dk))
+    for b in range(B):
+        for h in range(H):
+            S = np.zeros((dv, dk)) if S0 is None else S0[b, h].copy()
+            for c0 in range(0, T, C):
+                sl = slice(c0, min(c0 + C, T))
+                Q, K, V = q[b, sl, h], k[b, sl, h], v[b, sl, h]
+                beta = be[b, sl, h]
+                g = np.cumsum(la[b, sl, h])
+                n = len(g)
+                ratio = np.exp(g[:, None] - g[None, :])
+                strict = np.tril(np.ones((n, n)), -1)
+                incl = np.tril(np.ones((n, n)))
+                A = strict * (beta[:, None] * ratio * (K @ K.T))
+                Tm = np.linalg.inv(np.eye(n) + A)
+                Ug = Tm @ (beta[:, None] * V)
+                W = Tm @ ((beta * np.exp(g))[:, None] * K)
+                U = Ug - W @ S.T
+                o[b, sl, h] = np.exp(g)[:, None] * (Q @ S.T) + ((Q @ K.T) * ratio * incl) @ U
+                S = np.exp(g[-1]) * S + U.T @ (np.exp(g[-1] - g)[:, None] * K)
+            ST[b, h] = S
+    return o, ST
+
+
+def chunkwise_gdr2(q, k, v, la, bg, wg, S0, C):
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    o = np.zeros((B, T, H, dv))
+    ST = np.zeros((B, H, dv, dk))
+    for b in range(B):
+        for h in range(H):
+            S = np.zeros((dv, dk)) if S0 is None else S0[b, h].copy()
+            for c0 in range(0, T, C):
+                sl = slice(c0, min(c0 + C, T))
+                Q, K, V = q[b, sl, h], k[b, sl, h], v[b, sl, h]
+                G = np.cumsum(la[b, sl, h], axis=0)
+                E = np.exp(G)
+                n = G.shape[0]
+                strict = np.tril(np.ones((n, n)), -1)
+                incl = np.tril(np.ones((n, n)))
+                KBE = K * bg[b, sl, h] * E
+                A = strict * (KBE @ (K / E).T)
+                Tm = np.linalg.inv(np.eye(n) + A)
+                U = Tm @ (wg[b, sl, h] * V - KBE @ S.T)
+                QE = Q * E
+                o[b, sl, h] = QE @ S.T + ((QE @ (K / E).T) * incl) @ U
+                S = S * E[-1][None, :] + U.T @ (K * np.exp(G[-1][None, :] - G))
+            ST[b, h] = S
+    return o, ST
+
+
+@pytest.mark.parametrize("C", [1, 4, 64])
+@pytest.mark.parametrize("T", [64, 100, 256])
+def test_chunkwise_gdr_equals_recurrence(C, T):
+    rng = np.random.default_rng(C * 1000 + T)
+    q, k, v, la, be, S0 = rand_inputs(rng, 1, T, 2, 8, 6)
+    o, ST = oracle.gdr_fwd(q, k, v, la, be, S0)
+    oc, STc = chunkwise_gdr(q, k, v, la, be, S0, C)
+    assert rel_err(oc, o) < 1e-11
+    assert rel_err(STc, ST) < 1e-11
+
+
+@pytest.mark.parametrize("C", [1, 4, 64])
+@pytest.mark.parametrize("T", [64, 100])
+def test_chunkwise_gdr2_equals_recurrence(C, T):
+    rng = np.random.default_rng(7 * C + T)
+    q, k, v, _, _, S0 = rand_inputs(rng, 1, T, 2, 8, 6)
+    la = -np.log1p(np.exp(rng.normal(-2.0, 1.0, size=(1, T, 2, 8))))
+    bg = 1.0 / (1.0 + np.exp(-rng.normal(size=(1, T, 2, 8))))
+    wg = 1.0 / (1.0 + np.exp(-rng.normal(size=(1, T, 2, 6))))
+    o, ST = oracle.gdr2_fwd(q, k, v, la, bg, wg, S0)
+    oc, STc = chunkwise_gdr2(q, k, v, la, bg, wg, S0, C)
+    assert rel_err(oc, o) < 1e-10
+    assert rel_err(STc, ST) < 1e-10
+
+
+def test_mask_without_decay_is_wrong():
+    """The literal printed mask (no decay on the intra-chunk term) disagrees
+    with the recurrence, which is why the decayed mask is the reading."""
+    rng = np.random.default_rng(9)
+    q, k, v, la, be, S0 = rand_inputs(rng, 1, 64, 1, 8, 6)
+    o, _ = oracle.gdr_fwd(q, k, v, la, be, S0)
+    Q, K, V = q[0, :, 0], k[0, :, 0], v[0, :, 0]
+    beta = be[0, :, 0]
+    g = np.cumsum(la[0, :, 0])
+    n = 64
+    ratio = np.exp(g[:, None] - g[None, :])
+    A = np.tril(np.ones((n, n)), -1) * (beta[:, None] * ratio * (K @ K.T))
+    Tm = np.linalg.inv(np.eye(n) + A)
+    S = S0[0, 0]
+    U = Tm @ (beta[:, None] * V) - Tm @ ((beta * np.exp(g))[:, None] * K) @ S.T
+    o_bad = np.exp(g)[:, None] * (Q @ S.T) + ((Q @ K.T) * np.tril(np.ones((n, n)))) @ U
+    assert rel_err(o_bad, o[0, :, 0]) > 1e-2
