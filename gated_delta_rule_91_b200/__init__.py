@@ -1,0 +1,184 @@
+"""Python binding of libgdr.so, the B200 (sm_100a) gated delta rule library.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI declared in include/gdr.h.  PyTorch supplies device
+memory (outputs, workspace) and the current CUDA stream.  There is no CPU
+path: if libgdr.so is missing or no GPU is present the calls raise.
+
+Functions (same names as the C entry points):
+    gdr_fwd(q, k, v, log_alpha, beta, S0=None)          -> (o, S_T)
+    gdr_step(q, k, v, log_alpha, beta, S)                -> o  (S advanced in place)
+    gdr_bwd(q, k, v, log_alpha, beta, S0, dO, dS_T=None) -> dict of gradients
+    gdr2_fwd(q, k, v, log_alpha, b, w, S0=None)          -> (o, S_T)
+"""
+import ctypes
+import os
+
+import torch
+
+PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG_DIR, "libgdr.so")
+
+GDR_OK, GDR_ERR_INVALID_ARGUMENT, GDR_ERR_UNSUPPORTED, GDR_ERR_WORKSPACE, GDR_ERR_CUDA, \
+    GDR_ERR_TIMEOUT = range(6)
+GDR_F32, GDR_BF16 = 0, 1
+STATUS_NAMES = {0: "GDR_OK", 1: "GDR_ERR_INVALID_ARGUMENT", 2: "GDR_ERR_UNSUPPORTED",
+                3: "GDR_ERR_WORKSPACE", 4: "GDR_ERR_CUDA", 5: "GDR_ERR_TIMEOUT"}
+
+# name -> (restype, argtypes); mirrors include/gdr.h
+_I, _SZ, _P = ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p
+SIGNATURES = {
+    "gdr_fwd": (_I, [_I] * 6 + [_P] * 8 + [_P, _SZ, _P]),
+    "gdr_fwd_workspace_bytes": (_SZ, [_I] * 6),
+    "gdr_step": (_I, [_I] * 5 + [_P] * 7 + [_P]),
+    "gdr_bwd": (_I, [_I] * 6 + [_P] * 14 + [_P, _SZ, _P]),
+    "gdr_bwd_workspace_bytes": (_SZ, [_I] * 6),
+    "gdr2_fwd": (_I, [_I] * 6 + [_P] * 9 + [_P, _SZ, _P]),
+    "gdr2_fwd_workspace_bytes": (_SZ, [_I] * 6),
+    "gdr_check_status": (_I, [_P]),
+    "gdr_last_error_string": (ctypes.c_char_p, []),
+    "gdr_launch_count": (ctypes.c_uint64, []),
+    "gdr_version": (_I, []),
+}
+
+
+class GdrError(RuntimeError):
+    def __init__(self, status, msg):
+        super().__init__("%s: %s" % (STATUS_NAMES.get(status, status), msg))
+        self.status = status
+
+
+_lib = None
+
+
+def lib():
+    """The loaded libgdr.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError("libgdr.so not found at %s; build it with "
+                               "`python -m gated_delta_rule_91_b200._build`" % LIB_PATH)
+        h = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(h, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = h
+    return _lib
+
+
+def check(status):
+    if status != GDR_OK:
+        raise GdrError(status, lib().gdr_last_error_string().decode())
+
+
+def launch_count() -> int:
+    return int(lib().gdr_launch_count())
+
+
+def check_status(stream=None):
+    """Synchronise the stream and raise if a kernel recorded a timeout."""
+    s = torch.cuda.current_stream() if stream is None else stream
+    check(lib().gdr_check_status(ctypes.c_void_p(s.cuda_stream)))
+
+
+def _dt(x: torch.Tensor) -> int:
+    if x.dtype == torch.float32:
+        return GDR_F32
+    if x.dtype == torch.bfloat16:
+        return GDR_BF16
+    raise TypeError("q/k/v must be float32 or bfloat16, got %s" % x.dtype)
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if not x.is_cuda:
+        raise ValueError("tensors must be on a CUDA device")
+    if not x.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return ctypes.c_void_p(x.data_ptr())
+
+
+def _f32(x, name):
+    if x is not None and x.dtype != torch.float32:
+        raise TypeError("%s must be float32" % name)
+    return x
+
+
+def _stream(x):
+    return ctypes.c_void_p(torch.cuda.current_stream(x.device).cuda_stream)
+
+
+def _workspace(nbytes, device, workspace):
+    if nbytes == 0:
+        return None, 0
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    return workspace, workspace.numel() * workspace.element_size()
+
+
+def gdr_fwd(q, k, v, log_alpha, beta, S0=None, *, o=None, S_T=None, return_state=True,
+            workspace=None):
+    """Chunkwise forward on the current stream.  Returns (o, S_T or None)."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = _dt(q)
+    _f32(log_alpha, "log_alpha"), _f32(beta, "beta"), _f32(S0, "S0")
+    if o is None:
+        o = torch.empty(B, T, H, dv, dtype=q.dtype, device=q.device)
+    if S_T is None and return_state:
+        S_T = torch.empty(B, H, dv, dk, dtype=torch.float32, device=q.device)
+    L = lib()
+    ws, ws_bytes = _workspace(L.gdr_fwd_workspace_bytes(B, T, H, dk, dv, dt), q.device, workspace)
+    check(L.gdr_fwd(B, T, H, dk, dv, dt, _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+                    _ptr(S0), _ptr(o), _ptr(S_T), _ptr(ws), ws_bytes, _stream(q)))
+    return o, S_T
+
+
+def gdr_step(q, k, v, log_alpha, beta, S, *, o=None):
+    """One decode token; S [B,H,dv,dk] fp32 is advanced in place.  Returns o."""
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = _dt(q)
+    _f32(S, "S")
+    if o is None:
+        o = torch.empty(B, H, dv, dtype=q.dtype, device=q.device)
+    check(lib().gdr_step(B, H, dk, dv, dt, _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
+                         _ptr(beta), _ptr(S), _ptr(o), _stream(q)))
+    return o
+
+
+def gdr_bwd(q, k, v, log_alpha, beta, S0, dO, dS_T=None, *, want_dS0=True, workspace=None):
+    """Backward of gdr_fwd.  Returns dict(dq, dk, dv, dlog_alpha, dbeta, dS0)."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = _dt(q)
+    out = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dv=torch.empty_like(v),
+               dlog_alpha=torch.empty_like(log_alpha), dbeta=torch.empty_like(beta),
+               dS0=torch.empty(B, H, dv, dk, dtype=torch.float32, device=q.device)
+               if want_dS0 else None)
+    L = lib()
+    ws, ws_bytes = _workspace(L.gdr_bwd_workspace_bytes(B, T, H, dk, dv, dt), q.device, workspace)
+    check(L.gdr_bwd(B, T, H, dk, dv, dt, _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+                    _ptr(S0), _ptr(dO), _ptr(dS_T), _ptr(out["dq"]), _ptr(out["dk"]),
+                    _ptr(out["dv"]), _ptr(out["dlog_alpha"]), _ptr(out["dbeta"]),
+                    _ptr(out["dS0"]), _ptr(ws), ws_bytes, _stream(q)))
+    return out
+
+
+def gdr2_fwd(q, k, v, log_alpha, b, w, S0=None, *, o=None, S_T=None, return_state=True,
+             workspace=None):
+    """Gated DeltaNet-2 forward.  Returns (o, S_T or None)."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = _dt(q)
+    if o is None:
+        o = torch.empty(B, T, H, dv, dtype=q.dtype, device=q.device)
+    if S_T is None and return_state:
+        S_T = torch.empty(B, H, dv, dk, dtype=torch.float32, device=q.device)
+    L = lib()
+    ws, ws_bytes = _workspace(L.gdr2_fwd_workspace_bytes(B, T, H, dk, dv, dt), q.device, workspace)
+    check(L.gdr2_fwd(B, T, H, dk, dv, dt, _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b),
+                     _ptr(w), _ptr(S0), _ptr(o), _ptr(S_T), _ptr(ws), ws_bytes, _stream(q)))
+    return o, S_T

@@ -1,0 +1,247 @@
+// gdr_lib.cu -- the C ABI of libgdr.so (declared in include/gdr.h): argument
+// validation, workspace sizing, kernel selection and the device status word.
+// Every kernel header is included here so the library is one translation
+// unit (the device status word is then a single symbol).
+#include <stdarg.h>
+#include <stdio.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <string>
+
+#include "common.cuh"
+#include "step_kernel.cuh"
+#include "fwd_simt.cuh"
+#include "bwd_simt.cuh"
+#include "gdr2_simt.cuh"
+#include "fwd_tc.cuh"
+
+namespace gdr {
+std::atomic<uint64_t> g_launches{0};
+}  // namespace gdr
+
+using namespace gdr;
+
+namespace {
+
+thread_local std::string t_last_error;
+
+gdr_status fail(gdr_status s, const char *fmt, ...) __attribute__((format(printf, 2, 3)));
+gdr_status fail(gdr_status s, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    t_last_error = buf;
+    return s;
+}
+
+gdr_status cuda_fail(cudaError_t e, const char *where) {
+    return fail(GDR_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+#define GDR_REQUIRE_PTR(p)                                                                   \
+    do {                                                                                     \
+        if ((p) == nullptr) return fail(GDR_ERR_INVALID_ARGUMENT, "%s: %s is NULL", fn, #p); \
+        if (!aligned16(p))                                                                   \
+            return fail(GDR_ERR_INVALID_ARGUMENT, "%s: %s is not 16-byte aligned", fn, #p);  \
+    } while (0)
+#define GDR_OPTIONAL_PTR(p)                                                                 \
+    do {                                                                                    \
+        if ((p) != nullptr && !aligned16(p))                                                \
+            return fail(GDR_ERR_INVALID_ARGUMENT, "%s: %s is not 16-byte aligned", fn, #p); \
+    } while (0)
+
+gdr_status check_dims(const char *fn, int B, int T, int H, int dk, int dv, gdr_dtype dt) {
+    if (B < 1 || T < 1 || H < 1 || dk < 1 || dv < 1)
+        return fail(GDR_ERR_INVALID_ARGUMENT, "%s: sizes must be positive (B=%d T=%d H=%d dk=%d dv=%d)",
+                    fn, B, T, H, dk, dv);
+    if (dt != GDR_F32 && dt != GDR_BF16)
+        return fail(GDR_ERR_UNSUPPORTED, "%s: unknown dtype %d", fn, (int)dt);
+    if ((dk != 64 && dk != 128) || (dv != 64 && dv != 128))
+        return fail(GDR_ERR_UNSUPPORTED, "%s: dk=%d dv=%d (supported: 64 or 128 each)", fn, dk, dv);
+    const long long elems = (long long)B * T * H * (dk > dv ? dk : dv);
+    if (elems >= (1LL << 31))
+        return fail(GDR_ERR_UNSUPPORTED, "%s: B*T*H*max(dk,dv) = %lld exceeds 2^31-1", fn, elems);
+    if ((long long)B * H * (dv / 64) >= (1LL << 31))
+        return fail(GDR_ERR_UNSUPPORTED, "%s: too many (batch, head) units", fn);
+    return GDR_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int gdr_version(void) { return (0 << 16) | 1; }
+
+uint64_t gdr_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+const char *gdr_last_error_string(void) { return t_last_error.c_str(); }
+
+gdr_status gdr_check_status(gdr_stream_t stream) {
+    cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "gdr_check_status: synchronize");
+    int host = 0, zero = 0;
+    e = cudaMemcpyFromSymbol(&host, g_status, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e, "gdr_check_status: read status");
+    if (host != 0) {
+        e = cudaMemcpyToSymbol(g_status, &zero, sizeof(int));
+        if (e != cudaSuccess) return cuda_fail(e, "gdr_check_status: clear status");
+        return fail((gdr_status)host, "device status %d: a bounded on-chip wait gave up", host);
+    }
+    return GDR_OK;
+}
+
+size_t gdr_fwd_workspace_bytes(int, int, int, int, int, gdr_dtype) { return 0; }
+
+gdr_status gdr_fwd(int B, int T, int H, int dk, int dv, gdr_dtype dt, const void *q, const void *k,
+                   const void *v, const float *log_alpha, const float *beta, const float *S0,
+                   void *o, float *S_T, void *workspace, size_t workspace_bytes,
+                   gdr_stream_t stream) {
+    const char *fn = "gdr_fwd";
+    gdr_status st = check_dims(fn, B, T, H, dk, dv, dt);
+    if (st != GDR_OK) return st;
+    GDR_REQUIRE_PTR(q);
+    GDR_REQUIRE_PTR(k);
+    GDR_REQUIRE_PTR(v);
+    GDR_REQUIRE_PTR(log_alpha);
+    GDR_REQUIRE_PTR(beta);
+    GDR_REQUIRE_PTR(o);
+    GDR_OPTIONAL_PTR(S0);
+    GDR_OPTIONAL_PTR(S_T);
+    GDR_OPTIONAL_PTR(workspace);
+    const size_t need = gdr_fwd_workspace_bytes(B, T, H, dk, dv, dt);
+    if (need > 0 && (workspace == nullptr || workspace_bytes < need))
+        return fail(GDR_ERR_WORKSPACE, "%s: workspace of %zu bytes needed, %zu given", fn, need,
+                    workspace ? workspace_bytes : (size_t)0);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    // bf16 with dk = dv = 128 runs on the tensor cores; GDR_FWD_KERNEL=simt
+    // selects the CUDA-core kernel instead (used to cross-check the two).
+    const char *sel = getenv("GDR_FWD_KERNEL");
+    const bool force_simt = sel != nullptr && strcmp(sel, "simt") == 0;
+    if (dt == GDR_BF16 && dk == 128 && dv == 128 && !force_simt) {
+        e = launch_fwd_tc(B, T, H, q, k, v, log_alpha, beta, S0, o, S_T, s);
+        if (e != cudaSuccess) return cuda_fail(e, fn);
+        return GDR_OK;
+    }
+    if (dt == GDR_F32)
+        e = dk == 128 ? launch_fwd_simt<float, 128>(B, T, H, dv, q, k, v, log_alpha, beta, S0, o, S_T, s)
+                      : launch_fwd_simt<float, 64>(B, T, H, dv, q, k, v, log_alpha, beta, S0, o, S_T, s);
+    else
+        e = dk == 128
+                ? launch_fwd_simt<__nv_bfloat16, 128>(B, T, H, dv, q, k, v, log_alpha, beta, S0, o, S_T, s)
+                : launch_fwd_simt<__nv_bfloat16, 64>(B, T, H, dv, q, k, v, log_alpha, beta, S0, o, S_T, s);
+    if (e != cudaSuccess) return cuda_fail(e, fn);
+    return GDR_OK;
+}
+
+gdr_status gdr_step(int B, int H, int dk, int dv, gdr_dtype dt, const void *q, const void *k,
+                    const void *v, const float *log_alpha, const float *beta, float *S, void *o,
+                    gdr_stream_t stream) {
+    const char *fn = "gdr_step";
+    gdr_status st = check_dims(fn, B, 1, H, dk, dv, dt);
+    if (st != GDR_OK) return st;
+    GDR_REQUIRE_PTR(q);
+    GDR_REQUIRE_PTR(k);
+    GDR_REQUIRE_PTR(v);
+    GDR_REQUIRE_PTR(log_alpha);
+    GDR_REQUIRE_PTR(beta);
+    GDR_REQUIRE_PTR(S);
+    GDR_REQUIRE_PTR(o);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    if (dt == GDR_F32)
+        e = dk == 128 ? launch_step<float, 128>(B, H, dv, q, k, v, log_alpha, beta, S, o, s)
+                      : launch_step<float, 64>(B, H, dv, q, k, v, log_alpha, beta, S, o, s);
+    else
+        e = dk == 128 ? launch_step<__nv_bfloat16, 128>(B, H, dv, q, k, v, log_alpha, beta, S, o, s)
+                      : launch_step<__nv_bfloat16, 64>(B, H, dv, q, k, v, log_alpha, beta, S, o, s);
+    if (e != cudaSuccess) return cuda_fail(e, fn);
+    return GDR_OK;
+}
+
+size_t gdr_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, gdr_dtype) {
+    if (B < 1 || T < 1 || H < 1 || (dk != 64 && dk != 128) || (dv != 64 && dv != 128)) return 0;
+    return bwd_workspace_bytes(B, T, H, dk, dv);
+}
+
+gdr_status gdr_bwd(int B, int T, int H, int dk, int dv, gdr_dtype dt, const void *q, const void *k,
+                   const void *v, const float *log_alpha, const float *beta, const float *S0,
+                   const void *dO, const float *dS_T, void *dq, void *dk_out, void *dv_out,
+                   float *dlog_alpha, float *dbeta, float *dS0, void *workspace,
+                   size_t workspace_bytes, gdr_stream_t stream) {
+    const char *fn = "gdr_bwd";
+    gdr_status st = check_dims(fn, B, T, H, dk, dv, dt);
+    if (st != GDR_OK) return st;
+    GDR_REQUIRE_PTR(q);
+    GDR_REQUIRE_PTR(k);
+    GDR_REQUIRE_PTR(v);
+    GDR_REQUIRE_PTR(log_alpha);
+    GDR_REQUIRE_PTR(beta);
+    GDR_REQUIRE_PTR(dO);
+    GDR_REQUIRE_PTR(dq);
+    GDR_REQUIRE_PTR(dk_out);
+    GDR_REQUIRE_PTR(dv_out);
+    GDR_REQUIRE_PTR(dlog_alpha);
+    GDR_REQUIRE_PTR(dbeta);
+    GDR_OPTIONAL_PTR(S0);
+    GDR_OPTIONAL_PTR(dS_T);
+    GDR_OPTIONAL_PTR(dS0);
+    const size_t need = gdr_bwd_workspace_bytes(B, T, H, dk, dv, dt);
+    if (workspace == nullptr || workspace_bytes < need)
+        return fail(GDR_ERR_WORKSPACE, "%s: workspace of %zu bytes needed, %zu given", fn, need,
+                    workspace ? workspace_bytes : (size_t)0);
+    if (!aligned16(workspace))
+        return fail(GDR_ERR_INVALID_ARGUMENT, "%s: workspace is not 16-byte aligned", fn);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e;
+#define GDR_BWD_ARGS B, T, H, dv, q, k, v, log_alpha, beta, S0, dO, dS_T, dq, dk_out, dv_out, \
+                     dlog_alpha, dbeta, dS0, workspace, s
+    if (dt == GDR_F32)
+        e = dk == 128 ? launch_bwd_simt<float, 128>(GDR_BWD_ARGS) : launch_bwd_simt<float, 64>(GDR_BWD_ARGS);
+    else
+        e = dk == 128 ? launch_bwd_simt<__nv_bfloat16, 128>(GDR_BWD_ARGS)
+                      : launch_bwd_simt<__nv_bfloat16, 64>(GDR_BWD_ARGS);
+#undef GDR_BWD_ARGS
+    if (e != cudaSuccess) return cuda_fail(e, fn);
+    return GDR_OK;
+}
+
+size_t gdr2_fwd_workspace_bytes(int, int, int, int, int, gdr_dtype) { return 0; }
+
+gdr_status gdr2_fwd(int B, int T, int H, int dk, int dv, gdr_dtype dt, const void *q, const void *k,
+                    const void *v, const float *log_alpha, const float *b, const float *w,
+                    const float *S0, void *o, float *S_T, void *workspace, size_t workspace_bytes,
+                    gdr_stream_t stream) {
+    const char *fn = "gdr2_fwd";
+    gdr_status st = check_dims(fn, B, T, H, dk, dv, dt);
+    if (st != GDR_OK) return st;
+    GDR_REQUIRE_PTR(q);
+    GDR_REQUIRE_PTR(k);
+    GDR_REQUIRE_PTR(v);
+    GDR_REQUIRE_PTR(log_alpha);
+    GDR_REQUIRE_PTR(b);
+    GDR_REQUIRE_PTR(w);
+    GDR_REQUIRE_PTR(o);
+    GDR_OPTIONAL_PTR(S0);
+    GDR_OPTIONAL_PTR(S_T);
+    GDR_OPTIONAL_PTR(workspace);
+    (void)workspace_bytes;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e;
+#define GDR2_ARGS B, T, H, dv, q, k, v, log_alpha, b, w, S0, o, S_T, s
+    if (dt == GDR_F32)
+        e = dk == 128 ? launch_gdr2_simt<float, 128>(GDR2_ARGS) : launch_gdr2_simt<float, 64>(GDR2_ARGS);
+    else
+        e = dk == 128 ? launch_gdr2_simt<__nv_bfloat16, 128>(GDR2_ARGS)
+                      : launch_gdr2_simt<__nv_bfloat16, 64>(GDR2_ARGS);
+#undef GDR2_ARGS
+    if (e != cudaSuccess) return cuda_fail(e, fn);
+    return GDR_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,162 @@
+/*
+ * gdr.h -- C ABI of the B200 (sm_100a) gated delta rule library, libgdr.so.
+ *
+ * The operation (per batch b and head h, state S of dv rows x dk columns):
+ *
+ *     S_t = S_{t-1} . alpha_t (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,
+ *     o_t = S_t q_t                          (readout after the update)
+ *
+ * with alpha_t = exp(log_alpha_t) in (0,1) and beta_t in (0,1) one scalar per
+ * (b, t, h).  Sources: the Gated DeltaNet review at meaningful96.github.io/nr/GDN,
+ * section 1 (inputs q, k, v, alpha, beta; outputs S_t and o_t = S_t q_t) and
+ * section 3.4 (the gated delta rule); the same rule is stated in section
+ * "Method" of "Gated DeltaNet: Merging Gating and the Delta Rule to Beat
+ * Mamba2 on Language and Retrieval" (agihunt.info/en/papers/2412.06464).
+ * The forward and backward are computed chunkwise (64 tokens per chunk, UT
+ * transform / WY form, review section 3.7); the result equals the token
+ * recurrence up to rounding.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  * Pointers are DEVICE pointers (cudaMalloc / torch CUDA memory) on the
+ *    current device unless stated otherwise.  The caller owns every buffer;
+ *    the library never allocates device memory and keeps no state between
+ *    calls other than a per-device table of kernel attributes.
+ *  * All tensors are dense, row-major, contiguous:
+ *      q, k          [B, T, H, dk]      v, o, dO        [B, T, H, dv]
+ *      log_alpha     [B, T, H] fp32     beta            [B, T, H] fp32
+ *      S0, S_T, dS   [B, H, dv, dk] fp32 (always fp32)
+ *    q, k, v, o, dO, dq, dk, dv have the dtype `dt` (GDR_F32 or GDR_BF16).
+ *  * q and k are consumed as given: the library does not L2-normalise them
+ *    and applies no 1/sqrt(dk) scale (the block normalises them upstream).
+ *  * Supported sizes: dk, dv in {64, 128}; B, H >= 1; T >= 1 (a partial last
+ *    chunk is handled); B*T*H*max(dk,dv) < 2^31.  Others return
+ *    GDR_ERR_UNSUPPORTED (sizes) or GDR_ERR_INVALID_ARGUMENT (non-positive).
+ *  * Every pointer must be 16-byte aligned.  Required pointers that are
+ *    NULL, or misaligned pointers, return GDR_ERR_INVALID_ARGUMENT.
+ *  * Work is enqueued on `stream` (NULL = legacy default stream) and the call
+ *    returns without synchronising.  Argument errors are detected on the host
+ *    BEFORE anything is launched; nothing is written in that case.
+ *  * A launch failure returns GDR_ERR_CUDA.  Kernels that wait on on-chip
+ *    barriers give up after a bounded number of polls and record
+ *    GDR_ERR_TIMEOUT in a device status word, read by gdr_check_status().
+ *  * Outputs must not alias inputs (except S in gdr_step, which is in-out).
+ *  * gdr_last_error_string() describes the last non-OK status returned on the
+ *    calling thread.
+ */
+#ifndef GDR_H_
+#define GDR_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define GDR_API __attribute__((visibility("default")))
+#else
+#define GDR_API
+#endif
+
+/* Same type as cudaStream_t / CUstream; declared here so the header needs no
+ * CUDA include. */
+typedef struct CUstream_st *gdr_stream_t;
+
+typedef enum {
+    GDR_OK = 0,
+    GDR_ERR_INVALID_ARGUMENT = 1, /* NULL/misaligned pointer, non-positive size */
+    GDR_ERR_UNSUPPORTED = 2,      /* size or dtype this build does not handle  */
+    GDR_ERR_WORKSPACE = 3,        /* workspace NULL or smaller than required  */
+    GDR_ERR_CUDA = 4,             /* a CUDA runtime call or launch failed      */
+    GDR_ERR_TIMEOUT = 5           /* a bounded on-chip wait gave up (device)   */
+} gdr_status;
+
+typedef enum { GDR_F32 = 0, GDR_BF16 = 1 } gdr_dtype;
+
+/*
+ * Chunkwise forward.
+ *   in : q, k [B,T,H,dk]; v [B,T,H,dv] (dtype dt); log_alpha, beta [B,T,H]
+ *        fp32; S0 [B,H,dv,dk] fp32 or NULL (zero initial state).
+ *   out: o [B,T,H,dv] (dtype dt); S_T [B,H,dv,dk] fp32, or NULL to skip.
+ *   workspace: device scratch of at least gdr_fwd_workspace_bytes(...) bytes
+ *        (may be NULL when that is 0).
+ */
+GDR_API gdr_status gdr_fwd(int B, int T, int H, int dk, int dv, gdr_dtype dt,
+                   const void *q, const void *k, const void *v,
+                   const float *log_alpha, const float *beta, const float *S0,
+                   void *o, float *S_T, void *workspace, size_t workspace_bytes,
+                   gdr_stream_t stream);
+GDR_API size_t gdr_fwd_workspace_bytes(int B, int T, int H, int dk, int dv, gdr_dtype dt);
+
+/*
+ * Single-token recurrent decode (recurrent inference, review section 3.1:
+ * keeping only S_t makes token-by-token inference possible).
+ *   in : q, k [B,H,dk]; v [B,H,dv] (dtype dt); log_alpha, beta [B,H] fp32.
+ *   in/out: S [B,H,dv,dk] fp32, advanced by one token in place.
+ *   out: o [B,H,dv] (dtype dt) = S_t q.
+ */
+GDR_API gdr_status gdr_step(int B, int H, int dk, int dv, gdr_dtype dt,
+                    const void *q, const void *k, const void *v,
+                    const float *log_alpha, const float *beta,
+                    float *S, void *o, gdr_stream_t stream);
+
+/*
+ * Backward of gdr_fwd (reverse mode; the pages give none, it is the chain
+ * rule of the recurrence).  Loss gradients are taken with respect to the
+ * given q, k, v, log_alpha, beta and S0.
+ *   in : the forward's inputs (S0 may be NULL = 0); dO [B,T,H,dv] (dtype dt);
+ *        dS_T [B,H,dv,dk] fp32 or NULL (zero).
+ *   out: dq, dk [B,T,H,dk], dv [B,T,H,dv] (dtype dt); dlog_alpha, dbeta
+ *        [B,T,H] fp32; dS0 [B,H,dv,dk] fp32 or NULL to skip.
+ *   workspace: at least gdr_bwd_workspace_bytes(...) bytes (required): it
+ *        holds every chunk's starting state and per-slice partial gradients.
+ */
+GDR_API gdr_status gdr_bwd(int B, int T, int H, int dk, int dv, gdr_dtype dt,
+                   const void *q, const void *k, const void *v,
+                   const float *log_alpha, const float *beta, const float *S0,
+                   const void *dO, const float *dS_T,
+                   void *dq, void *dk_out, void *dv_out,
+                   float *dlog_alpha, float *dbeta, float *dS0,
+                   void *workspace, size_t workspace_bytes, gdr_stream_t stream);
+GDR_API size_t gdr_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, gdr_dtype dt);
+
+/*
+ * Gated Delta Rule-2 forward ("Gated DeltaNet-2: Decoupling Erase and Write
+ * in Linear Attention", agihunt.info/papers/2605.22791, Gated Delta Rule-2
+ * paragraph): per token, decay each key channel, read along b_t*k_t, write the
+ * residual of w_t*v_t along k_t:
+ *     S' = S_{t-1} Diag(alpha_t);  S_t = S' - (S'(b_t*k_t) - w_t*v_t) k_t^T;
+ *     o_t = S_t q_t.
+ *   in : q, k, v as gdr_fwd; log_alpha [B,T,H,dk] fp32 (per key channel);
+ *        b [B,T,H,dk] fp32 (erase gate); w [B,T,H,dv] fp32 (write gate);
+ *        S0 [B,H,dv,dk] fp32 or NULL.
+ *   out: o [B,T,H,dv] (dtype dt); S_T fp32 or NULL.
+ */
+GDR_API gdr_status gdr2_fwd(int B, int T, int H, int dk, int dv, gdr_dtype dt,
+                    const void *q, const void *k, const void *v,
+                    const float *log_alpha, const float *b, const float *w,
+                    const float *S0, void *o, float *S_T,
+                    void *workspace, size_t workspace_bytes, gdr_stream_t stream);
+GDR_API size_t gdr2_fwd_workspace_bytes(int B, int T, int H, int dk, int dv, gdr_dtype dt);
+
+/* Synchronise `stream`, then read and clear the device status word that
+ * kernels set when a bounded wait gives up.  Returns GDR_OK or
+ * GDR_ERR_TIMEOUT (or GDR_ERR_CUDA if the synchronisation itself failed). */
+GDR_API gdr_status gdr_check_status(gdr_stream_t stream);
+
+/* Text for the last non-OK status returned on this host thread. */
+GDR_API const char *gdr_last_error_string(void);
+
+/* Number of kernels this library has launched in this process (all
+ * threads); lets a caller count launches inside a timed region. */
+GDR_API uint64_t gdr_launch_count(void);
+
+/* Library version, (major << 16) | minor. */
+GDR_API int gdr_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GDR_H_ */

@@ -1,0 +1,80 @@
+"""The C-ABI library loads, exports every symbol include/gdr.h declares, and
+rejects bad arguments on the host before launching anything (CPU only)."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import gated_delta_rule_91_b200 as gdr
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "gdr.h")
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"GDR_API\s+[\w\s\*]*?\b(gdr\w*)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    names = declared_symbols()
+    assert len(names) >= 11
+    L = gdr.lib()
+    for n in names:
+        assert hasattr(L, n), n
+        assert n in gdr.SIGNATURES, n
+
+
+def test_version_and_counter():
+    assert gdr.lib().gdr_version() >= 1
+    assert gdr.launch_count() >= 0
+
+
+FAKE = 0x10000  # aligned, never dereferenced: every call below fails validation first
+
+
+def _fwd(B=1, T=4, H=1, dk=64, dv=64, dt=gdr.GDR_F32, q=FAKE, k=FAKE, v=FAKE, la=FAKE,
+         be=FAKE, S0=None, o=FAKE, ST=None):
+    P = ctypes.c_void_p
+    return gdr.lib().gdr_fwd(B, T, H, dk, dv, dt, P(q), P(k), P(v), P(la), P(be), P(S0), P(o),
+                             P(ST), None, 0, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(B=0), gdr.GDR_ERR_INVALID_ARGUMENT),
+    (dict(T=0), gdr.GDR_ERR_INVALID_ARGUMENT),
+    (dict(H=-1), gdr.GDR_ERR_INVALID_ARGUMENT),
+    (dict(dk=96), gdr.GDR_ERR_UNSUPPORTED),
+    (dict(dv=32), gdr.GDR_ERR_UNSUPPORTED),
+    (dict(dt=7), gdr.GDR_ERR_UNSUPPORTED),
+    (dict(q=None), gdr.GDR_ERR_INVALID_ARGUMENT),
+    (dict(o=None), gdr.GDR_ERR_INVALID_ARGUMENT),
+    (dict(k=FAKE + 4), gdr.GDR_ERR_INVALID_ARGUMENT),
+    (dict(S0=FAKE + 8), gdr.GDR_ERR_INVALID_ARGUMENT),
+    (dict(B=1 << 20, T=1 << 12, H=16), gdr.GDR_ERR_UNSUPPORTED),
+])
+def test_fwd_rejects_bad_arguments(kw, status):
+    assert _fwd(**kw) == status
+    assert gdr.lib().gdr_last_error_string().decode().startswith("gdr_fwd")
+
+
+def test_step_rejects_bad_arguments():
+    P = ctypes.c_void_p
+    L = gdr.lib()
+    assert L.gdr_step(1, 1, 64, 64, gdr.GDR_BF16, P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(FAKE),
+                      None, P(FAKE), None) == gdr.GDR_ERR_INVALID_ARGUMENT
+    assert L.gdr_step(1, 1, 48, 64, gdr.GDR_BF16, P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(FAKE),
+                      P(FAKE), P(FAKE), None) == gdr.GDR_ERR_UNSUPPORTED
+
+
+def test_python_binding_refuses_cpu_tensors():
+    x = torch.zeros(1, 4, 1, 64)
+    with pytest.raises((ValueError, RuntimeError)):
+        gdr.gdr_fwd(x, x, x, torch.zeros(1, 4, 1), torch.zeros(1, 4, 1))
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="only meaningful without a GPU")
+def test_valid_arguments_without_gpu_report_cuda_error():
+    # arguments pass validation; the launch then fails cleanly with no device
+    assert _fwd() == gdr.GDR_ERR_CUDA

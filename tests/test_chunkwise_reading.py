@@ -134,3 +134,90 @@ def test_mask_without_decay_is_wrong():
     U = Tm @ (beta[:, None] * V) - Tm @ ((beta * np.exp(g))[:, None] * K) @ S.T
     o_bad = np.exp(g)[:, None] * (Q @ S.T) + ((Q @ K.T) * np.tril(np.ones((n, n)))) @ U
     assert rel_err(o_bad, o[0, :, 0]) > 1e-2
+
+
+def chunkwise_gdr_bwd(q, k, v, la, be, S0, dO, dST, C=64):
+    """Per-chunk reverse mode of the chunkwise reading above (the formulas
+    the CUDA backward evaluates), fp64."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    g_all = {n: np.zeros_like(x) for n, x in (("dq", q), ("dk", k), ("dv", v), ("dla", la),
+                                              ("dbe", be))}
+    dS0 = np.zeros((B, H, dv, dk))
+    for b in range(B):
+        for h in range(H):
+            # forward: chunk entry states
+            S = np.zeros((dv, dk)) if S0 is None else S0[b, h].copy()
+            starts = []
+            for c0 in range(0, T, C):
+                starts.append(S.copy())
+                sl = slice(c0, min(c0 + C, T))
+                _, S = _chunk_fwd(q[b, sl, h], k[b, sl, h], v[b, sl, h], la[b, sl, h],
+                                  be[b, sl, h], S)
+            D = dST[b, h].copy() if dST is not None else np.zeros((dv, dk))
+            for ci in reversed(range(len(starts))):
+                c0 = ci * C
+                sl = slice(c0, min(c0 + C, T))
+                Q, K, V, dOc = q[b, sl, h], k[b, sl, h], v[b, sl, h], dO[b, sl, h]
+                beta = be[b, sl, h]
+                S = starts[ci]
+                n = Q.shape[0]
+                g = np.cumsum(la[b, sl, h])
+                gam = np.exp(g)
+                dec = np.exp(g[-1] - g)
+                ratio = np.exp(g[:, None] - g[None, :])
+                strict = np.tril(np.ones((n, n)), -1)
+                incl = np.tril(np.ones((n, n)))
+                G = strict * ratio * (K @ K.T)
+                A = beta[:, None] * G
+                P = incl * ratio * (Q @ K.T)
+                X = K @ S.T
+                Y = Q @ S.T
+                R = beta[:, None] * (V - gam[:, None] * X)
+                U = np.linalg.solve(np.eye(n) + A, R)
+                dU = dec[:, None] * (K @ D.T) + P.T @ dOc
+                dP = incl * (dOc @ U.T)
+                dR = np.linalg.solve((np.eye(n) + A).T, dU)
+                dA = -strict * (dR @ U.T)
+                dPL = dP * incl * ratio
+                dKK = dA * beta[:, None] * ratio * strict
+                UD = dec[:, None] * (U @ D)
+                dQ = gam[:, None] * (dOc @ S) + dPL @ K
+                dK = dPL.T @ Q + dKK @ K + dKK.T @ K + UD - (beta * gam)[:, None] * (dR @ S)
+                db = np.sum(dR * (V - gam[:, None] * X), 1) + np.sum(dA * G, 1)
+                E, F = dP * P, dA * A
+                z = np.sum(UD * K, 1)
+                dg = (gam * np.sum(dOc * Y, 1) - beta * gam * np.sum(dR * X, 1) - z
+                      + E.sum(1) - E.sum(0) + F.sum(1) - F.sum(0))
+                dg[-1] += gam[-1] * np.sum(D * S) + z.sum()
+                g_all["dq"][b, sl, h] = dQ
+                g_all["dk"][b, sl, h] = dK
+                g_all["dv"][b, sl, h] = beta[:, None] * dR
+                g_all["dbe"][b, sl, h] = db
+                g_all["dla"][b, sl, h] = np.cumsum(dg[::-1])[::-1]
+                D = gam[-1] * D + dOc.T @ (gam[:, None] * Q) - dR.T @ ((beta * gam)[:, None] * K)
+            dS0[b, h] = D
+    return dict(dq=g_all["dq"], dk=g_all["dk"], dv=g_all["dv"], dlog_alpha=g_all["dla"],
+                dbeta=g_all["dbe"], dS0=dS0)
+
+
+def _chunk_fwd(Q, K, V, la, beta, S):
+    g = np.cumsum(la)
+    n = len(g)
+    ratio = np.exp(g[:, None] - g[None, :])
+    A = np.tril(np.ones((n, n)), -1) * (beta[:, None] * ratio * (K @ K.T))
+    U = np.linalg.solve(np.eye(n) + A, beta[:, None] * (V - np.exp(g)[:, None] * (K @ S.T)))
+    O = np.exp(g)[:, None] * (Q @ S.T) + ((Q @ K.T) * ratio * np.tril(np.ones((n, n)))) @ U
+    return O, np.exp(g[-1]) * S + U.T @ (np.exp(g[-1] - g)[:, None] * K)
+
+
+@pytest.mark.parametrize("T,C", [(64, 64), (100, 64), (150, 16), (37, 8)])
+def test_chunkwise_backward_equals_oracle_reverse_mode(T, C):
+    rng = np.random.default_rng(T + C)
+    q, k, v, la, be, S0 = rand_inputs(rng, 1, T, 2, 8, 6)
+    dO = rng.normal(size=v.shape)
+    dST = rng.normal(size=(1, 2, 6, 8))
+    ref = oracle.gdr_bwd(q, k, v, la, be, S0, dO, dST)
+    got = chunkwise_gdr_bwd(q, k, v, la, be, S0, dO, dST, C)
+    for name in ref:
+        assert rel_err(got[name], ref[name]) < 1e-10, name
