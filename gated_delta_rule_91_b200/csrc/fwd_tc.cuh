@@ -53,9 +53,9 @@ struct FwdTcSmem {
     static constexpr uint32_t oSB = oW + 16384;               // S bf16 [c][j]    K-major, 32 KB
     static constexpr uint32_t oU = oSB;                       //   aliased later: U^T  [c][r] 16 KB
     static constexpr uint32_t oUt = oSB + 16384;              //                  U~^T [c][r] 16 KB
-    static constexpr uint32_t oA = oSB + 32768;               // fp32 A  64 x 65
-    static constexpr uint32_t oT = oA + 64 * 65 * 4;          // fp32 T  64 x 65
-    static constexpr uint32_t oGate = oT + 64 * 65 * 4;       // g, gamma, beta, dec (4 x 64 fp32)
+    static constexpr uint32_t oA = oSB + 32768;               // fp32 A  64 x 68
+    static constexpr uint32_t oT = oA + 64 * 68 * 4;          // fp32 T  64 x 68
+    static constexpr uint32_t oGate = oT + 64 * 68 * 4;       // g, gamma, beta, dec (4 x 64 fp32)
     static constexpr uint32_t oBar = oGate + 4 * 64 * 4;      // 3 mbarriers, tmem slot, abort flag
     static constexpr uint32_t kBytes = oBar + 64;
     static constexpr uint32_t kAlloc = kBytes + 1024;         // + alignment slack
@@ -64,45 +64,95 @@ struct FwdTcSmem {
 // TMEM column map (512 columns allocated)
 constexpr uint32_t kTmS = 0, kTmKQ = 128, kTmW = 192, kTmU = 256, kTmO1 = 320, kTmO2 = 384;
 
-// T = (I + A)^{-1} for strictly lower 64 x 64 A (fp32, row stride 65), using
-// 128 threads.  Only the lower triangle (incl. diagonal) of T is written; the
-// upper triangle of A is used as scratch.
+// Row stride (floats) of the fp32 64 x 64 matrices A and T: rows start on
+// 16-byte boundaries (vector loads) and 68 = 4 mod 32 spreads rows over banks.
+constexpr int kLdT = 68;
+
+// T = (I + A)^{-1} for strictly lower 64 x 64 A (fp32, row stride kLdT), with
+// 128 threads, by recursive doubling: 16 x 16 diagonal inverses by
+// substitution, then [[T1,0],[L21,T2]]^-1 = [[T1,0],[-T2 L21 T1, T2]] at the
+// 32 and 64 levels.  Only the lower triangle (incl. diagonal) of T is
+// meaningful.  The upper triangle of A holds the intermediate products.
 __device__ __forceinline__ void invert_unit_lower_64(float *sA, float *sT) {
-    constexpr int LD = 65;
+    constexpr int LD = kLdT;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    // diagonal 16 x 16 blocks: warp w solves block w, lane j owns column j
-    if (lane < 16) {
+    {   // zero T[0:16,16:32] and T[32:48,48:64] (upper parts of the 32-blocks)
+        const int idx = tid * 4, blk = idx >> 8, e = idx & 255;
+        float4 *p = reinterpret_cast<float4 *>(sT + (blk * 32 + (e >> 4)) * LD + blk * 32 + 16 + (e & 15));
+        *p = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    if (lane < 16) {  // 16 x 16 diagonal block `warp`, column `lane`
         const int base = warp * 16, j = lane;
         float t[16];
 #pragma unroll
         for (int r = 0; r < 16; ++r) {
-            float acc = (r == j) ? 1.f : 0.f;
+            float acc0 = (r == j) ? 1.f : 0.f, acc1 = 0.f;
 #pragma unroll
-            for (int i = 0; i < r; ++i) acc = fmaf(-sA[(base + r) * LD + base + i], t[i], acc);
-            t[r] = (r < j) ? 0.f : acc;
+            for (int i = 0; i + 1 < r; i += 2) {
+                acc0 = fmaf(-sA[(base + r) * LD + base + i], t[i], acc0);
+                acc1 = fmaf(-sA[(base + r) * LD + base + i + 1], t[i + 1], acc1);
+            }
+            if (r & 1) acc0 = fmaf(-sA[(base + r) * LD + base + r - 1], t[r - 1], acc0);
+            t[r] = (r < j) ? 0.f : acc0 + acc1;
         }
 #pragma unroll
         for (int r = 0; r < 16; ++r) sT[(base + r) * LD + base + j] = t[r];
     }
     __syncthreads();
-    // block rows I = 1..3: X_IJ = sum_{K=J}^{I-1} A_IK T_KJ, then T_IJ = -T_II X_IJ
-#pragma unroll 1
-    for (int I = 1; I < 4; ++I) {
-        for (int o = tid; o < I * 256; o += blockDim.x) {
-            const int J = o >> 8, r = (o >> 4) & 15, c = o & 15;
-            float acc = 0.f;
-            for (int kk = J * 16; kk < I * 16; ++kk)
-                acc = fmaf(sA[(I * 16 + r) * LD + kk], sT[kk * LD + J * 16 + c], acc);
-            sA[(J * 16 + c) * LD + I * 16 + r] = acc;  // X_IJ[r][c] parked in A's upper block (J, I)
+    // 32 level: for P in {0,1}: X = A[32P+16:32P+32, 32P:32P+16] t_{2P};  T21 = -t_{2P+1} X
+    {
+        const int P = tid >> 6, rr = (tid & 63) >> 2, cq = (tid & 3) * 4, o = 32 * P;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            const float a = sA[(o + 16 + rr) * LD + o + k];
+            const float4 t4 = *reinterpret_cast<const float4 *>(sT + (o + k) * LD + o + cq);
+            acc.x = fmaf(a, t4.x, acc.x); acc.y = fmaf(a, t4.y, acc.y);
+            acc.z = fmaf(a, t4.z, acc.z); acc.w = fmaf(a, t4.w, acc.w);
         }
+        *reinterpret_cast<float4 *>(sA + (o + rr) * LD + o + 16 + cq) = acc;  // X parked above the diagonal
         __syncthreads();
-        for (int o = tid; o < I * 256; o += blockDim.x) {
-            const int J = o >> 8, r = (o >> 4) & 15, c = o & 15;
-            float acc = 0.f;
-            for (int kk = 0; kk <= r; ++kk)
-                acc = fmaf(sT[(I * 16 + r) * LD + I * 16 + kk], sA[(J * 16 + c) * LD + I * 16 + kk], acc);
-            sT[(I * 16 + r) * LD + J * 16 + c] = -acc;
+        acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            const float t = sT[(o + 16 + rr) * LD + o + 16 + k];
+            const float4 x4 = *reinterpret_cast<const float4 *>(sA + (o + k) * LD + o + 16 + cq);
+            acc.x = fmaf(t, x4.x, acc.x); acc.y = fmaf(t, x4.y, acc.y);
+            acc.z = fmaf(t, x4.z, acc.z); acc.w = fmaf(t, x4.w, acc.w);
         }
+        *reinterpret_cast<float4 *>(sT + (o + 16 + rr) * LD + o + cq) =
+            make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
+        __syncthreads();
+    }
+    // 64 level: X = A[32:64, 0:32] T[0:32, 0:32];  T[32:64, 0:32] = -T[32:64, 32:64] X
+    {
+        const int r0 = (tid >> 3) * 2, cq = (tid & 7) * 4;
+        float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f), acc1 = acc0;
+#pragma unroll 8
+        for (int k = 0; k < 32; ++k) {
+            const float a0 = sA[(32 + r0) * LD + k], a1 = sA[(33 + r0) * LD + k];
+            const float4 t4 = *reinterpret_cast<const float4 *>(sT + k * LD + cq);
+            acc0.x = fmaf(a0, t4.x, acc0.x); acc0.y = fmaf(a0, t4.y, acc0.y);
+            acc0.z = fmaf(a0, t4.z, acc0.z); acc0.w = fmaf(a0, t4.w, acc0.w);
+            acc1.x = fmaf(a1, t4.x, acc1.x); acc1.y = fmaf(a1, t4.y, acc1.y);
+            acc1.z = fmaf(a1, t4.z, acc1.z); acc1.w = fmaf(a1, t4.w, acc1.w);
+        }
+        *reinterpret_cast<float4 *>(sA + r0 * LD + 32 + cq) = acc0;        // X parked in A[0:32, 32:64]
+        *reinterpret_cast<float4 *>(sA + (r0 + 1) * LD + 32 + cq) = acc1;
+        __syncthreads();
+        acc0 = make_float4(0.f, 0.f, 0.f, 0.f);
+        acc1 = acc0;
+#pragma unroll 8
+        for (int k = 0; k < 32; ++k) {
+            const float t0 = sT[(32 + r0) * LD + 32 + k], t1 = sT[(33 + r0) * LD + 32 + k];
+            const float4 x4 = *reinterpret_cast<const float4 *>(sA + k * LD + 32 + cq);
+            acc0.x = fmaf(t0, x4.x, acc0.x); acc0.y = fmaf(t0, x4.y, acc0.y);
+            acc0.z = fmaf(t0, x4.z, acc0.z); acc0.w = fmaf(t0, x4.w, acc0.w);
+            acc1.x = fmaf(t1, x4.x, acc1.x); acc1.y = fmaf(t1, x4.y, acc1.y);
+            acc1.z = fmaf(t1, x4.z, acc1.z); acc1.w = fmaf(t1, x4.w, acc1.w);
+        }
+        *reinterpret_cast<float4 *>(sT + (32 + r0) * LD + cq) = make_float4(-acc0.x, -acc0.y, -acc0.z, -acc0.w);
+        *reinterpret_cast<float4 *>(sT + (33 + r0) * LD + cq) = make_float4(-acc1.x, -acc1.y, -acc1.z, -acc1.w);
         __syncthreads();
     }
 }
@@ -261,7 +311,7 @@ gdr_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 const float gr = sg[r], br = sbeta[r];
 #pragma unroll
                 for (int i = 0; i < 64; ++i)
-                    sA[r * 65 + i] = (i < r) ? br * expf(gr - sg[i]) * v[i] : 0.f;
+                    sA[r * kLdT + i] = (i < r) ? br * expf(gr - sg[i]) * v[i] : 0.f;
             } else {
                 const int r = tid - 64;
                 const float gr = sg[r];
@@ -284,7 +334,7 @@ gdr_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const int i = ch * 8 + e;
-                    const float t = (i <= r) ? sT[r * 65 + i] : 0.f;
+                    const float t = (i <= r) ? sT[r * kLdT + i] : 0.f;
                     v[e] = t * sbeta[i] * (second ? sgam[i] : 1.f);
                 }
                 st_bf16x8(sm + (second ? L::oT2 : L::oT1) + sw128_offset(r, ch), v);
