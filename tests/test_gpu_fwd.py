@@ -101,8 +101,11 @@ def test_fwd_split_sequence_resume():
                          cut("log_alpha", 0, T1), cut("beta", 0, T1), d["S0"])
     o2, S2 = gdr.gdr_fwd(cut("q", T1, 300), cut("k", T1, 300), cut("v", T1, 300),
                          cut("log_alpha", T1, 300), cut("beta", T1, 300), S1)
-    assert max_rel(np64(torch.cat([o1, o2], 1)), np64(o)) <= 2e-2
-    assert fro_rel(np64(S2), np64(ST)) <= 1e-3
+    # The two runs place chunk boundaries differently, so the bf16 rounding of
+    # the MMA operands (S, U, W: unit roundoff 2^-8) happens at different
+    # points: agreement is bounded by the parity tolerances, not by fp32.
+    assert max_rel(np64(torch.cat([o1, o2], 1)), np64(o)) <= TOL_O["bf16"]
+    assert fro_rel(np64(S2), np64(ST)) <= TOL_S
 
 
 def test_fwd_deterministic():
