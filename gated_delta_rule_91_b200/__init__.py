@@ -33,6 +33,7 @@ SIGNATURES = {
     "gdr_step": (_I, [_I] * 5 + [_P] * 7 + [_P]),
     "gdr_bwd": (_I, [_I] * 6 + [_P] * 14 + [_P, _SZ, _P]),
     "gdr_bwd_workspace_bytes": (_SZ, [_I] * 6),
+    "gdr_bwd_noalloc": (_I, [_I] * 6 + [_P] * 14 + [_P]),
     "gdr2_fwd": (_I, [_I] * 6 + [_P] * 9 + [_P, _SZ, _P]),
     "gdr2_fwd_workspace_bytes": (_SZ, [_I] * 6),
     "gdr_check_status": (_I, [_P]),

@@ -7,6 +7,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <mutex>
 #include <string>
 
 #include "common.cuh"
@@ -245,3 +246,75 @@ gdr_status gdr2_fwd(int B, int T, int H, int dk, int dv, gdr_dtype dt, const voi
 }
 
 }  // extern "C"
+
+// ---- gdr_bwd_noalloc: backward with library-owned static scratch -------------
+// For callers that cannot allocate device memory: the scratch is this
+// file-scope device array (64 MiB on every GPU that loads the library).  In
+// host code `g_bwd_static_scratch` only names the symbol; its device address
+// comes from cudaGetSymbolAddress, resolved once per device.
+namespace {
+constexpr size_t kBwdStaticScratchBytes = (size_t)64 << 20;
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void *g_scratch_ptr[kMaxDevices] = {};
+}  // namespace
+static __device__ __align__(256) unsigned char g_bwd_static_scratch[kBwdStaticScratchBytes];
+
+extern "C" gdr_status gdr_bwd_noalloc(int B, int T, int H, int dk, int dv, gdr_dtype dt,
+                                      const void *q, const void *k, const void *v,
+                                      const float *log_alpha, const float *beta, const float *S0,
+                                      const void *dO, const float *dS_T, void *dq, void *dk_out,
+                                      void *dv_out, float *dlog_alpha, float *dbeta, float *dS0,
+                                      gdr_stream_t stream) {
+    const char *fn = "gdr_bwd_noalloc";
+    gdr_status st = check_dims(fn, B, T, H, dk, dv, dt);
+    if (st != GDR_OK) return st;
+    GDR_REQUIRE_PTR(q);
+    GDR_REQUIRE_PTR(k);
+    GDR_REQUIRE_PTR(v);
+    GDR_REQUIRE_PTR(log_alpha);
+    GDR_REQUIRE_PTR(beta);
+    GDR_REQUIRE_PTR(dO);
+    GDR_REQUIRE_PTR(dq);
+    GDR_REQUIRE_PTR(dk_out);
+    GDR_REQUIRE_PTR(dv_out);
+    GDR_REQUIRE_PTR(dlog_alpha);
+    GDR_REQUIRE_PTR(dbeta);
+    GDR_OPTIONAL_PTR(S0);
+    GDR_OPTIONAL_PTR(dS_T);
+    GDR_OPTIONAL_PTR(dS0);
+    const size_t need = bwd_workspace_bytes(B, T, H, dk, dv);
+    if (need > kBwdStaticScratchBytes)
+        return fail(GDR_ERR_WORKSPACE,
+                    "%s: this problem needs %zu bytes of scratch; the static scratch holds %zu "
+                    "(use gdr_bwd with a caller workspace)",
+                    fn, need, kBwdStaticScratchBytes);
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "gdr_bwd_noalloc: cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices)
+        return fail(GDR_ERR_UNSUPPORTED, "%s: device ordinal %d out of range", fn, dev);
+    void *scratch = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_scratch_mu);
+        if (g_scratch_ptr[dev] == nullptr) {
+            e = cudaGetSymbolAddress(&g_scratch_ptr[dev], g_bwd_static_scratch);
+            if (e != cudaSuccess) {
+                g_scratch_ptr[dev] = nullptr;
+                return cuda_fail(e, "gdr_bwd_noalloc: cudaGetSymbolAddress");
+            }
+        }
+        scratch = g_scratch_ptr[dev];
+    }
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+#define GDR_BWD_ARGS B, T, H, dv, q, k, v, log_alpha, beta, S0, dO, dS_T, dq, dk_out, dv_out, \
+                     dlog_alpha, dbeta, dS0, scratch, s
+    if (dt == GDR_F32)
+        e = dk == 128 ? launch_bwd_simt<float, 128>(GDR_BWD_ARGS) : launch_bwd_simt<float, 64>(GDR_BWD_ARGS);
+    else
+        e = dk == 128 ? launch_bwd_simt<__nv_bfloat16, 128>(GDR_BWD_ARGS)
+                      : launch_bwd_simt<__nv_bfloat16, 64>(GDR_BWD_ARGS);
+#undef GDR_BWD_ARGS
+    if (e != cudaSuccess) return cuda_fail(e, fn);
+    return GDR_OK;
+}

@@ -123,6 +123,39 @@ GDR_API gdr_status gdr_bwd(int B, int T, int H, int dk, int dv, gdr_dtype dt,
 GDR_API size_t gdr_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, gdr_dtype dt);
 
 /*
+ * gdr_bwd without caller-provided workspace.  This entry point has no
+ * counterpart in the pages; it exists for callers that cannot allocate
+ * device memory at the point where they need the backward -- for example
+ * code running inside a pool or arena that owns all device memory, an
+ * embedding runtime that forbids cudaMalloc after start-up, or an
+ * allocation-free hot loop.  The caller still owns and passes every input
+ * and output buffer (same arguments and meaning as gdr_bwd, minus the
+ * workspace).
+ *
+ * The scratch it needs (chunk-entry states and per-slice partial
+ * gradients) lives in a fixed 64 MiB static device array inside libgdr.so,
+ * so every GPU that loads the library holds those 64 MiB until the
+ * process exits.  Problems whose scratch exceeds 64 MiB
+ * (gdr_bwd_workspace_bytes(...) > 64 MiB) are rejected on the host with
+ * GDR_ERR_WORKSPACE before anything is launched.  It calls no cudaMalloc,
+ * cudaFree or other allocating routine.
+ *
+ * The first call on each device resolves the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  All calls share the one array and it keeps
+ * the last call's contents (nothing in it needs to start at zero: every
+ * byte a call reads is written earlier in the same call), so calls whose
+ * work overlaps on the GPU (different streams, or threads racing on one
+ * device) race on the scratch: serialise them.
+ */
+GDR_API gdr_status gdr_bwd_noalloc(int B, int T, int H, int dk, int dv, gdr_dtype dt,
+                   const void *q, const void *k, const void *v,
+                   const float *log_alpha, const float *beta, const float *S0,
+                   const void *dO, const float *dS_T,
+                   void *dq, void *dk_out, void *dv_out,
+                   float *dlog_alpha, float *dbeta, float *dS0, gdr_stream_t stream);
+
+/*
  * Gated Delta Rule-2 forward ("Gated DeltaNet-2: Decoupling Erase and Write
  * in Linear Attention", agihunt.info/papers/2605.22791, Gated Delta Rule-2
  * paragraph): per token, decay each key channel, read along b_t*k_t, write the
