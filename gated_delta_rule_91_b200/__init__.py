@@ -37,6 +37,7 @@ SIGNATURES = {
     "gdr2_fwd": (_I, [_I] * 6 + [_P] * 9 + [_P, _SZ, _P]),
     "gdr2_fwd_workspace_bytes": (_SZ, [_I] * 6),
     "gdr_check_status": (_I, [_P]),
+    "gdr_debug_wait_timeout": (_I, [_I, _P]),
     "gdr_last_error_string": (ctypes.c_char_p, []),
     "gdr_launch_count": (ctypes.c_uint64, []),
     "gdr_version": (_I, []),

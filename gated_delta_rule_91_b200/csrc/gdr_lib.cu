@@ -16,6 +16,7 @@
 #include "bwd_simt.cuh"
 #include "gdr2_simt.cuh"
 #include "fwd_tc.cuh"
+#include "fwd_tc2.cuh"
 
 namespace gdr {
 std::atomic<uint64_t> g_launches{0};
@@ -96,6 +97,28 @@ gdr_status gdr_check_status(gdr_stream_t stream) {
     return GDR_OK;
 }
 
+// One thread waits, with a short bound, on a barrier that never completes.
+__global__ void gdr_timeout_probe_kernel(uint64_t limit_ns) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        sm100::mbar_init(&bar, 1);
+        sm100::fence_mbar_init();
+        if (!sm100::mbar_wait(&bar, 0, limit_ns)) record_status(GDR_ERR_TIMEOUT);
+    }
+}
+
+gdr_status gdr_debug_wait_timeout(int timeout_ms, gdr_stream_t stream) {
+    const char *fn = "gdr_debug_wait_timeout";
+    if (timeout_ms < 1 || timeout_ms > 10000)
+        return fail(GDR_ERR_INVALID_ARGUMENT, "%s: timeout_ms=%d (1..10000)", fn, timeout_ms);
+    gdr_timeout_probe_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        (uint64_t)timeout_ms * 1000000ull);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, fn);
+    return GDR_OK;
+}
+
 size_t gdr_fwd_workspace_bytes(int, int, int, int, int, gdr_dtype) { return 0; }
 
 gdr_status gdr_fwd(int B, int T, int H, int dk, int dv, gdr_dtype dt, const void *q, const void *k,
@@ -120,12 +143,15 @@ gdr_status gdr_fwd(int B, int T, int H, int dk, int dv, gdr_dtype dt, const void
                     workspace ? workspace_bytes : (size_t)0);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e;
-    // bf16 with dk = dv = 128 runs on the tensor cores; GDR_FWD_KERNEL=simt
-    // selects the CUDA-core kernel instead (used to cross-check the two).
+    // bf16 with dk = dv = 128 runs on the tensor cores (the two-SM cluster
+    // kernel); GDR_FWD_KERNEL=tc1 selects the single-CTA tensor-core kernel and
+    // GDR_FWD_KERNEL=simt the CUDA-core kernel (used to cross-check them).
     const char *sel = getenv("GDR_FWD_KERNEL");
     const bool force_simt = sel != nullptr && strcmp(sel, "simt") == 0;
+    const bool force_tc1 = sel != nullptr && strcmp(sel, "tc1") == 0;
     if (dt == GDR_BF16 && dk == 128 && dv == 128 && !force_simt) {
-        e = launch_fwd_tc(B, T, H, q, k, v, log_alpha, beta, S0, o, S_T, s);
+        e = force_tc1 ? launch_fwd_tc(B, T, H, q, k, v, log_alpha, beta, S0, o, S_T, s)
+                      : launch_fwd_tc2(B, T, H, q, k, v, log_alpha, beta, S0, o, S_T, s);
         if (e != cudaSuccess) return cuda_fail(e, fn);
         return GDR_OK;
     }

@@ -25,9 +25,18 @@
 namespace gdr {
 namespace sm100 {
 
-// Polls before a wait gives up.  At ~100 ns per failed try_wait this is
-// seconds, far beyond any legitimate wait inside one chunk.
-constexpr uint32_t kWaitLimit = 1u << 26;
+// A wait gives up after this much wall-clock time (global timer, ns): far
+// beyond any legitimate wait inside one chunk (microseconds), short enough
+// that a lost arrival ends the kernel with an error instead of a hang.
+// (try_wait may suspend the thread between polls, so the bound is in time,
+// not in polls.)
+constexpr uint64_t kWaitNs = 4000000000ull;
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -46,9 +55,10 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
                  : "memory");
 }
 // Wait until the phase with parity `parity` has completed; false on timeout.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64_t limit_ns = kWaitNs) {
     const uint32_t addr = smem_u32(bar);
-    for (uint32_t it = 0; it < kWaitLimit; ++it) {
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 1;; ++it) {
         uint32_t done;
         asm volatile(
             "{\n .reg .pred p;\n"
@@ -58,8 +68,59 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
             : "r"(addr), "r"(parity)
             : "memory");
         if (done) return true;
+        if ((it & 255u) == 0 && global_timer_ns() - t0 > limit_ns) return false;
     }
-    return false;
+}
+
+// Same wait, acquiring at cluster scope (the phase was completed by another
+// CTA of the cluster: a remote arrive or a DSMEM bulk copy).
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity) {
+    const uint32_t addr = smem_u32(bar);
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 1;; ++it) {
+        uint32_t done;
+        asm volatile(
+            "{\n .reg .pred p;\n"
+            " mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n"
+            " selp.u32 %0, 1, 0, p;\n}\n"
+            : "=r"(done)
+            : "r"(addr), "r"(parity)
+            : "memory");
+        if (done) return true;
+        if ((it & 255u) == 0 && global_timer_ns() - t0 > kWaitNs) return false;
+    }
+}
+
+// ---- thread-block cluster ---------------------------------------------------
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// Shared::cluster address of the same offset as `p` in cluster CTA `rank`.
+__device__ __forceinline__ uint32_t cluster_addr(const void *p, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Arrive once on a barrier in another CTA of the cluster (release at cluster scope).
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_bar_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar_addr)
+                 : "memory");
+}
+// Bulk copy of `bytes` (multiple of 16) from this CTA's shared memory into
+// another CTA's shared memory; completes `bytes` of transaction count on the
+// destination CTA's barrier.
+__device__ __forceinline__ void bulk_copy_to_cluster(uint32_t dst_cluster_addr, const void *src,
+                                                     uint32_t bytes, uint32_t bar_cluster_addr) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            dst_cluster_addr),
+        "r"(smem_u32(src)), "r"(bytes), "r"(bar_cluster_addr)
+        : "memory");
 }
 
 // ---- TMA ----------------------------------------------------------------------

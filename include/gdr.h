@@ -179,6 +179,14 @@ GDR_API size_t gdr2_fwd_workspace_bytes(int B, int T, int H, int dk, int dv, gdr
  * GDR_ERR_TIMEOUT (or GDR_ERR_CUDA if the synchronisation itself failed). */
 GDR_API gdr_status gdr_check_status(gdr_stream_t stream);
 
+/* Test hook for the timeout path: launches a one-thread kernel that waits on
+ * an on-chip barrier nothing ever arrives on, with a bound of `timeout_ms`
+ * milliseconds (1..10000).  The wait runs out, the kernel records
+ * GDR_ERR_TIMEOUT in the device status word and returns normally: no fault,
+ * no trap, the context stays usable.  A following gdr_check_status(stream)
+ * returns GDR_ERR_TIMEOUT (and clears the word). */
+GDR_API gdr_status gdr_debug_wait_timeout(int timeout_ms, gdr_stream_t stream);
+
 /* Text for the last non-OK status returned on this host thread. */
 GDR_API const char *gdr_last_error_string(void);
 

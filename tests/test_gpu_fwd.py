@@ -115,12 +115,18 @@ def test_fwd_deterministic():
     assert torch.equal(o1, o2) and torch.equal(S1, S2)
 
 
+@pytest.mark.parametrize("kernel", ["default", "tc1"])
 @pytest.mark.parametrize("T", [64, 129, 1000])
-def test_tensor_core_forward_matches_cuda_core_forward(T, monkeypatch):
-    """bf16 d=128 runs on tcgen05; the fp32 CUDA-core kernel on the same
-    inputs must agree within the bf16 tolerance (and both with the oracle)."""
+def test_tensor_core_forward_matches_cuda_core_forward(T, kernel, monkeypatch):
+    """bf16 d=128 runs on tcgen05 (the two-SM cluster kernel by default, the
+    single-CTA kernel with GDR_FWD_KERNEL=tc1); the fp32 CUDA-core kernel on
+    the same inputs must agree within the bf16 tolerance (and both with the
+    oracle)."""
     x = synth.gdr_inputs(2, T, 3, 128, 128, "bf16", seed=40 + T, s0_std=0.02)
+    if kernel != "default":
+        monkeypatch.setenv("GDR_FWD_KERNEL", kernel)
     o_tc, S_tc = _run(x)
+    gdr.check_status()
     monkeypatch.setenv("GDR_FWD_KERNEL", "simt")
     o_si, S_si = _run(x)
     assert max_rel(np64(o_tc), np64(o_si)) <= TOL_O["bf16"]
