@@ -1,5 +1,5 @@
 // fwd_tc2.cuh -- chunkwise forward on tcgen05, split over a 2-CTA cluster
-// per (b, h): a "prep" CTA and a "state" CTA on two SMs.
+// per (b, h): a "prep" CTA and a "state" CTA on two SMs, 256 threads each.
 //
 // Same chunk algebra and operand orientation as fwd_tc.cuh (Gated DeltaNet
 // review, meaningful96.github.io/nr/GDN, section 3.7: UT transform / WY form
@@ -16,12 +16,18 @@
 //     W^T = K^T T''^T, U^gT = V^T T'^T       (issued one chunk ahead)
 //     U^T -= S W^T,  O^T = S Q~^T           (S read as bf16 operand)
 //     O^T += U^T P^T,  S = gamma_C S + U~^T K
-// so the state CTA's critical path per chunk is: S -> bf16 operand, two MMA
-// groups and one U round trip; the epilogue of chunk n-1 and the W/U^g
-// products of chunk n+1 overlap its MMAs (double-buffered U and O
-// accumulators).  Hand-off slots are released back to the prep CTA with a
-// remote mbarrier arrive.  No TMA multicast anywhere; each CTA loads its own
-// tiles (the shared K/Q tiles hit L2 for the second reader).
+//     O staged in shared memory and written by a TMA store.
+// The decay ratio exp(g_r - g_i) of the masks is formed as
+// gamma'_r * (1/gamma'_i) with gamma' = exp(g - g_31) taken about the chunk's
+// middle token (two multiplies per element, no exponential); a chunk whose
+// decay range exceeds e^80 (where those factors could overflow) takes the
+// exact per-element exponential instead.
+//
+// Warps 0-3 and 4-7 of each CTA own TMEM lane quarters 0-3 and split the
+// columns; thread 0 issues TMA and MMA.  The prep waits for a free hand-off
+// slot only after the inverse, so the state CTA's tail overlaps it.  Slots go
+// back to the prep CTA with a remote mbarrier arrive.  No TMA multicast; each
+// CTA loads its own tiles (the shared K/Q tiles hit L2 for the second reader).
 #pragma once
 #include <cuda.h>
 
@@ -30,6 +36,8 @@
 #include "sm100.cuh"
 
 namespace gdr {
+
+constexpr int kTc2Threads = 256;
 
 struct Tc2Layout {
     // hand-off slot (identical offsets in the prep staging area and the state slots)
@@ -46,7 +54,8 @@ struct Tc2Layout {
     static constexpr uint32_t S_H = S_V + 2 * 16384;      // 2 hand-off slots
     static constexpr uint32_t S_W = S_H + 2 * H_SLOT;     // W [j][r] MN-major, 16 KB
     static constexpr uint32_t S_SB = S_W + 16384;         // S bf16 [c][j] (32 KB); later U^T, U~^T
-    static constexpr uint32_t S_GL = S_SB + 32768;        // gamma of chunks n, n-1: [2][64] fp32
+    static constexpr uint32_t S_OST = S_SB + 32768;       // O tile for the TMA store, 2 halves x 8 KB
+    static constexpr uint32_t S_GL = S_OST + 16384;       // gamma of chunks by parity: [2][64] fp32
     static constexpr uint32_t S_BAR = S_GL + 512;
     static constexpr uint32_t S_BYTES = S_BAR + 128;
     // prep CTA
@@ -54,12 +63,13 @@ struct Tc2Layout {
     static constexpr uint32_t P_A = P_KQ + 2 * 32768;
     static constexpr uint32_t P_T = P_A + 64 * kLdT * 4;
     static constexpr uint32_t P_STG = P_T + 64 * kLdT * 4;  // 2 staging slots
-    static constexpr uint32_t P_GATE = P_STG + 2 * H_SLOT;  // g[64], beta[64]
-    static constexpr uint32_t P_BAR = P_GATE + 512;
+    static constexpr uint32_t P_GATE = P_STG + 2 * H_SLOT;  // g, beta, gamma, dec, gamma', 1/gamma' [64] + flag
+    static constexpr uint32_t P_BAR = P_GATE + 6 * 256 + 16;
     static constexpr uint32_t P_BYTES = P_BAR + 128;
     static constexpr uint32_t kAlloc = (S_BYTES > P_BYTES ? S_BYTES : P_BYTES) + 1024;
 };
-static_assert(Tc2Layout::S_H % 1024 == 0 && Tc2Layout::S_W % 1024 == 0 && Tc2Layout::S_SB % 1024 == 0,
+static_assert(Tc2Layout::S_H % 1024 == 0 && Tc2Layout::S_W % 1024 == 0 && Tc2Layout::S_SB % 1024 == 0 &&
+                  Tc2Layout::S_OST % 1024 == 0,
               "state tiles must be 1024-aligned");
 static_assert(Tc2Layout::P_STG % 1024 == 0 && Tc2Layout::H_SLOT % 1024 == 0, "slots must be 1024-aligned");
 static_assert(Tc2Layout::kAlloc <= 232448, "shared memory budget");
@@ -67,24 +77,83 @@ static_assert(Tc2Layout::kAlloc <= 232448, "shared memory budget");
 // state TMEM columns (512 allocated)
 constexpr uint32_t kT2S = 0, kT2W = 128, kT2U = 192, kT2O = 320;  // U, O double-buffered (+64)
 
-__device__ __forceinline__ void tc2_gates(int lane, int nv, const float *la, const float *bt, size_t H,
-                                          float *g, float *gam, float *beta, float *dec) {
-    const int r0 = 2 * lane, r1 = r0 + 1;
-    const float l0 = r0 < nv ? la[(size_t)r0 * H] : 0.f;
-    const float l1 = r1 < nv ? la[(size_t)r1 * H] : 0.f;
-    float incl = l0 + l1;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-        const float y = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += y;
+// T = (I + A)^{-1} for strictly lower 64 x 64 A (fp32, row stride kLdT) with
+// 256 threads; same recursive doubling as invert_unit_lower_64 (16 x 16
+// diagonal inverses by substitution, then the 32 and 64 levels), retiled for
+// eight warps.  Only the lower triangle of T is meaningful; the upper
+// triangle of A holds the intermediate products.
+__device__ __forceinline__ void invert_unit_lower_64_w8(float *sA, float *sT) {
+    constexpr int LD = kLdT;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    {   // zero T[0:16,16:32] and T[32:48,48:64]
+        const int idx = tid * 2, blk = idx >> 8, e = idx & 255;
+        float2 *p = reinterpret_cast<float2 *>(sT + (blk * 32 + (e >> 4)) * LD + blk * 32 + 16 + (e & 15));
+        *p = make_float2(0.f, 0.f);
     }
-    const float g1 = incl, g0 = incl - l1;
-    const float gC = __shfl_sync(0xffffffffu, incl, 31);
-    g[r0] = g0; g[r1] = g1;
-    gam[r0] = expf(g0); gam[r1] = expf(g1);
-    dec[r0] = expf(gC - g0); dec[r1] = expf(gC - g1);
-    beta[r0] = r0 < nv ? bt[(size_t)r0 * H] : 0.f;
-    beta[r1] = r1 < nv ? bt[(size_t)r1 * H] : 0.f;
+    if (warp < 4 && lane < 16) {  // 16 x 16 diagonal block `warp`, column `lane`
+        const int base = warp * 16, j = lane;
+        float t[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+            float acc0 = (r == j) ? 1.f : 0.f, acc1 = 0.f;
+#pragma unroll
+            for (int i = 0; i + 1 < r; i += 2) {
+                acc0 = fmaf(-sA[(base + r) * LD + base + i], t[i], acc0);
+                acc1 = fmaf(-sA[(base + r) * LD + base + i + 1], t[i + 1], acc1);
+            }
+            if (r & 1) acc0 = fmaf(-sA[(base + r) * LD + base + r - 1], t[r - 1], acc0);
+            t[r] = (r < j) ? 0.f : acc0 + acc1;
+        }
+#pragma unroll
+        for (int r = 0; r < 16; ++r) sT[(base + r) * LD + base + j] = t[r];
+    }
+    __syncthreads();
+    {   // 32 level: X = A[o+16:o+32, o:o+16] t_{2P};  T[o+16:o+32, o:o+16] = -t_{2P+1} X
+        const int P = tid >> 7, rr = (tid & 127) >> 3, cq = (tid & 7) * 2, o = 32 * P;
+        float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            const float a = sA[(o + 16 + rr) * LD + o + k];
+            const float2 t2 = *reinterpret_cast<const float2 *>(sT + (o + k) * LD + o + cq);
+            acc.x = fmaf(a, t2.x, acc.x);
+            acc.y = fmaf(a, t2.y, acc.y);
+        }
+        *reinterpret_cast<float2 *>(sA + (o + rr) * LD + o + 16 + cq) = acc;
+        __syncthreads();
+        acc = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            const float t = sT[(o + 16 + rr) * LD + o + 16 + k];
+            const float2 x2 = *reinterpret_cast<const float2 *>(sA + (o + k) * LD + o + 16 + cq);
+            acc.x = fmaf(t, x2.x, acc.x);
+            acc.y = fmaf(t, x2.y, acc.y);
+        }
+        *reinterpret_cast<float2 *>(sT + (o + 16 + rr) * LD + o + cq) = make_float2(-acc.x, -acc.y);
+        __syncthreads();
+    }
+    {   // 64 level: X = A[32:64, 0:32] T[0:32, 0:32];  T[32:64, 0:32] = -T[32:64, 32:64] X
+        const int r = tid >> 3, cq = (tid & 7) * 4;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+        for (int k = 0; k < 32; ++k) {
+            const float a = sA[(32 + r) * LD + k];
+            const float4 t4 = *reinterpret_cast<const float4 *>(sT + k * LD + cq);
+            acc.x = fmaf(a, t4.x, acc.x); acc.y = fmaf(a, t4.y, acc.y);
+            acc.z = fmaf(a, t4.z, acc.z); acc.w = fmaf(a, t4.w, acc.w);
+        }
+        *reinterpret_cast<float4 *>(sA + r * LD + 32 + cq) = acc;
+        __syncthreads();
+        acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+        for (int k = 0; k < 32; ++k) {
+            const float t = sT[(32 + r) * LD + 32 + k];
+            const float4 x4 = *reinterpret_cast<const float4 *>(sA + k * LD + 32 + cq);
+            acc.x = fmaf(t, x4.x, acc.x); acc.y = fmaf(t, x4.y, acc.y);
+            acc.z = fmaf(t, x4.z, acc.z); acc.w = fmaf(t, x4.w, acc.w);
+        }
+        *reinterpret_cast<float4 *>(sT + (32 + r) * LD + cq) = make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
+        __syncthreads();
+    }
 }
 
 // ------------------------------------------------------------------ prep CTA --
@@ -93,14 +162,17 @@ __device__ __forceinline__ void tc2_prep(uint8_t *sm, const CUtensorMap *tm_q, c
                                          const float *beta) {
     using L = Tc2Layout;
     using namespace sm100;
-    const int tid = threadIdx.x, warp = tid >> 5;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int wq = warp & 3, wh = warp >> 2;  // TMEM lane quarter, column half
     const int nch = (T + kChunk - 1) / kChunk;
     uint64_t *tma_full = reinterpret_cast<uint64_t *>(sm + L::P_BAR);  // [2]
     uint64_t *empty = tma_full + 2;                                      // [2], arrived by the state CTA
     uint64_t *mma_bar = tma_full + 4;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tma_full + 5);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    float *sg = reinterpret_cast<float *>(sm + L::P_GATE), *sbeta = sg + 64;
+    float *sg = reinterpret_cast<float *>(sm + L::P_GATE);
+    float *sbeta = sg + 64, *sgam = sg + 128, *sdec = sg + 192, *sgp = sg + 256, *sinv = sg + 320;
+    volatile int *exact_flag = reinterpret_cast<volatile int *>(sg + 384);
     float *sA = reinterpret_cast<float *>(sm + L::P_A), *sT = reinterpret_cast<float *>(sm + L::P_T);
     const uint32_t sbase = smem_u32(sm);
 
@@ -121,7 +193,7 @@ __device__ __forceinline__ void tc2_prep(uint8_t *sm, const CUtensorMap *tm_q, c
     tc_after_sync();
     cluster_sync();  // both CTAs' barriers are initialised (and the state's slots armed)
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
+    const uint32_t tl = tmem + ((uint32_t)(wq * 32) << 16);
     const uint32_t remote_slot0 = cluster_addr(sm + L::S_H, 1);
     const uint32_t remote_full0 = cluster_addr(sm + L::S_BAR + 16, 1);  // state's hand_full[0]
 
@@ -143,6 +215,18 @@ __device__ __forceinline__ void tc2_prep(uint8_t *sm, const CUtensorMap *tm_q, c
         }
         mma_commit(mma_bar);
     };
+    // gates of one chunk, held by warp 0 (lane l: rows 2l, 2l+1) between load and use
+    float pl0 = 0.f, pl1 = 0.f, pb0 = 0.f, pb1 = 0.f;
+    auto load_gates = [&](int n) {
+        const int c0 = n * kChunk, nv = min(kChunk, T - c0);
+        const size_t tok0 = ((size_t)b * T + c0) * H + h;
+        const int r0 = 2 * lane, r1 = r0 + 1;
+        pl0 = r0 < nv ? log_alpha[tok0 + (size_t)r0 * H] : 0.f;
+        pl1 = r1 < nv ? log_alpha[tok0 + (size_t)r1 * H] : 0.f;
+        pb0 = r0 < nv ? beta[tok0 + (size_t)r0 * H] : 0.f;
+        pb1 = r1 < nv ? beta[tok0 + (size_t)r1 * H] : 0.f;
+    };
+    if (warp == 0) load_gates(0);
 
     int tma_issued = 0, tma_done = 0;
     uint32_t mma_phase = 0;
@@ -164,62 +248,68 @@ __device__ __forceinline__ void tc2_prep(uint8_t *sm, const CUtensorMap *tm_q, c
 #pragma unroll 1
     for (int n = 0; n < nch; ++n) {
         const int s = n & 1;
-        const int c0 = n * kChunk, nv = min(kChunk, T - c0);
-        const size_t tok0 = ((size_t)b * T + c0) * H + h;
         uint8_t *stg = sm + L::P_STG + s * L::H_SLOT;
-        float *hg = reinterpret_cast<float *>(stg + L::H_G);
         __syncthreads();
         if (*abort_flag) break;
-        if (tid == 0) {
-            // staging slot s (and the state's slot s) must have been consumed (chunk n-2)
-            if (n >= 2 && !mbar_wait_cluster(&empty[s], (uint32_t)(((n >> 1) - 1) & 1))) *abort_flag = 1;
-            if (!mbar_wait(mma_bar, mma_phase)) *abort_flag = 1;
+        if (warp == 0) {  // gates: g (inclusive prefix sum), gamma, dec, gamma' = exp(g - g_31), 1/gamma'
+            const int r0 = 2 * lane, r1 = r0 + 1;
+            float incl = pl0 + pl1;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, incl, off);
+                if (lane >= off) incl += y;
+            }
+            const float g1 = incl, g0 = incl - pl1;
+            const float gC = __shfl_sync(0xffffffffu, incl, 31);
+            const float gM = __shfl_sync(0xffffffffu, g1, 15);  // g_31
+            const float gF = __shfl_sync(0xffffffffu, g0, 0);   // g_0
+            sg[r0] = g0; sg[r1] = g1;
+            sbeta[r0] = pb0; sbeta[r1] = pb1;
+            sgam[r0] = expf(g0); sgam[r1] = expf(g1);
+            sdec[r0] = expf(gC - g0); sdec[r1] = expf(gC - g1);
+            sgp[r0] = expf(g0 - gM); sgp[r1] = expf(g1 - gM);
+            sinv[r0] = expf(gM - g0); sinv[r1] = expf(gM - g1);
+            if (lane == 0) *exact_flag = (gF - gC) > 80.f;
+            if (n + 1 < nch) load_gates(n + 1);  // prefetch: consumed next chunk
         }
+        if (tid == 0 && !mbar_wait(mma_bar, mma_phase)) *abort_flag = 1;
         mma_phase ^= 1;
-        if (warp == 0) tc2_gates(tid, nv, log_alpha + tok0, beta + tok0, (size_t)H, sg, hg, sbeta, hg + 64);
         tc_before_sync();
         __syncthreads();
         if (*abort_flag) break;
         tc_after_sync();
 
-        // A (fp32, rows 0-63) and P (bf16 into the staging slot, rows 64-127)
+        // A (fp32, rows 0-63 -> sA) and P (rows 64-127, kept in registers), this
+        // thread's 32 columns of its TMEM lane
+        const int row = wq * 32 + lane;  // 0..127
+        const int c0 = wh * 32;
+        float pv[32];
         {
-            float v[64];
-            tmem_ld32(tl, v);
-            tmem_ld32(tl + 32, v + 32);
-            if (tid < 64) {
-                const int r = tid;
-                const float gr = sg[r], br = sbeta[r];
+            tmem_ld32(tl + c0, pv);
+            const bool exact = *exact_flag;
+            if (row < 64) {
+                const int r = row;
+                const float gr = sg[r], f = sbeta[r] * sgp[r], br = sbeta[r];
 #pragma unroll
-                for (int i = 0; i < 64; ++i) sA[r * kLdT + i] = (i < r) ? br * __expf(gr - sg[i]) * v[i] : 0.f;
+                for (int i = 0; i < 32; ++i) {
+                    const int col = c0 + i;
+                    const float d = exact ? br * __expf(gr - sg[col]) : f * sinv[col];
+                    sA[r * kLdT + col] = (col < r) ? d * pv[i] : 0.f;
+                }
             } else {
-                const int r = tid - 64;
-                const float gr = sg[r];
+                const int r = row - 64;
+                const float gr = sg[r], f = sgp[r];
 #pragma unroll
-                for (int i = 0; i < 64; ++i) v[i] = (i <= r) ? __expf(gr - sg[i]) * v[i] : 0.f;
-#pragma unroll
-                for (int ch = 0; ch < 8; ++ch) st_bf16x8(stg + L::H_P + sw128_offset(r, ch), v + 8 * ch);
-            }
-        }
-        // Q~ = diag(gamma) Q: same swizzled positions as the Q tile
-        {
-            const uint8_t *qt = sm + L::P_KQ + s * 32768 + 8192;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const int ci = tid * 8 + e;  // 16-byte chunk 0..1023
-                const int half = ci >> 9;
-                const uint32_t ob = (uint32_t)(ci & 511) * 16;
-                const float gm = hg[ob >> 7];
-                float f[8];
-                load8(reinterpret_cast<const __nv_bfloat16 *>(qt + half * 16384 + ob), f);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) f[i] *= gm;
-                st_bf16x8(stg + L::H_QT + half * 8192 + ob, f);
+                for (int i = 0; i < 32; ++i) {
+                    const int col = c0 + i;
+                    const float d = exact ? __expf(gr - sg[col]) : f * sinv[col];
+                    pv[i] = (col <= r) ? d * pv[i] : 0.f;
+                }
             }
         }
         tc_before_sync();
         __syncthreads();
-        if (tid == 0 && n + 1 < nch) {  // next chunk's K K^T / Q K^T overlaps this chunk's solve
+        if (tid == 0 && n + 1 < nch) {  // next chunk's K K^T / Q K^T overlaps this chunk's inverse
             tc_after_sync();
             if (!mbar_wait(&tma_full[s ^ 1], (uint32_t)(((n + 1) >> 1) & 1))) *abort_flag = 1;
             else {
@@ -227,20 +317,53 @@ __device__ __forceinline__ void tc2_prep(uint8_t *sm, const CUtensorMap *tm_q, c
                 issue_mma1(s ^ 1);
             }
         }
-        invert_unit_lower_64(sA, sT);
-        {   // T' = T diag(beta), T'' = T diag(beta gamma)
-            const int r = tid & 63;
-            const bool second = tid >= 64;
-            float v[8];
+        invert_unit_lower_64_w8(sA, sT);
+        // staging slot s (and the state's slot s) must have been consumed (chunk n-2)
+        if (tid == 0 && n >= 2 && !mbar_wait_cluster(&empty[s], (uint32_t)(((n >> 1) - 1) & 1))) *abort_flag = 1;
+        __syncthreads();
+        if (*abort_flag) break;
+        {
+            float *hg = reinterpret_cast<float *>(stg + L::H_G);
+            if (tid < 64) hg[tid] = sgam[tid];
+            else if (tid < 128) hg[tid] = sdec[tid - 64];
+            // P rows
+            if (row >= 64) {
 #pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
+                for (int ch = 0; ch < 4; ++ch)
+                    st_bf16x8(stg + L::H_P + sw128_offset(row - 64, wh * 4 + ch), pv + 8 * ch);
+            }
+            // T' = T diag(beta) (rows 0-63), T'' = T diag(beta gamma) (rows 64-127), 32 columns each
+            {
+                const int r = tid & 63;
+                const bool second = (tid & 64) != 0;
+                const int cb = (tid >> 7) * 32;
+                float v[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int i = ch * 8 + e;
-                    const float t = (i <= r) ? sT[r * kLdT + i] : 0.f;
-                    v[e] = t * sbeta[i] * (second ? hg[i] : 1.f);
+                for (int ch = 0; ch < 4; ++ch) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int i = cb + ch * 8 + e;
+                        const float t = (i <= r) ? sT[r * kLdT + i] : 0.f;
+                        v[e] = t * sbeta[i] * (second ? sgam[i] : 1.f);
+                    }
+                    st_bf16x8(stg + (second ? L::H_T2 : L::H_T1) + sw128_offset(r, (cb >> 3) + ch), v);
                 }
-                st_bf16x8(stg + (second ? L::H_T2 : L::H_T1) + sw128_offset(r, ch), v);
+            }
+            // Q~ = diag(gamma) Q: same swizzled positions as the Q tile
+            {
+                const uint8_t *qt = sm + L::P_KQ + s * 32768 + 8192;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int ci = tid * 4 + e;  // 16-byte chunk 0..1023
+                    const int half = ci >> 9;
+                    const uint32_t ob = (uint32_t)(ci & 511) * 16;
+                    const float gm = sgam[ob >> 7];
+                    float f[8];
+                    load8(reinterpret_cast<const __nv_bfloat16 *>(qt + half * 16384 + ob), f);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) f[i] *= gm;
+                    st_bf16x8(stg + L::H_QT + half * 8192 + ob, f);
+                }
             }
         }
         fence_async_smem();
@@ -271,12 +394,14 @@ __device__ __forceinline__ void tc2_prep(uint8_t *sm, const CUtensorMap *tm_q, c
 
 // ----------------------------------------------------------------- state CTA --
 __device__ __forceinline__ void tc2_state(uint8_t *sm, const CUtensorMap *tm_k, const CUtensorMap *tm_v,
-                                          int T, int H, int b, int h, const float *S0,
-                                          __nv_bfloat16 *o, float *S_T) {
+                                          const CUtensorMap *tm_o, int T, int H, int b, int h,
+                                          const float *S0, float *S_T) {
     using L = Tc2Layout;
     using namespace sm100;
     constexpr int D = 128;
-    const int tid = threadIdx.x, warp = tid >> 5;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int wq = warp & 3, wh = warp >> 2;
+    const int row = wq * 32 + lane;  // TMEM lane = row of S / U^T / O^T / W^T
     const int bh = b * H + h;
     const int nch = (T + kChunk - 1) / kChunk;
     uint64_t *tma_full = reinterpret_cast<uint64_t *>(sm + L::S_BAR);  // [2]
@@ -298,6 +423,7 @@ __device__ __forceinline__ void tc2_state(uint8_t *sm, const CUtensorMap *tm_k, 
         *abort_flag = 0;
         prefetch_tmap(tm_k);
         prefetch_tmap(tm_v);
+        prefetch_tmap(tm_o);
         mbar_expect_tx(&hand_full[0], L::H_BYTES);  // arm the slots for chunks 0 and 1
         if (nch > 1) mbar_expect_tx(&hand_full[1], L::H_BYTES);
     }
@@ -307,15 +433,16 @@ __device__ __forceinline__ void tc2_state(uint8_t *sm, const CUtensorMap *tm_k, 
     tc_after_sync();
     cluster_sync();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
+    const uint32_t tl = tmem + ((uint32_t)(wq * 32) << 16);
     const uint32_t remote_empty0 = cluster_addr(sm + L::P_BAR + 16, 0);  // prep's empty[0]
 
-    {   // entry state -> TMEM (row tid)
+    {   // entry state -> TMEM (row `row`, columns of this column half)
         float v[32];
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
+            const int col = wh * 64 + c * 32;
             if (S0) {
-                const float4 *src = reinterpret_cast<const float4 *>(S0 + ((size_t)bh * D + tid) * D + c * 32);
+                const float4 *src = reinterpret_cast<const float4 *>(S0 + ((size_t)bh * D + row) * D + col);
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     const float4 x = src[i];
@@ -325,7 +452,7 @@ __device__ __forceinline__ void tc2_state(uint8_t *sm, const CUtensorMap *tm_k, 
 #pragma unroll
                 for (int i = 0; i < 32; ++i) v[i] = 0.f;
             }
-            tmem_st32(tl + kT2S + c * 32, v);
+            tmem_st32(tl + kT2S + col, v);
         }
         tmem_wait_st();
     }
@@ -362,19 +489,24 @@ __device__ __forceinline__ void tc2_state(uint8_t *sm, const CUtensorMap *tm_k, 
         mma_commit(bar_b);
         return true;
     };
-    auto epilogue = [&](int n) {  // O^T (lane = value channel, column = token) -> o
-        const int c0 = n * kChunk, nv = min(kChunk, T - c0);
-        const size_t tok0 = ((size_t)b * T + c0) * H + h;
+    // O^T of chunk n (lane = value channel, column = token) -> bf16 tile [token][channel]
+    auto stage_o = [&](int n) {
         float v[32];
-#pragma unroll 1
-        for (int half = 0; half < 2; ++half) {
-            tmem_ld32(tl + kT2O + 64 * (n & 1) + half * 32, v);
+        tmem_ld32(tl + kT2O + 64 * (n & 1) + wh * 32, v);
+        uint8_t *half = sm + L::S_OST + (row >> 6) * 8192;
+        const int cc = row & 63;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const int r = half * 32 + i;
-                if (r < nv) o[(tok0 + (size_t)r * H) * D + tid] = __float2bfloat16_rn(v[i]);
-            }
+        for (int i = 0; i < 32; ++i) {
+            const int r = wh * 32 + i;
+            *reinterpret_cast<__nv_bfloat16 *>(half + sw128_offset(r, cc >> 3) + (cc & 7) * 2) =
+                __float2bfloat16_rn(v[i]);
         }
+        fence_async_smem();
+    };
+    auto store_o = [&](int n) {  // thread 0, after a barrier that follows stage_o
+        tma_store_4d(tm_o, sm + L::S_OST, 0, h, n * kChunk, b);
+        tma_store_4d(tm_o, sm + L::S_OST + 8192, 64, h, n * kChunk, b);
+        bulk_commit();
     };
     auto stash_gamma = [&](int n) {  // keep gamma of chunk n after its slot is released
         if (tid < 64) gl[64 * (n & 1) + tid] =
@@ -399,11 +531,10 @@ __device__ __forceinline__ void tc2_state(uint8_t *sm, const CUtensorMap *tm_k, 
     __syncthreads();
     tc_after_sync();
     if (!*abort_flag) {
-        float v[64];
-        tmem_ld32(tl + kT2W, v);
-        tmem_ld32(tl + kT2W + 32, v + 32);
+        float v[32];
+        tmem_ld32(tl + kT2W + wh * 32, v);
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) st_bf16x8(sm + L::S_W + sw128_offset(tid, ch), v + 8 * ch);
+        for (int ch = 0; ch < 4; ++ch) st_bf16x8(sm + L::S_W + sw128_offset(row, wh * 4 + ch), v + 8 * ch);
         stash_gamma(0);
         fence_async_smem();
     }
@@ -423,18 +554,20 @@ __device__ __forceinline__ void tc2_state(uint8_t *sm, const CUtensorMap *tm_k, 
             const float gC = gl[64 * s + kChunk - 1];
             float v[32];
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-                tmem_ld32(tl + kT2S + c * 32, v);
-                uint8_t *half = sm + L::S_SB + (c >> 1) * 16384;
+            for (int c = 0; c < 2; ++c) {
+                const int col = wh * 64 + c * 32;
+                tmem_ld32(tl + kT2S + col, v);
+                uint8_t *half = sm + L::S_SB + wh * 16384;
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) st_bf16x8(half + sw128_offset(tid, (c & 1) * 4 + q4), v + 8 * q4);
+                for (int q4 = 0; q4 < 4; ++q4) st_bf16x8(half + sw128_offset(row, c * 4 + q4), v + 8 * q4);
 #pragma unroll
                 for (int i = 0; i < 32; ++i) v[i] *= gC;
-                tmem_st32(tl + kT2S + c * 32, v);
+                tmem_st32(tl + kT2S + col, v);
             }
             tmem_wait_st();
         }
         fence_async_smem();
+        if (tid == 0) bulk_wait_read_all();  // the O tile of chunk n-2 has left shared memory
         tc_before_sync();
         __syncthreads();
 
@@ -457,8 +590,8 @@ __device__ __forceinline__ void tc2_state(uint8_t *sm, const CUtensorMap *tm_k, 
             mma_commit(bar_a);
         }
         __syncwarp();
-        // (c) epilogue of the previous chunk, then W/U^g of the next chunk
-        if (n > 0) epilogue(n - 1);
+        // (c) stage the previous chunk's output, then W/U^g of the next chunk
+        if (n > 0) stage_o(n - 1);
         if (tid == 0 && n + 1 < nch) {
             if (!issue_wu(n + 1)) *abort_flag = 1;
             else ++tma_done_n;
@@ -471,16 +604,17 @@ __device__ __forceinline__ void tc2_state(uint8_t *sm, const CUtensorMap *tm_k, 
         __syncthreads();
         if (*abort_flag) break;
         tc_after_sync();
+        if (tid == 0 && n > 0) store_o(n - 1);
         {
-            float v[64];
-            tmem_ld32(tl + kT2U + 64 * s, v);
-            tmem_ld32(tl + kT2U + 64 * s + 32, v + 32);
+            float v[32];
+            tmem_ld32(tl + kT2U + 64 * s + wh * 32, v);
 #pragma unroll
-            for (int ch = 0; ch < 8; ++ch) st_bf16x8(sm + L::S_SB + sw128_offset(tid, ch), v + 8 * ch);
+            for (int ch = 0; ch < 4; ++ch) st_bf16x8(sm + L::S_SB + sw128_offset(row, wh * 4 + ch), v + 8 * ch);
 #pragma unroll
-            for (int i = 0; i < 64; ++i) v[i] *= hgate[64 + i];
+            for (int i = 0; i < 32; ++i) v[i] *= hgate[64 + wh * 32 + i];
 #pragma unroll
-            for (int ch = 0; ch < 8; ++ch) st_bf16x8(sm + L::S_SB + 16384 + sw128_offset(tid, ch), v + 8 * ch);
+            for (int ch = 0; ch < 4; ++ch)
+                st_bf16x8(sm + L::S_SB + 16384 + sw128_offset(row, wh * 4 + ch), v + 8 * ch);
         }
         fence_async_smem();
         tc_before_sync();
@@ -509,11 +643,10 @@ __device__ __forceinline__ void tc2_state(uint8_t *sm, const CUtensorMap *tm_k, 
         tc_after_sync();
         // (f) W of the next chunk -> MN-major B operand (W buffer free: its MMA is done)
         if (n + 1 < nch) {
-            float v[64];
-            tmem_ld32(tl + kT2W, v);
-            tmem_ld32(tl + kT2W + 32, v + 32);
+            float v[32];
+            tmem_ld32(tl + kT2W + wh * 32, v);
 #pragma unroll
-            for (int ch = 0; ch < 8; ++ch) st_bf16x8(sm + L::S_W + sw128_offset(tid, ch), v + 8 * ch);
+            for (int ch = 0; ch < 4; ++ch) st_bf16x8(sm + L::S_W + sw128_offset(row, wh * 4 + ch), v + 8 * ch);
             stash_gamma(n + 1);
             fence_async_smem();
         }
@@ -537,18 +670,24 @@ __device__ __forceinline__ void tc2_state(uint8_t *sm, const CUtensorMap *tm_k, 
     }
 
     if (!*abort_flag && nch > 0) {
-        epilogue(nch - 1);
+        if (tid == 0) bulk_wait_read_all();
+        __syncthreads();
+        stage_o(nch - 1);
+        __syncthreads();
+        if (tid == 0) store_o(nch - 1);
         if (S_T) {
             float v[32];
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-                tmem_ld32(tl + kT2S + c * 32, v);
-                float4 *dst = reinterpret_cast<float4 *>(S_T + ((size_t)bh * D + tid) * D + c * 32);
+            for (int c = 0; c < 2; ++c) {
+                const int col = wh * 64 + c * 32;
+                tmem_ld32(tl + kT2S + col, v);
+                float4 *dst = reinterpret_cast<float4 *>(S_T + ((size_t)bh * D + row) * D + col);
 #pragma unroll
                 for (int i = 0; i < 8; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
             }
         }
     }
+    if (tid == 0) bulk_wait_all();  // output stores complete before the CTA exits
     if (*abort_flag && tid == 0) {
         record_status(GDR_ERR_TIMEOUT);
         // drain: this CTA's TMA loads, its MMAs, and the prep CTA's copies into it
@@ -558,7 +697,6 @@ __device__ __forceinline__ void tc2_state(uint8_t *sm, const CUtensorMap *tm_k, 
         for (int k2 = n_done; k2 < nch && k2 < n_done + 2; ++k2)
             mbar_wait_cluster(&hand_full[k2 & 1], (uint32_t)((k2 >> 1) & 1));
     }
-    (void)n_done;
     tc_before_sync();
     __syncthreads();
     cluster_sync();
@@ -568,11 +706,11 @@ __device__ __forceinline__ void tc2_state(uint8_t *sm, const CUtensorMap *tm_k, 
     }
 }
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTc2Threads, 1)
 gdr_fwd_tc2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                   const __grid_constant__ CUtensorMap tm_v, int T, int H,
-                   const float *__restrict__ log_alpha, const float *__restrict__ beta,
-                   const float *__restrict__ S0, __nv_bfloat16 *__restrict__ o, float *__restrict__ S_T) {
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                   int T, int H, const float *__restrict__ log_alpha, const float *__restrict__ beta,
+                   const float *__restrict__ S0, float *__restrict__ S_T) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
@@ -580,21 +718,21 @@ gdr_fwd_tc2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     if (sm100::cluster_ctarank() == 0)
         tc2_prep(sm, &tm_q, &tm_k, T, H, b, h, log_alpha, beta);
     else
-        tc2_state(sm, &tm_k, &tm_v, T, H, b, h, S0, o, S_T);
+        tc2_state(sm, &tm_k, &tm_v, &tm_o, T, H, b, h, S0, S_T);
 }
 
 inline cudaError_t launch_fwd_tc2(int B, int T, int H, const void *q, const void *k, const void *v,
                                   const float *la, const float *beta, const float *S0, void *o,
                                   float *S_T, cudaStream_t stream) {
-    CUtensorMap mq, mk, mv;
+    CUtensorMap mq, mk, mv, mo;
     if (!make_token_map(&mq, q, B, T, H, 128) || !make_token_map(&mk, k, B, T, H, 128) ||
-        !make_token_map(&mv, v, B, T, H, 128))
+        !make_token_map(&mv, v, B, T, H, 128) || !make_token_map(&mo, o, B, T, H, 128))
         return cudaErrorInvalidValue;
     cudaError_t err = cudaFuncSetAttribute(gdr_fwd_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            (int)Tc2Layout::kAlloc);
     if (err != cudaSuccess) return err;
-    gdr_fwd_tc2_kernel<<<(unsigned)(2 * B * H), kTcThreads, Tc2Layout::kAlloc, stream>>>(
-        mq, mk, mv, T, H, la, beta, S0, static_cast<__nv_bfloat16 *>(o), S_T);
+    gdr_fwd_tc2_kernel<<<(unsigned)(2 * B * H), kTc2Threads, Tc2Layout::kAlloc, stream>>>(
+        mq, mk, mv, mo, T, H, la, beta, S0, S_T);
     g_launches.fetch_add(1, std::memory_order_relaxed);
     return cudaGetLastError();
 }
