@@ -1,5 +1,5 @@
 // fwd_tc2.cuh -- chunkwise forward on tcgen05, split over a 2-CTA cluster
-// per (b, h): a "prep" CTA and a "state" CTA on two SMs, 256 threads each.
+// per (b, h): a "prep" CTA and a "state" CTA on two SMs, 512 threads each.
 //
 // Same chunk algebra and operand orientation as fwd_tc.cuh (Gated DeltaNet
 // review, meaningful96.github.io/nr/GDN, section 3.7: UT transform / WY form
@@ -23,8 +23,10 @@
 // decay range exceeds e^80 (where those factors could overflow) takes the
 // exact per-element exponential instead.
 //
-// Warps 0-3 and 4-7 of each CTA own TMEM lane quarters 0-3 and split the
-// columns; thread 0 issues TMA and MMA.  The prep waits for a free hand-off
+// Warp w of each CTA owns TMEM lane quarter w % 4 and column group w / 4 (of
+// four); thread 0 issues TMA and MMA.  Sixteen warps (four per SM
+// sub-partition) hide the latency of the CUDA-core phases, each written as
+// vector loads, then arithmetic, then vector stores.  The prep waits for a free hand-off
 // slot only after the inverse, so the state CTA's tail overlaps it.  Slots go
 // back to the prep CTA with a remote mbarrier arrive.  No TMA multicast; each
 // CTA loads its own tiles (the shared K/Q tiles hit L2 for the second reader).
@@ -37,7 +39,7 @@
 
 namespace gdr {
 
-constexpr int kTc2Threads = 256;
+constexpr int kTc2Threads = 512;
 
 struct Tc2Layout {
     // hand-off slot (identical offsets in the prep staging area and the state slots)
@@ -78,17 +80,16 @@ static_assert(Tc2Layout::kAlloc <= 232448, "shared memory budget");
 constexpr uint32_t kT2S = 0, kT2W = 128, kT2U = 192, kT2O = 320;  // U, O double-buffered (+64)
 
 // T = (I + A)^{-1} for strictly lower 64 x 64 A (fp32, row stride kLdT) with
-// 256 threads; same recursive doubling as invert_unit_lower_64 (16 x 16
+// 512 threads; same recursive doubling as invert_unit_lower_64 (16 x 16
 // diagonal inverses by substitution, then the 32 and 64 levels), retiled for
-// eight warps.  Only the lower triangle of T is meaningful; the upper
+// sixteen warps.  Only the lower triangle of T is meaningful; the upper
 // triangle of A holds the intermediate products.
-__device__ __forceinline__ void invert_unit_lower_64_w8(float *sA, float *sT) {
+__device__ __forceinline__ void invert_unit_lower_64_w16(float *sA, float *sT) {
     constexpr int LD = kLdT;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     {   // zero T[0:16,16:32] and T[32:48,48:64]
-        const int idx = tid * 2, blk = idx >> 8, e = idx & 255;
-        float2 *p = reinterpret_cast<float2 *>(sT + (blk * 32 + (e >> 4)) * LD + blk * 32 + 16 + (e & 15));
-        *p = make_float2(0.f, 0.f);
+        const int blk = tid >> 8, e = tid & 255;
+        sT[(blk * 32 + (e >> 4)) * LD + blk * 32 + 16 + (e & 15)] = 0.f;
     }
     if (warp < 4 && lane < 16) {  // 16 x 16 diagonal block `warp`, column `lane`
         const int base = warp * 16, j = lane;
@@ -109,49 +110,57 @@ __device__ __forceinline__ void invert_unit_lower_64_w8(float *sA, float *sT) {
     }
     __syncthreads();
     {   // 32 level: X = A[o+16:o+32, o:o+16] t_{2P};  T[o+16:o+32, o:o+16] = -t_{2P+1} X
-        const int P = tid >> 7, rr = (tid & 127) >> 3, cq = (tid & 7) * 2, o = 32 * P;
-        float2 acc = make_float2(0.f, 0.f);
+        const int P = tid >> 8, rr = (tid & 255) >> 4, c = tid & 15, o = 32 * P;
+        float a[16], acc = 0.f;
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-            const float a = sA[(o + 16 + rr) * LD + o + k];
-            const float2 t2 = *reinterpret_cast<const float2 *>(sT + (o + k) * LD + o + cq);
-            acc.x = fmaf(a, t2.x, acc.x);
-            acc.y = fmaf(a, t2.y, acc.y);
+        for (int k4 = 0; k4 < 4; ++k4) {
+            const float4 x = *reinterpret_cast<const float4 *>(sA + (o + 16 + rr) * LD + o + 4 * k4);
+            a[4 * k4] = x.x; a[4 * k4 + 1] = x.y; a[4 * k4 + 2] = x.z; a[4 * k4 + 3] = x.w;
         }
-        *reinterpret_cast<float2 *>(sA + (o + rr) * LD + o + 16 + cq) = acc;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) acc = fmaf(a[k], sT[(o + k) * LD + o + c], acc);
+        sA[(o + rr) * LD + o + 16 + c] = acc;  // X parked above the diagonal
         __syncthreads();
-        acc = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-            const float t = sT[(o + 16 + rr) * LD + o + 16 + k];
-            const float2 x2 = *reinterpret_cast<const float2 *>(sA + (o + k) * LD + o + 16 + cq);
-            acc.x = fmaf(t, x2.x, acc.x);
-            acc.y = fmaf(t, x2.y, acc.y);
+        for (int k4 = 0; k4 < 4; ++k4) {
+            const float4 x = *reinterpret_cast<const float4 *>(sT + (o + 16 + rr) * LD + o + 16 + 4 * k4);
+            a[4 * k4] = x.x; a[4 * k4 + 1] = x.y; a[4 * k4 + 2] = x.z; a[4 * k4 + 3] = x.w;
         }
-        *reinterpret_cast<float2 *>(sT + (o + 16 + rr) * LD + o + cq) = make_float2(-acc.x, -acc.y);
+        acc = 0.f;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) acc = fmaf(a[k], sA[(o + k) * LD + o + 16 + c], acc);
+        sT[(o + 16 + rr) * LD + o + c] = -acc;
         __syncthreads();
     }
     {   // 64 level: X = A[32:64, 0:32] T[0:32, 0:32];  T[32:64, 0:32] = -T[32:64, 32:64] X
-        const int r = tid >> 3, cq = (tid & 7) * 4;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 8
-        for (int k = 0; k < 32; ++k) {
-            const float a = sA[(32 + r) * LD + k];
-            const float4 t4 = *reinterpret_cast<const float4 *>(sT + k * LD + cq);
-            acc.x = fmaf(a, t4.x, acc.x); acc.y = fmaf(a, t4.y, acc.y);
-            acc.z = fmaf(a, t4.z, acc.z); acc.w = fmaf(a, t4.w, acc.w);
+        const int r = tid >> 4, cq = (tid & 15) * 2;
+        float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int k4 = 0; k4 < 8; ++k4) {
+            const float4 a4 = *reinterpret_cast<const float4 *>(sA + (32 + r) * LD + 4 * k4);
+            const float a[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                const float2 t2 = *reinterpret_cast<const float2 *>(sT + (4 * k4 + kk) * LD + cq);
+                acc.x = fmaf(a[kk], t2.x, acc.x);
+                acc.y = fmaf(a[kk], t2.y, acc.y);
+            }
         }
-        *reinterpret_cast<float4 *>(sA + r * LD + 32 + cq) = acc;
+        *reinterpret_cast<float2 *>(sA + r * LD + 32 + cq) = acc;  // X parked in A[0:32, 32:64]
         __syncthreads();
-        acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 8
-        for (int k = 0; k < 32; ++k) {
-            const float t = sT[(32 + r) * LD + 32 + k];
-            const float4 x4 = *reinterpret_cast<const float4 *>(sA + k * LD + 32 + cq);
-            acc.x = fmaf(t, x4.x, acc.x); acc.y = fmaf(t, x4.y, acc.y);
-            acc.z = fmaf(t, x4.z, acc.z); acc.w = fmaf(t, x4.w, acc.w);
+        acc = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int k4 = 0; k4 < 8; ++k4) {
+            const float4 t4 = *reinterpret_cast<const float4 *>(sT + (32 + r) * LD + 32 + 4 * k4);
+            const float t[4] = {t4.x, t4.y, t4.z, t4.w};
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                const float2 x2 = *reinterpret_cast<const float2 *>(sA + (4 * k4 + kk) * LD + 32 + cq);
+                acc.x = fmaf(t[kk], x2.x, acc.x);
+                acc.y = fmaf(t[kk], x2.y, acc.y);
+            }
         }
-        *reinterpret_cast<float4 *>(sT + (32 + r) * LD + cq) = make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
+        *reinterpret_cast<float2 *>(sT + (32 + r) * LD + cq) = make_float2(-acc.x, -acc.y);
         __syncthreads();
     }
 }
@@ -163,7 +172,7 @@ __device__ __forceinline__ void tc2_prep(uint8_t *sm, const CUtensorMap *tm_q, c
     using L = Tc2Layout;
     using namespace sm100;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int wq = warp & 3, wh = warp >> 2;  // TMEM lane quarter, column half
+    const int wq = warp & 3, wc = warp >> 2;  // TMEM lane quarter, column group (of 4)
     const int nch = (T + kChunk - 1) / kChunk;
     uint64_t *tma_full = reinterpret_cast<uint64_t *>(sm + L::P_BAR);  // [2]
     uint64_t *empty = tma_full + 2;                                      // [2], arrived by the state CTA
@@ -280,31 +289,35 @@ __device__ __forceinline__ void tc2_prep(uint8_t *sm, const CUtensorMap *tm_q, c
         tc_after_sync();
 
         // A (fp32, rows 0-63 -> sA) and P (rows 64-127, kept in registers), this
-        // thread's 32 columns of its TMEM lane
+        // thread's 16 columns of its TMEM lane
         const int row = wq * 32 + lane;  // 0..127
-        const int c0 = wh * 32;
-        float pv[32];
+        const int c0 = wc * 16;
+        float pv[16];
         {
-            tmem_ld32(tl + c0, pv);
+            tmem_ld16(tl + c0, pv);
             const bool exact = *exact_flag;
+            float sv[16], gv[16];
+#pragma unroll
+            for (int k4 = 0; k4 < 4; ++k4) {
+                const float4 x = *reinterpret_cast<const float4 *>(sinv + c0 + 4 * k4);
+                const float4 y = *reinterpret_cast<const float4 *>(sg + c0 + 4 * k4);
+                sv[4 * k4] = x.x; sv[4 * k4 + 1] = x.y; sv[4 * k4 + 2] = x.z; sv[4 * k4 + 3] = x.w;
+                gv[4 * k4] = y.x; gv[4 * k4 + 1] = y.y; gv[4 * k4 + 2] = y.z; gv[4 * k4 + 3] = y.w;
+            }
+            const int r = row & 63;
+            const float gr = sg[r], br = row < 64 ? sbeta[r] : 1.f;
+            const float f = br * sgp[r];
+            const int lim = row < 64 ? r : r + 1;  // strictly lower for A, incl. diagonal for P
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const float d = exact ? br * __expf(gr - gv[i]) : f * sv[i];
+                pv[i] = (c0 + i < lim) ? d * pv[i] : 0.f;
+            }
             if (row < 64) {
-                const int r = row;
-                const float gr = sg[r], f = sbeta[r] * sgp[r], br = sbeta[r];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int col = c0 + i;
-                    const float d = exact ? br * __expf(gr - sg[col]) : f * sinv[col];
-                    sA[r * kLdT + col] = (col < r) ? d * pv[i] : 0.f;
-                }
-            } else {
-                const int r = row - 64;
-                const float gr = sg[r], f = sgp[r];
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int col = c0 + i;
-                    const float d = exact ? __expf(gr - sg[col]) : f * sinv[col];
-                    pv[i] = (col <= r) ? d * pv[i] : 0.f;
-                }
+                for (int k4 = 0; k4 < 4; ++k4)
+                    *reinterpret_cast<float4 *>(sA + r * kLdT + c0 + 4 * k4) =
+                        make_float4(pv[4 * k4], pv[4 * k4 + 1], pv[4 * k4 + 2], pv[4 * k4 + 3]);
             }
         }
         tc_before_sync();
@@ -317,7 +330,7 @@ __device__ __forceinline__ void tc2_prep(uint8_t *sm, const CUtensorMap *tm_q, c
                 issue_mma1(s ^ 1);
             }
         }
-        invert_unit_lower_64_w8(sA, sT);
+        invert_unit_lower_64_w16(sA, sT);
         // staging slot s (and the state's slot s) must have been consumed (chunk n-2)
         if (tid == 0 && n >= 2 && !mbar_wait_cluster(&empty[s], (uint32_t)(((n >> 1) - 1) & 1))) *abort_flag = 1;
         __syncthreads();
@@ -329,39 +342,44 @@ __device__ __forceinline__ void tc2_prep(uint8_t *sm, const CUtensorMap *tm_q, c
             // P rows
             if (row >= 64) {
 #pragma unroll
-                for (int ch = 0; ch < 4; ++ch)
-                    st_bf16x8(stg + L::H_P + sw128_offset(row - 64, wh * 4 + ch), pv + 8 * ch);
+                for (int ch = 0; ch < 2; ++ch)
+                    st_bf16x8(stg + L::H_P + sw128_offset(row - 64, wc * 2 + ch), pv + 8 * ch);
             }
-            // T' = T diag(beta) (rows 0-63), T'' = T diag(beta gamma) (rows 64-127), 32 columns each
+            // T' = T diag(beta) (rows 0-63), T'' = T diag(beta gamma) (rows 64-127), 16 columns each
             {
                 const int r = tid & 63;
                 const bool second = (tid & 64) != 0;
-                const int cb = (tid >> 7) * 32;
-                float v[8];
+                const int cb = (tid >> 7) * 16;
+                float t[16], bv[16], gm[16];
 #pragma unroll
-                for (int ch = 0; ch < 4; ++ch) {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int i = cb + ch * 8 + e;
-                        const float t = (i <= r) ? sT[r * kLdT + i] : 0.f;
-                        v[e] = t * sbeta[i] * (second ? sgam[i] : 1.f);
-                    }
-                    st_bf16x8(stg + (second ? L::H_T2 : L::H_T1) + sw128_offset(r, (cb >> 3) + ch), v);
+                for (int k4 = 0; k4 < 4; ++k4) {
+                    const float4 x = *reinterpret_cast<const float4 *>(sT + r * kLdT + cb + 4 * k4);
+                    const float4 y = *reinterpret_cast<const float4 *>(sbeta + cb + 4 * k4);
+                    const float4 z = *reinterpret_cast<const float4 *>(sgam + cb + 4 * k4);
+                    t[4 * k4] = x.x; t[4 * k4 + 1] = x.y; t[4 * k4 + 2] = x.z; t[4 * k4 + 3] = x.w;
+                    bv[4 * k4] = y.x; bv[4 * k4 + 1] = y.y; bv[4 * k4 + 2] = y.z; bv[4 * k4 + 3] = y.w;
+                    gm[4 * k4] = z.x; gm[4 * k4 + 1] = z.y; gm[4 * k4 + 2] = z.z; gm[4 * k4 + 3] = z.w;
                 }
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    t[i] = (cb + i <= r) ? t[i] * bv[i] * (second ? gm[i] : 1.f) : 0.f;
+#pragma unroll
+                for (int ch = 0; ch < 2; ++ch)
+                    st_bf16x8(stg + (second ? L::H_T2 : L::H_T1) + sw128_offset(r, (cb >> 3) + ch), t + 8 * ch);
             }
             // Q~ = diag(gamma) Q: same swizzled positions as the Q tile
             {
                 const uint8_t *qt = sm + L::P_KQ + s * 32768 + 8192;
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int ci = tid * 4 + e;  // 16-byte chunk 0..1023
+                for (int e = 0; e < 2; ++e) {
+                    const int ci = tid * 2 + e;  // 16-byte chunk 0..1023
                     const int half = ci >> 9;
                     const uint32_t ob = (uint32_t)(ci & 511) * 16;
-                    const float gm = sgam[ob >> 7];
+                    const float g = sgam[ob >> 7];
                     float f[8];
                     load8(reinterpret_cast<const __nv_bfloat16 *>(qt + half * 16384 + ob), f);
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) f[i] *= gm;
+                    for (int i = 0; i < 8; ++i) f[i] *= g;
                     st_bf16x8(stg + L::H_QT + half * 8192 + ob, f);
                 }
             }
@@ -400,7 +418,7 @@ __device__ __forceinline__ void tc2_state(uint8_t *sm, const CUtensorMap *tm_k, 
     using namespace sm100;
     constexpr int D = 128;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int wq = warp & 3, wh = warp >> 2;
+    const int wq = warp & 3, wc = warp >> 2;  // TMEM lane quarter, column group (of 4)
     const int row = wq * 32 + lane;  // TMEM lane = row of S / U^T / O^T / W^T
     const int bh = b * H + h;
     const int nch = (T + kChunk - 1) / kChunk;
@@ -436,11 +454,10 @@ __device__ __forceinline__ void tc2_state(uint8_t *sm, const CUtensorMap *tm_k, 
     const uint32_t tl = tmem + ((uint32_t)(wq * 32) << 16);
     const uint32_t remote_empty0 = cluster_addr(sm + L::P_BAR + 16, 0);  // prep's empty[0]
 
-    {   // entry state -> TMEM (row `row`, columns of this column half)
+    {   // entry state -> TMEM (row `row`, this column group's 32 columns)
         float v[32];
-#pragma unroll 1
-        for (int c = 0; c < 2; ++c) {
-            const int col = wh * 64 + c * 32;
+        {
+            const int col = wc * 32;
             if (S0) {
                 const float4 *src = reinterpret_cast<const float4 *>(S0 + ((size_t)bh * D + row) * D + col);
 #pragma unroll
@@ -491,13 +508,13 @@ __device__ __forceinline__ void tc2_state(uint8_t *sm, const CUtensorMap *tm_k, 
     };
     // O^T of chunk n (lane = value channel, column = token) -> bf16 tile [token][channel]
     auto stage_o = [&](int n) {
-        float v[32];
-        tmem_ld32(tl + kT2O + 64 * (n & 1) + wh * 32, v);
+        float v[16];
+        tmem_ld16(tl + kT2O + 64 * (n & 1) + wc * 16, v);
         uint8_t *half = sm + L::S_OST + (row >> 6) * 8192;
         const int cc = row & 63;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const int r = wh * 32 + i;
+        for (int i = 0; i < 16; ++i) {
+            const int r = wc * 16 + i;
             *reinterpret_cast<__nv_bfloat16 *>(half + sw128_offset(r, cc >> 3) + (cc & 7) * 2) =
                 __float2bfloat16_rn(v[i]);
         }
@@ -531,10 +548,10 @@ __device__ __forceinline__ void tc2_state(uint8_t *sm, const CUtensorMap *tm_k, 
     __syncthreads();
     tc_after_sync();
     if (!*abort_flag) {
-        float v[32];
-        tmem_ld32(tl + kT2W + wh * 32, v);
+        float v[16];
+        tmem_ld16(tl + kT2W + wc * 16, v);
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) st_bf16x8(sm + L::S_W + sw128_offset(row, wh * 4 + ch), v + 8 * ch);
+        for (int ch = 0; ch < 2; ++ch) st_bf16x8(sm + L::S_W + sw128_offset(row, wc * 2 + ch), v + 8 * ch);
         stash_gamma(0);
         fence_async_smem();
     }
@@ -553,13 +570,12 @@ __device__ __forceinline__ void tc2_state(uint8_t *sm, const CUtensorMap *tm_k, 
         {
             const float gC = gl[64 * s + kChunk - 1];
             float v[32];
-#pragma unroll 1
-            for (int c = 0; c < 2; ++c) {
-                const int col = wh * 64 + c * 32;
+            {
+                const int col = wc * 32;
                 tmem_ld32(tl + kT2S + col, v);
-                uint8_t *half = sm + L::S_SB + wh * 16384;
+                uint8_t *half = sm + L::S_SB + (wc >> 1) * 16384;
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) st_bf16x8(half + sw128_offset(row, c * 4 + q4), v + 8 * q4);
+                for (int q4 = 0; q4 < 4; ++q4) st_bf16x8(half + sw128_offset(row, (wc & 1) * 4 + q4), v + 8 * q4);
 #pragma unroll
                 for (int i = 0; i < 32; ++i) v[i] *= gC;
                 tmem_st32(tl + kT2S + col, v);
@@ -606,15 +622,18 @@ __device__ __forceinline__ void tc2_state(uint8_t *sm, const CUtensorMap *tm_k, 
         tc_after_sync();
         if (tid == 0 && n > 0) store_o(n - 1);
         {
-            float v[32];
-            tmem_ld32(tl + kT2U + 64 * s + wh * 32, v);
+            float v[16];
+            tmem_ld16(tl + kT2U + 64 * s + wc * 16, v);
 #pragma unroll
-            for (int ch = 0; ch < 4; ++ch) st_bf16x8(sm + L::S_SB + sw128_offset(row, wh * 4 + ch), v + 8 * ch);
+            for (int ch = 0; ch < 2; ++ch) st_bf16x8(sm + L::S_SB + sw128_offset(row, wc * 2 + ch), v + 8 * ch);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] *= hgate[64 + wh * 32 + i];
+            for (int k4 = 0; k4 < 4; ++k4) {
+                const float4 dv4 = *reinterpret_cast<const float4 *>(hgate + 64 + wc * 16 + 4 * k4);
+                v[4 * k4] *= dv4.x; v[4 * k4 + 1] *= dv4.y; v[4 * k4 + 2] *= dv4.z; v[4 * k4 + 3] *= dv4.w;
+            }
 #pragma unroll
-            for (int ch = 0; ch < 4; ++ch)
-                st_bf16x8(sm + L::S_SB + 16384 + sw128_offset(row, wh * 4 + ch), v + 8 * ch);
+            for (int ch = 0; ch < 2; ++ch)
+                st_bf16x8(sm + L::S_SB + 16384 + sw128_offset(row, wc * 2 + ch), v + 8 * ch);
         }
         fence_async_smem();
         tc_before_sync();
@@ -643,10 +662,10 @@ __device__ __forceinline__ void tc2_state(uint8_t *sm, const CUtensorMap *tm_k, 
         tc_after_sync();
         // (f) W of the next chunk -> MN-major B operand (W buffer free: its MMA is done)
         if (n + 1 < nch) {
-            float v[32];
-            tmem_ld32(tl + kT2W + wh * 32, v);
+            float v[16];
+            tmem_ld16(tl + kT2W + wc * 16, v);
 #pragma unroll
-            for (int ch = 0; ch < 4; ++ch) st_bf16x8(sm + L::S_W + sw128_offset(row, wh * 4 + ch), v + 8 * ch);
+            for (int ch = 0; ch < 2; ++ch) st_bf16x8(sm + L::S_W + sw128_offset(row, wc * 2 + ch), v + 8 * ch);
             stash_gamma(n + 1);
             fence_async_smem();
         }
@@ -677,9 +696,8 @@ __device__ __forceinline__ void tc2_state(uint8_t *sm, const CUtensorMap *tm_k, 
         if (tid == 0) store_o(nch - 1);
         if (S_T) {
             float v[32];
-#pragma unroll 1
-            for (int c = 0; c < 2; ++c) {
-                const int col = wh * 64 + c * 32;
+            {
+                const int col = wc * 32;
                 tmem_ld32(tl + kT2S + col, v);
                 float4 *dst = reinterpret_cast<float4 *>(S_T + ((size_t)bh * D + row) * D + col);
 #pragma unroll
