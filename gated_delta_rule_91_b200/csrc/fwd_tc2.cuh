@@ -413,7 +413,7 @@ __device__ __forceinline__ void tc2_prep(uint8_t *sm, const CUtensorMap *tm_q, c
 // ----------------------------------------------------------------- state CTA --
 __device__ __forceinline__ void tc2_state(uint8_t *sm, const CUtensorMap *tm_k, const CUtensorMap *tm_v,
                                           const CUtensorMap *tm_o, int T, int H, int b, int h,
-                                          const float *S0, float *S_T) {
+                                          const float *S0, float *S_T, bool store_o, float *S_chunks) {
     using L = Tc2Layout;
     using namespace sm100;
     constexpr int D = 128;
@@ -520,7 +520,7 @@ __device__ __forceinline__ void tc2_state(uint8_t *sm, const CUtensorMap *tm_k, 
         }
         fence_async_smem();
     };
-    auto store_o = [&](int n) {  // thread 0, after a barrier that follows stage_o
+    auto store_o_tile = [&](int n) {  // thread 0, after a barrier that follows stage_o
         tma_store_4d(tm_o, sm + L::S_OST, 0, h, n * kChunk, b);
         tma_store_4d(tm_o, sm + L::S_OST + 8192, 64, h, n * kChunk, b);
         bulk_commit();
@@ -573,6 +573,13 @@ __device__ __forceinline__ void tc2_state(uint8_t *sm, const CUtensorMap *tm_k, 
             {
                 const int col = wc * 32;
                 tmem_ld32(tl + kT2S + col, v);
+                if (S_chunks) {  // entry state of chunk n, for the backward's recompute
+                    float4 *dst = reinterpret_cast<float4 *>(
+                        S_chunks + (((size_t)bh * nch + n) * D + row) * D + col);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                }
                 uint8_t *half = sm + L::S_SB + (wc >> 1) * 16384;
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4) st_bf16x8(half + sw128_offset(row, (wc & 1) * 4 + q4), v + 8 * q4);
@@ -607,7 +614,7 @@ __device__ __forceinline__ void tc2_state(uint8_t *sm, const CUtensorMap *tm_k, 
         }
         __syncwarp();
         // (c) stage the previous chunk's output, then W/U^g of the next chunk
-        if (n > 0) stage_o(n - 1);
+        if (store_o && n > 0) stage_o(n - 1);
         if (tid == 0 && n + 1 < nch) {
             if (!issue_wu(n + 1)) *abort_flag = 1;
             else ++tma_done_n;
@@ -620,7 +627,7 @@ __device__ __forceinline__ void tc2_state(uint8_t *sm, const CUtensorMap *tm_k, 
         __syncthreads();
         if (*abort_flag) break;
         tc_after_sync();
-        if (tid == 0 && n > 0) store_o(n - 1);
+        if (tid == 0 && store_o && n > 0) store_o_tile(n - 1);
         {
             float v[16];
             tmem_ld16(tl + kT2U + 64 * s + wc * 16, v);
@@ -689,11 +696,13 @@ __device__ __forceinline__ void tc2_state(uint8_t *sm, const CUtensorMap *tm_k, 
     }
 
     if (!*abort_flag && nch > 0) {
-        if (tid == 0) bulk_wait_read_all();
-        __syncthreads();
-        stage_o(nch - 1);
-        __syncthreads();
-        if (tid == 0) store_o(nch - 1);
+        if (store_o) {
+            if (tid == 0) bulk_wait_read_all();
+            __syncthreads();
+            stage_o(nch - 1);
+            __syncthreads();
+            if (tid == 0) store_o_tile(nch - 1);
+        }
         if (S_T) {
             float v[32];
             {
@@ -728,7 +737,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTc2Threads, 1)
 gdr_fwd_tc2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                    int T, int H, const float *__restrict__ log_alpha, const float *__restrict__ beta,
-                   const float *__restrict__ S0, float *__restrict__ S_T) {
+                   const float *__restrict__ S0, float *__restrict__ S_T, int store_o,
+                   float *__restrict__ S_chunks) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
@@ -736,21 +746,24 @@ gdr_fwd_tc2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     if (sm100::cluster_ctarank() == 0)
         tc2_prep(sm, &tm_q, &tm_k, T, H, b, h, log_alpha, beta);
     else
-        tc2_state(sm, &tm_k, &tm_v, &tm_o, T, H, b, h, S0, S_T);
+        tc2_state(sm, &tm_k, &tm_v, &tm_o, T, H, b, h, S0, S_T, store_o != 0, S_chunks);
 }
 
+// o == nullptr runs the recurrence without writing outputs (the backward's
+// recompute); S_chunks (nullable) receives every chunk's entry state,
+// [B, H, nchunks, 128, 128] fp32.
 inline cudaError_t launch_fwd_tc2(int B, int T, int H, const void *q, const void *k, const void *v,
                                   const float *la, const float *beta, const float *S0, void *o,
-                                  float *S_T, cudaStream_t stream) {
+                                  float *S_T, cudaStream_t stream, float *S_chunks = nullptr) {
     CUtensorMap mq, mk, mv, mo;
     if (!make_token_map(&mq, q, B, T, H, 128) || !make_token_map(&mk, k, B, T, H, 128) ||
-        !make_token_map(&mv, v, B, T, H, 128) || !make_token_map(&mo, o, B, T, H, 128))
+        !make_token_map(&mv, v, B, T, H, 128) || !make_token_map(&mo, o ? o : q, B, T, H, 128))
         return cudaErrorInvalidValue;
     cudaError_t err = cudaFuncSetAttribute(gdr_fwd_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            (int)Tc2Layout::kAlloc);
     if (err != cudaSuccess) return err;
     gdr_fwd_tc2_kernel<<<(unsigned)(2 * B * H), kTc2Threads, Tc2Layout::kAlloc, stream>>>(
-        mq, mk, mv, mo, T, H, la, beta, S0, S_T);
+        mq, mk, mv, mo, T, H, la, beta, S0, S_T, o != nullptr ? 1 : 0, S_chunks);
     g_launches.fetch_add(1, std::memory_order_relaxed);
     return cudaGetLastError();
 }

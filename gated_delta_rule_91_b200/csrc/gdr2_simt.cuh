@@ -12,9 +12,14 @@
 //     U    = (I + A)^{-1} (W*V - (K*B*exp(G)) S^T)
 //     O    = (Q*exp(G)) S^T + P U,  P_ri = sum_j q_r[j] k_i[j] exp(G_r[j] - G_i[j])  (i <= r)
 //     S'   = S Diag(exp(G_C)) + U^T (K * exp(G_C - G))
-// The decay ratios exp(G_r - G_i) are evaluated per element (never as a
-// product of exp(G_r) and exp(-G_i)), so no factor can overflow whatever the
-// gates are.  Same CTA / slice structure as fwd_simt.cuh.
+// The decay ratios exp(G_r[j] - G_i[j]) enter the products through operands
+// scaled about the chunk's middle token: Q*E', K*B*E' and K/E' with
+// E' = exp(G - G_31) per (token, channel), so the dot products carry no
+// exponential; S is scaled by exp(G_31) on the fly for the S products and the
+// state update uses K/E' times exp(G_C - G_31).  A chunk in which some
+// channel decays by more than e^80 (where E' or 1/E' could overflow) takes
+// the exact path, which evaluates exp(G_r[j] - G_i[j]) per element.  Same
+// CTA / slice structure as fwd_simt.cuh.
 #pragma once
 #include "common.cuh"
 #include "fwd_simt.cuh"
@@ -35,7 +40,8 @@ struct Gdr2Layout {
     static constexpr int oU = oS + kSimtDvs * LDK;
     static constexpr int oA = oU + C * LDV;
     static constexpr int oP = oA + C * LDC;
-    static constexpr int kFloats = oP + C * LDC;
+    static constexpr int oVec = oP + C * LDC;  // exp(G_31), exp(G_C), exp(G_C - G_31) per channel; flag
+    static constexpr int kFloats = oVec + 3 * DK + 4;
     static constexpr size_t kBytes = (size_t)kFloats * sizeof(float);
 };
 
@@ -50,6 +56,8 @@ gdr2_fwd_simt_kernel(int T, int H, int dv, const Tio *__restrict__ q, const Tio 
     extern __shared__ float smem[];
     float *sQ = smem + L::oQ, *sK = smem + L::oK, *sKB = smem + L::oKB, *sG = smem + L::oG;
     float *sS = smem + L::oS, *sU = smem + L::oU, *sA = smem + L::oA, *sP = smem + L::oP;
+    float *sE31 = smem + L::oVec, *sEC = sE31 + DK, *sEpC = sEC + DK;
+    int *s_exact = reinterpret_cast<int *>(sEpC + DK);
 
     const int nslice = dv / kSimtDvs;
     const int slice = blockIdx.x % nslice;
@@ -96,7 +104,28 @@ gdr2_fwd_simt_kernel(int T, int H, int dv, const Tio *__restrict__ q, const Tio 
                 sKB[r * L::LDK + j] = bg * sK[r * L::LDK + j];
             }
         }
+        if (tid == 0) *s_exact = 0;
         __syncthreads();
+        for (int j = tid; j < DK; j += blockDim.x) {
+            const float g0 = sG[j], gM = sG[31 * L::LDK + j], gC = sG[(kChunk - 1) * L::LDK + j];
+            if (g0 - gC > 80.f) *s_exact = 1;
+            sE31[j] = expf(gM);
+            sEC[j] = expf(gC);
+            sEpC[j] = expf(gC - gM);
+        }
+        __syncthreads();
+        const bool exact = *s_exact != 0;
+        if (!exact) {  // Q*E', (K*B)*E', K/E' with E' = exp(G - G_31)
+            for (int idx = tid; idx < kChunk * DK; idx += blockDim.x) {
+                const int r = idx / DK, j = idx % DK;
+                const float d = sG[r * L::LDK + j] - sG[31 * L::LDK + j];
+                const float e = __expf(d), ie = __expf(-d);
+                sQ[r * L::LDK + j] *= e;
+                sKB[r * L::LDK + j] *= e;
+                sK[r * L::LDK + j] *= ie;
+            }
+            __syncthreads();
+        }
 
         // ---- phase 1: A, P (decay inside the dot products); X, Y against S ----
         float o_acc[4][4];
@@ -106,6 +135,7 @@ gdr2_fwd_simt_kernel(int T, int H, int dv, const Tio *__restrict__ q, const Tio 
             for (int a = 0; a < 4; ++a)
 #pragma unroll
                 for (int c = 0; c < 4; ++c) o_acc[a][c] = 0.f;
+            if (exact) {
 #pragma unroll 2
             for (int j = 0; j < DK; ++j) {
                 float kbr[4], qr[4], gr[4], ki[4], gi[4], sc[4];
@@ -130,6 +160,29 @@ gdr2_fwd_simt_kernel(int T, int H, int dv, const Tio *__restrict__ q, const Tio 
                         xs[a][c] = fmaf(kbr[a] * er, sc[c], xs[a][c]);
                         o_acc[a][c] = fmaf(qr[a] * er, sc[c], o_acc[a][c]);
                     }
+                }
+            }
+            } else {
+#pragma unroll 4
+                for (int j = 0; j < DK; ++j) {
+                    float kbr[4], qr[4], ki[4], sc[4];
+                    const float e31 = sE31[j];
+#pragma unroll
+                    for (int a = 0; a < 4; ++a) {
+                        kbr[a] = sKB[(ty + 16 * a) * L::LDK + j];
+                        qr[a] = sQ[(ty + 16 * a) * L::LDK + j];
+                        ki[a] = sK[(tx + 16 * a) * L::LDK + j];
+                        sc[a] = sS[(tx + 16 * a) * L::LDK + j] * e31;
+                    }
+#pragma unroll
+                    for (int a = 0; a < 4; ++a)
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            aa[a][c] = fmaf(kbr[a], ki[c], aa[a][c]);
+                            pp[a][c] = fmaf(qr[a], ki[c], pp[a][c]);
+                            xs[a][c] = fmaf(kbr[a], sc[c], xs[a][c]);
+                            o_acc[a][c] = fmaf(qr[a], sc[c], o_acc[a][c]);
+                        }
                 }
             }
 #pragma unroll
@@ -191,12 +244,21 @@ gdr2_fwd_simt_kernel(int T, int H, int dv, const Tio *__restrict__ q, const Tio 
 #pragma unroll
                 for (int c = 0; c < NB; ++c) {
                     const int j = tx + 16 * c;
-                    kr[c] = sK[r * L::LDK + j] * expf(gC[c] - sG[r * L::LDK + j]);
+                    // exact: k * exp(G_C - G_r); scaled: (K/E') times exp(G_C - G_31), applied below
+                    kr[c] = exact ? sK[r * L::LDK + j] * expf(gC[c] - sG[r * L::LDK + j]) : sK[r * L::LDK + j];
                 }
 #pragma unroll
                 for (int a = 0; a < 4; ++a)
 #pragma unroll
                     for (int c = 0; c < NB; ++c) acc[a][c] = fmaf(ur[a], kr[c], acc[a][c]);
+            }
+            if (!exact) {
+#pragma unroll
+                for (int c = 0; c < NB; ++c) {
+                    const float f = sEpC[tx + 16 * c];
+#pragma unroll
+                    for (int a = 0; a < 4; ++a) acc[a][c] *= f;
+                }
             }
             __syncthreads();  // everyone finished reading S (phase 1) and U
 #pragma unroll
