@@ -24,7 +24,7 @@
 // exact per-element exponential instead.
 //
 // Warp w of each CTA owns TMEM lane quarter w % 4 and column group w / 4 (of
-// four); thread 0 issues TMA and MMA.  Sixteen warps (four per SM
+// four); one thread per CTA issues TMA and MMA.  Sixteen warps (four per SM
 // sub-partition) hide the latency of the CUDA-core phases, each written as
 // vector loads, then arithmetic, then vector stores.  The prep waits for a free hand-off
 // slot only after the inverse, so the state CTA's tail overlaps it.  Slots go
@@ -64,9 +64,10 @@ struct Tc2Layout {
     static constexpr uint32_t P_KQ = 0;                   // 2 stages x 32 KB ([K;Q] per dk half)
     static constexpr uint32_t P_A = P_KQ + 2 * 32768;
     static constexpr uint32_t P_T = P_A + 64 * kLdT * 4;
-    static constexpr uint32_t P_STG = P_T + 64 * kLdT * 4;  // 2 staging slots
-    static constexpr uint32_t P_GATE = P_STG + 2 * H_SLOT;  // g, beta, gamma, dec, gamma', 1/gamma' [64] + flag
-    static constexpr uint32_t P_BAR = P_GATE + 6 * 256 + 16;
+    static constexpr uint32_t P_STG = P_T + 64 * kLdT * 4;  // 3 staging slots
+    static constexpr uint32_t P_GATE = P_STG + 3 * H_SLOT;  // 2 x {g, beta, gamma, dec, gamma', 1/gamma' [64], flag}
+    static constexpr uint32_t P_GATE_BYTES = 6 * 256 + 16;
+    static constexpr uint32_t P_BAR = P_GATE + 2 * P_GATE_BYTES;
     static constexpr uint32_t P_BYTES = P_BAR + 128;
     static constexpr uint32_t kAlloc = (S_BYTES > P_BYTES ? S_BYTES : P_BYTES) + 1024;
 };
@@ -79,93 +80,167 @@ static_assert(Tc2Layout::kAlloc <= 232448, "shared memory budget");
 // state TMEM columns (512 allocated)
 constexpr uint32_t kT2S = 0, kT2W = 128, kT2U = 192, kT2O = 320;  // U, O double-buffered (+64)
 
-// T = (I + A)^{-1} for strictly lower 64 x 64 A (fp32, row stride kLdT) with
-// 512 threads; same recursive doubling as invert_unit_lower_64 (16 x 16
-// diagonal inverses by substitution, then the 32 and 64 levels), retiled for
-// sixteen warps.  Only the lower triangle of T is meaningful; the upper
-// triangle of A holds the intermediate products.
-__device__ __forceinline__ void invert_unit_lower_64_w16(float *sA, float *sT) {
+// T = (I + A)^{-1} for strictly lower 64 x 64 A (fp32, row stride kLdT) by
+// recursive doubling over 16 x 16 blocks, solved by two warps:
+//   diagonal blocks t_0..t_3 by substitution (lane j owns column j of one
+//   block; each warp takes two blocks);
+//   32 level, block P (o = 32P, one warp each):
+//     T[o+16:o+32, o:o+16] = -t_{2P+1} (A[o+16:o+32, o:o+16] t_{2P});
+//   64 level, in 8-column slabs (two per warp):
+//     T[32:64, 0:32] = -T22 (A[32:64, 0:32] T11).
+// Products run on warp-level tensor-core tiles (m16n8k8, tf32 operands,
+// fp32 accumulation); the known zero blocks of T11 and T22 are skipped.  Intermediate products are parked in A's unused upper
+// triangle; only the lower triangle of T is written.
+__device__ __forceinline__ void inverse_diag16(const float *sA, float *sT, int blk, int j) {
     constexpr int LD = kLdT;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    {   // zero T[0:16,16:32] and T[32:48,48:64]
-        const int blk = tid >> 8, e = tid & 255;
-        sT[(blk * 32 + (e >> 4)) * LD + blk * 32 + 16 + (e & 15)] = 0.f;
-    }
-    if (warp < 4 && lane < 16) {  // 16 x 16 diagonal block `warp`, column `lane`
-        const int base = warp * 16, j = lane;
-        float t[16];
+    const int base = blk * 16;
+    float t[16];
 #pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            float acc0 = (r == j) ? 1.f : 0.f, acc1 = 0.f;
+    for (int r = 0; r < 16; ++r) {
+        float acc0 = (r == j) ? 1.f : 0.f, acc1 = 0.f;
 #pragma unroll
-            for (int i = 0; i + 1 < r; i += 2) {
-                acc0 = fmaf(-sA[(base + r) * LD + base + i], t[i], acc0);
-                acc1 = fmaf(-sA[(base + r) * LD + base + i + 1], t[i + 1], acc1);
-            }
-            if (r & 1) acc0 = fmaf(-sA[(base + r) * LD + base + r - 1], t[r - 1], acc0);
-            t[r] = (r < j) ? 0.f : acc0 + acc1;
+        for (int i = 0; i + 1 < r; i += 2) {
+            acc0 = fmaf(-sA[(base + r) * LD + base + i], t[i], acc0);
+            acc1 = fmaf(-sA[(base + r) * LD + base + i + 1], t[i + 1], acc1);
         }
-#pragma unroll
-        for (int r = 0; r < 16; ++r) sT[(base + r) * LD + base + j] = t[r];
+        if (r & 1) acc0 = fmaf(-sA[(base + r) * LD + base + r - 1], t[r - 1], acc0);
+        t[r] = (r < j) ? 0.f : acc0 + acc1;
     }
-    __syncthreads();
-    {   // 32 level: X = A[o+16:o+32, o:o+16] t_{2P};  T[o+16:o+32, o:o+16] = -t_{2P+1} X
-        const int P = tid >> 8, rr = (tid & 255) >> 4, c = tid & 15, o = 32 * P;
-        float a[16], acc = 0.f;
 #pragma unroll
-        for (int k4 = 0; k4 < 4; ++k4) {
-            const float4 x = *reinterpret_cast<const float4 *>(sA + (o + 16 + rr) * LD + o + 4 * k4);
-            a[4 * k4] = x.x; a[4 * k4 + 1] = x.y; a[4 * k4 + 2] = x.z; a[4 * k4 + 3] = x.w;
-        }
+    for (int r = 0; r < 16; ++r) sT[(base + r) * LD + base + j] = t[r];
+}
+
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+__device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// acc[m][n] (16 x 8 tiles) += A (16*MT x 8*NK8, from Ab) * B (8*NK8 x 8*NT,
+// from Bb); both fp32 row-major with stride kLdT.  Tile (m, k) is skipped
+// when k >= kmax[m] (a known zero block of A).  Fragment ownership (lane =
+// 4g + t): A rows g, g+8 and columns t, t+4; B rows t, t+4 and column g; acc
+// rows g, g+8 and columns 2t, 2t+1.  With kInverseSplitTf32 each operand is
+// split into tf32 hi + lo and the product keeps hi*hi + hi*lo + lo*hi.
+constexpr bool kInverseSplitTf32 = false;
+template <int MT, int NT, int NK8>
+__device__ __forceinline__ void warp_mm(float (&acc)[MT][NT][4], const float *Ab, const float *Bb,
+                                        const int (&kmax)[MT], int lane) {
+    constexpr int LD = kLdT;
+    const int g = lane >> 2, t = lane & 3;
 #pragma unroll
-        for (int k = 0; k < 16; ++k) acc = fmaf(a[k], sT[(o + k) * LD + o + c], acc);
-        sA[(o + rr) * LD + o + 16 + c] = acc;  // X parked above the diagonal
-        __syncthreads();
+    for (int kk = 0; kk < NK8; ++kk) {
+        uint32_t ah[MT][4], al[MT][4], bh[NT][2], bl[NT][2];
 #pragma unroll
-        for (int k4 = 0; k4 < 4; ++k4) {
-            const float4 x = *reinterpret_cast<const float4 *>(sT + (o + 16 + rr) * LD + o + 16 + 4 * k4);
-            a[4 * k4] = x.x; a[4 * k4 + 1] = x.y; a[4 * k4 + 2] = x.z; a[4 * k4 + 3] = x.w;
-        }
-        acc = 0.f;
+        for (int m = 0; m < MT; ++m) {
+            const float *ap = Ab + m * 16 * LD + kk * 8;
+            const float av[4] = {ap[g * LD + t], ap[(g + 8) * LD + t], ap[g * LD + t + 4], ap[(g + 8) * LD + t + 4]};
 #pragma unroll
-        for (int k = 0; k < 16; ++k) acc = fmaf(a[k], sA[(o + k) * LD + o + 16 + c], acc);
-        sT[(o + 16 + rr) * LD + o + c] = -acc;
-        __syncthreads();
-    }
-    {   // 64 level: X = A[32:64, 0:32] T[0:32, 0:32];  T[32:64, 0:32] = -T[32:64, 32:64] X
-        const int r = tid >> 4, cq = (tid & 15) * 2;
-        float2 acc = make_float2(0.f, 0.f);
-#pragma unroll
-        for (int k4 = 0; k4 < 8; ++k4) {
-            const float4 a4 = *reinterpret_cast<const float4 *>(sA + (32 + r) * LD + 4 * k4);
-            const float a[4] = {a4.x, a4.y, a4.z, a4.w};
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                const float2 t2 = *reinterpret_cast<const float2 *>(sT + (4 * k4 + kk) * LD + cq);
-                acc.x = fmaf(a[kk], t2.x, acc.x);
-                acc.y = fmaf(a[kk], t2.y, acc.y);
+            for (int i = 0; i < 4; ++i) {
+                ah[m][i] = to_tf32(av[i]);
+                al[m][i] = kInverseSplitTf32 ? to_tf32(av[i] - __uint_as_float(ah[m][i])) : 0u;
             }
         }
-        *reinterpret_cast<float2 *>(sA + r * LD + 32 + cq) = acc;  // X parked in A[0:32, 32:64]
-        __syncthreads();
-        acc = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int k4 = 0; k4 < 8; ++k4) {
-            const float4 t4 = *reinterpret_cast<const float4 *>(sT + (32 + r) * LD + 32 + 4 * k4);
-            const float t[4] = {t4.x, t4.y, t4.z, t4.w};
+        for (int n = 0; n < NT; ++n) {
+            const float *bp = Bb + kk * 8 * LD + n * 8;
+            const float bv[2] = {bp[t * LD + g], bp[(t + 4) * LD + g]};
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                const float2 x2 = *reinterpret_cast<const float2 *>(sA + (4 * k4 + kk) * LD + 32 + cq);
-                acc.x = fmaf(t[kk], x2.x, acc.x);
-                acc.y = fmaf(t[kk], x2.y, acc.y);
+            for (int i = 0; i < 2; ++i) {
+                bh[n][i] = to_tf32(bv[i]);
+                bl[n][i] = kInverseSplitTf32 ? to_tf32(bv[i] - __uint_as_float(bh[n][i])) : 0u;
             }
         }
-        *reinterpret_cast<float2 *>(sT + (32 + r) * LD + cq) = make_float2(-acc.x, -acc.y);
-        __syncthreads();
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+            if (kk >= kmax[m]) continue;
+#pragma unroll
+            for (int n = 0; n < NT; ++n) {
+                if (kInverseSplitTf32) {
+                    mma_tf32_16x8x8(acc[m][n], al[m], bh[n][0], bh[n][1]);
+                    mma_tf32_16x8x8(acc[m][n], ah[m], bl[n][0], bl[n][1]);
+                }
+                mma_tf32_16x8x8(acc[m][n], ah[m], bh[n][0], bh[n][1]);
+            }
+        }
+    }
+}
+__device__ __forceinline__ void warp_store16x8(float *Db, const float (&acc)[4], float scale, int lane) {
+    constexpr int LD = kLdT;
+    const int g = lane >> 2, t = lane & 3;
+    *reinterpret_cast<float2 *>(Db + g * LD + 2 * t) = make_float2(scale * acc[0], scale * acc[1]);
+    *reinterpret_cast<float2 *>(Db + (g + 8) * LD + 2 * t) = make_float2(scale * acc[2], scale * acc[3]);
+}
+
+// The whole inverse, run by the two warps w = 0, 1 of the calling CTA;
+// `bar_id` names a 64-thread barrier between the 32 and 64 levels.
+__device__ __forceinline__ void inverse_two_warps(float *sA, float *sT, int w, int lane, int bar_id) {
+    constexpr int LD = kLdT;
+    inverse_diag16(sA, sT, 2 * w + (lane >> 4), lane & 15);
+    __syncwarp();
+    {   // 32 level, block P = w
+        const int o = 32 * w;
+        const int k2[1] = {2};
+        float acc[1][2][4] = {};
+        // X = A[o+16:o+32, o:o+16] t_{2P} -> parked in A[o:o+16, o+16:o+32]
+        warp_mm<1, 2, 2>(acc, sA + (o + 16) * LD + o, sT + o * LD + o, k2, lane);
+        warp_store16x8(sA + o * LD + o + 16, acc[0][0], 1.f, lane);
+        warp_store16x8(sA + o * LD + o + 24, acc[0][1], 1.f, lane);
+        __syncwarp();
+        float acc2[1][2][4] = {};
+        // T[o+16:o+32, o:o+16] = -t_{2P+1} X
+        warp_mm<1, 2, 2>(acc2, sT + (o + 16) * LD + o + 16, sA + o * LD + o + 16, k2, lane);
+        warp_store16x8(sT + (o + 16) * LD + o, acc2[0][0], -1.f, lane);
+        warp_store16x8(sT + (o + 16) * LD + o + 8, acc2[0][1], -1.f, lane);
+    }
+    asm volatile("barrier.sync %0, 64;" ::"r"(bar_id) : "memory");
+    {   // 64 level: slabs c0 = 8w (T11 rows 0:32) and 16 + 8w (T11 rows 16:32 only)
+        const int c0 = 8 * w, c1 = 16 + 8 * w;
+        const int k4[2] = {4, 4}, k2[2] = {2, 2};
+        float x0[2][1][4] = {}, x1[2][1][4] = {};
+        // X = A[32:64, 0:32] T11[:, slab] -> parked in A[0:32, 32 + slab]
+        warp_mm<2, 1, 4>(x0, sA + 32 * LD, sT + c0, k4, lane);
+        warp_mm<2, 1, 2>(x1, sA + 32 * LD + 16, sT + 16 * LD + c1, k2, lane);
+#pragma unroll
+        for (int m = 0; m < 2; ++m) {
+            warp_store16x8(sA + 16 * m * LD + 32 + c0, x0[m][0], 1.f, lane);
+            warp_store16x8(sA + 16 * m * LD + 32 + c1, x1[m][0], 1.f, lane);
+        }
+        __syncwarp();
+        // T[32:64, slab] = -T22 X  (T22[0:16, 16:32] = 0)
+        const int kt[2] = {2, 4};
+        float y0[2][1][4] = {}, y1[2][1][4] = {};
+        warp_mm<2, 1, 4>(y0, sT + 32 * LD + 32, sA + 32 + c0, kt, lane);
+        warp_mm<2, 1, 4>(y1, sT + 32 * LD + 32, sA + 32 + c1, kt, lane);
+#pragma unroll
+        for (int m = 0; m < 2; ++m) {
+            warp_store16x8(sT + (32 + 16 * m) * LD + c0, y0[m][0], -1.f, lane);
+            warp_store16x8(sT + (32 + 16 * m) * LD + c1, y1[m][0], -1.f, lane);
+        }
     }
 }
 
 // ------------------------------------------------------------------ prep CTA --
+// Prep-CTA roles: warps 0 and 1 (which hold only rows of A in the mask step)
+// solve the inverse while the other fourteen warps stage P, Q~ and the gates
+// into a local slot and warp 8 computes the next chunk's gates; lane 0 of the
+// last warp issues TMA, MMA and the bulk copy.  Three local staging slots feed the state CTA's two: the
+// local slot of chunk n was last read by the copy of chunk n-3, which the
+// state CTA confirmed before chunk n-1 went out, so staging never waits; only
+// the copy waits for the state CTA's slot.
+constexpr int kPrepIssuer = kTc2Threads - 32;
+constexpr int kPrepGateWarp = 8;
+constexpr int kPrepStagers = kTc2Threads - 2 * 32;  // warps 2-15 (named barrier 1)
+constexpr int kPrepQtStagers = kPrepStagers - 32;  // the issuer's warp skips the Q~ copy
+constexpr int kPrepSolverBarrier = 2;               // the two solver warps
+
 __device__ __forceinline__ void tc2_prep(uint8_t *sm, const CUtensorMap *tm_q, const CUtensorMap *tm_k,
                                          int T, int H, int b, int h, const float *log_alpha,
                                          const float *beta) {
@@ -174,16 +249,18 @@ __device__ __forceinline__ void tc2_prep(uint8_t *sm, const CUtensorMap *tm_q, c
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int wq = warp & 3, wc = warp >> 2;  // TMEM lane quarter, column group (of 4)
     const int nch = (T + kChunk - 1) / kChunk;
+    const bool issuer = tid == kPrepIssuer;
+    const bool solver = warp < 2;
+    const int srank = tid - 64;  // rank among the staging warps
     uint64_t *tma_full = reinterpret_cast<uint64_t *>(sm + L::P_BAR);  // [2]
     uint64_t *empty = tma_full + 2;                                      // [2], arrived by the state CTA
     uint64_t *mma_bar = tma_full + 4;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tma_full + 5);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    float *sg = reinterpret_cast<float *>(sm + L::P_GATE);
-    float *sbeta = sg + 64, *sgam = sg + 128, *sdec = sg + 192, *sgp = sg + 256, *sinv = sg + 320;
-    volatile int *exact_flag = reinterpret_cast<volatile int *>(sg + 384);
     float *sA = reinterpret_cast<float *>(sm + L::P_A), *sT = reinterpret_cast<float *>(sm + L::P_T);
     const uint32_t sbase = smem_u32(sm);
+    // gate arrays of chunk parity `par`: g, beta, gamma, dec, gamma', 1/gamma', exact flag
+    auto gates_of = [&](int par) { return reinterpret_cast<float *>(sm + L::P_GATE + par * L::P_GATE_BYTES); };
 
     if (tid == 0) {
         mbar_init(&tma_full[0], 1);
@@ -224,7 +301,7 @@ __device__ __forceinline__ void tc2_prep(uint8_t *sm, const CUtensorMap *tm_q, c
         }
         mma_commit(mma_bar);
     };
-    // gates of one chunk, held by warp 0 (lane l: rows 2l, 2l+1) between load and use
+    // gates of one chunk, held by the gate warp (lane l: rows 2l, 2l+1) between load and use
     float pl0 = 0.f, pl1 = 0.f, pb0 = 0.f, pb1 = 0.f;
     auto load_gates = [&](int n) {
         const int c0 = n * kChunk, nv = min(kChunk, T - c0);
@@ -235,11 +312,37 @@ __device__ __forceinline__ void tc2_prep(uint8_t *sm, const CUtensorMap *tm_q, c
         pb0 = r0 < nv ? beta[tok0 + (size_t)r0 * H] : 0.f;
         pb1 = r1 < nv ? beta[tok0 + (size_t)r1 * H] : 0.f;
     };
-    if (warp == 0) load_gates(0);
+    // g (inclusive prefix sum), gamma, dec, gamma' = exp(g - g_31), 1/gamma', exact flag
+    auto compute_gates = [&](float *G) {
+        const int r0 = 2 * lane, r1 = r0 + 1;
+        float incl = pl0 + pl1;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const float y = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += y;
+        }
+        const float g1 = incl, g0 = incl - pl1;
+        const float gC = __shfl_sync(0xffffffffu, incl, 31);
+        const float gM = __shfl_sync(0xffffffffu, g1, 15);  // g_31
+        const float gF = __shfl_sync(0xffffffffu, g0, 0);   // g_0
+        G[r0] = g0; G[r1] = g1;
+        G[64 + r0] = pb0; G[64 + r1] = pb1;
+        G[128 + r0] = expf(g0); G[128 + r1] = expf(g1);
+        G[192 + r0] = expf(gC - g0); G[192 + r1] = expf(gC - g1);
+        G[256 + r0] = expf(g0 - gM); G[256 + r1] = expf(g1 - gM);
+        G[320 + r0] = expf(gM - g0); G[320 + r1] = expf(gM - g1);
+        if (lane == 0) reinterpret_cast<volatile int *>(G + 384)[0] = (gF - gC) > 80.f;
+    };
+    if (warp == kPrepGateWarp) {
+        load_gates(0);
+        compute_gates(gates_of(0));
+        if (nch > 1) load_gates(1);  // prefetch: consumed during chunk 0
+    }
 
     int tma_issued = 0, tma_done = 0;
     uint32_t mma_phase = 0;
-    if (tid == 0) {
+    int ls = 0;  // local staging slot of chunk n (n mod 3)
+    if (issuer) {
         issue_tma(0, 0);
         ++tma_issued;
         if (nch > 1) {
@@ -257,31 +360,12 @@ __device__ __forceinline__ void tc2_prep(uint8_t *sm, const CUtensorMap *tm_q, c
 #pragma unroll 1
     for (int n = 0; n < nch; ++n) {
         const int s = n & 1;
-        uint8_t *stg = sm + L::P_STG + s * L::H_SLOT;
+        uint8_t *stg = sm + L::P_STG + ls * L::H_SLOT;
+        const float *G = gates_of(s);
+        const float *sg = G, *sbeta = G + 64, *sgam = G + 128, *sdec = G + 192, *sgp = G + 256, *sinv = G + 320;
         __syncthreads();
         if (*abort_flag) break;
-        if (warp == 0) {  // gates: g (inclusive prefix sum), gamma, dec, gamma' = exp(g - g_31), 1/gamma'
-            const int r0 = 2 * lane, r1 = r0 + 1;
-            float incl = pl0 + pl1;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const float y = __shfl_up_sync(0xffffffffu, incl, off);
-                if (lane >= off) incl += y;
-            }
-            const float g1 = incl, g0 = incl - pl1;
-            const float gC = __shfl_sync(0xffffffffu, incl, 31);
-            const float gM = __shfl_sync(0xffffffffu, g1, 15);  // g_31
-            const float gF = __shfl_sync(0xffffffffu, g0, 0);   // g_0
-            sg[r0] = g0; sg[r1] = g1;
-            sbeta[r0] = pb0; sbeta[r1] = pb1;
-            sgam[r0] = expf(g0); sgam[r1] = expf(g1);
-            sdec[r0] = expf(gC - g0); sdec[r1] = expf(gC - g1);
-            sgp[r0] = expf(g0 - gM); sgp[r1] = expf(g1 - gM);
-            sinv[r0] = expf(gM - g0); sinv[r1] = expf(gM - g1);
-            if (lane == 0) *exact_flag = (gF - gC) > 80.f;
-            if (n + 1 < nch) load_gates(n + 1);  // prefetch: consumed next chunk
-        }
-        if (tid == 0 && !mbar_wait(mma_bar, mma_phase)) *abort_flag = 1;
+        if (issuer && !mbar_wait(mma_bar, mma_phase)) *abort_flag = 1;
         mma_phase ^= 1;
         tc_before_sync();
         __syncthreads();
@@ -295,7 +379,7 @@ __device__ __forceinline__ void tc2_prep(uint8_t *sm, const CUtensorMap *tm_q, c
         float pv[16];
         {
             tmem_ld16(tl + c0, pv);
-            const bool exact = *exact_flag;
+            const bool exact = reinterpret_cast<const volatile int *>(G + 384)[0] != 0;
             float sv[16], gv[16];
 #pragma unroll
             for (int k4 = 0; k4 < 4; ++k4) {
@@ -322,57 +406,29 @@ __device__ __forceinline__ void tc2_prep(uint8_t *sm, const CUtensorMap *tm_q, c
         }
         tc_before_sync();
         __syncthreads();
-        if (tid == 0 && n + 1 < nch) {  // next chunk's K K^T / Q K^T overlaps this chunk's inverse
-            tc_after_sync();
-            if (!mbar_wait(&tma_full[s ^ 1], (uint32_t)(((n + 1) >> 1) & 1))) *abort_flag = 1;
-            else {
-                ++tma_done;
-                issue_mma1(s ^ 1);
+
+        if (solver) {
+            inverse_two_warps(sA, sT, warp, lane, kPrepSolverBarrier);
+        } else {
+            if (issuer && n + 1 < nch) {  // next chunk's K K^T / Q K^T overlaps this chunk's inverse
+                tc_after_sync();
+                if (!mbar_wait(&tma_full[s ^ 1], (uint32_t)(((n + 1) >> 1) & 1))) *abort_flag = 1;
+                else {
+                    ++tma_done;
+                    issue_mma1(s ^ 1);
+                }
             }
-        }
-        invert_unit_lower_64_w16(sA, sT);
-        // staging slot s (and the state's slot s) must have been consumed (chunk n-2)
-        if (tid == 0 && n >= 2 && !mbar_wait_cluster(&empty[s], (uint32_t)(((n >> 1) - 1) & 1))) *abort_flag = 1;
-        __syncthreads();
-        if (*abort_flag) break;
-        {
             float *hg = reinterpret_cast<float *>(stg + L::H_G);
-            if (tid < 64) hg[tid] = sgam[tid];
-            else if (tid < 128) hg[tid] = sdec[tid - 64];
-            // P rows
-            if (row >= 64) {
+            if (srank < 128) hg[srank] = srank < 64 ? sgam[srank] : sdec[srank - 64];
+            if (row >= 64) {  // P rows
 #pragma unroll
                 for (int ch = 0; ch < 2; ++ch)
                     st_bf16x8(stg + L::H_P + sw128_offset(row - 64, wc * 2 + ch), pv + 8 * ch);
             }
-            // T' = T diag(beta) (rows 0-63), T'' = T diag(beta gamma) (rows 64-127), 16 columns each
-            {
-                const int r = tid & 63;
-                const bool second = (tid & 64) != 0;
-                const int cb = (tid >> 7) * 16;
-                float t[16], bv[16], gm[16];
-#pragma unroll
-                for (int k4 = 0; k4 < 4; ++k4) {
-                    const float4 x = *reinterpret_cast<const float4 *>(sT + r * kLdT + cb + 4 * k4);
-                    const float4 y = *reinterpret_cast<const float4 *>(sbeta + cb + 4 * k4);
-                    const float4 z = *reinterpret_cast<const float4 *>(sgam + cb + 4 * k4);
-                    t[4 * k4] = x.x; t[4 * k4 + 1] = x.y; t[4 * k4 + 2] = x.z; t[4 * k4 + 3] = x.w;
-                    bv[4 * k4] = y.x; bv[4 * k4 + 1] = y.y; bv[4 * k4 + 2] = y.z; bv[4 * k4 + 3] = y.w;
-                    gm[4 * k4] = z.x; gm[4 * k4 + 1] = z.y; gm[4 * k4 + 2] = z.z; gm[4 * k4 + 3] = z.w;
-                }
-#pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    t[i] = (cb + i <= r) ? t[i] * bv[i] * (second ? gm[i] : 1.f) : 0.f;
-#pragma unroll
-                for (int ch = 0; ch < 2; ++ch)
-                    st_bf16x8(stg + (second ? L::H_T2 : L::H_T1) + sw128_offset(r, (cb >> 3) + ch), t + 8 * ch);
-            }
             // Q~ = diag(gamma) Q: same swizzled positions as the Q tile
-            {
-                const uint8_t *qt = sm + L::P_KQ + s * 32768 + 8192;
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int ci = tid * 2 + e;  // 16-byte chunk 0..1023
+            const uint8_t *qt = sm + L::P_KQ + s * 32768 + 8192;
+            if (srank < kPrepQtStagers) {
+                for (int ci = srank; ci < 1024; ci += kPrepQtStagers) {  // 16-byte chunks
                     const int half = ci >> 9;
                     const uint32_t ob = (uint32_t)(ci & 511) * 16;
                     const float g = sgam[ob >> 7];
@@ -383,19 +439,50 @@ __device__ __forceinline__ void tc2_prep(uint8_t *sm, const CUtensorMap *tm_q, c
                     st_bf16x8(stg + L::H_QT + half * 8192 + ob, f);
                 }
             }
-        }
-        fence_async_smem();
-        __syncthreads();
-        if (tid == 0) {
-            bulk_copy_to_cluster(remote_slot0 + s * L::H_SLOT, stg, L::H_BYTES, remote_full0 + 8 * s);
-            if (n + 2 < nch) {  // K/Q stage s is free: its MMA is done and Q~ has been read
+            asm volatile("barrier.sync 1, %0;" ::"n"(kPrepStagers) : "memory");
+            if (issuer && n + 2 < nch && !*abort_flag) {  // K/Q stage s is free: MMA done, Q read
                 issue_tma(n + 2, s);
                 ++tma_issued;
             }
+            if (warp == kPrepGateWarp && n + 1 < nch) {  // next chunk's gates (other buffer)
+                compute_gates(gates_of(s ^ 1));
+                if (n + 2 < nch) load_gates(n + 2);
+            }
         }
+        __syncthreads();
+        if (*abort_flag) break;
+        {   // T' = T diag(beta) (rows 0-63), T'' = T diag(beta gamma) (rows 64-127), 16 columns each
+            const int r = tid & 63;
+            const bool second = (tid & 64) != 0;
+            const int cb = (tid >> 7) * 16;
+            float t[16], bv[16], gm[16];
+#pragma unroll
+            for (int k4 = 0; k4 < 4; ++k4) {
+                const float4 x = *reinterpret_cast<const float4 *>(sT + r * kLdT + cb + 4 * k4);
+                const float4 y = *reinterpret_cast<const float4 *>(sbeta + cb + 4 * k4);
+                const float4 z = *reinterpret_cast<const float4 *>(sgam + cb + 4 * k4);
+                t[4 * k4] = x.x; t[4 * k4 + 1] = x.y; t[4 * k4 + 2] = x.z; t[4 * k4 + 3] = x.w;
+                bv[4 * k4] = y.x; bv[4 * k4 + 1] = y.y; bv[4 * k4 + 2] = y.z; bv[4 * k4 + 3] = y.w;
+                gm[4 * k4] = z.x; gm[4 * k4 + 1] = z.y; gm[4 * k4 + 2] = z.z; gm[4 * k4 + 3] = z.w;
+            }
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                t[i] = (cb + i <= r) ? t[i] * bv[i] * (second ? gm[i] : 1.f) : 0.f;
+#pragma unroll
+            for (int ch = 0; ch < 2; ++ch)
+                st_bf16x8(stg + (second ? L::H_T2 : L::H_T1) + sw128_offset(r, (cb >> 3) + ch), t + 8 * ch);
+        }
+        fence_async_smem();
+        __syncthreads();
+        if (issuer) {
+            // the state CTA's slot s must have been consumed (chunk n-2)
+            if (n >= 2 && !mbar_wait_cluster(&empty[s], (uint32_t)(((n >> 1) - 1) & 1))) *abort_flag = 1;
+            else bulk_copy_to_cluster(remote_slot0 + s * L::H_SLOT, stg, L::H_BYTES, remote_full0 + 8 * s);
+        }
+        ls = ls == 2 ? 0 : ls + 1;
     }
 
-    if (*abort_flag && tid == 0) {
+    if (*abort_flag && issuer) {
         record_status(GDR_ERR_TIMEOUT);
         for (int k2 = tma_done; k2 < tma_issued; ++k2) mbar_wait(&tma_full[k2 & 1], (uint32_t)((k2 >> 1) & 1));
         mma_commit(mma_bar);
