@@ -241,9 +241,11 @@ constexpr int kPrepStagers = kTc2Threads - 2 * 32;  // warps 2-15 (named barrier
 constexpr int kPrepQtStagers = kPrepStagers - 32;  // the issuer's warp skips the Q~ copy
 constexpr int kPrepSolverBarrier = 2;               // the two solver warps
 
+// `reverse` walks the chunks from last to first (the backward's dS pass):
+// step n then works on chunk nch-1-n; everything else is unchanged.
 __device__ __forceinline__ void tc2_prep(uint8_t *sm, const CUtensorMap *tm_q, const CUtensorMap *tm_k,
                                          int T, int H, int b, int h, const float *log_alpha,
-                                         const float *beta) {
+                                         const float *beta, bool reverse = false) {
     using L = Tc2Layout;
     using namespace sm100;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -285,11 +287,12 @@ __device__ __forceinline__ void tc2_prep(uint8_t *sm, const CUtensorMap *tm_q, c
 
     auto issue_tma = [&](int n, int s) {
         uint8_t *kq = sm + L::P_KQ + s * 32768;
+        const int c = reverse ? nch - 1 - n : n;
         mbar_expect_tx(&tma_full[s], 32768);
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
-            tma_load_4d(kq + half * 16384, tm_k, &tma_full[s], half * 64, h, n * kChunk, b);
-            tma_load_4d(kq + half * 16384 + 8192, tm_q, &tma_full[s], half * 64, h, n * kChunk, b);
+            tma_load_4d(kq + half * 16384, tm_k, &tma_full[s], half * 64, h, c * kChunk, b);
+            tma_load_4d(kq + half * 16384 + 8192, tm_q, &tma_full[s], half * 64, h, c * kChunk, b);
         }
     };
     auto issue_mma1 = [&](int s) {  // [K;Q] K^T -> TMEM (lanes 0-63 K K^T, 64-127 Q K^T)
@@ -304,7 +307,7 @@ __device__ __forceinline__ void tc2_prep(uint8_t *sm, const CUtensorMap *tm_q, c
     // gates of one chunk, held by the gate warp (lane l: rows 2l, 2l+1) between load and use
     float pl0 = 0.f, pl1 = 0.f, pb0 = 0.f, pb1 = 0.f;
     auto load_gates = [&](int n) {
-        const int c0 = n * kChunk, nv = min(kChunk, T - c0);
+        const int c0 = (reverse ? nch - 1 - n : n) * kChunk, nv = min(kChunk, T - c0);
         const size_t tok0 = ((size_t)b * T + c0) * H + h;
         const int r0 = 2 * lane, r1 = r0 + 1;
         pl0 = r0 < nv ? log_alpha[tok0 + (size_t)r0 * H] : 0.f;

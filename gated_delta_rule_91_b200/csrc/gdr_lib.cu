@@ -17,6 +17,7 @@
 #include "gdr2_simt.cuh"
 #include "fwd_tc.cuh"
 #include "fwd_tc2.cuh"
+#include "bwd_tc.cuh"
 
 namespace gdr {
 std::atomic<uint64_t> g_launches{0};
@@ -73,6 +74,27 @@ gdr_status check_dims(const char *fn, int B, int T, int H, int dk, int dv, gdr_d
     return GDR_OK;
 }
 
+
+// The backward's kernels for one call (shared by gdr_bwd and gdr_bwd_noalloc).
+// bf16 with dk = dv = 128 runs on the tensor cores (recompute, dS pass,
+// chunk-parallel gradients); GDR_BWD_KERNEL=simt selects the CUDA-core
+// backward (used to cross-check them).
+cudaError_t run_bwd(int B, int T, int H, int dk, int dv, gdr_dtype dt, const void *q, const void *k,
+                    const void *v, const float *log_alpha, const float *beta, const float *S0, const void *dO,
+                    const float *dS_T, void *dq, void *dk_out, void *dv_out, float *dlog_alpha, float *dbeta,
+                    float *dS0, void *workspace, cudaStream_t s) {
+    const char *sel = getenv("GDR_BWD_KERNEL");
+    if (dt == GDR_BF16 && dk == 128 && dv == 128 && !(sel != nullptr && strcmp(sel, "simt") == 0))
+        return launch_bwd_tc(B, T, H, q, k, v, log_alpha, beta, S0, dO, dS_T, dq, dk_out, dv_out, dlog_alpha,
+                             dbeta, dS0, workspace, s);
+#define GDR_BWD_ARGS B, T, H, dv, q, k, v, log_alpha, beta, S0, dO, dS_T, dq, dk_out, dv_out, \
+                     dlog_alpha, dbeta, dS0, workspace, s
+    if (dt == GDR_F32)
+        return dk == 128 ? launch_bwd_simt<float, 128>(GDR_BWD_ARGS) : launch_bwd_simt<float, 64>(GDR_BWD_ARGS);
+    return dk == 128 ? launch_bwd_simt<__nv_bfloat16, 128>(GDR_BWD_ARGS)
+                     : launch_bwd_simt<__nv_bfloat16, 64>(GDR_BWD_ARGS);
+#undef GDR_BWD_ARGS
+}
 }  // namespace
 
 extern "C" {
@@ -226,14 +248,8 @@ gdr_status gdr_bwd(int B, int T, int H, int dk, int dv, gdr_dtype dt, const void
         return fail(GDR_ERR_INVALID_ARGUMENT, "%s: workspace is not 16-byte aligned", fn);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e;
-#define GDR_BWD_ARGS B, T, H, dv, q, k, v, log_alpha, beta, S0, dO, dS_T, dq, dk_out, dv_out, \
-                     dlog_alpha, dbeta, dS0, workspace, s
-    if (dt == GDR_F32)
-        e = dk == 128 ? launch_bwd_simt<float, 128>(GDR_BWD_ARGS) : launch_bwd_simt<float, 64>(GDR_BWD_ARGS);
-    else
-        e = dk == 128 ? launch_bwd_simt<__nv_bfloat16, 128>(GDR_BWD_ARGS)
-                      : launch_bwd_simt<__nv_bfloat16, 64>(GDR_BWD_ARGS);
-#undef GDR_BWD_ARGS
+    e = run_bwd(B, T, H, dk, dv, dt, q, k, v, log_alpha, beta, S0, dO, dS_T, dq, dk_out, dv_out, dlog_alpha,
+                dbeta, dS0, workspace, s);
     if (e != cudaSuccess) return cuda_fail(e, fn);
     return GDR_OK;
 }
@@ -333,14 +349,8 @@ extern "C" gdr_status gdr_bwd_noalloc(int B, int T, int H, int dk, int dv, gdr_d
         scratch = g_scratch_ptr[dev];
     }
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-#define GDR_BWD_ARGS B, T, H, dv, q, k, v, log_alpha, beta, S0, dO, dS_T, dq, dk_out, dv_out, \
-                     dlog_alpha, dbeta, dS0, scratch, s
-    if (dt == GDR_F32)
-        e = dk == 128 ? launch_bwd_simt<float, 128>(GDR_BWD_ARGS) : launch_bwd_simt<float, 64>(GDR_BWD_ARGS);
-    else
-        e = dk == 128 ? launch_bwd_simt<__nv_bfloat16, 128>(GDR_BWD_ARGS)
-                      : launch_bwd_simt<__nv_bfloat16, 64>(GDR_BWD_ARGS);
-#undef GDR_BWD_ARGS
+    e = run_bwd(B, T, H, dk, dv, dt, q, k, v, log_alpha, beta, S0, dO, dS_T, dq, dk_out, dv_out, dlog_alpha,
+                dbeta, dS0, scratch, s);
     if (e != cudaSuccess) return cuda_fail(e, fn);
     return GDR_OK;
 }

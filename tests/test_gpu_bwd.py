@@ -104,3 +104,20 @@ def test_bwd_deterministic():
     b = _gpu(x, None)
     for n in NAMES + ["dS0"]:
         assert torch.equal(a[n], b[n]), n
+
+
+@pytest.mark.parametrize("T", [64, 129, 1000])
+def test_tensor_core_backward_matches_cuda_core_backward(T, monkeypatch):
+    """bf16 d=128 runs on tcgen05 (recompute, dS pass, chunk-parallel
+    gradients); the fp32 CUDA-core backward (GDR_BWD_KERNEL=simt) on the same
+    inputs must agree within the bf16 tolerance, and both with the oracle."""
+    x = synth.gdr_inputs(2, T, 3, 128, 128, "bf16", seed=60 + T, s0_std=0.02, with_dO=True)
+    dST = torch.randn(2, 3, 128, 128, generator=torch.Generator().manual_seed(T)) * 0.05
+    got = _gpu(x, dST)
+    gdr.check_status()
+    monkeypatch.setenv("GDR_BWD_KERNEL", "simt")
+    ref_si = _gpu(x, dST)
+    for n in NAMES:
+        assert max_rel(np64(got[n]), np64(ref_si[n])) <= TOL_G["bf16"], n
+    assert fro_rel(np64(got["dS0"]), np64(ref_si["dS0"])) <= 1e-2
+    _compare(got, _oracle(x, dST), "bf16")
