@@ -28,10 +28,8 @@
 // fixed order by gdr_bwd_reduce_kernel (deterministic, no atomics).
 #pragma once
 #include "common.cuh"
-#include <type_traits>
 
 #include "fwd_simt.cuh"
-#include "fwd_tc2.cuh"
 
 namespace gdr {
 
@@ -689,12 +687,11 @@ cudaError_t launch_bwd_simt(int B, int T, int H, int dv, const void *q, const vo
                             void *dv_out, float *dla, float *dbeta, float *dS0, void *ws,
                             cudaStream_t stream) {
     BwdWorkspace w = bwd_carve(ws, B, T, H, DK, dv);
-    // 1) forward recompute, keeping every chunk's entry state (tensor-core
-    //    kernel for bf16 with dk = dv = 128, CUDA cores otherwise)
-    cudaError_t err = (std::is_same<Tio, __nv_bfloat16>::value && DK == 128 && dv == 128)
-                          ? launch_fwd_tc2(B, T, H, q, k, v, la, beta, S0, nullptr, nullptr, stream, w.states)
-                          : launch_fwd_simt<Tio, DK>(B, T, H, dv, q, k, v, la, beta, S0, nullptr, nullptr,
-                                                     stream, w.states);
+    // 1) forward recompute on the CUDA cores, keeping every chunk's fp32 entry
+    //    state (this backward is also the cross-check of the tensor-core one,
+    //    so it shares none of its kernels)
+    cudaError_t err = launch_fwd_simt<Tio, DK>(B, T, H, dv, q, k, v, la, beta, S0, nullptr, nullptr, stream,
+                                               w.states);
     if (err != cudaSuccess) return err;
     // 2) reverse chunk pass per (b, h, slice)
     using L = BwdLayout<DK>;

@@ -7,14 +7,15 @@
 // are listed at the top of bwd_simt.cuh).  Three launches:
 //
 //  1. the forward, recomputed without outputs, keeps every chunk's entry
-//     state S_n (fp32);
+//     state S_n as its bf16 MMA operand tile (32 KB, 128B-swizzled);
 //  2. the dS pass (gdr_bwd_chain_kernel), one 2-CTA cluster per (b, h), walks
 //     the chunks from last to first.  Its prep CTA is the forward's (masks,
 //     inverse, P, Q~ = diag(gamma) Q, T'' = T diag(beta gamma)); its state CTA
 //     carries D = dL/dS (exit state of the current chunk) in TMEM:
 //        dU^T = D K^T diag(exp(g_C - g)) + dO^T P
 //        D   <- gamma_C D + dO^T Q~ - dU^T W,   W = T'' K,
-//     and stores every chunk's D (fp32) for step 3;  dS0 is the final D;
+//     and stores every chunk's D the same way for step 3;  dS0 is the final
+//     D (fp32);
 //  3. the gradients (gdr_bwd_grad_kernel), one CTA per (b, h, chunk), all
 //     chunks in parallel, from S_n, D_n and the chunk's inputs.
 #pragma once
@@ -26,11 +27,12 @@ namespace gdr {
 constexpr uint32_t kBcD = 0, kBcX1 = 128, kBcX2 = 192, kBcW = 256;
 
 // State CTA of the dS pass.  Shared memory follows Tc2Layout (the prep CTA's
-// DSMEM copies land in S_H): K tiles in S_K, dO tiles in S_V, W in S_W and
-// S_OST by step parity, bf16 D and then dU^T in S_SB.
+// DSMEM copies land in S_H): K tiles in S_K, dO tiles in S_V, W in S_W, bf16
+// D and then dU^T in S_SB.  W of step n+1 is computed behind step n's D
+// update and converted in step n+1, so the hand-off wait stays off the chain.
 __device__ __forceinline__ void bwd_chain_state(uint8_t *sm, const CUtensorMap *tm_k, const CUtensorMap *tm_do,
                                                 int T, int H, int b, int h, const float *dS_T, float *dS0,
-                                                float *D_chunks) {
+                                                uint8_t *D_tiles) {
     using L = Tc2Layout;
     using namespace sm100;
     constexpr int D = 128;
@@ -45,7 +47,6 @@ __device__ __forceinline__ void bwd_chain_state(uint8_t *sm, const CUtensorMap *
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tma_full + 6);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     const uint32_t sbase = smem_u32(sm);
-    auto wbuf = [](int n) -> uint32_t { return (n & 1) ? L::S_OST : L::S_W; };
     auto chunk_of = [&](int n) { return nch - 1 - n; };
 
     if (tid == 0) {
@@ -113,12 +114,11 @@ __device__ __forceinline__ void bwd_chain_state(uint8_t *sm, const CUtensorMap *
         mma_commit(bar_b);
         return true;
     };
-    auto convert_w = [&](int n) {  // W^T (lane j, column r) -> [j][r] bf16, the K-major B of D -= dU^T W
+    auto convert_w = [&]() {  // W^T (lane j, column r) -> [j][r] bf16, the K-major B of D -= dU^T W
         float v[16];
         tmem_ld16(tl + kBcW + wc * 16, v);
 #pragma unroll
-        for (int ch = 0; ch < 2; ++ch) st_bf16x8(sm + wbuf(n) + sw128_offset(row, wc * 2 + ch), v + 8 * ch);
-        fence_async_smem();
+        for (int ch = 0; ch < 2; ++ch) st_bf16x8(sm + L::S_W + sw128_offset(row, wc * 2 + ch), v + 8 * ch);
     };
 
     int tma_issued = 0, tma_done_n = 0;
@@ -131,15 +131,8 @@ __device__ __forceinline__ void bwd_chain_state(uint8_t *sm, const CUtensorMap *
             ++tma_issued;
         }
         if (!issue_w(0)) *abort_flag = 1;
-        else if (!mbar_wait(bar_b, bphase)) *abort_flag = 1;
         else tma_done_n = 1;
     }
-    bphase ^= 1;
-    tc_before_sync();
-    __syncthreads();
-    tc_after_sync();
-    if (!*abort_flag) convert_w(0);
-    tc_before_sync();
     __syncthreads();
 
     int n_done = 0;  // steps whose MMAs all completed
@@ -150,17 +143,12 @@ __device__ __forceinline__ void bwd_chain_state(uint8_t *sm, const CUtensorMap *
         const uint32_t hs = sbase + L::S_H + s * L::H_SLOT;
         const float *hgate = reinterpret_cast<const float *>(sm + L::S_H + s * L::H_SLOT + L::H_G);
 
-        // (a) store D (the exit-state gradient of chunk c); D -> bf16 operand; D *= gamma_C
+        // (a) D (the exit-state gradient of chunk c) -> bf16 operand; D *= gamma_C
         {
             const float gC = hgate[kChunk - 1];
             const int col = wc * 32;
             float v[32];
             tmem_ld32(tl + kBcD + col, v);
-            if (D_chunks) {
-                float4 *dst = reinterpret_cast<float4 *>(D_chunks + (((size_t)bh * nch + c) * D + row) * D + col);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-            }
             uint8_t *half = sm + L::S_SB + (wc >> 1) * 16384;
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4) st_bf16x8(half + sw128_offset(row, (wc & 1) * 4 + q4), v + 8 * q4);
@@ -176,6 +164,10 @@ __device__ __forceinline__ void bwd_chain_state(uint8_t *sm, const CUtensorMap *
         // (b) X1 = D K^T, X2 = dO^T P (-> bar_a); then D += dO^T Q~
         if (tid == 0) {
             tc_after_sync();
+            if (D_tiles) {  // the bf16 tile of D, as swizzled, for the gradient kernel
+                bulk_store_s2g(D_tiles + ((size_t)bh * nch + c) * 32768, sm + L::S_SB, 32768);
+                bulk_commit();
+            }
             const uint32_t sb = sbase + L::S_SB;
             const uint32_t kt = sbase + L::S_K + s * 16384, dt = sbase + L::S_V + s * 16384;
 #pragma unroll
@@ -193,16 +185,15 @@ __device__ __forceinline__ void bwd_chain_state(uint8_t *sm, const CUtensorMap *
             for (int kk = 0; kk < 4; ++kk)
                 mma_bf16(tmem + kBcD, smem_desc_sw128(dt + kk * 2048, 8192, 1024),
                          smem_desc_sw128(hs + L::H_QT + kk * 2048, 8192, 1024), idesc_bf16(128, 128, true, true), 1);
-            // (c) W of the next step
-            if (n + 1 < nch) {
-                if (!issue_w(n + 1)) *abort_flag = 1;
-                else ++tma_done_n;
-            }
         }
         __syncwarp();
-        // (d) dU^T = X1 diag(exp(g_C - g)) + X2 -> bf16 A operand
-        if (tid == 0 && !mbar_wait(bar_a, aphase)) *abort_flag = 1;
+        // (d) dU^T = X1 diag(exp(g_C - g)) + X2 -> bf16 A operand; W of this step -> S_W
+        if (tid == 0) {
+            if (!mbar_wait(bar_a, aphase) || !mbar_wait(bar_b, bphase)) *abort_flag = 1;
+            if (D_tiles) bulk_wait_read_all();  // the copy of D has left S_SB
+        }
         aphase ^= 1;
+        bphase ^= 1;
         tc_before_sync();
         __syncthreads();
         if (*abort_flag) break;
@@ -222,28 +213,25 @@ __device__ __forceinline__ void bwd_chain_state(uint8_t *sm, const CUtensorMap *
 #pragma unroll
             for (int ch = 0; ch < 2; ++ch) st_bf16x8(sm + L::S_SB + sw128_offset(row, wc * 2 + ch), x1 + 8 * ch);
         }
+        convert_w();
         fence_async_smem();
         tc_before_sync();
         __syncthreads();
 
-        // (e) D -= dU^T W
+        // (e) D -= dU^T W, then W of the next step
         if (tid == 0) {
             tc_after_sync();
-            const uint32_t du = sbase + L::S_SB, wb = sbase + wbuf(n);
+            const uint32_t du = sbase + L::S_SB, wb = sbase + L::S_W;
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
                 mma_bf16(tmem + kBcD, smem_desc_sw128(du + kk * 32, 16, 1024), smem_desc_sw128(wb + kk * 32, 16, 1024),
                          idesc_bf16(128, 128, false, false, true), 1);
             mma_commit(bar_a);
-            if (n + 1 < nch && !mbar_wait(bar_b, bphase)) *abort_flag = 1;
+            if (n + 1 < nch) {
+                if (!issue_w(n + 1)) *abort_flag = 1;
+                else ++tma_done_n;
+            }
         }
-        if (n + 1 < nch) bphase ^= 1;
-        tc_before_sync();
-        __syncthreads();
-        if (*abort_flag) break;
-        tc_after_sync();
-        // (f) W of the next step -> the other W buffer (its last reader, step n-1, is done)
-        if (n + 1 < nch) convert_w(n + 1);
         // (g) step n finished: release its hand-off slot and K/dO stage
         if (tid == 0) {
             if (!mbar_wait(bar_a, aphase)) *abort_flag = 1;
@@ -271,6 +259,7 @@ __device__ __forceinline__ void bwd_chain_state(uint8_t *sm, const CUtensorMap *
 #pragma unroll
         for (int i = 0; i < 8; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
     }
+    if (tid == 0) bulk_wait_all();  // the copies of D are complete before the CTA exits
     if (*abort_flag && tid == 0) {
         record_status(GDR_ERR_TIMEOUT);
         // drain: this CTA's TMA loads, its MMAs, and the prep CTA's copies into it
@@ -293,7 +282,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTc2Threads, 1)
 gdr_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_do, int T, int H,
                      const float *__restrict__ log_alpha, const float *__restrict__ beta,
-                     const float *__restrict__ dS_T, float *__restrict__ dS0, float *__restrict__ D_chunks) {
+                     const float *__restrict__ dS_T, float *__restrict__ dS0, uint8_t *__restrict__ D_tiles) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
@@ -301,7 +290,7 @@ gdr_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     if (sm100::cluster_ctarank() == 0)
         tc2_prep(sm, &tm_q, &tm_k, T, H, b, h, log_alpha, beta, true);
     else
-        bwd_chain_state(sm, &tm_k, &tm_do, T, H, b, h, dS_T, dS0, D_chunks);
+        bwd_chain_state(sm, &tm_k, &tm_do, T, H, b, h, dS_T, dS0, D_tiles);
 }
 
 // ------------------------------------------------------------ gradient kernel --
@@ -404,7 +393,7 @@ __global__ void __launch_bounds__(kTc2Threads, 1)
 gdr_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                     int T, int H, const float *__restrict__ log_alpha, const float *__restrict__ beta,
-                    const float *__restrict__ S_chunks, const float *__restrict__ D_chunks,
+                    const uint8_t *__restrict__ S_tiles, const uint8_t *__restrict__ D_tiles,
                     __nv_bfloat16 *__restrict__ dq, __nv_bfloat16 *__restrict__ dk,
                     __nv_bfloat16 *__restrict__ dv, float *__restrict__ dlog_alpha, float *__restrict__ dbeta) {
     using L = BgLayout;
@@ -428,7 +417,7 @@ gdr_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const uint32_t sbase = smem_u32(sm);
     const uint32_t kq = sbase + L::KQ, dor = sbase + L::DOR, sb = sbase + L::SB, db = sbase + L::DB;
     const uint32_t ru = sbase + L::RU, ub = sbase + L::UB, tb = sbase + L::TB, pb = sbase + L::PB;
-    const size_t chunk_state = ((size_t)bh * nch + c) * D * D;
+    const size_t chunk_tile = ((size_t)bh * nch + c) * 32768;
     auto tok = [&](int r) { return ((size_t)(b * T + t0 + r) * H + h); };
 
     if (tid == 0) {
@@ -436,7 +425,9 @@ gdr_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         mbar_init(bar_mma, 1);
         fence_mbar_init();
         *abort_flag = 0;
-        mbar_expect_tx(bar_tma, 65536);
+        mbar_expect_tx(bar_tma, 65536 + 2 * 32768);
+        bulk_load_g2s(sm + L::SB, S_tiles + chunk_tile, 32768, bar_tma);
+        bulk_load_g2s(sm + L::DB, D_tiles + chunk_tile, 32768, bar_tma);
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
             tma_load_4d(sm + L::KQ + half * 16384, &tm_k, bar_tma, half * 64, h, t0, b);
@@ -446,28 +437,6 @@ gdr_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
     }
     if (warp == 0) tmem_alloc(tmem_slot, 512);
-    {   // S, D -> bf16 [c][j] tiles; <D, S> partial
-        const int r = tid & 127, cq = tid >> 7;
-        const float4 *ps = reinterpret_cast<const float4 *>(S_chunks + chunk_state + (size_t)r * D + cq * 32);
-        const float4 *pd = reinterpret_cast<const float4 *>(D_chunks + chunk_state + (size_t)r * D + cq * 32);
-        float vs[32], vd[32];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const float4 x = ps[i], y = pd[i];
-            vs[4 * i] = x.x; vs[4 * i + 1] = x.y; vs[4 * i + 2] = x.z; vs[4 * i + 3] = x.w;
-            vd[4 * i] = y.x; vd[4 * i + 1] = y.y; vd[4 * i + 2] = y.z; vd[4 * i + 3] = y.w;
-        }
-        float ds = 0.f;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) ds = fmaf(vd[i], vs[i], ds);
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-            st_bf16x8(sm + L::SB + (cq >> 1) * 16384 + sw128_offset(r, (cq & 1) * 4 + q4), vs + 8 * q4);
-            st_bf16x8(sm + L::DB + (cq >> 1) * 16384 + sw128_offset(r, (cq & 1) * 4 + q4), vd + 8 * q4);
-        }
-        ds = warp_sum32(ds);
-        if (lane == 0) red[L::RDS + warp] = ds;
-    }
     if (warp == 15) {  // gates: g (inclusive prefix sum of log alpha), beta, gamma, exp(g_C - g)
         const int r0 = 2 * lane, r1 = r0 + 1;
         const float l0 = r0 < nv ? log_alpha[tok(r0)] : 0.f, l1 = r1 < nv ? log_alpha[tok(r1)] : 0.f;
@@ -542,6 +511,20 @@ gdr_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
         if (!mma_wait_all()) break;
 
+        {   // <D, S> over the bf16 tiles (same layout, so elementwise by byte offset)
+            float ds = 0.f;
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                float fs[8], fd[8];
+                const uint32_t off = (uint32_t)(tid + m * kTc2Threads) * 16;
+                load8(reinterpret_cast<const __nv_bfloat16 *>(sm + L::SB + off), fs);
+                load8(reinterpret_cast<const __nv_bfloat16 *>(sm + L::DB + off), fd);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) ds = fmaf(fs[i], fd[i], ds);
+            }
+            ds = warp_sum32(ds);
+            if (lane == 0) red[L::RDS + warp] = ds;
+        }
         // ---- masks: A (fp32, rows 0-63) and P (bf16, rows 64-127); R^T from X^T
         {
             float v[16];
@@ -866,18 +849,19 @@ gdr_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     }
 }
 
-// Workspace of the tensor-core backward: S_n, then D_n, both [B, H, nchunks, 128, 128] fp32.
+// Workspace of the tensor-core backward: the tiles of S_n, then those of D_n,
+// [B, H, nchunks] x 32 KB each.
 inline size_t bwd_tc_state_bytes(int B, int T, int H) {
     const size_t nch = (size_t)(T + kChunk - 1) / kChunk;
-    return ((size_t)B * H * nch * 128 * 128 * 4 + 255) / 256 * 256;
+    return ((size_t)B * H * nch * 32768 + 255) / 256 * 256;
 }
 
 inline cudaError_t launch_bwd_tc(int B, int T, int H, const void *q, const void *k, const void *v,
                                  const float *la, const float *beta, const float *S0, const void *dO,
                                  const float *dS_T, void *dq, void *dk_out, void *dv_out, float *dla,
                                  float *dbeta, float *dS0, void *ws, cudaStream_t stream) {
-    float *states = static_cast<float *>(ws);
-    float *dchunks = reinterpret_cast<float *>(static_cast<char *>(ws) + bwd_tc_state_bytes(B, T, H));
+    uint8_t *states = static_cast<uint8_t *>(ws);
+    uint8_t *dchunks = states + bwd_tc_state_bytes(B, T, H);
     // 1) forward recompute, keeping every chunk's entry state
     cudaError_t err = launch_fwd_tc2(B, T, H, q, k, v, la, beta, S0, nullptr, nullptr, stream, states);
     if (err != cudaSuccess) return err;

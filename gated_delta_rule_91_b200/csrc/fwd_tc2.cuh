@@ -503,7 +503,7 @@ __device__ __forceinline__ void tc2_prep(uint8_t *sm, const CUtensorMap *tm_q, c
 // ----------------------------------------------------------------- state CTA --
 __device__ __forceinline__ void tc2_state(uint8_t *sm, const CUtensorMap *tm_k, const CUtensorMap *tm_v,
                                           const CUtensorMap *tm_o, int T, int H, int b, int h,
-                                          const float *S0, float *S_T, bool store_o, float *S_chunks) {
+                                          const float *S0, float *S_T, bool store_o, uint8_t *S_tiles) {
     using L = Tc2Layout;
     using namespace sm100;
     constexpr int D = 128;
@@ -663,13 +663,6 @@ __device__ __forceinline__ void tc2_state(uint8_t *sm, const CUtensorMap *tm_k, 
             {
                 const int col = wc * 32;
                 tmem_ld32(tl + kT2S + col, v);
-                if (S_chunks) {  // entry state of chunk n, for the backward's recompute
-                    float4 *dst = reinterpret_cast<float4 *>(
-                        S_chunks + (((size_t)bh * nch + n) * D + row) * D + col);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-                }
                 uint8_t *half = sm + L::S_SB + (wc >> 1) * 16384;
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4) st_bf16x8(half + sw128_offset(row, (wc & 1) * 4 + q4), v + 8 * q4);
@@ -687,6 +680,10 @@ __device__ __forceinline__ void tc2_state(uint8_t *sm, const CUtensorMap *tm_k, 
         // (b) U^T -= S W^T ; O^T = S Q~^T
         if (tid == 0) {
             tc_after_sync();
+            if (S_tiles) {  // the bf16 entry state of chunk n, as swizzled, for the backward
+                bulk_store_s2g(S_tiles + ((size_t)bh * nch + n) * 32768, sm + L::S_SB, 32768);
+                bulk_commit();
+            }
             const uint32_t sb = sbase + L::S_SB, w = sbase + L::S_W;
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
@@ -712,6 +709,7 @@ __device__ __forceinline__ void tc2_state(uint8_t *sm, const CUtensorMap *tm_k, 
         __syncwarp();
         // (d) U^T, U~^T = U^T diag(exp(g_C - g)) -> bf16 A operands
         if (tid == 0 && !mbar_wait(bar_a, aphase)) *abort_flag = 1;
+        if (tid == 0 && S_tiles) bulk_wait_read_all();  // the state copy has left S_SB
         aphase ^= 1;
         tc_before_sync();
         __syncthreads();
@@ -828,7 +826,7 @@ gdr_fwd_tc2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                    int T, int H, const float *__restrict__ log_alpha, const float *__restrict__ beta,
                    const float *__restrict__ S0, float *__restrict__ S_T, int store_o,
-                   float *__restrict__ S_chunks) {
+                   uint8_t *__restrict__ S_tiles) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
@@ -836,15 +834,16 @@ gdr_fwd_tc2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     if (sm100::cluster_ctarank() == 0)
         tc2_prep(sm, &tm_q, &tm_k, T, H, b, h, log_alpha, beta);
     else
-        tc2_state(sm, &tm_k, &tm_v, &tm_o, T, H, b, h, S0, S_T, store_o != 0, S_chunks);
+        tc2_state(sm, &tm_k, &tm_v, &tm_o, T, H, b, h, S0, S_T, store_o != 0, S_tiles);
 }
 
 // o == nullptr runs the recurrence without writing outputs (the backward's
-// recompute); S_chunks (nullable) receives every chunk's entry state,
-// [B, H, nchunks, 128, 128] fp32.
+// recompute); S_tiles (nullable) receives every chunk's entry state as the
+// bf16 MMA operand tile, [B, H, nchunks] x 32 KB: two 64-column halves of
+// [128 rows][64 columns], 128-byte rows, 128B-swizzled.
 inline cudaError_t launch_fwd_tc2(int B, int T, int H, const void *q, const void *k, const void *v,
                                   const float *la, const float *beta, const float *S0, void *o,
-                                  float *S_T, cudaStream_t stream, float *S_chunks = nullptr) {
+                                  float *S_T, cudaStream_t stream, uint8_t *S_tiles = nullptr) {
     CUtensorMap mq, mk, mv, mo;
     if (!make_token_map(&mq, q, B, T, H, 128) || !make_token_map(&mk, k, B, T, H, 128) ||
         !make_token_map(&mv, v, B, T, H, 128) || !make_token_map(&mo, o ? o : q, B, T, H, 128))
@@ -853,7 +852,7 @@ inline cudaError_t launch_fwd_tc2(int B, int T, int H, const void *q, const void
                                            (int)Tc2Layout::kAlloc);
     if (err != cudaSuccess) return err;
     gdr_fwd_tc2_kernel<<<(unsigned)(2 * B * H), kTc2Threads, Tc2Layout::kAlloc, stream>>>(
-        mq, mk, mv, mo, T, H, la, beta, S0, S_T, o != nullptr ? 1 : 0, S_chunks);
+        mq, mk, mv, mo, T, H, la, beta, S0, S_T, o != nullptr ? 1 : 0, S_tiles);
     g_launches.fetch_add(1, std::memory_order_relaxed);
     return cudaGetLastError();
 }

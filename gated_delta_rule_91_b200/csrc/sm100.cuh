@@ -143,6 +143,22 @@ __device__ __forceinline__ void tma_store_4d(const CUtensorMap *map, const void 
         "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z), "r"(w)
         : "memory");
 }
+// Plain bulk copies between global and shared memory (16-byte aligned
+// addresses, size a multiple of 16).  Shared -> global is tracked by bulk
+// async-groups; global -> shared completes `bytes` on the mbarrier.
+__device__ __forceinline__ void bulk_store_s2g(void *dst, const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(
+                     reinterpret_cast<uint64_t>(dst)),
+                 "r"(smem_u32(src)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_load_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Wait until every committed bulk group has finished reading shared memory.
 __device__ __forceinline__ void bulk_wait_read_all() {
