@@ -655,10 +655,7 @@ inline size_t bwd_workspace_bytes(int B, int T, int H, int dk, int dv) {
     const size_t ns = (size_t)dv / kBwdDvs;
     const size_t bth = (size_t)B * T * H;
     auto al = [](size_t x) { return (x + 255) / 256 * 256; };
-    const size_t states = al((size_t)B * H * nch * dv * dk * 4);
-    const size_t simt = states + 2 * al(ns * bth * dk * 4) + 2 * al(ns * bth * 4);
-    // the tensor-core backward keeps S_n and D_n, two arrays of `states` bytes
-    return simt > 2 * states ? simt : 2 * states;
+    return al((size_t)B * H * nch * dv * dk * 4) + 2 * al(ns * bth * dk * 4) + 2 * al(ns * bth * 4);
 }
 
 inline BwdWorkspace bwd_carve(void *ws, int B, int T, int H, int dk, int dv) {

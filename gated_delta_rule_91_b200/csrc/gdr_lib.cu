@@ -75,16 +75,24 @@ gdr_status check_dims(const char *fn, int B, int T, int H, int dk, int dv, gdr_d
 }
 
 
+// bf16 with dk = dv = 128 runs the backward on the tensor cores (recompute,
+// dS pass, chunk-parallel gradients); GDR_BWD_KERNEL=simt selects the
+// CUDA-core backward (used to cross-check them).  The workspace size follows
+// the same choice.
+bool bwd_uses_tc(int dk, int dv, gdr_dtype dt) {
+    const char *sel = getenv("GDR_BWD_KERNEL");
+    return dt == GDR_BF16 && dk == 128 && dv == 128 && !(sel != nullptr && strcmp(sel, "simt") == 0);
+}
+size_t bwd_scratch_bytes(int B, int T, int H, int dk, int dv, gdr_dtype dt) {
+    return bwd_uses_tc(dk, dv, dt) ? 2 * bwd_tc_state_bytes(B, T, H) : bwd_workspace_bytes(B, T, H, dk, dv);
+}
+
 // The backward's kernels for one call (shared by gdr_bwd and gdr_bwd_noalloc).
-// bf16 with dk = dv = 128 runs on the tensor cores (recompute, dS pass,
-// chunk-parallel gradients); GDR_BWD_KERNEL=simt selects the CUDA-core
-// backward (used to cross-check them).
 cudaError_t run_bwd(int B, int T, int H, int dk, int dv, gdr_dtype dt, const void *q, const void *k,
                     const void *v, const float *log_alpha, const float *beta, const float *S0, const void *dO,
                     const float *dS_T, void *dq, void *dk_out, void *dv_out, float *dlog_alpha, float *dbeta,
                     float *dS0, void *workspace, cudaStream_t s) {
-    const char *sel = getenv("GDR_BWD_KERNEL");
-    if (dt == GDR_BF16 && dk == 128 && dv == 128 && !(sel != nullptr && strcmp(sel, "simt") == 0))
+    if (bwd_uses_tc(dk, dv, dt))
         return launch_bwd_tc(B, T, H, q, k, v, log_alpha, beta, S0, dO, dS_T, dq, dk_out, dv_out, dlog_alpha,
                              dbeta, dS0, workspace, s);
 #define GDR_BWD_ARGS B, T, H, dv, q, k, v, log_alpha, beta, S0, dO, dS_T, dq, dk_out, dv_out, \
@@ -213,9 +221,9 @@ gdr_status gdr_step(int B, int H, int dk, int dv, gdr_dtype dt, const void *q, c
     return GDR_OK;
 }
 
-size_t gdr_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, gdr_dtype) {
+size_t gdr_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, gdr_dtype dt) {
     if (B < 1 || T < 1 || H < 1 || (dk != 64 && dk != 128) || (dv != 64 && dv != 128)) return 0;
-    return bwd_workspace_bytes(B, T, H, dk, dv);
+    return bwd_scratch_bytes(B, T, H, dk, dv, dt);
 }
 
 gdr_status gdr_bwd(int B, int T, int H, int dk, int dv, gdr_dtype dt, const void *q, const void *k,
@@ -325,7 +333,7 @@ extern "C" gdr_status gdr_bwd_noalloc(int B, int T, int H, int dk, int dv, gdr_d
     GDR_OPTIONAL_PTR(S0);
     GDR_OPTIONAL_PTR(dS_T);
     GDR_OPTIONAL_PTR(dS0);
-    const size_t need = bwd_workspace_bytes(B, T, H, dk, dv);
+    const size_t need = bwd_scratch_bytes(B, T, H, dk, dv, dt);
     if (need > kBwdStaticScratchBytes)
         return fail(GDR_ERR_WORKSPACE,
                     "%s: this problem needs %zu bytes of scratch; the static scratch holds %zu "
