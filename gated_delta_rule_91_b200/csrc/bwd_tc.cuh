@@ -4,11 +4,12 @@
 // The pages give no backward; the reverse mode here is the chain rule applied
 // to the chunk map of the forward (chunkwise form of the Gated DeltaNet
 // review, meaningful96.github.io/nr/GDN, section 3.7; the per-chunk formulas
-// are listed at the top of bwd_simt.cuh).  Three launches:
+// are listed at the top of bwd_simt.cuh).  Three steps in two launches (1
+// and 2 share one launch, gdr_bwd_passes_kernel, as they are independent):
 //
 //  1. the forward, recomputed without outputs, keeps every chunk's entry
 //     state S_n as its bf16 MMA operand tile (32 KB, 128B-swizzled);
-//  2. the dS pass (gdr_bwd_chain_kernel), one 2-CTA cluster per (b, h), walks
+//  2. the dS pass, one 2-CTA cluster per (b, h), walks
 //     the chunks from last to first.  Its prep CTA is the forward's (masks,
 //     inverse, P, Q~ = diag(gamma) Q, T'' = T diag(beta gamma)); its state CTA
 //     carries D = dL/dS (exit state of the current chunk) in TMEM:
@@ -278,19 +279,27 @@ __device__ __forceinline__ void bwd_chain_state(uint8_t *sm, const CUtensorMap *
     }
 }
 
+// The recompute and the dS pass need nothing from each other, so one launch
+// runs both: clusters [0, B*H) recompute the forward (no outputs, bf16 state
+// tiles kept), clusters [B*H, 2*B*H) run the dS pass.
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTc2Threads, 1)
-gdr_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                     const __grid_constant__ CUtensorMap tm_do, int T, int H,
-                     const float *__restrict__ log_alpha, const float *__restrict__ beta,
-                     const float *__restrict__ dS_T, float *__restrict__ dS0, uint8_t *__restrict__ D_tiles) {
+gdr_bwd_passes_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                      int T, int H, const float *__restrict__ log_alpha, const float *__restrict__ beta,
+                      const float *__restrict__ S0, const float *__restrict__ dS_T, float *__restrict__ dS0,
+                      uint8_t *__restrict__ S_tiles, uint8_t *__restrict__ D_tiles) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
-    const int bh = blockIdx.x >> 1, b = bh / H, h = bh % H;
+    const int nbh = (int)(gridDim.x >> 2), cl = (int)(blockIdx.x >> 1);
+    const bool dS_pass = cl >= nbh;
+    const int bh = dS_pass ? cl - nbh : cl, b = bh / H, h = bh % H;
     if (sm100::cluster_ctarank() == 0)
-        tc2_prep(sm, &tm_q, &tm_k, T, H, b, h, log_alpha, beta, true);
-    else
+        tc2_prep(sm, &tm_q, &tm_k, T, H, b, h, log_alpha, beta, dS_pass);
+    else if (dS_pass)
         bwd_chain_state(sm, &tm_k, &tm_do, T, H, b, h, dS_T, dS0, D_tiles);
+    else  // no output: the q map stands in for the unused output map
+        tc2_state(sm, &tm_k, &tm_v, &tm_q, T, H, b, h, S0, nullptr, false, S_tiles);
 }
 
 // ------------------------------------------------------------ gradient kernel --
@@ -862,19 +871,16 @@ inline cudaError_t launch_bwd_tc(int B, int T, int H, const void *q, const void 
                                  float *dbeta, float *dS0, void *ws, cudaStream_t stream) {
     uint8_t *states = static_cast<uint8_t *>(ws);
     uint8_t *dchunks = states + bwd_tc_state_bytes(B, T, H);
-    // 1) forward recompute, keeping every chunk's entry state
-    cudaError_t err = launch_fwd_tc2(B, T, H, q, k, v, la, beta, S0, nullptr, nullptr, stream, states);
-    if (err != cudaSuccess) return err;
     CUtensorMap mq, mk, mv, mdo;
     if (!make_token_map(&mq, q, B, T, H, 128) || !make_token_map(&mk, k, B, T, H, 128) ||
         !make_token_map(&mv, v, B, T, H, 128) || !make_token_map(&mdo, dO, B, T, H, 128))
         return cudaErrorInvalidValue;
-    // 2) dS pass, chunks from last to first
-    err = cudaFuncSetAttribute(gdr_bwd_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)Tc2Layout::kAlloc);
+    // 1+2) forward recompute (every chunk's entry state) and dS pass, one launch
+    cudaError_t err = cudaFuncSetAttribute(gdr_bwd_passes_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)Tc2Layout::kAlloc);
     if (err != cudaSuccess) return err;
-    gdr_bwd_chain_kernel<<<(unsigned)(2 * B * H), kTc2Threads, Tc2Layout::kAlloc, stream>>>(
-        mq, mk, mdo, T, H, la, beta, dS_T, dS0, dchunks);
+    gdr_bwd_passes_kernel<<<(unsigned)(4 * B * H), kTc2Threads, Tc2Layout::kAlloc, stream>>>(
+        mq, mk, mv, mdo, T, H, la, beta, S0, dS_T, dS0, states, dchunks);
     g_launches.fetch_add(1, std::memory_order_relaxed);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
