@@ -389,15 +389,6 @@ __device__ __forceinline__ float warp_sum32(float x) {
     return x;
 }
 
-// Element (row, col) of a 128B-swizzled bf16 tile with 128-byte rows.
-__device__ __forceinline__ float ld_sw_bf16(const uint8_t *tile, int row, int col) {
-    return __bfloat162float(
-        *reinterpret_cast<const __nv_bfloat16 *>(tile + sm100::sw128_offset(row, col >> 3) + (col & 7) * 2));
-}
-__device__ __forceinline__ void st_sw_bf16(uint8_t *tile, int row, int col, float x) {
-    *reinterpret_cast<__nv_bfloat16 *>(tile + sm100::sw128_offset(row, col >> 3) + (col & 7) * 2) = __float2bfloat16_rn(x);
-}
-
 __global__ void __launch_bounds__(kTc2Threads, 1)
 gdr_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -571,7 +562,7 @@ gdr_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             for (int ch = 0; ch < 2; ++ch) st_bf16x8(sm + L::RU + sw128_offset(cc, wc * 2 + ch), x + 8 * ch);
         }
         __syncthreads();
-        if (warp < 2) inverse_two_warps(sA, sT, warp, lane, 1);
+        if (warp < 2) inverse_two_warps(sA, sT, warp, lane, 1, TEmit{nullptr, nullptr, nullptr, nullptr});
         __syncthreads();
         {   // T fp32 -> bf16 [r][i] (lower triangle; the fp32 scratch overlaps TB)
             const int r = tid & 63, cb = (tid >> 6) * 8;

@@ -76,6 +76,7 @@ static_assert(Tc2Layout::S_H % 1024 == 0 && Tc2Layout::S_W % 1024 == 0 && Tc2Lay
               "state tiles must be 1024-aligned");
 static_assert(Tc2Layout::P_STG % 1024 == 0 && Tc2Layout::H_SLOT % 1024 == 0, "slots must be 1024-aligned");
 static_assert(Tc2Layout::kAlloc <= 232448, "shared memory budget");
+static_assert(Tc2Layout::H_T2 == Tc2Layout::H_T1 + 8192, "T' and T'' are adjacent");
 
 // state TMEM columns (512 allocated)
 constexpr uint32_t kT2S = 0, kT2W = 128, kT2U = 192, kT2O = 320;  // U, O double-buffered (+64)
@@ -91,7 +92,15 @@ constexpr uint32_t kT2S = 0, kT2W = 128, kT2U = 192, kT2O = 320;  // U, O double
 // Products run on warp-level tensor-core tiles (m16n8k8, tf32 operands,
 // fp32 accumulation); the known zero blocks of T11 and T22 are skipped.  Intermediate products are parked in A's unused upper
 // triangle; only the lower triangle of T is written.
-__device__ __forceinline__ void inverse_diag16(const float *sA, float *sT, int blk, int j) {
+// Optional bf16 copies of T with scaled columns, written as the blocks of T are
+// produced: t1 = T diag(beta), t2 = T diag(beta gamma), 128B-swizzled [r][i]
+// tiles; only the lower triangle (diagonal blocks whole) is written.
+struct TEmit {
+    uint8_t *t1, *t2;           // nullptr: no copies
+    const float *beta, *gamma;  // [64]
+};
+
+__device__ __forceinline__ void inverse_diag16(const float *sA, float *sT, int blk, int j, const TEmit &em) {
     constexpr int LD = kLdT;
     const int base = blk * 16;
     float t[16];
@@ -108,6 +117,15 @@ __device__ __forceinline__ void inverse_diag16(const float *sA, float *sT, int b
     }
 #pragma unroll
     for (int r = 0; r < 16; ++r) sT[(base + r) * LD + base + j] = t[r];
+    if (em.t1) {
+        const int c = base + j;
+        const float b1 = em.beta[c], b2 = b1 * em.gamma[c];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+            sm100::st_sw_bf16(em.t1, base + r, c, t[r] * b1);
+            sm100::st_sw_bf16(em.t2, base + r, c, t[r] * b2);
+        }
+    }
 }
 
 __device__ __forceinline__ uint32_t to_tf32(float x) {
@@ -179,11 +197,24 @@ __device__ __forceinline__ void warp_store16x8(float *Db, const float (&acc)[4],
     *reinterpret_cast<float2 *>(Db + (g + 8) * LD + 2 * t) = make_float2(scale * acc[2], scale * acc[3]);
 }
 
+// The bf16 copies of one 16 x 8 fragment of T (scaled by `scale`) at (row0, col0).
+__device__ __forceinline__ void emit16x8(const TEmit &em, int row0, int col0, const float (&acc)[4], float scale,
+                                         int lane) {
+    const int g = lane >> 2, c = col0 + 2 * (lane & 3);
+    const float ba = scale * em.beta[c], bb = scale * em.beta[c + 1];
+    const float ga = ba * em.gamma[c], gb = bb * em.gamma[c + 1];
+    sm100::st_sw_bf16x2(em.t1, row0 + g, c, acc[0] * ba, acc[1] * bb);
+    sm100::st_sw_bf16x2(em.t1, row0 + g + 8, c, acc[2] * ba, acc[3] * bb);
+    sm100::st_sw_bf16x2(em.t2, row0 + g, c, acc[0] * ga, acc[1] * gb);
+    sm100::st_sw_bf16x2(em.t2, row0 + g + 8, c, acc[2] * ga, acc[3] * gb);
+}
+
 // The whole inverse, run by the two warps w = 0, 1 of the calling CTA;
 // `bar_id` names a 64-thread barrier between the 32 and 64 levels.
-__device__ __forceinline__ void inverse_two_warps(float *sA, float *sT, int w, int lane, int bar_id) {
+__device__ __forceinline__ void inverse_two_warps(float *sA, float *sT, int w, int lane, int bar_id,
+                                                  const TEmit &em) {
     constexpr int LD = kLdT;
-    inverse_diag16(sA, sT, 2 * w + (lane >> 4), lane & 15);
+    inverse_diag16(sA, sT, 2 * w + (lane >> 4), lane & 15, em);
     __syncwarp();
     {   // 32 level, block P = w
         const int o = 32 * w;
@@ -199,6 +230,10 @@ __device__ __forceinline__ void inverse_two_warps(float *sA, float *sT, int w, i
         warp_mm<1, 2, 2>(acc2, sT + (o + 16) * LD + o + 16, sA + o * LD + o + 16, k2, lane);
         warp_store16x8(sT + (o + 16) * LD + o, acc2[0][0], -1.f, lane);
         warp_store16x8(sT + (o + 16) * LD + o + 8, acc2[0][1], -1.f, lane);
+        if (em.t1) {
+            emit16x8(em, o + 16, o, acc2[0][0], -1.f, lane);
+            emit16x8(em, o + 16, o + 8, acc2[0][1], -1.f, lane);
+        }
     }
     asm volatile("barrier.sync %0, 64;" ::"r"(bar_id) : "memory");
     {   // 64 level: slabs c0 = 8w (T11 rows 0:32) and 16 + 8w (T11 rows 16:32 only)
@@ -223,6 +258,10 @@ __device__ __forceinline__ void inverse_two_warps(float *sA, float *sT, int w, i
         for (int m = 0; m < 2; ++m) {
             warp_store16x8(sT + (32 + 16 * m) * LD + c0, y0[m][0], -1.f, lane);
             warp_store16x8(sT + (32 + 16 * m) * LD + c1, y1[m][0], -1.f, lane);
+            if (em.t1) {
+                emit16x8(em, 32 + 16 * m, c0, y0[m][0], -1.f, lane);
+                emit16x8(em, 32 + 16 * m, c1, y1[m][0], -1.f, lane);
+            }
         }
     }
 }
@@ -274,6 +313,12 @@ __device__ __forceinline__ void tc2_prep(uint8_t *sm, const CUtensorMap *tm_q, c
         *abort_flag = 0;
         prefetch_tmap(tm_q);
         prefetch_tmap(tm_k);
+    }
+    // T' and T'' of every staging slot: zero once; the inverse writes only the
+    // lower triangle, so the upper blocks stay zero
+    for (int k = tid; k < 3 * 1024; k += kTc2Threads) {
+        const int slot = k >> 10, off = (k & 1023) * 16;  // H_T1 and H_T2 are adjacent (16 KB)
+        *reinterpret_cast<uint4 *>(sm + L::P_STG + slot * L::H_SLOT + L::H_T1 + off) = make_uint4(0, 0, 0, 0);
     }
     if (warp == 0) tmem_alloc(tmem_slot, 64);
     tc_before_sync();
@@ -411,7 +456,8 @@ __device__ __forceinline__ void tc2_prep(uint8_t *sm, const CUtensorMap *tm_q, c
         __syncthreads();
 
         if (solver) {
-            inverse_two_warps(sA, sT, warp, lane, kPrepSolverBarrier);
+            inverse_two_warps(sA, sT, warp, lane, kPrepSolverBarrier,
+                              TEmit{stg + L::H_T1, stg + L::H_T2, sbeta, sgam});
         } else {
             if (issuer && n + 1 < nch) {  // next chunk's K K^T / Q K^T overlaps this chunk's inverse
                 tc_after_sync();
@@ -452,31 +498,9 @@ __device__ __forceinline__ void tc2_prep(uint8_t *sm, const CUtensorMap *tm_q, c
                 if (n + 2 < nch) load_gates(n + 2);
             }
         }
-        __syncthreads();
-        if (*abort_flag) break;
-        {   // T' = T diag(beta) (rows 0-63), T'' = T diag(beta gamma) (rows 64-127), 16 columns each
-            const int r = tid & 63;
-            const bool second = (tid & 64) != 0;
-            const int cb = (tid >> 7) * 16;
-            float t[16], bv[16], gm[16];
-#pragma unroll
-            for (int k4 = 0; k4 < 4; ++k4) {
-                const float4 x = *reinterpret_cast<const float4 *>(sT + r * kLdT + cb + 4 * k4);
-                const float4 y = *reinterpret_cast<const float4 *>(sbeta + cb + 4 * k4);
-                const float4 z = *reinterpret_cast<const float4 *>(sgam + cb + 4 * k4);
-                t[4 * k4] = x.x; t[4 * k4 + 1] = x.y; t[4 * k4 + 2] = x.z; t[4 * k4 + 3] = x.w;
-                bv[4 * k4] = y.x; bv[4 * k4 + 1] = y.y; bv[4 * k4 + 2] = y.z; bv[4 * k4 + 3] = y.w;
-                gm[4 * k4] = z.x; gm[4 * k4 + 1] = z.y; gm[4 * k4 + 2] = z.z; gm[4 * k4 + 3] = z.w;
-            }
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-                t[i] = (cb + i <= r) ? t[i] * bv[i] * (second ? gm[i] : 1.f) : 0.f;
-#pragma unroll
-            for (int ch = 0; ch < 2; ++ch)
-                st_bf16x8(stg + (second ? L::H_T2 : L::H_T1) + sw128_offset(r, (cb >> 3) + ch), t + 8 * ch);
-        }
         fence_async_smem();
         __syncthreads();
+        if (*abort_flag) break;
         if (issuer) {
             // the state CTA's slot s must have been consumed (chunk n-2)
             if (n >= 2 && !mbar_wait_cluster(&empty[s], (uint32_t)(((n >> 1) - 1) & 1))) *abort_flag = 1;

@@ -283,6 +283,20 @@ __device__ __forceinline__ uint32_t sw128_offset(int row, int chunk) {
     return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
 }
 
+// Element (row, col) of a 128B-swizzled bf16 tile with 128-byte rows.
+__device__ __forceinline__ float ld_sw_bf16(const uint8_t *tile, int row, int col) {
+    return __bfloat162float(
+        *reinterpret_cast<const __nv_bfloat16 *>(tile + sw128_offset(row, col >> 3) + (col & 7) * 2));
+}
+__device__ __forceinline__ void st_sw_bf16(uint8_t *tile, int row, int col, float x) {
+    *reinterpret_cast<__nv_bfloat16 *>(tile + sw128_offset(row, col >> 3) + (col & 7) * 2) = __float2bfloat16_rn(x);
+}
+// Elements (row, col) and (row, col + 1), col even.
+__device__ __forceinline__ void st_sw_bf16x2(uint8_t *tile, int row, int col, float x, float y) {
+    *reinterpret_cast<__nv_bfloat162 *>(tile + sw128_offset(row, col >> 3) + (col & 7) * 2) =
+        __floats2bfloat162_rn(x, y);
+}
+
 // Pack 8 floats as bf16 and store as one 16-byte chunk.
 __device__ __forceinline__ void st_bf16x8(uint8_t *dst, const float *v) {
     uint4 u;
