@@ -106,10 +106,14 @@ __device__ __forceinline__ uint32_t cluster_addr(const void *p, uint32_t rank) {
 __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
-// Arrive once on a barrier in another CTA of the cluster (release at cluster scope).
+// Arrive once on a barrier in another CTA of the cluster.  Used to hand a
+// buffer back to its producer: everything that read the buffer (this CTA's
+// MMAs, observed complete through an mbarrier, and its threads' loads, done
+// before a CTA barrier) is finished, and the producer refills it with an async
+// copy only after its cluster-scope acquire on this barrier, so the default
+// release semantics suffice; a cluster-scope release costs about 1K cycles.
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_bar_addr) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar_addr)
-                 : "memory");
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar_addr) : "memory");
 }
 // Bulk copy of `bytes` (multiple of 16) from this CTA's shared memory into
 // another CTA's shared memory; completes `bytes` of transaction count on the
