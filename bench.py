@@ -53,7 +53,25 @@ def parse_args():
     p.add_argument("--no-secondary", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--e2e-steps", type=int, default=5)
+    p.add_argument("--profile-bwd", metavar="B,T,H", default=None,
+                   help="only run gdr_bwd twice on seeded bf16 d=128 inputs of this shape "
+                        "(a short command for profilers) and exit")
     return p.parse_args()
+
+
+def profile_bwd(shape):
+    """Two backward calls on seeded layer-recipe inputs (bf16, d = 128,
+    S0 ~ N(0, 0.02), dO drawn with the inputs), then a status check."""
+    import gated_delta_rule_91_b200 as gdr
+    B, T, H = (int(x) for x in shape.split(","))
+    x = synth.gdr_inputs(B, T, H, 128, 128, "bf16", seed=1, s0_std=0.02, with_dO=True)
+    d = {n: (x[n].cuda() if x[n] is not None else None)
+         for n in ("q", "k", "v", "log_alpha", "beta", "S0", "dO")}
+    for _ in range(2):
+        gdr.gdr_bwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["S0"], d["dO"])
+    torch.cuda.synchronize()
+    gdr.check_status()
+    print(json.dumps({"profile_bwd": shape, "status": "ok"}))
 
 
 def peaks():
@@ -362,6 +380,9 @@ def secondary(pk):
 
 def main():
     args = parse_args()
+    if args.profile_bwd:
+        profile_bwd(args.profile_bwd)
+        return
     rank, world, local = dist_init(args)
     if args.impl == "reference":
         run_reference(args, rank, world)  # no process group: rank 0 alone works
