@@ -96,7 +96,7 @@ constexpr uint32_t kT2S = 0, kT2W = 128, kT2U = 192, kT2O = 320;  // U, O double
 // produced: t1 = T diag(beta), t2 = T diag(beta gamma), 128B-swizzled [r][i]
 // tiles; only the lower triangle (diagonal blocks whole) is written.
 struct TEmit {
-    uint8_t *t1, *t2;           // nullptr: no copies
+    uint8_t *t1, *t2;           // t1 nullptr: no copies; t2 nullptr: t1 only
     const float *beta, *gamma;  // [64]
 };
 
@@ -123,7 +123,7 @@ __device__ __forceinline__ void inverse_diag16(const float *sA, float *sT, int b
 #pragma unroll
         for (int r = 0; r < 16; ++r) {
             sm100::st_sw_bf16(em.t1, base + r, c, t[r] * b1);
-            sm100::st_sw_bf16(em.t2, base + r, c, t[r] * b2);
+            if (em.t2) sm100::st_sw_bf16(em.t2, base + r, c, t[r] * b2);
         }
     }
 }
@@ -205,8 +205,10 @@ __device__ __forceinline__ void emit16x8(const TEmit &em, int row0, int col0, co
     const float ga = ba * em.gamma[c], gb = bb * em.gamma[c + 1];
     sm100::st_sw_bf16x2(em.t1, row0 + g, c, acc[0] * ba, acc[1] * bb);
     sm100::st_sw_bf16x2(em.t1, row0 + g + 8, c, acc[2] * ba, acc[3] * bb);
-    sm100::st_sw_bf16x2(em.t2, row0 + g, c, acc[0] * ga, acc[1] * gb);
-    sm100::st_sw_bf16x2(em.t2, row0 + g + 8, c, acc[2] * ga, acc[3] * gb);
+    if (em.t2) {
+        sm100::st_sw_bf16x2(em.t2, row0 + g, c, acc[0] * ga, acc[1] * gb);
+        sm100::st_sw_bf16x2(em.t2, row0 + g + 8, c, acc[2] * ga, acc[3] * gb);
+    }
 }
 
 // The whole inverse, run by the two warps w = 0, 1 of the calling CTA;

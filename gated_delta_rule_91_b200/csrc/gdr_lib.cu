@@ -18,6 +18,7 @@
 #include "fwd_tc.cuh"
 #include "fwd_tc2.cuh"
 #include "bwd_tc.cuh"
+#include "fwd2_tc.cuh"
 
 namespace gdr {
 std::atomic<uint64_t> g_launches{0};
@@ -284,6 +285,14 @@ gdr_status gdr2_fwd(int B, int T, int H, int dk, int dv, gdr_dtype dt, const voi
     (void)workspace_bytes;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e;
+    // bf16 with dk = dv = 128 runs on the tensor cores; GDR2_FWD_KERNEL=simt
+    // selects the CUDA-core kernel (used to cross-check it).
+    const char *sel = getenv("GDR2_FWD_KERNEL");
+    if (dt == GDR_BF16 && dk == 128 && dv == 128 && !(sel != nullptr && strcmp(sel, "simt") == 0)) {
+        e = launch_fwd2_tc(B, T, H, q, k, v, log_alpha, b, w, S0, o, S_T, s);
+        if (e != cudaSuccess) return cuda_fail(e, fn);
+        return GDR_OK;
+    }
 #define GDR2_ARGS B, T, H, dv, q, k, v, log_alpha, b, w, S0, o, S_T, s
     if (dt == GDR_F32)
         e = dk == 128 ? launch_gdr2_simt<float, 128>(GDR2_ARGS) : launch_gdr2_simt<float, 64>(GDR2_ARGS);

@@ -62,3 +62,36 @@ def test_gdr2_collapses_to_gated_delta_rule_on_gpu():
     o2, S2 = gdr.gdr2_fwd(d["q"], d["k"], d["v"], la, bw, bw, d["S0"])
     assert max_rel(np64(o2), np64(o1)) <= 1e-4
     assert fro_rel(np64(S2), np64(S1)) <= 1e-4
+
+
+@pytest.mark.parametrize("T", [64, 129, 1000])
+def test_tensor_core_gdr2_matches_cuda_core_gdr2(T, monkeypatch):
+    """bf16 d=128 runs on tcgen05; the fp32 CUDA-core kernel
+    (GDR2_FWD_KERNEL=simt) on the same inputs must agree within the bf16
+    tolerance, and both with the oracle."""
+    x = synth.gdr2_inputs(2, T, 3, 128, 128, "bf16", seed=90 + T, s0_std=0.02)
+    o_tc, S_tc = _gpu(x)
+    gdr.check_status()
+    monkeypatch.setenv("GDR2_FWD_KERNEL", "simt")
+    o_si, S_si = _gpu(x)
+    assert max_rel(np64(o_tc), np64(o_si)) <= TOL_O["bf16"]
+    assert fro_rel(np64(S_tc), np64(S_si)) <= TOL_S
+    o_ref, S_ref = _oracle(x)
+    assert max_rel(np64(o_tc), o_ref) <= TOL_O["bf16"]
+    assert fro_rel(np64(S_tc), S_ref) <= TOL_S
+
+
+def test_gdr2_strong_decay_takes_the_exact_path():
+    """Channels that decay by e^-3 per token fall by e^-192 over a chunk, past
+    what K/E can hold in a bf16 operand; those chunks evaluate A and P term
+    by term.  Half the heads decay strongly in half the channels; all must
+    still match the oracle."""
+    x = synth.gdr2_inputs(1, 200, 4, 128, 128, "bf16", seed=77, s0_std=0.02)
+    la = x["log_alpha"].clone()
+    la[:, :, :2, :64] = -3.0
+    x["log_alpha"] = la
+    o, S = _gpu(x)
+    gdr.check_status()
+    o_ref, S_ref = _oracle(x)
+    assert max_rel(np64(o), o_ref) <= TOL_O["bf16"]
+    assert fro_rel(np64(S), S_ref) <= TOL_S
