@@ -63,66 +63,100 @@ static_assert(G2Layout::kAlloc <= 232448, "shared memory budget");
 // TMEM columns (512 allocated)
 constexpr uint32_t kG2S = 0, kG2AP = 128, kG2W = 192, kG2U = 256, kG2O = 320;
 
-// Step 1 for the chunk at t0 (nv valid tokens): thread (j = tid % 128, row
-// group rg = tid / 128) owns channel j of rows 16 rg .. 16 rg + 15.  Writes
-// the operand tiles, E_C and the chunk's exact-path flag (cleared by the
-// caller before the call).
+// Step 1 for the chunk at tok0 (nv valid tokens), in two passes.
+// Scan: thread (j = tid % 128, row group rg = tid / 128) takes channel j of
+// rows 16 rg .. 16 rg + 15 and writes G (fp32 [r][j], into the S operand's
+// space, which is free until step 3; the exact path reads it too), E_C and
+// the chunk's exact-path flag (cleared by the caller).
+// Tiles: thread items (row r, 8 channels) build 16 bytes of every operand
+// tile at once, at the swizzled position of the TMA tile they come from.
 __device__ __forceinline__ void g2_tiles(uint8_t *sm, const float *log_alpha, const float *bgate,
                                          const float *wgate, size_t tok0, int H, int nv) {
     using L = G2Layout;
     using namespace sm100;
-    const int tid = threadIdx.x, j = tid & 127, rg = tid >> 7;
+    const int tid = threadIdx.x;
     float *ec = reinterpret_cast<float *>(sm + L::MISC), *scan = ec + 128;
     volatile int *flag = reinterpret_cast<volatile int *>(ec + 128 + 512 + 64);
-    float la[16], g[16];
+    float *sg = reinterpret_cast<float *>(sm + L::SB);
+    // the b and w gates of this thread's two tile items are loaded first, so
+    // their latency overlaps the scan's
+    float4 bq[2][2], wq[2][2];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        const int r = rg * 16 + i;
-        la[i] = r < nv ? log_alpha[(tok0 + (size_t)r * H) * 128 + j] : 0.f;
+    for (int m = 0; m < 2; ++m) {
+        const int item = tid + m * kG2Threads, r = item >> 4, c8 = (item & 15) * 8;
+        const size_t e = (tok0 + (size_t)r * H) * 128 + c8;
+        const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+        bq[m][0] = r < nv ? *reinterpret_cast<const float4 *>(bgate + e) : z;
+        bq[m][1] = r < nv ? *reinterpret_cast<const float4 *>(bgate + e + 4) : z;
+        wq[m][0] = r < nv ? *reinterpret_cast<const float4 *>(wgate + e) : z;
+        wq[m][1] = r < nv ? *reinterpret_cast<const float4 *>(wgate + e + 4) : z;
     }
-    float run = 0.f;
+    {
+        const int j = tid & 127, rg = tid >> 7;
+        float g[16];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        run += la[i];
-        g[i] = run;
+        for (int i = 0; i < 16; ++i) {
+            const int r = rg * 16 + i;
+            g[i] = r < nv ? log_alpha[(tok0 + (size_t)r * H) * 128 + j] : 0.f;
+        }
+#pragma unroll
+        for (int i = 1; i < 16; ++i) g[i] += g[i - 1];
+        scan[rg * 128 + j] = g[15];
+        __syncthreads();
+        float off = 0.f, tot = 0.f;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float x = scan[q * 128 + j];
+            off += q < rg ? x : 0.f;
+            tot += x;
+        }
+        if (rg == 0) {
+            ec[j] = expf(tot);
+            if (-tot > 80.f) *flag = 1;
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) sg[(rg * 16 + i) * 128 + j] = g[i] + off;
     }
-    scan[rg * 128 + j] = run;
     __syncthreads();
-    float off = 0.f, tot = 0.f;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const float x = scan[q * 128 + j];
-        off += q < rg ? x : 0.f;
-        tot += x;
-    }
-    if (rg == 0) {
-        ec[j] = expf(tot);
-        if (-tot > 80.f) *flag = 1;
-    }
-    const int hj = (j >> 6), cj = j & 63;
-    const uint8_t *tk = sm + L::TK + hj * 8192, *tq = sm + L::TQ + hj * 8192, *tv = sm + L::TV + hj * 8192;
-    uint8_t *kbe = sm + L::KQE + hj * 16384, *qe = kbe + 8192;
-    uint8_t *kie = sm + L::KIE + hj * 8192, *ktl = sm + L::KTL + hj * 8192, *wv = sm + L::WV + hj * 8192;
+    for (int m = 0; m < 2; ++m) {
+        const int item = tid + m * kG2Threads, r = item >> 4, c8 = (item & 15) * 8;
+        const int hj = c8 >> 6;
+        const uint32_t off = sw128_offset(r, (c8 & 63) >> 3);
+        float G[8], Gc[8], kk[8], qq[8], vv[8];
+        const bool exact = *flag != 0;
+        const float bb[8] = {bq[m][0].x, bq[m][0].y, bq[m][0].z, bq[m][0].w,
+                             bq[m][1].x, bq[m][1].y, bq[m][1].z, bq[m][1].w};
+        const float ww[8] = {wq[m][0].x, wq[m][0].y, wq[m][0].z, wq[m][0].w,
+                             wq[m][1].x, wq[m][1].y, wq[m][1].z, wq[m][1].w};
+        load8(sg + r * 128 + c8, G);
+        load8(sg + 63 * 128 + c8, Gc);
+        load8(reinterpret_cast<const __nv_bfloat16 *>(sm + L::TK + hj * 8192 + off), kk);
+        load8(reinterpret_cast<const __nv_bfloat16 *>(sm + L::TQ + hj * 8192 + off), qq);
+        load8(reinterpret_cast<const __nv_bfloat16 *>(sm + L::TV + hj * 8192 + off), vv);
+        float kbe[8], qe[8], kie[8], ktl[8], wv[8];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        const int r = rg * 16 + i;
-        const float G = g[i] + off;
-        const float e = __expf(G), kv = ld_sw_bf16(tk, r, cj);
-        const float bb = r < nv ? bgate[(tok0 + (size_t)r * H) * 128 + j] : 0.f;
-        const float ww = r < nv ? wgate[(tok0 + (size_t)r * H) * 128 + j] : 0.f;
-        st_sw_bf16(kbe, r, cj, kv * bb * e);
-        st_sw_bf16(qe, r, cj, ld_sw_bf16(tq, r, cj) * e);
-        st_sw_bf16(kie, r, cj, -G <= 80.f ? __fdividef(kv, e) : 0.f);
-        st_sw_bf16(ktl, r, cj, kv * __expf(tot - G));
-        st_sw_bf16(wv, r, cj, ww * ld_sw_bf16(tv, r, cj));
-        g[i] = G;
-    }
-    // the exact path needs G of every (token, channel): park it in the S operand's space
-    __syncthreads();
-    if (*flag) {
-        float *sg = reinterpret_cast<float *>(sm + L::SB);
+        for (int i = 0; i < 8; ++i) {
+            const float e = __expf(G[i]);
+            kbe[i] = kk[i] * bb[i] * e;
+            qe[i] = qq[i] * e;
+            kie[i] = -G[i] <= 80.f ? __fdividef(kk[i], e) : 0.f;
+            wv[i] = ww[i] * vv[i];
+        }
+        if (!exact) {  // K exp(G_C - G) = (K/E) exp(G_C), with E_C = exp(G_C) <= 1
+            const float4 e0 = *reinterpret_cast<const float4 *>(ec + c8), e1 = *reinterpret_cast<const float4 *>(ec + c8 + 4);
+            const float ecv[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
 #pragma unroll
-        for (int i = 0; i < 16; ++i) sg[(rg * 16 + i) * 128 + j] = g[i];
+            for (int i = 0; i < 8; ++i) ktl[i] = kie[i] * ecv[i];
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) ktl[i] = kk[i] * __expf(Gc[i] - G[i]);
+        }
+        st_bf16x8(sm + L::KQE + hj * 16384 + off, kbe);
+        st_bf16x8(sm + L::KQE + hj * 16384 + 8192 + off, qe);
+        st_bf16x8(sm + L::KIE + hj * 8192 + off, kie);
+        st_bf16x8(sm + L::KTL + hj * 8192 + off, ktl);
+        st_bf16x8(sm + L::WV + hj * 8192 + off, wv);
     }
 }
 
@@ -235,6 +269,16 @@ gdr2_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 
         // 1. gates and operand tiles
         g2_tiles(sm, log_alpha, bgate, wgate, tok0, H, nv);
+        if (n + 1 < nch) {  // the next chunk's gate rows -> L2 (3 gates x 64 rows x 4 lines of 128 B)
+            const int nv1 = min(kChunk, T - t0 - kChunk);
+            for (int k = tid; k < 3 * 64 * 4; k += kG2Threads) {
+                const int gate = k >> 8, r = (k >> 2) & 63, line = k & 3;
+                if (r < nv1) {
+                    const float *base = gate == 0 ? log_alpha : gate == 1 ? bgate : wgate;
+                    prefetch_l2(base + (tok0 + (size_t)(kChunk + r) * H) * 128 + line * 32);
+                }
+            }
+        }
         operands_ready();
 
         // 2. [K*B*E; Q*E] (K/E)^T -> A (rows 0-63), P (rows 64-127)
