@@ -449,12 +449,33 @@ def main():
     h2d = sum(t.numel() * t.element_size() for t in h.values())
     d2h = oh.numel() * oh.element_size() + sh.numel() * sh.element_size()
 
+    # one batch element at a time on two streams, so element b+1's upload
+    # overlaps element b's forward and download (the copy engines run both
+    # directions at once); every call is the public gdr_fwd on a batch slice
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+
     def e2e_step():
-        for n in h:
-            d[n].copy_(h[n], non_blocking=True)
-        step()
-        oh.copy_(o, non_blocking=True)
-        sh.copy_(ST, non_blocking=True)
+        start = torch.cuda.Event()
+        start.record(stream)
+        done = []
+        for bi in range(B):
+            sb = streams[bi % 2]
+            sb.wait_event(start)
+            with torch.cuda.stream(sb):
+                for n in h:
+                    if h[n] is not None:
+                        d[n][bi].copy_(h[n][bi], non_blocking=True)
+                gdr.gdr_fwd(d["q"][bi:bi + 1], d["k"][bi:bi + 1], d["v"][bi:bi + 1],
+                            d["log_alpha"][bi:bi + 1], d["beta"][bi:bi + 1],
+                            d["S0"][bi:bi + 1] if d["S0"] is not None else None,
+                            o=o[bi:bi + 1], S_T=ST[bi:bi + 1])
+                oh[bi].copy_(o[bi], non_blocking=True)
+                sh[bi].copy_(ST[bi], non_blocking=True)
+                ev = torch.cuda.Event()
+                ev.record(sb)
+                done.append(ev)
+        for ev in done:
+            stream.wait_event(ev)
 
     e2e_step()
     torch.cuda.synchronize()
