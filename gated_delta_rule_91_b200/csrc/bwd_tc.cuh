@@ -201,8 +201,7 @@ __device__ __forceinline__ void bwd_chain_state(uint8_t *sm, const CUtensorMap *
         tc_after_sync();
         {
             float x1[16], x2[16];
-            tmem_ld16(tl + kBcX1 + wc * 16, x1);
-            tmem_ld16(tl + kBcX2 + wc * 16, x2);
+            tmem_ld16x2(tl + kBcX1 + wc * 16, x1, tl + kBcX2 + wc * 16, x2);
 #pragma unroll
             for (int k4 = 0; k4 < 4; ++k4) {
                 const float4 dv4 = *reinterpret_cast<const float4 *>(hgate + 64 + wc * 16 + 4 * k4);
@@ -394,8 +393,9 @@ gdr_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                     int T, int H, const float *__restrict__ log_alpha, const float *__restrict__ beta,
                     const uint8_t *__restrict__ S_tiles, const uint8_t *__restrict__ D_tiles,
-                    __nv_bfloat16 *__restrict__ dq, __nv_bfloat16 *__restrict__ dk,
-                    __nv_bfloat16 *__restrict__ dv, float *__restrict__ dlog_alpha, float *__restrict__ dbeta) {
+                    const __grid_constant__ CUtensorMap tm_dq, const __grid_constant__ CUtensorMap tm_dk,
+                    const __grid_constant__ CUtensorMap tm_dv, float *__restrict__ dlog_alpha,
+                    float *__restrict__ dbeta) {
     using L = BgLayout;
     using namespace sm100;
     constexpr int D = 128;
@@ -595,8 +595,7 @@ gdr_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 #pragma unroll
             for (int ch = 0; ch < 2; ++ch) st_bf16x8(sm + L::UB + sw128_offset(row, wc * 2 + ch), u + 8 * ch);
             float x1[16], x2[16];
-            tmem_ld16(tl + kBgX1 + wc * 16, x1);
-            tmem_ld16(tl + kBgX2 + wc * 16, x2);
+            tmem_ld16x2(tl + kBgX1 + wc * 16, x1, tl + kBgX2 + wc * 16, x2);
 #pragma unroll
             for (int i = 0; i < 16; ++i) x1[i] = fmaf(x1[i], sdec[wc * 16 + i], x2[i]);
 #pragma unroll
@@ -626,9 +625,8 @@ gdr_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             float rb[16], rg[16], rc = 0.f;
             {
                 float dr[16], x[16];
-                tmem_ld16(tl + kBgDR + wc * 16, dr);
-                tmem_ld16(tl + kBgX + wc * 16, x);
-                uint8_t *drh = sm + L::DOR + (cc >> 6) * 16384;
+                tmem_ld16x2(tl + kBgDR + wc * 16, dr, tl + kBgX + wc * 16, x);
+                uint8_t *drh = sm + L::DOR + (cc >> 6) * 16384, *dvh = sm + L::DB + (cc >> 6) * 8192;
                 const uint8_t *vh = sm + L::V + (cc >> 6) * 8192;
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
@@ -637,7 +635,7 @@ gdr_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     rb[i] = dr[i] * (ld_sw_bf16(vh, r, cc & 63) - gr * x[i]);
                     rg[i] = -br * gr * dr[i] * x[i];
                     st_sw_bf16(drh, r, cc & 63, dr[i]);
-                    if (r < nv) dv[tok(r) * D + cc] = __float2bfloat16_rn(br * dr[i]);
+                    st_sw_bf16(dvh, r, cc & 63, br * dr[i]);  // dv tile (D is dead by now)
                 }
             }
             {
@@ -675,6 +673,9 @@ gdr_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 
         // ---- G4: [dA'; dP] = [dR; dO] U^T, (dR S)^T = S^T dR^T
         if (tid == 0) {
+            tma_store_4d(&tm_dv, sm + L::DB, 0, h, t0, b);  // dv [token][channel], tokens past T clipped
+            tma_store_4d(&tm_dv, sm + L::DB + 8192, 64, h, t0, b);
+            bulk_commit();
             tc_after_sync();
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
@@ -691,8 +692,7 @@ gdr_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         if (!mma_wait_all()) break;
         {   // rows 0-63: dA, dKK (fp32 -> FA); rows 64-127: dP, dP*L (bf16 -> PB); row and column sums
             float pa[16], kv[16], cs[16];
-            tmem_ld16(tl + kBgPA + wc * 16, pa);
-            tmem_ld16(tl + kBgKQ + wc * 16, kv);
+            tmem_ld16x2(tl + kBgPA + wc * 16, pa, tl + kBgKQ + wc * 16, kv);
             const int i0 = wc * 16;
             float rs_b = 0.f, rs_g = 0.f;
             if (row < 64) {
@@ -773,23 +773,31 @@ gdr_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         {
             const int j = row;
             float a[16], e[16];
-            tmem_ld16(tl + kBgDQ1 + wc * 16, a);
-            tmem_ld16(tl + kBgDQ2 + wc * 16, e);
+            tmem_ld16x2(tl + kBgDQ1 + wc * 16, a, tl + kBgDQ2 + wc * 16, e);
+            uint8_t *tq = sm + L::SB + (j >> 6) * 8192, *tk = sm + L::SB + 16384 + (j >> 6) * 8192;  // S is dead
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
                 const int r = wc * 16 + i;
-                if (r < nv) dq[tok(r) * D + j] = __float2bfloat16_rn(fmaf(sgam[r], a[i], e[i]));
+                st_sw_bf16(tq, r, j & 63, fmaf(sgam[r], a[i], e[i]));
             }
-            tmem_ld16(tl + kBgDK + wc * 16, a);
-            tmem_ld16(tl + kBgUD + wc * 16, e);
-            float f[16];
-            tmem_ld16(tl + kBgDRS + wc * 16, f);
+            tmem_ld16x2(tl + kBgDK + wc * 16, a, tl + kBgUD + wc * 16, e);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) a[i] = fmaf(sdec[wc * 16 + i], e[i], a[i]);
+            tmem_ld16(tl + kBgDRS + wc * 16, e);
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
                 const int r = wc * 16 + i;
-                const float x = fmaf(sdec[r], e[i], a[i]) - sbeta[r] * sgam[r] * f[i];
-                if (r < nv) dk[tok(r) * D + j] = __float2bfloat16_rn(x);
+                st_sw_bf16(tk, r, j & 63, a[i] - sbeta[r] * sgam[r] * e[i]);
             }
+        }
+        fence_async_smem();
+        __syncthreads();
+        if (tid == 0) {
+            tma_store_4d(&tm_dq, sm + L::SB, 0, h, t0, b);
+            tma_store_4d(&tm_dq, sm + L::SB + 8192, 64, h, t0, b);
+            tma_store_4d(&tm_dk, sm + L::SB + 16384, 0, h, t0, b);
+            tma_store_4d(&tm_dk, sm + L::SB + 16384 + 8192, 64, h, t0, b);
+            bulk_commit();
         }
         // ---- dbeta, dg -> dlog alpha (suffix sums inside the chunk)
         if (warp == 0) {
@@ -835,6 +843,7 @@ gdr_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
     } while (0);
 
+    if (tid == 0) bulk_wait_all();  // the gradient tiles have left shared memory
     if (*abort_flag && tid == 0) {
         record_status(GDR_ERR_TIMEOUT);
         if (tma_pending) mbar_wait(bar_tma, 0);
@@ -880,9 +889,12 @@ inline cudaError_t launch_bwd_tc(int B, int T, int H, const void *q, const void 
                                (int)BgLayout::kAlloc);
     if (err != cudaSuccess) return err;
     const int nch = (T + kChunk - 1) / kChunk;
+    CUtensorMap mdq, mdk, mdv;
+    if (!make_token_map(&mdq, dq, B, T, H, 128) || !make_token_map(&mdk, dk_out, B, T, H, 128) ||
+        !make_token_map(&mdv, dv_out, B, T, H, 128))
+        return cudaErrorInvalidValue;
     gdr_bwd_grad_kernel<<<(unsigned)(B * H * nch), kTc2Threads, BgLayout::kAlloc, stream>>>(
-        mq, mk, mv, mdo, T, H, la, beta, states, dchunks, static_cast<__nv_bfloat16 *>(dq),
-        static_cast<__nv_bfloat16 *>(dk_out), static_cast<__nv_bfloat16 *>(dv_out), dla, dbeta);
+        mq, mk, mv, mdo, T, H, la, beta, states, dchunks, mdq, mdk, mdv, dla, dbeta);
     g_launches.fetch_add(1, std::memory_order_relaxed);
     return cudaGetLastError();
 }
