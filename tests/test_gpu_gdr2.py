@@ -95,3 +95,38 @@ def test_gdr2_strong_decay_takes_the_exact_path():
     o_ref, S_ref = _oracle(x)
     assert max_rel(np64(o), o_ref) <= TOL_O["bf16"]
     assert fro_rel(np64(S), S_ref) <= TOL_S
+
+
+def test_gdr2_deterministic():
+    x = synth.gdr2_inputs(2, 300, 3, 128, 128, "bf16", seed=55, s0_std=0.02)
+    o1, S1 = _gpu(x)
+    o2, S2 = _gpu(x)
+    assert torch.equal(o1, o2) and torch.equal(S1, S2)
+
+
+def test_gdr2_split_sequence_resume():
+    """Running [0, t) then [t, T) from the first part's final state gives the
+    same outputs and state as one pass (the state is the whole carry)."""
+    x = synth.gdr2_inputs(1, 700, 2, 128, 128, "bf16", seed=56, s0_std=0.02)
+    o, S = _gpu(x)
+    t = 320  # a chunk boundary; the second part starts a fresh chunk grid
+    a = {n: (v[:, :t].contiguous() if v is not None and v.dim() == 4 and v.shape[1] == 700 else v)
+         for n, v in x.items()}
+    b = {n: (v[:, t:].contiguous() if v is not None and v.dim() == 4 and v.shape[1] == 700 else v)
+         for n, v in x.items()}
+    oa, Sa = _gpu(a)
+    b["S0"] = Sa.cpu()
+    ob, Sb = _gpu(b)
+    o2 = torch.cat([oa, ob], dim=1)
+    assert max_rel(np64(o2), np64(o)) <= TOL_O["bf16"]
+    assert fro_rel(np64(Sb), np64(S)) <= TOL_S
+
+
+def test_gdr2_null_state_and_no_final_state():
+    x = synth.gdr2_inputs(1, 150, 2, 128, 128, "bf16", seed=57)
+    assert x["S0"] is None
+    o, S = gdr.gdr2_fwd(dev(x["q"]), dev(x["k"]), dev(x["v"]), dev(x["log_alpha"]), dev(x["b"]),
+                        dev(x["w"]), None, return_state=False)
+    assert S is None
+    o_ref, _ = _oracle(x)
+    assert max_rel(np64(o), o_ref) <= TOL_O["bf16"]
