@@ -56,7 +56,23 @@ def parse_args():
     p.add_argument("--profile-bwd", metavar="B,T,H", default=None,
                    help="only run gdr_bwd twice on seeded bf16 d=128 inputs of this shape "
                         "(a short command for profilers) and exit")
+    p.add_argument("--profile-gdn2", metavar="B,T,H", default=None,
+                   help="only run gdr2_fwd twice on seeded bf16 d=128 inputs of this shape and exit")
     return p.parse_args()
+
+
+def profile_gdn2(shape):
+    """Two Gated DeltaNet-2 forward calls on the seeded GDN-2 recipe
+    (bf16, d = 128, S0 ~ N(0, 0.02)), then a status check."""
+    import gated_delta_rule_91_b200 as gdr
+    B, T, H = (int(x) for x in shape.split(","))
+    x = synth.gdr2_inputs(B, T, H, 128, 128, "bf16", seed=4, s0_std=0.02)
+    d = {n: (x[n].cuda() if x[n] is not None else None) for n in ("q", "k", "v", "log_alpha", "b", "w", "S0")}
+    for _ in range(2):
+        gdr.gdr2_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["b"], d["w"], d["S0"])
+    torch.cuda.synchronize()
+    gdr.check_status()
+    print(json.dumps({"profile_gdn2": shape, "status": "ok"}))
 
 
 def profile_bwd(shape):
@@ -382,6 +398,9 @@ def main():
     args = parse_args()
     if args.profile_bwd:
         profile_bwd(args.profile_bwd)
+        return
+    if args.profile_gdn2:
+        profile_gdn2(args.profile_gdn2)
         return
     rank, world, local = dist_init(args)
     if args.impl == "reference":
