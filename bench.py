@@ -389,6 +389,18 @@ def secondary(pk):
                            "mtok_per_s": w.B * w.T / (ms * 1e-3) / 1e6,
                            "tc_frac": fwd_flops(w.B, w.T, w.H, w.dk, w.dv) / (ms * 1e-3) / (pk["bf16_tflops"] * 1e12),
                            "hbm_frac": gdr2_bytes(w.B, w.T, w.H, w.dk, w.dv) / (ms * 1e-3) / 1e9 / pk["hbm_gbs"]}
+        # the same workload with the erase gate in (0, 2) (negative-eigenvalue range)
+        d["b"].mul_(2.0)
+        call()
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(5):
+            call()
+        e1.record()
+        torch.cuda.synchronize()
+        ms2 = e0.elapsed_time(e1) / 5
+        out["gdn2_fwd_b_0_2"] = {"workload": "B=4 T=4096 H=16 d=128 bf16, b in (0, 2)", "ms": ms2,
+                                 "mtok_per_s": w.B * w.T / (ms2 * 1e-3) / 1e6}
     except Exception as e:
         out["gdn2_fwd"] = {"unavailable": str(e).splitlines()[0][:200]}
     return out

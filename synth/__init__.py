@@ -86,9 +86,10 @@ def gdr_inputs(B: int, T: int, H: int, dk: int, dv: int, dtype: str = "bf16",
 
 
 def gdr2_inputs(B: int, T: int, H: int, dk: int, dv: int, dtype: str = "bf16",
-                seed: int = 0, s0_std: float = 0.0) -> dict:
+                seed: int = 0, s0_std: float = 0.0, b_max: float = 1.0) -> dict:
     """Inputs of Gated DeltaNet-2: q, k, v as above; log_alpha, b
-    [B,T,H,dk] fp32; w [B,T,H,dv] fp32; S0 or None."""
+    [B,T,H,dk] fp32; w [B,T,H,dv] fp32; S0 or None.  b = b_max * sigmoid(x):
+    b_max = 2 gives the negative-eigenvalue range b in (0, 2)."""
     g = torch.Generator().manual_seed(seed)
     dt = DTYPES[dtype]
     q = _l2n(torch.randn(B, T, H, dk, generator=g)).to(dt)
@@ -98,7 +99,7 @@ def gdr2_inputs(B: int, T: int, H: int, dk: int, dv: int, dtype: str = "bf16",
     S0 = None
     if s0_std > 0.0:
         S0 = torch.randn(B, H, dv, dk, generator=g) * s0_std
-    b = torch.sigmoid(torch.randn(B, T, H, dk, generator=g))
+    b = b_max * torch.sigmoid(torch.randn(B, T, H, dk, generator=g))
     w = torch.sigmoid(torch.randn(B, T, H, dv, generator=g))
     return dict(q=q, k=k, v=v, log_alpha=log_alpha, b=b, w=w, S0=S0)
 

@@ -130,3 +130,19 @@ def test_gdr2_null_state_and_no_final_state():
     assert S is None
     o_ref, _ = _oracle(x)
     assert max_rel(np64(o), o_ref) <= TOL_O["bf16"]
+
+
+@pytest.mark.parametrize("kernel", ["default", "simt"])
+def test_gdr2_negative_eigenvalue_erase_gate(kernel, monkeypatch):
+    """Erase gate b in (0, 2) (the negative-eigenvalue range): the erase
+    factor's eigenvalue along k reaches -1, and over 1000 tokens both
+    kernels must still match the oracle."""
+    if kernel != "default":
+        monkeypatch.setenv("GDR2_FWD_KERNEL", kernel)
+    x = synth.gdr2_inputs(2, 1000, 2, 128, 128, "bf16", seed=58, s0_std=0.02, b_max=2.0)
+    assert float(x["b"].max()) > 1.5
+    o, S = _gpu(x)
+    gdr.check_status()
+    o_ref, S_ref = _oracle(x)
+    assert max_rel(np64(o), o_ref) <= TOL_O["bf16"]
+    assert fro_rel(np64(S), S_ref) <= TOL_S

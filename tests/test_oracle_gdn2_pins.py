@@ -108,3 +108,32 @@ def test_transition_products(T):
     for t in range(T):
         S = S + np.outer(w[0, t, 0] * v[0, t, 0], k[0, t, 0]) @ prod(t + 1)
     np.testing.assert_allclose(ST[0, 0], S, rtol=1e-11, atol=1e-12)
+
+
+def test_erase_gate_two_is_a_householder_reflection():
+    """Negative-eigenvalue range (erase gate b in [0, 2], the Gated DeltaNet-2
+    page's remark on extending the erase gate): with unit keys, no decay and
+    b = 2 on every channel, the erase factor I - 2 k k^T is a reflection, so
+    each step gives S_t k_t = -S_{t-1} k_t + w_t*v_t exactly (fp64)."""
+    rng = np.random.default_rng(44)
+    B, T, H, dk, dv = 1, 12, 1, 6, 4
+    k = rng.normal(size=(B, T, H, dk))
+    k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    q = rng.normal(size=(B, T, H, dk))
+    v = rng.normal(size=(B, T, H, dv))
+    w = rng.uniform(0.1, 1.0, size=(B, T, H, dv))
+    b = np.full((B, T, H, dk), 2.0)
+    la = np.zeros((B, T, H, dk))
+    S = rng.normal(size=(B, H, dv, dk))
+    for t in range(T):
+        sl = lambda x: x[:, t:t + 1]
+        _, S_next = oracle.gdr2_fwd(sl(q), sl(k), sl(v), sl(la), sl(b), sl(w), S)
+        kt = k[0, t, 0]
+        lhs = S_next[0, 0] @ kt
+        rhs = -(S[0, 0] @ kt) + w[0, t, 0] * v[0, t, 0]
+        assert np.abs(lhs - rhs).max() < 1e-12
+        # the reflection preserves the part of the state orthogonal to k
+        u = rng.normal(size=dk)
+        u -= (u @ kt) * kt
+        assert np.abs(S_next[0, 0] @ u - S[0, 0] @ u).max() < 1e-12
+        S = S_next
