@@ -30,6 +30,7 @@ def _load():
         lib.oracle_gdr_step.argtypes = [i, i, i, i] + [dp] * 7
         lib.oracle_gdr_bwd.argtypes = [i, i, i, i, i] + [dp] * 14
         lib.oracle_gdr2_fwd.argtypes = [i, i, i, i, i] + [dp] * 9
+        lib.oracle_gdr2_bwd.argtypes = [i, i, i, i, i] + [dp] * 16
         lib.oracle_num_threads.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -106,3 +107,19 @@ def gdr2_fwd(q, k, v, log_alpha, b, w, S0=None):
     _load().oracle_gdr2_fwd(B, T, H, dk, dv, _p(q), _p(k), _p(v), _p(la), _p(bb),
                             _p(ww), _p(S0), _p(o), _p(ST))
     return o, ST
+
+
+def gdr2_bwd(q, k, v, log_alpha, b, w, S0, dO, dS_T=None):
+    """Hand-derived reverse mode of gdr2_fwd.  Returns a dict with dq, dk, dv,
+    dlog_alpha, db, dw, dS0 (float64)."""
+    q, k, v, la, bb, ww, S0, dO, dST = map(_in, (q, k, v, log_alpha, b, w, S0, dO, dS_T))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    out = dict(dq=np.zeros_like(q), dk=np.zeros_like(k), dv=np.zeros_like(v),
+               dlog_alpha=np.zeros_like(la), db=np.zeros_like(bb), dw=np.zeros_like(ww),
+               dS0=np.zeros((B, H, dv, dk)))
+    _load().oracle_gdr2_bwd(B, T, H, dk, dv, _p(q), _p(k), _p(v), _p(la), _p(bb), _p(ww),
+                            _p(S0), _p(dO), _p(dST), _p(out["dq"]), _p(out["dk"]),
+                            _p(out["dv"]), _p(out["dlog_alpha"]), _p(out["db"]), _p(out["dw"]),
+                            _p(out["dS0"]))
+    return out

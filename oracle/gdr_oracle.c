@@ -309,3 +309,130 @@ void oracle_gdr2_fwd(int B, int T, int H, int dk, int dv,
         free(S); free(bk); free(al);
     }
 }
+
+/* One Gated Delta Rule-2 step on S in place (the update of oracle_gdr2_fwd). */
+static void gdr2_token(int dk, int dv, double *S, const double *kt, const double *vt,
+                       const double *la, const double *bt, const double *wt) {
+    for (int i = 0; i < dv; ++i) {
+        double *row = S + (size_t)i * dk;
+        double rd = 0.0;
+        for (int j = 0; j < dk; ++j) { row[j] *= exp(la[j]); rd += row[j] * bt[j] * kt[j]; }
+        double res = rd - wt[i] * vt[i];
+        for (int j = 0; j < dk; ++j) row[j] -= res * kt[j];
+    }
+}
+
+/*
+ * Gated Delta Rule-2 backward: reverse mode of the step of oracle_gdr2_fwd
+ * (the pages give no backward).  With S = S_{t-1}, P = S Diag(alpha),
+ * e = w*v - P(b*k) (so S_t = P + e k^T), and G = dL/dS_t once the readout's
+ * do q^T is added:
+ *   dq    = S_t^T do                 gk = G k
+ *   dv    = w * gk                   dw = v * gk
+ *   dk    = G^T e - b * (P^T gk)     db = -k * (P^T gk)
+ *   dlog alpha_j = sum_i P_ij (G_ij - gk_i b_j k_j)
+ *   dL/dS_{t-1} = (G - gk (b*k)^T) Diag(alpha)
+ * The state entering each block of ORACLE_CK tokens is kept from a forward
+ * pass and the block's states are recomputed before walking it backwards.
+ * Gradient layouts match the inputs; dS_T and dS0 may be NULL.
+ */
+void oracle_gdr2_bwd(int B, int T, int H, int dk, int dv,
+                     const double *q, const double *k, const double *v,
+                     const double *log_alpha, const double *bgate, const double *wgate,
+                     const double *S0, const double *dO, const double *dS_T,
+                     double *dq, double *dk_out, double *dv_out,
+                     double *dlog_alpha, double *db_out, double *dw_out, double *dS0) {
+    long units = (long)B * H;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long bh = 0; bh < units; ++bh) {
+        int b = (int)(bh / H), h = (int)(bh % H);
+        size_t ssz = (size_t)dv * dk;
+        int nblk = (T + ORACLE_CK - 1) / ORACLE_CK;
+        double *ckpt = (double *)malloc((size_t)(nblk > 0 ? nblk : 1) * ssz * sizeof(double));
+        double *Sb = (double *)malloc((size_t)(ORACLE_CK + 1) * ssz * sizeof(double));
+        double *G = (double *)malloc(ssz * sizeof(double));
+        double *P = (double *)malloc(ssz * sizeof(double));
+        double *e = (double *)malloc((size_t)dv * sizeof(double));
+        double *gk = (double *)malloc((size_t)dv * sizeof(double));
+        double *bk = (double *)malloc((size_t)dk * sizeof(double));
+        double *al = (double *)malloc((size_t)dk * sizeof(double));
+
+        double *S = Sb;
+        if (S0) memcpy(S, S0 + (size_t)bh * ssz, ssz * sizeof(double));
+        else memset(S, 0, ssz * sizeof(double));
+        for (int t = 0; t < T; ++t) {
+            if (t % ORACLE_CK == 0)
+                memcpy(ckpt + (size_t)(t / ORACLE_CK) * ssz, S, ssz * sizeof(double));
+            size_t ti = tok_index(b, t, h, T, H);
+            gdr2_token(dk, dv, S, k + ti * dk, v + ti * dv, log_alpha + ti * dk, bgate + ti * dk,
+                       wgate + ti * dv);
+        }
+
+        if (dS_T) memcpy(G, dS_T + (size_t)bh * ssz, ssz * sizeof(double));
+        else memset(G, 0, ssz * sizeof(double));
+
+        for (int blk = nblk - 1; blk >= 0; --blk) {
+            int t0 = blk * ORACLE_CK;
+            int t1 = t0 + ORACLE_CK < T ? t0 + ORACLE_CK : T;
+            memcpy(Sb, ckpt + (size_t)blk * ssz, ssz * sizeof(double));
+            for (int t = t0; t < t1; ++t) {
+                size_t ti = tok_index(b, t, h, T, H);
+                double *nxt = Sb + (size_t)(t - t0 + 1) * ssz;
+                memcpy(nxt, Sb + (size_t)(t - t0) * ssz, ssz * sizeof(double));
+                gdr2_token(dk, dv, nxt, k + ti * dk, v + ti * dv, log_alpha + ti * dk, bgate + ti * dk,
+                           wgate + ti * dv);
+            }
+            for (int t = t1 - 1; t >= t0; --t) {
+                size_t ti = tok_index(b, t, h, T, H);
+                const double *Sp = Sb + (size_t)(t - t0) * ssz;      /* S_{t-1} */
+                const double *St = Sb + (size_t)(t - t0 + 1) * ssz;  /* S_t */
+                const double *qt = q + ti * dk, *kt = k + ti * dk, *vt = v + ti * dv;
+                const double *la = log_alpha + ti * dk, *bt = bgate + ti * dk, *wt = wgate + ti * dv;
+                const double *dot = dO + ti * dv;
+                for (int j = 0; j < dk; ++j) { al[j] = exp(la[j]); bk[j] = bt[j] * kt[j]; }
+                for (int i = 0; i < dv; ++i)
+                    for (int j = 0; j < dk; ++j) P[(size_t)i * dk + j] = Sp[(size_t)i * dk + j] * al[j];
+
+                /* readout: G += do q^T ; dq = S_t^T do */
+                for (int i = 0; i < dv; ++i)
+                    for (int j = 0; j < dk; ++j) G[(size_t)i * dk + j] += dot[i] * qt[j];
+                for (int j = 0; j < dk; ++j) {
+                    double acc = 0.0;
+                    for (int i = 0; i < dv; ++i) acc += St[(size_t)i * dk + j] * dot[i];
+                    dq[ti * dk + j] = acc;
+                }
+                /* e = w*v - P(b*k), gk = G k; dv, dw */
+                for (int i = 0; i < dv; ++i) {
+                    double rd = 0.0, g = 0.0;
+                    for (int j = 0; j < dk; ++j) {
+                        rd += P[(size_t)i * dk + j] * bk[j];
+                        g += G[(size_t)i * dk + j] * kt[j];
+                    }
+                    e[i] = wt[i] * vt[i] - rd;
+                    gk[i] = g;
+                    dv_out[ti * dv + i] = wt[i] * g;
+                    dw_out[ti * dv + i] = vt[i] * g;
+                }
+                /* dk, db, dlog alpha (column sums over the value channels) */
+                for (int j = 0; j < dk; ++j) {
+                    double ge = 0.0, pg = 0.0, da = 0.0;
+                    for (int i = 0; i < dv; ++i) {
+                        double pij = P[(size_t)i * dk + j], gij = G[(size_t)i * dk + j];
+                        ge += gij * e[i];
+                        pg += pij * gk[i];
+                        da += pij * (gij - gk[i] * bk[j]);
+                    }
+                    dk_out[ti * dk + j] = ge - bt[j] * pg;
+                    db_out[ti * dk + j] = -kt[j] * pg;
+                    dlog_alpha[ti * dk + j] = da;
+                }
+                /* dL/dS_{t-1} = (G - gk (b*k)^T) Diag(alpha) */
+                for (int i = 0; i < dv; ++i)
+                    for (int j = 0; j < dk; ++j)
+                        G[(size_t)i * dk + j] = (G[(size_t)i * dk + j] - gk[i] * bk[j]) * al[j];
+            }
+        }
+        if (dS0) memcpy(dS0 + (size_t)bh * ssz, G, ssz * sizeof(double));
+        free(ckpt); free(Sb); free(G); free(P); free(e); free(gk); free(bk); free(al);
+    }
+}
