@@ -36,6 +36,8 @@ SIGNATURES = {
     "gdr_bwd_noalloc": (_I, [_I] * 6 + [_P] * 14 + [_P]),
     "gdr2_fwd": (_I, [_I] * 6 + [_P] * 9 + [_P, _SZ, _P]),
     "gdr2_fwd_workspace_bytes": (_SZ, [_I] * 6),
+    "gdr2_bwd": (_I, [_I] * 6 + [_P] * 16 + [_P, _SZ, _P]),
+    "gdr2_bwd_workspace_bytes": (_SZ, [_I] * 6),
     "gdr_check_status": (_I, [_P]),
     "gdr_debug_wait_timeout": (_I, [_I, _P]),
     "gdr_last_error_string": (ctypes.c_char_p, []),
@@ -184,3 +186,20 @@ def gdr2_fwd(q, k, v, log_alpha, b, w, S0=None, *, o=None, S_T=None, return_stat
     check(L.gdr2_fwd(B, T, H, dk, dv, dt, _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b),
                      _ptr(w), _ptr(S0), _ptr(o), _ptr(S_T), _ptr(ws), ws_bytes, _stream(q)))
     return o, S_T
+
+
+def gdr2_bwd(q, k, v, log_alpha, b, w, S0, dO, dS_T=None, *, want_dS0=True, workspace=None):
+    """Backward of gdr2_fwd.  Returns dict(dq, dk, dv, dlog_alpha, db, dw, dS0)."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = _dt(q)
+    out = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dv=torch.empty_like(v),
+               dlog_alpha=torch.empty_like(log_alpha), db=torch.empty_like(b), dw=torch.empty_like(w),
+               dS0=torch.empty(B, H, dv, dk, dtype=torch.float32, device=q.device) if want_dS0 else None)
+    L = lib()
+    ws, ws_bytes = _workspace(L.gdr2_bwd_workspace_bytes(B, T, H, dk, dv, dt), q.device, workspace)
+    check(L.gdr2_bwd(B, T, H, dk, dv, dt, _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w),
+                     _ptr(S0), _ptr(dO), _ptr(dS_T), _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]),
+                     _ptr(out["dlog_alpha"]), _ptr(out["db"]), _ptr(out["dw"]), _ptr(out["dS0"]),
+                     _ptr(ws), ws_bytes, _stream(q)))
+    return out

@@ -1,0 +1,528 @@
+// bwd2_simt.cuh -- chunkwise backward of Gated DeltaNet-2 on CUDA cores (fp32
+// arithmetic; fp32 or bf16 q/k/v/dO).
+//
+// The pages give no backward; this is the chain rule applied to the chunk
+// map of the Gated Delta Rule-2 forward ("Gated DeltaNet-2: Decoupling Erase
+// and Write in Linear Attention", agihunt.info/papers/2605.22791, the Gated
+// Delta Rule-2 paragraph; the chunk form is restated in gdr2_simt.cuh).  Per
+// chunk, with G the per-channel cumulative log decay, E = exp(G),
+//     KBE = K*B*E, QE = Q*E, KiE = K/E, Kt = K*exp(G_C - G) = KiE Diag(E_C),
+//     A = strictLower(KBE KiE^T), P = inclLower(QE KiE^T), T = (I + A)^{-1},
+//     R = W*V - KBE S^T, U = T R, O = QE S^T + P U, S' = S Diag(E_C) + U^T Kt,
+// and D = dL/dS', dO:
+//     dU = Kt D^T + P^T dO          dR = T^T dU          dA = -dR U^T (i < r)
+//     dP = dO U^T (i <= r)          dV = W*dR            dW = V*dR
+//     dKBE = -dR S + dA KiE         dQE = dO S + dP KiE
+//     dKiE = dA^T KBE + dP^T QE + (U D) Diag(E_C)
+//     dS = D Diag(E_C) + dO^T QE - dR^T KBE            (D of the previous chunk)
+//     dE_C = colsum(S * D) + colsum((U D) * KiE)
+// then per element dK = dKBE B E + dKiE / E, dB = dKBE K E, dQ = dQE E,
+// dG = dKBE KBE + dQE QE - dKiE KiE, plus E_C dE_C on the chunk's last token,
+// and dlog alpha = the in-chunk suffix sums of dG per channel.
+//
+// One CTA owns one (b, h) and a slice of kBwd2Dvs state rows and walks the
+// chunks from last to first.  dV, dW and dS are slice-local; dKBE, dQE,
+// dKiE and dE_C are sums over slices, written per slice and summed in a
+// fixed order by gdr2_bwd_reduce_kernel, which also applies the per-element
+// chain rule (deterministic, no atomics).  A chunk in which some channel
+// decays by more than e^80 (K/E would overflow) is not handled: the kernel
+// reports GDR_ERR_UNSUPPORTED through the status word.
+#pragma once
+#include "common.cuh"
+#include "bwd_simt.cuh"
+#include "gdr2_simt.cuh"
+
+namespace gdr {
+
+constexpr int kBwd2Dvs = 32;  // state rows per CTA
+
+template <int DK>
+struct Bwd2Layout {
+    static constexpr int C = kChunk;
+    static constexpr int LDK = DK + 1;
+    static constexpr int LDV = kBwd2Dvs + 1;
+    static constexpr int LDC = C + 1;
+    static constexpr int oKB = 0;                    // K*B*E      [C][LDK]
+    static constexpr int oQE = oKB + C * LDK;        // Q*E        [C][LDK]
+    static constexpr int oKI = oQE + C * LDK;        // K/E        [C][LDK]
+    static constexpr int oG = oKI + C * LDK;         // log alpha [C][LDK]; later dP, dA [C][LDC] each
+    static constexpr int kGFloats = C * LDK > 2 * C * LDC ? C * LDK : 2 * C * LDC;
+    static constexpr int oS = oG + kGFloats;         // entry state slice [kBwd2Dvs][LDK]
+    static constexpr int oD = oS + kBwd2Dvs * LDK;   // dL/dS' slice      [kBwd2Dvs][LDK]
+    static constexpr int odO = oD + kBwd2Dvs * LDK;  // [C][LDV] each below
+    static constexpr int oU = odO + C * LDV;         // R, then U
+    static constexpr int odR = oU + C * LDV;         // dU, then dR
+    static constexpr int oA = odR + C * LDV;         // [C][LDC] each below
+    static constexpr int oP = oA + C * LDC;
+    static constexpr int oVec = oP + C * LDC;        // E_C [DK], ones [C], flag
+    static constexpr int kFloats = oVec + DK + C + 4;
+    static constexpr size_t kBytes = (size_t)kFloats * sizeof(float);
+    static_assert(kBytes <= 232448, "shared memory budget");
+};
+
+template <typename Tio, int DK>
+__global__ void __launch_bounds__(kSimtThreads, 1)
+gdr2_bwd_simt_kernel(int T, int H, int dv, const Tio *__restrict__ q, const Tio *__restrict__ k,
+                     const Tio *__restrict__ v, const float *__restrict__ log_alpha,
+                     const float *__restrict__ bgate, const float *__restrict__ wgate,
+                     const Tio *__restrict__ dO, const float *__restrict__ dS_T,
+                     const float *__restrict__ S_chunks, Tio *__restrict__ dv_out,
+                     float *__restrict__ dw_out, float *__restrict__ dS0, float *__restrict__ part_kb,
+                     float *__restrict__ part_qe, float *__restrict__ part_ki, float *__restrict__ part_ec) {
+    using L = Bwd2Layout<DK>;
+    constexpr int NB = DK / 16;
+    extern __shared__ float smem[];
+    float *sKB = smem + L::oKB, *sQE = smem + L::oQE, *sKI = smem + L::oKI, *sG = smem + L::oG;
+    float *sdP = sG, *sdA = sG + kChunk * L::LDC;
+    float *sS = smem + L::oS, *sD = smem + L::oD, *sdO = smem + L::odO, *sU = smem + L::oU;
+    float *sdR = smem + L::odR, *sA = smem + L::oA, *sP = smem + L::oP;
+    float *sEC = smem + L::oVec, *sOne = sEC + DK;
+    int *s_flag = reinterpret_cast<int *>(sOne + kChunk);
+
+    const int nslice = dv / kBwd2Dvs;
+    const int slice = blockIdx.x % nslice;
+    const int bh = blockIdx.x / nslice;
+    const int b = bh / H, h = bh % H;
+    const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+    const int vcol0 = slice * kBwd2Dvs;
+    const int nchunks = (T + kChunk - 1) / kChunk;
+    const size_t BTH = (size_t)gridDim.x / nslice * T;  // B*H*T token-heads
+    const size_t pslice = (size_t)slice * BTH;
+
+    for (int idx = tid; idx < kBwd2Dvs * DK; idx += blockDim.x) {
+        const int r = idx / DK, c = idx % DK;
+        sD[r * L::LDK + c] = dS_T ? dS_T[((size_t)bh * dv + vcol0 + r) * DK + c] : 0.f;
+    }
+    if (tid < kChunk) sOne[tid] = 1.f;
+
+#pragma unroll 1
+    for (int ch = nchunks - 1; ch >= 0; --ch) {
+        const int c0 = ch * kChunk;
+        const int n = min(kChunk, T - c0);
+        const size_t tok0 = ((size_t)b * T + c0) * H + h;
+        __syncthreads();
+        // ---- gates: G (per-channel cumulative log decay), E_C; K, Q, B, dO, S
+        if (tid == 0) *s_flag = 0;
+        for (int idx = tid; idx < kChunk * DK; idx += blockDim.x) {
+            const int r = idx / DK, j = idx % DK;
+            const size_t off = (tok0 + (size_t)r * H) * DK + j;
+            const bool ok = r < n;
+            sG[r * L::LDK + j] = ok ? log_alpha[off] : 0.f;
+            sKB[r * L::LDK + j] = ok ? to_f32(k[off]) * bgate[off] : 0.f;  // K*B, scaled by E below
+            sKI[r * L::LDK + j] = ok ? to_f32(k[off]) : 0.f;               // K, divided by E below
+            sQE[r * L::LDK + j] = ok ? to_f32(q[off]) : 0.f;               // Q, scaled by E below
+        }
+        load_tile(sdO, L::LDV, dO + tok0 * dv + vcol0, (size_t)H * dv, n, kBwd2Dvs);
+        {
+            const float *src = S_chunks + (((size_t)bh * nchunks + ch) * dv + vcol0) * DK;
+            for (int idx = tid; idx < kBwd2Dvs * DK; idx += blockDim.x)
+                sS[(idx / DK) * L::LDK + idx % DK] = src[idx];
+        }
+        __syncthreads();
+        for (int j = tid; j < DK; j += blockDim.x) {
+            float g = 0.f;
+            for (int r = 0; r < kChunk; ++r) {
+                g += sG[r * L::LDK + j];
+                const float e = expf(g);
+                sKB[r * L::LDK + j] *= e;
+                sQE[r * L::LDK + j] *= e;
+                sKI[r * L::LDK + j] = -g <= 80.f ? sKI[r * L::LDK + j] / e : 0.f;
+            }
+            sEC[j] = expf(g);
+            if (-g > 80.f) *s_flag = 1;
+        }
+        __syncthreads();
+        if (*s_flag && tid == 0) record_status(GDR_ERR_UNSUPPORTED);
+
+        // ---- P1: A, P (C x C); R = W*V - KBE S^T -> sU
+        {
+            float aa[4][4] = {}, pp[4][4] = {}, xs[4][2] = {};
+#pragma unroll 2
+            for (int j = 0; j < DK; ++j) {
+                float kb[4], qe[4], ki[4], sc[2];
+#pragma unroll
+                for (int a = 0; a < 4; ++a) {
+                    kb[a] = sKB[(ty + 16 * a) * L::LDK + j];
+                    qe[a] = sQE[(ty + 16 * a) * L::LDK + j];
+                    ki[a] = sKI[(tx + 16 * a) * L::LDK + j];
+                }
+#pragma unroll
+                for (int c = 0; c < 2; ++c) sc[c] = sS[(tx + 16 * c) * L::LDK + j];
+#pragma unroll
+                for (int a = 0; a < 4; ++a) {
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        aa[a][c] = fmaf(kb[a], ki[c], aa[a][c]);
+                        pp[a][c] = fmaf(qe[a], ki[c], pp[a][c]);
+                    }
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) xs[a][c] = fmaf(kb[a], sc[c], xs[a][c]);
+                }
+            }
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+                const int r = ty + 16 * a;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int i = tx + 16 * c;
+                    sA[r * L::LDC + i] = (i < r) ? aa[a][c] : 0.f;
+                    sP[r * L::LDC + i] = (i <= r) ? pp[a][c] : 0.f;
+                }
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    const int cc = tx + 16 * c;
+                    float wv = 0.f;
+                    if (r < n) {
+                        const size_t off = (tok0 + (size_t)r * H) * dv + vcol0 + cc;
+                        wv = wgate[off] * to_f32(v[off]);
+                    }
+                    sU[r * L::LDV + cc] = wv - xs[a][c];
+                }
+            }
+        }
+        __syncthreads();
+
+        // ---- P2: U = (I + A)^{-1} R
+        fwd_solve<L::LDC, L::LDV, kBwd2Dvs>(sA, sOne, sU);
+
+        // ---- P3: dU = Kt D^T + P^T dO -> sdR ; dP = dO U^T (i <= r) -> sdP
+        {
+            float du[4][2] = {};
+#pragma unroll 2
+            for (int j = 0; j < DK; ++j) {
+                float kr[4], dd[2];
+                const float ec = sEC[j];
+#pragma unroll
+                for (int a = 0; a < 4; ++a) kr[a] = sKI[(ty + 16 * a) * L::LDK + j] * ec;
+#pragma unroll
+                for (int c = 0; c < 2; ++c) dd[c] = sD[(tx + 16 * c) * L::LDK + j];
+#pragma unroll
+                for (int a = 0; a < 4; ++a)
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) du[a][c] = fmaf(kr[a], dd[c], du[a][c]);
+            }
+#pragma unroll 4
+            for (int i = 0; i < kChunk; ++i) {
+                float pr[4], od[2];
+#pragma unroll
+                for (int a = 0; a < 4; ++a) pr[a] = sP[i * L::LDC + ty + 16 * a];
+#pragma unroll
+                for (int c = 0; c < 2; ++c) od[c] = sdO[i * L::LDV + tx + 16 * c];
+#pragma unroll
+                for (int a = 0; a < 4; ++a)
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) du[a][c] = fmaf(pr[a], od[c], du[a][c]);
+            }
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int c = 0; c < 2; ++c) sdR[(ty + 16 * a) * L::LDV + tx + 16 * c] = du[a][c];
+            float dp[4][4] = {};
+#pragma unroll 4
+            for (int c = 0; c < kBwd2Dvs; ++c) {
+                float od[4], ui[4];
+#pragma unroll
+                for (int a = 0; a < 4; ++a) {
+                    od[a] = sdO[(ty + 16 * a) * L::LDV + c];
+                    ui[a] = sU[(tx + 16 * a) * L::LDV + c];
+                }
+#pragma unroll
+                for (int a = 0; a < 4; ++a)
+#pragma unroll
+                    for (int cc = 0; cc < 4; ++cc) dp[a][cc] = fmaf(od[a], ui[cc], dp[a][cc]);
+            }
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+                const int r = ty + 16 * a;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int i = tx + 16 * c;
+                    sdP[r * L::LDC + i] = (i <= r) ? dp[a][c] : 0.f;
+                }
+            }
+        }
+        __syncthreads();
+
+        // ---- P4: dR = (I + A)^{-T} dU (in sdR)
+        back_solve<L::LDC, L::LDV, kBwd2Dvs>(sA, sOne, sdR);
+
+        // ---- P5: dA = -dR U^T (i < r) -> sdA ; dV = W*dR, dW = V*dR
+        {
+            float da[4][4] = {};
+#pragma unroll 4
+            for (int c = 0; c < kBwd2Dvs; ++c) {
+                float dr[4], ui[4];
+#pragma unroll
+                for (int a = 0; a < 4; ++a) {
+                    dr[a] = sdR[(ty + 16 * a) * L::LDV + c];
+                    ui[a] = sU[(tx + 16 * a) * L::LDV + c];
+                }
+#pragma unroll
+                for (int a = 0; a < 4; ++a)
+#pragma unroll
+                    for (int cc = 0; cc < 4; ++cc) da[a][cc] = fmaf(-dr[a], ui[cc], da[a][cc]);
+            }
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+                const int r = ty + 16 * a;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int i = tx + 16 * c;
+                    sdA[r * L::LDC + i] = (i < r) ? da[a][c] : 0.f;
+                }
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    const int cc = tx + 16 * c;
+                    if (r < n) {
+                        const size_t off = (tok0 + (size_t)r * H) * dv + vcol0 + cc;
+                        const float dr = sdR[r * L::LDV + cc];
+                        dv_out[off] = from_f32<Tio>(wgate[off] * dr);
+                        dw_out[off] = to_f32(v[off]) * dr;
+                    }
+                }
+            }
+        }
+        __syncthreads();
+
+        // ---- P6: slice partials of dKBE, dQE, dKiE (C x DK) and of dE_C (DK)
+        {
+            float akb[4][NB] = {}, aqe[4][NB] = {}, aki[4][NB] = {}, ud[4][NB] = {};
+            // -dR S (-> dKBE), dO S (-> dQE), U D (-> dKiE via Diag(E_C))
+#pragma unroll 2
+            for (int c = 0; c < kBwd2Dvs; ++c) {
+                float dr[4], od[4], ur[4], ss[NB], dd[NB];
+#pragma unroll
+                for (int a = 0; a < 4; ++a) {
+                    const int r = ty + 16 * a;
+                    dr[a] = sdR[r * L::LDV + c];
+                    od[a] = sdO[r * L::LDV + c];
+                    ur[a] = sU[r * L::LDV + c];
+                }
+#pragma unroll
+                for (int bq = 0; bq < NB; ++bq) {
+                    ss[bq] = sS[c * L::LDK + tx + 16 * bq];
+                    dd[bq] = sD[c * L::LDK + tx + 16 * bq];
+                }
+#pragma unroll
+                for (int a = 0; a < 4; ++a)
+#pragma unroll
+                    for (int bq = 0; bq < NB; ++bq) {
+                        akb[a][bq] = fmaf(-dr[a], ss[bq], akb[a][bq]);
+                        aqe[a][bq] = fmaf(od[a], ss[bq], aqe[a][bq]);
+                        ud[a][bq] = fmaf(ur[a], dd[bq], ud[a][bq]);
+                    }
+            }
+            // dA KiE (-> dKBE), dP KiE (-> dQE), dA^T KBE + dP^T QE (-> dKiE)
+#pragma unroll 2
+            for (int i = 0; i < kChunk; ++i) {
+                float w_a[4], w_p[4], w_at[4], w_pt[4], ki[NB], kb[NB], qe[NB];
+#pragma unroll
+                for (int a = 0; a < 4; ++a) {
+                    const int r = ty + 16 * a;
+                    w_a[a] = sdA[r * L::LDC + i];
+                    w_p[a] = sdP[r * L::LDC + i];
+                    w_at[a] = sdA[i * L::LDC + r];
+                    w_pt[a] = sdP[i * L::LDC + r];
+                }
+#pragma unroll
+                for (int bq = 0; bq < NB; ++bq) {
+                    ki[bq] = sKI[i * L::LDK + tx + 16 * bq];
+                    kb[bq] = sKB[i * L::LDK + tx + 16 * bq];
+                    qe[bq] = sQE[i * L::LDK + tx + 16 * bq];
+                }
+#pragma unroll
+                for (int a = 0; a < 4; ++a)
+#pragma unroll
+                    for (int bq = 0; bq < NB; ++bq) {
+                        akb[a][bq] = fmaf(w_a[a], ki[bq], akb[a][bq]);
+                        aqe[a][bq] = fmaf(w_p[a], ki[bq], aqe[a][bq]);
+                        aki[a][bq] = fmaf(w_at[a], kb[bq], fmaf(w_pt[a], qe[bq], aki[a][bq]));
+                    }
+            }
+            // write the partials; colsum((U D) * KiE) of this thread's rows -> dE_C
+            float ecp[NB] = {};
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+                const int r = ty + 16 * a;
+                const size_t row = pslice * DK + (tok0 + (size_t)r * H) * DK;
+#pragma unroll
+                for (int bq = 0; bq < NB; ++bq) {
+                    const int j = tx + 16 * bq;
+                    ecp[bq] = fmaf(ud[a][bq], sKI[r * L::LDK + j], ecp[bq]);
+                    if (r < n) {
+                        part_kb[row + j] = akb[a][bq];
+                        part_qe[row + j] = aqe[a][bq];
+                        part_ki[row + j] = fmaf(ud[a][bq], sEC[j], aki[a][bq]);
+                    }
+                }
+            }
+            // colsum over the 16 row groups (ty) via shared memory, fixed order
+            __syncthreads();  // every read of dA / dP done: reuse their space
+            float *red = sdP;
+#pragma unroll
+            for (int bq = 0; bq < NB; ++bq) red[ty * DK + tx + 16 * bq] = ecp[bq];
+            __syncthreads();
+            for (int j = tid; j < DK; j += blockDim.x) {
+                float s = 0.f;
+                for (int g = 0; g < 16; ++g) s += red[g * DK + j];
+                for (int c = 0; c < kBwd2Dvs; ++c) s = fmaf(sS[c * L::LDK + j], sD[c * L::LDK + j], s);
+                part_ec[((size_t)slice * (BTH / T * nchunks) + (size_t)bh * nchunks + ch) * DK + j] = s;
+            }
+        }
+        __syncthreads();
+
+        // ---- P7: D <- D Diag(E_C) + dO^T QE - dR^T KBE (slice rows)
+        {
+            float dn[2][NB];
+#pragma unroll
+            for (int a = 0; a < 2; ++a)
+#pragma unroll
+                for (int bq = 0; bq < NB; ++bq) {
+                    const int c = ty + 16 * a, j = tx + 16 * bq;
+                    dn[a][bq] = sD[c * L::LDK + j] * sEC[j];
+                }
+#pragma unroll 4
+            for (int r = 0; r < kChunk; ++r) {
+                float w1[2], w2[2], qr[NB], kr[NB];
+#pragma unroll
+                for (int a = 0; a < 2; ++a) {
+                    w1[a] = sdO[r * L::LDV + ty + 16 * a];
+                    w2[a] = -sdR[r * L::LDV + ty + 16 * a];
+                }
+#pragma unroll
+                for (int bq = 0; bq < NB; ++bq) {
+                    qr[bq] = sQE[r * L::LDK + tx + 16 * bq];
+                    kr[bq] = sKB[r * L::LDK + tx + 16 * bq];
+                }
+#pragma unroll
+                for (int a = 0; a < 2; ++a)
+#pragma unroll
+                    for (int bq = 0; bq < NB; ++bq)
+                        dn[a][bq] = fmaf(w1[a], qr[bq], fmaf(w2[a], kr[bq], dn[a][bq]));
+            }
+            __syncthreads();  // every read of D done
+#pragma unroll
+            for (int a = 0; a < 2; ++a)
+#pragma unroll
+                for (int bq = 0; bq < NB; ++bq) sD[(ty + 16 * a) * L::LDK + tx + 16 * bq] = dn[a][bq];
+        }
+    }
+    __syncthreads();
+    if (dS0) {
+        for (int idx = tid; idx < kBwd2Dvs * DK; idx += blockDim.x) {
+            const int r = idx / DK, c = idx % DK;
+            dS0[((size_t)bh * dv + vcol0 + r) * DK + c] = sD[r * L::LDK + c];
+        }
+    }
+}
+
+// Sum the per-slice partials in a fixed order and apply the per-element chain
+// rule; dlog alpha = the reverse prefix sum of dG per channel inside each
+// chunk.  One CTA per (b, h, chunk), one thread per key channel.
+template <typename Tio, int DK>
+__global__ void __launch_bounds__(DK)
+gdr2_bwd_reduce_kernel(int T, int H, int nslice, const Tio *__restrict__ q, const Tio *__restrict__ k,
+                       const float *__restrict__ log_alpha, const float *__restrict__ bgate,
+                       const float *__restrict__ part_kb, const float *__restrict__ part_qe,
+                       const float *__restrict__ part_ki, const float *__restrict__ part_ec,
+                       Tio *__restrict__ dq, Tio *__restrict__ dk, float *__restrict__ dlog_alpha,
+                       float *__restrict__ db, size_t BTH) {
+    __shared__ float sg[kChunk][DK];
+    const int nchunks = (T + kChunk - 1) / kChunk;
+    const int ch = blockIdx.x % nchunks;
+    const int bh = blockIdx.x / nchunks;
+    const int b = bh / H, h = bh % H;
+    const int c0 = ch * kChunk, n = min(kChunk, T - c0);
+    const size_t tok0 = ((size_t)b * T + c0) * H + h;
+    const size_t nbh = BTH / T;
+    const int j = threadIdx.x;
+    float g = 0.f;
+    for (int r = 0; r < n; ++r) {
+        g += log_alpha[(tok0 + (size_t)r * H) * DK + j];
+        sg[r][j] = g;
+    }
+    float dec = 0.f;  // dL/dE_C of this channel
+    for (int s = 0; s < nslice; ++s) dec += part_ec[(((size_t)s * nbh + bh) * nchunks + ch) * DK + j];
+    float suffix = expf(g) * dec;  // dG_C, carried by the chunk's last token
+    for (int r = n - 1; r >= 0; --r) {
+        const size_t off = (tok0 + (size_t)r * H) * DK + j;
+        float skb = 0.f, sqe = 0.f, ski = 0.f;
+        for (int s = 0; s < nslice; ++s) {
+            skb += part_kb[(size_t)s * BTH * DK + off];
+            sqe += part_qe[(size_t)s * BTH * DK + off];
+            ski += part_ki[(size_t)s * BTH * DK + off];
+        }
+        const float G = sg[r][j], e = expf(G), kv = to_f32(k[off]), qv = to_f32(q[off]), bv = bgate[off];
+        const float ie = -G <= 80.f ? 1.f / e : 0.f;
+        dk[off] = from_f32<Tio>(fmaf(skb * bv, e, ski * ie));
+        db[off] = skb * kv * e;
+        dq[off] = from_f32<Tio>(sqe * e);
+        suffix += skb * kv * bv * e + sqe * qv * e - ski * kv * ie;
+        dlog_alpha[off] = suffix;
+    }
+}
+
+struct Bwd2Workspace {
+    float *states, *part_kb, *part_qe, *part_ki, *part_ec;
+};
+
+inline size_t bwd2_workspace_bytes(int B, int T, int H, int dk, int dv) {
+    const size_t nch = (size_t)(T + kChunk - 1) / kChunk;
+    const size_t ns = (size_t)dv / kBwd2Dvs;
+    const size_t bth = (size_t)B * T * H;
+    auto al = [](size_t x) { return (x + 255) / 256 * 256; };
+    return al((size_t)B * H * nch * dv * dk * 4) + 3 * al(ns * bth * dk * 4) + al(ns * B * H * nch * dk * 4);
+}
+
+inline Bwd2Workspace bwd2_carve(void *ws, int B, int T, int H, int dk, int dv) {
+    const size_t nch = (size_t)(T + kChunk - 1) / kChunk;
+    const size_t ns = (size_t)dv / kBwd2Dvs;
+    const size_t bth = (size_t)B * T * H;
+    auto al = [](size_t x) { return (x + 255) / 256 * 256; };
+    char *p = static_cast<char *>(ws);
+    Bwd2Workspace w;
+    w.states = reinterpret_cast<float *>(p);
+    p += al((size_t)B * H * nch * dv * dk * 4);
+    w.part_kb = reinterpret_cast<float *>(p);
+    p += al(ns * bth * dk * 4);
+    w.part_qe = reinterpret_cast<float *>(p);
+    p += al(ns * bth * dk * 4);
+    w.part_ki = reinterpret_cast<float *>(p);
+    p += al(ns * bth * dk * 4);
+    w.part_ec = reinterpret_cast<float *>(p);
+    return w;
+}
+
+template <typename Tio, int DK>
+cudaError_t launch_bwd2_simt(int B, int T, int H, int dv, const void *q, const void *k, const void *v,
+                             const float *la, const float *bg, const float *wg, const float *S0,
+                             const void *dO, const float *dS_T, void *dq, void *dk_out, void *dv_out,
+                             float *dla, float *db, float *dw, float *dS0, void *ws, cudaStream_t stream) {
+    Bwd2Workspace w = bwd2_carve(ws, B, T, H, DK, dv);
+    // 1) forward recompute on the CUDA cores, keeping every chunk's fp32 entry state
+    cudaError_t err = launch_gdr2_simt<Tio, DK>(B, T, H, dv, q, k, v, la, bg, wg, S0, nullptr, nullptr, stream,
+                                                w.states);
+    if (err != cudaSuccess) return err;
+    // 2) reverse chunk pass per (b, h, slice)
+    using L = Bwd2Layout<DK>;
+    auto kern = gdr2_bwd_simt_kernel<Tio, DK>;
+    err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kBytes);
+    if (err != cudaSuccess) return err;
+    const int nslice = dv / kBwd2Dvs;
+    kern<<<(unsigned)(B * H * nslice), kSimtThreads, L::kBytes, stream>>>(
+        T, H, dv, static_cast<const Tio *>(q), static_cast<const Tio *>(k), static_cast<const Tio *>(v), la, bg,
+        wg, static_cast<const Tio *>(dO), dS_T, w.states, static_cast<Tio *>(dv_out), dw, dS0, w.part_kb,
+        w.part_qe, w.part_ki, w.part_ec);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+    // 3) sum the slices, chain rule through the gates, dlog alpha by reverse prefix sums
+    const int nch = (T + kChunk - 1) / kChunk;
+    gdr2_bwd_reduce_kernel<Tio, DK><<<(unsigned)(B * H * nch), DK, 0, stream>>>(
+        T, H, nslice, static_cast<const Tio *>(q), static_cast<const Tio *>(k), la, bg, w.part_kb, w.part_qe,
+        w.part_ki, w.part_ec, static_cast<Tio *>(dq), static_cast<Tio *>(dk_out), dla, db, (size_t)B * T * H);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return cudaGetLastError();
+}
+
+}  // namespace gdr

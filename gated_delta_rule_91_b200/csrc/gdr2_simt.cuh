@@ -50,7 +50,8 @@ __global__ void __launch_bounds__(kSimtThreads, 1)
 gdr2_fwd_simt_kernel(int T, int H, int dv, const Tio *__restrict__ q, const Tio *__restrict__ k,
                      const Tio *__restrict__ v, const float *__restrict__ log_alpha,
                      const float *__restrict__ bgate, const float *__restrict__ wgate,
-                     const float *__restrict__ S0, Tio *__restrict__ o, float *__restrict__ S_T) {
+                     const float *__restrict__ S0, Tio *__restrict__ o, float *__restrict__ S_T,
+                     float *__restrict__ S_chunks) {
     using L = Gdr2Layout<DK>;
     constexpr int NB = DK / 16;
     extern __shared__ float smem[];
@@ -78,6 +79,11 @@ gdr2_fwd_simt_kernel(int T, int H, int dv, const Tio *__restrict__ q, const Tio 
         __syncthreads();
         load_tile(sQ, L::LDK, q + tok0 * DK, (size_t)H * DK, n, DK);
         load_tile(sK, L::LDK, k + tok0 * DK, (size_t)H * DK, n, DK);
+        if (S_chunks) {  // chunk-entry state for the backward's recompute pass
+            float *dst = S_chunks + (((size_t)bh * ((T + kChunk - 1) / kChunk) + c0 / kChunk) * dv + vcol0) * DK;
+            for (int idx = tid; idx < kSimtDvs * DK; idx += blockDim.x)
+                dst[idx] = sS[(idx / DK) * L::LDK + idx % DK];
+        }
         // R <- w * v (slice columns), zero past the end
         for (int idx = tid; idx < kChunk * kSimtDvs; idx += blockDim.x) {
             const int r = idx / kSimtDvs, c = idx % kSimtDvs;
@@ -219,7 +225,7 @@ gdr2_fwd_simt_kernel(int T, int H, int dv, const Tio *__restrict__ q, const Tio 
 #pragma unroll
         for (int a = 0; a < 4; ++a) {
             const int r = ty + 16 * a;
-            if (r < n) {
+            if (r < n && o) {
                 Tio *orow = o + (tok0 + (size_t)r * H) * dv + vcol0;
 #pragma unroll
                 for (int c = 0; c < 4; ++c) orow[tx + 16 * c] = from_f32<Tio>(o_acc[a][c]);
@@ -280,9 +286,12 @@ gdr2_fwd_simt_kernel(int T, int H, int dv, const Tio *__restrict__ q, const Tio 
 }
 
 template <typename Tio, int DK>
+// o == nullptr skips the outputs (the backward's recompute); S_chunks
+// (nullable) receives every chunk's entry state, [B, H, nchunks, dv, DK] fp32.
 cudaError_t launch_gdr2_simt(int B, int T, int H, int dv, const void *q, const void *k,
                              const void *v, const float *la, const float *bg, const float *wg,
-                             const float *S0, void *o, float *S_T, cudaStream_t stream) {
+                             const float *S0, void *o, float *S_T, cudaStream_t stream,
+                             float *S_chunks = nullptr) {
     using L = Gdr2Layout<DK>;
     auto kern = gdr2_fwd_simt_kernel<Tio, DK>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -290,7 +299,7 @@ cudaError_t launch_gdr2_simt(int B, int T, int H, int dv, const void *q, const v
     if (err != cudaSuccess) return err;
     kern<<<(unsigned)(B * H * (dv / kSimtDvs)), kSimtThreads, L::kBytes, stream>>>(
         T, H, dv, static_cast<const Tio *>(q), static_cast<const Tio *>(k),
-        static_cast<const Tio *>(v), la, bg, wg, S0, static_cast<Tio *>(o), S_T);
+        static_cast<const Tio *>(v), la, bg, wg, S0, static_cast<Tio *>(o), S_T, S_chunks);
     g_launches.fetch_add(1, std::memory_order_relaxed);
     return cudaGetLastError();
 }

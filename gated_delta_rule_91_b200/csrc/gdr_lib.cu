@@ -19,6 +19,7 @@
 #include "fwd_tc2.cuh"
 #include "bwd_tc.cuh"
 #include "fwd2_tc.cuh"
+#include "bwd2_simt.cuh"
 
 namespace gdr {
 std::atomic<uint64_t> g_launches{0};
@@ -123,7 +124,9 @@ gdr_status gdr_check_status(gdr_stream_t stream) {
     if (host != 0) {
         e = cudaMemcpyToSymbol(g_status, &zero, sizeof(int));
         if (e != cudaSuccess) return cuda_fail(e, "gdr_check_status: clear status");
-        return fail((gdr_status)host, "device status %d: a bounded on-chip wait gave up", host);
+        return fail((gdr_status)host, "device status %d: %s", host,
+                    host == GDR_ERR_TIMEOUT ? "a bounded on-chip wait gave up"
+                                            : "a chunk the kernel does not handle (gdr2_bwd: channel decay past e^80)");
     }
     return GDR_OK;
 }
@@ -300,6 +303,55 @@ gdr_status gdr2_fwd(int B, int T, int H, int dk, int dv, gdr_dtype dt, const voi
         e = dk == 128 ? launch_gdr2_simt<__nv_bfloat16, 128>(GDR2_ARGS)
                       : launch_gdr2_simt<__nv_bfloat16, 64>(GDR2_ARGS);
 #undef GDR2_ARGS
+    if (e != cudaSuccess) return cuda_fail(e, fn);
+    return GDR_OK;
+}
+
+size_t gdr2_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, gdr_dtype) {
+    if (B < 1 || T < 1 || H < 1 || (dk != 64 && dk != 128) || (dv != 64 && dv != 128)) return 0;
+    return bwd2_workspace_bytes(B, T, H, dk, dv);
+}
+
+gdr_status gdr2_bwd(int B, int T, int H, int dk, int dv, gdr_dtype dt, const void *q, const void *k,
+                    const void *v, const float *log_alpha, const float *b, const float *w, const float *S0,
+                    const void *dO, const float *dS_T, void *dq, void *dk_out, void *dv_out, float *dlog_alpha,
+                    float *db, float *dw, float *dS0, void *workspace, size_t workspace_bytes,
+                    gdr_stream_t stream) {
+    const char *fn = "gdr2_bwd";
+    gdr_status st = check_dims(fn, B, T, H, dk, dv, dt);
+    if (st != GDR_OK) return st;
+    GDR_REQUIRE_PTR(q);
+    GDR_REQUIRE_PTR(k);
+    GDR_REQUIRE_PTR(v);
+    GDR_REQUIRE_PTR(log_alpha);
+    GDR_REQUIRE_PTR(b);
+    GDR_REQUIRE_PTR(w);
+    GDR_REQUIRE_PTR(dO);
+    GDR_REQUIRE_PTR(dq);
+    GDR_REQUIRE_PTR(dk_out);
+    GDR_REQUIRE_PTR(dv_out);
+    GDR_REQUIRE_PTR(dlog_alpha);
+    GDR_REQUIRE_PTR(db);
+    GDR_REQUIRE_PTR(dw);
+    GDR_OPTIONAL_PTR(S0);
+    GDR_OPTIONAL_PTR(dS_T);
+    GDR_OPTIONAL_PTR(dS0);
+    const size_t need = bwd2_workspace_bytes(B, T, H, dk, dv);
+    if (workspace == nullptr || workspace_bytes < need)
+        return fail(GDR_ERR_WORKSPACE, "%s: workspace of %zu bytes needed, %zu given", fn, need,
+                    workspace ? workspace_bytes : (size_t)0);
+    if (!aligned16(workspace))
+        return fail(GDR_ERR_INVALID_ARGUMENT, "%s: workspace is not 16-byte aligned", fn);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e;
+#define GDR2_BWD_ARGS B, T, H, dv, q, k, v, log_alpha, b, w, S0, dO, dS_T, dq, dk_out, dv_out, dlog_alpha, \
+                      db, dw, dS0, workspace, s
+    if (dt == GDR_F32)
+        e = dk == 128 ? launch_bwd2_simt<float, 128>(GDR2_BWD_ARGS) : launch_bwd2_simt<float, 64>(GDR2_BWD_ARGS);
+    else
+        e = dk == 128 ? launch_bwd2_simt<__nv_bfloat16, 128>(GDR2_BWD_ARGS)
+                      : launch_bwd2_simt<__nv_bfloat16, 64>(GDR2_BWD_ARGS);
+#undef GDR2_BWD_ARGS
     if (e != cudaSuccess) return cuda_fail(e, fn);
     return GDR_OK;
 }

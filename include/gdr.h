@@ -174,9 +174,33 @@ GDR_API gdr_status gdr2_fwd(int B, int T, int H, int dk, int dv, gdr_dtype dt,
                     void *workspace, size_t workspace_bytes, gdr_stream_t stream);
 GDR_API size_t gdr2_fwd_workspace_bytes(int B, int T, int H, int dk, int dv, gdr_dtype dt);
 
+/*
+ * Gated Delta Rule-2 backward: gradients of gdr2_fwd (the pages give no
+ * backward; this is the chain rule of the step above).
+ *   in : the inputs of gdr2_fwd; dO [B,T,H,dv] (dtype dt); dS_T [B,H,dv,dk]
+ *        fp32 or NULL (= 0).
+ *   out: dq, dk_out [B,T,H,dk] and dv_out [B,T,H,dv] (dtype dt);
+ *        dlog_alpha, db [B,T,H,dk] fp32; dw [B,T,H,dv] fp32;
+ *        dS0 [B,H,dv,dk] fp32 or NULL.
+ * The caller-owned workspace (at least gdr2_bwd_workspace_bytes) holds the
+ * recomputed forward's chunk-entry states and per-slice partial sums.  A
+ * 64-token chunk in which some key channel decays by more than e^80 is not
+ * handled: its gradients are not valid, and gdr_check_status then returns
+ * GDR_ERR_UNSUPPORTED.
+ */
+GDR_API gdr_status gdr2_bwd(int B, int T, int H, int dk, int dv, gdr_dtype dt,
+                    const void *q, const void *k, const void *v,
+                    const float *log_alpha, const float *b, const float *w, const float *S0,
+                    const void *dO, const float *dS_T,
+                    void *dq, void *dk_out, void *dv_out,
+                    float *dlog_alpha, float *db, float *dw, float *dS0,
+                    void *workspace, size_t workspace_bytes, gdr_stream_t stream);
+GDR_API size_t gdr2_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, gdr_dtype dt);
+
 /* Synchronise `stream`, then read and clear the device status word that
- * kernels set when a bounded wait gives up.  Returns GDR_OK or
- * GDR_ERR_TIMEOUT (or GDR_ERR_CUDA if the synchronisation itself failed). */
+ * kernels set when a bounded wait gives up (GDR_ERR_TIMEOUT) or when
+ * gdr2_bwd meets a chunk it does not handle (GDR_ERR_UNSUPPORTED).  Returns
+ * GDR_OK, that status, or GDR_ERR_CUDA if the synchronisation itself failed. */
 GDR_API gdr_status gdr_check_status(gdr_stream_t stream);
 
 /* Test hook for the timeout path: launches a one-thread kernel that waits on

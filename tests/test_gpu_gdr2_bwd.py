@@ -1,0 +1,111 @@
+"""gdr2_bwd (Gated DeltaNet-2 backward) on the GPU vs the oracle's reverse
+mode, through the C ABI.  Tolerances as for gdr_bwd: per gradient tensor
+max|d|/max|ref| <= 1e-4 for fp32 inputs and 2e-2 for bf16 inputs; dS0
+relative Frobenius <= 1e-2 (bf16) / 1e-4 (fp32)."""
+import numpy as np
+import pytest
+import torch
+
+import gated_delta_rule_91_b200 as gdr
+import oracle
+import synth
+from gpu_common import TOL_G, dev, fro_rel, max_rel, np64
+
+pytestmark = pytest.mark.gpu
+
+NAMES = ["dq", "dk", "dv", "dlog_alpha", "db", "dw"]
+
+
+def _inputs(B, T, H, dk, dv, dtype, seed, b_max=1.0):
+    x = synth.gdr2_inputs(B, T, H, dk, dv, dtype, seed=seed, s0_std=0.02, b_max=b_max)
+    g = torch.Generator().manual_seed(seed + 1)
+    x["dO"] = torch.randn(B, T, H, dv, generator=g).to(x["q"].dtype)
+    return x
+
+
+def _gpu(x, dST):
+    d = {n: dev(x[n]) for n in ("q", "k", "v", "log_alpha", "b", "w", "S0", "dO")}
+    return gdr.gdr2_bwd(d["q"], d["k"], d["v"], d["log_alpha"], d["b"], d["w"], d["S0"], d["dO"], dev(dST))
+
+
+def _oracle(x, dST, heads=None):
+    a = {n: np64(x[n]) for n in ("q", "k", "v", "log_alpha", "b", "w", "S0", "dO")}
+    dST = np64(dST)
+    if heads is not None:
+        for n in ("q", "k", "v", "log_alpha", "b", "w", "dO"):
+            a[n] = np.stack([a[n][b, :, h] for b, h in heads])[:, :, None]
+        a["S0"] = np.stack([a["S0"][b, h] for b, h in heads])[:, None]
+        if dST is not None:
+            dST = np.stack([dST[b, h] for b, h in heads])[:, None]
+    return oracle.gdr2_bwd(a["q"], a["k"], a["v"], a["log_alpha"], a["b"], a["w"], a["S0"], a["dO"], dST)
+
+
+def _compare(got, ref, dtype, heads=None):
+    for n in NAMES:
+        g = np64(got[n])
+        if heads is not None:
+            g = np.stack([g[b, :, h] for b, h in heads])[:, :, None]
+        assert max_rel(g, ref[n]) <= TOL_G[dtype], (n, max_rel(g, ref[n]))
+    g = np64(got["dS0"])
+    if heads is not None:
+        g = np.stack([g[b, h] for b, h in heads])[:, None]
+    assert fro_rel(g, ref["dS0"]) <= (TOL_G["f32"] if dtype == "f32" else 1e-2)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("T", [1, 64, 100, 130])
+@pytest.mark.parametrize("dk,dv", [(64, 64), (128, 128), (64, 128), (128, 64)])
+def test_gdr2_bwd_small(dtype, T, dk, dv):
+    x = _inputs(2, T, 2, dk, dv, dtype, seed=5 * T + dk + dv)
+    dST = torch.randn(2, 2, dv, dk, generator=torch.Generator().manual_seed(T)) * 0.1
+    got = _gpu(x, dST)
+    gdr.check_status()
+    _compare(got, _oracle(x, dST), dtype)
+
+
+def test_gdr2_bwd_workload_sampled_heads():
+    """The Gated DeltaNet-2 workload shape (B4 T4096 H16 d128 bf16): two heads
+    against the oracle over the whole sequence."""
+    x = _inputs(4, 4096, 16, 128, 128, "bf16", seed=4)
+    got = _gpu(x, None)
+    torch.cuda.synchronize()
+    gdr.check_status()
+    heads = [(0, 3), (3, 12)]
+    _compare(got, _oracle(x, None, heads), "bf16", heads)
+
+
+def test_gdr2_bwd_deterministic():
+    x = _inputs(1, 200, 2, 128, 128, "bf16", seed=9)
+    a = _gpu(x, None)
+    b = _gpu(x, None)
+    for n in NAMES + ["dS0"]:
+        assert torch.equal(a[n], b[n]), n
+
+
+def test_gdr2_bwd_collapses_to_gdr_bwd_on_gpu():
+    """b = w = beta*1 and a scalar decay broadcast to every channel: the
+    Gated DeltaNet-2 gradients reduce to the scalar-gate rule's (dlog alpha
+    summed over channels, dbeta = sum db + sum dw), across the two GPU
+    backward paths."""
+    x = synth.gdr_inputs(2, 150, 2, 128, 128, "f32", seed=33, s0_std=0.02, with_dO=True)
+    d = {n: dev(x[n]) for n in ("q", "k", "v", "log_alpha", "beta", "S0", "dO")}
+    g1 = gdr.gdr_bwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["S0"], d["dO"])
+    la = d["log_alpha"][..., None].expand(-1, -1, -1, 128).contiguous()
+    bw = d["beta"][..., None].expand(-1, -1, -1, 128).contiguous()
+    g2 = gdr.gdr2_bwd(d["q"], d["k"], d["v"], la, bw, bw, d["S0"], d["dO"])
+    for n in ("dq", "dk", "dv", "dS0"):
+        assert max_rel(np64(g2[n]), np64(g1[n])) <= 1e-4, n
+    assert max_rel(np64(g2["dlog_alpha"].sum(-1)), np64(g1["dlog_alpha"])) <= 1e-4
+    assert max_rel(np64(g2["db"].sum(-1) + g2["dw"].sum(-1)), np64(g1["dbeta"])) <= 1e-4
+
+
+def test_gdr2_bwd_reports_a_chunk_it_does_not_handle():
+    """A chunk in which some channel decays by more than e^80 is reported
+    through gdr_check_status as GDR_ERR_UNSUPPORTED (no fault)."""
+    x = _inputs(1, 100, 1, 128, 128, "bf16", seed=10)
+    x["log_alpha"][:, :, :, :8] = -3.0
+    _gpu(x, None)
+    with pytest.raises(gdr.GdrError) as e:
+        gdr.check_status()
+    assert e.value.status == gdr.GDR_ERR_UNSUPPORTED
+    gdr.check_status()  # the status word was cleared
