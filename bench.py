@@ -401,6 +401,22 @@ def secondary(pk):
         ms2 = e0.elapsed_time(e1) / 5
         out["gdn2_fwd_b_0_2"] = {"workload": "B=4 T=4096 H=16 d=128 bf16, b in (0, 2)", "ms": ms2,
                                  "mtok_per_s": w.B * w.T / (ms2 * 1e-3) / 1e6}
+        # Gated DeltaNet-2 backward on the same workload (dO ~ N(0, 1), dS_T = 0)
+        d["b"].mul_(0.5)
+        dO = torch.randn(d["q"].shape, generator=torch.Generator().manual_seed(7)).to(d["q"].dtype).cuda()
+        bcall = lambda: gdr.gdr2_bwd(d["q"], d["k"], d["v"], d["log_alpha"], d["b"], d["w"], d["S0"], dO)
+        bcall()
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(3):
+            bcall()
+        e1.record()
+        torch.cuda.synchronize()
+        bms = e0.elapsed_time(e1) / 3
+        out["gdn2_bwd"] = {"workload": "B=4 T=4096 H=16 d=128 bf16", "ms": bms,
+                           "mtok_per_s": w.B * w.T / (bms * 1e-3) / 1e6,
+                           "tc_frac": bwd_flops(w.B, w.T, w.H, w.dk) / (bms * 1e-3) / (pk["bf16_tflops"] * 1e12),
+                           "kernels": "CUDA cores (recompute, reverse chunk pass, reduce)"}
     except Exception as e:
         out["gdn2_fwd"] = {"unavailable": str(e).splitlines()[0][:200]}
     return out
