@@ -31,6 +31,8 @@
 #include "common.cuh"
 #include "bwd_simt.cuh"
 #include "gdr2_simt.cuh"
+#include "fwd2_tc.cuh"
+#include <type_traits>
 
 namespace gdr {
 
@@ -499,9 +501,12 @@ cudaError_t launch_bwd2_simt(int B, int T, int H, int dv, const void *q, const v
                              const void *dO, const float *dS_T, void *dq, void *dk_out, void *dv_out,
                              float *dla, float *db, float *dw, float *dS0, void *ws, cudaStream_t stream) {
     Bwd2Workspace w = bwd2_carve(ws, B, T, H, DK, dv);
-    // 1) forward recompute on the CUDA cores, keeping every chunk's fp32 entry state
-    cudaError_t err = launch_gdr2_simt<Tio, DK>(B, T, H, dv, q, k, v, la, bg, wg, S0, nullptr, nullptr, stream,
-                                                w.states);
+    // 1) forward recompute keeping every chunk's fp32 entry state (the
+    //    tensor-core forward for bf16 with dk = dv = 128, else CUDA cores)
+    cudaError_t err = (std::is_same<Tio, __nv_bfloat16>::value && DK == 128 && dv == 128)
+                          ? launch_fwd2_tc(B, T, H, q, k, v, la, bg, wg, S0, nullptr, nullptr, stream, w.states)
+                          : launch_gdr2_simt<Tio, DK>(B, T, H, dv, q, k, v, la, bg, wg, S0, nullptr, nullptr, stream,
+                                                      w.states);
     if (err != cudaSuccess) return err;
     // 2) reverse chunk pass per (b, h, slice)
     using L = Bwd2Layout<DK>;

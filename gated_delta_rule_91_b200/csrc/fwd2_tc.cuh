@@ -164,7 +164,8 @@ __global__ void __launch_bounds__(kG2Threads, 1)
 gdr2_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                    int T, int H, const float *__restrict__ log_alpha, const float *__restrict__ bgate,
-                   const float *__restrict__ wgate, const float *__restrict__ S0, float *__restrict__ S_T) {
+                   const float *__restrict__ wgate, const float *__restrict__ S0, float *__restrict__ S_T,
+                   int store_o, float *__restrict__ S_chunks) {
     using L = G2Layout;
     using namespace sm100;
     constexpr int D = 128;
@@ -351,6 +352,11 @@ gdr2_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             const int col = wc * 32;
             float v[32];
             tmem_ld32(tl + kG2S + col, v);
+            if (S_chunks) {  // entry state of chunk n, fp32, for the backward's recompute
+                float4 *dst = reinterpret_cast<float4 *>(S_chunks + (((size_t)bh * nch + n) * D + row) * D + col);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+            }
             uint8_t *half = sm + L::SB + (wc >> 1) * 16384;
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4) st_bf16x8(half + sw128_offset(row, (wc & 1) * 4 + q4), v + 8 * q4);
@@ -423,7 +429,7 @@ gdr2_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             ++ncommit;
         }
         if (!mma_wait_all()) break;
-        {   // O^T (lane = value channel, column = token) -> bf16 tile [token][channel] -> TMA store
+        if (store_o) {  // O^T (lane = value channel, column = token) -> bf16 tile [token][channel]
             float v[16];
             tmem_ld16(tl + kG2O + wc * 16, v);
             uint8_t *half = sm + L::OST + (row >> 6) * 8192;
@@ -433,7 +439,7 @@ gdr2_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         }
         fence_async_smem();
         __syncthreads();
-        if (tid == 0) {
+        if (tid == 0 && store_o) {
             tma_store_4d(&tm_o, sm + L::OST, 0, h, t0, b);
             tma_store_4d(&tm_o, sm + L::OST + 8192, 64, h, t0, b);
             bulk_commit();
@@ -463,18 +469,20 @@ gdr2_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     }
 }
 
+// o == nullptr runs without outputs (the backward's recompute); S_chunks
+// (nullable) receives every chunk's entry state, [B, H, nchunks, 128, 128] fp32.
 inline cudaError_t launch_fwd2_tc(int B, int T, int H, const void *q, const void *k, const void *v,
                                   const float *la, const float *bgate, const float *wgate, const float *S0,
-                                  void *o, float *S_T, cudaStream_t stream) {
+                                  void *o, float *S_T, cudaStream_t stream, float *S_chunks = nullptr) {
     CUtensorMap mq, mk, mv, mo;
     if (!make_token_map(&mq, q, B, T, H, 128) || !make_token_map(&mk, k, B, T, H, 128) ||
-        !make_token_map(&mv, v, B, T, H, 128) || !make_token_map(&mo, o, B, T, H, 128))
+        !make_token_map(&mv, v, B, T, H, 128) || !make_token_map(&mo, o ? o : q, B, T, H, 128))
         return cudaErrorInvalidValue;
     cudaError_t err = cudaFuncSetAttribute(gdr2_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            (int)G2Layout::kAlloc);
     if (err != cudaSuccess) return err;
-    gdr2_fwd_tc_kernel<<<(unsigned)(B * H), kG2Threads, G2Layout::kAlloc, stream>>>(mq, mk, mv, mo, T, H, la, bgate,
-                                                                                   wgate, S0, S_T);
+    gdr2_fwd_tc_kernel<<<(unsigned)(B * H), kG2Threads, G2Layout::kAlloc, stream>>>(
+        mq, mk, mv, mo, T, H, la, bgate, wgate, S0, S_T, o != nullptr ? 1 : 0, S_chunks);
     g_launches.fetch_add(1, std::memory_order_relaxed);
     return cudaGetLastError();
 }
