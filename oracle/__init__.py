@@ -31,6 +31,8 @@ def _load():
         lib.oracle_gdr_bwd.argtypes = [i, i, i, i, i] + [dp] * 14
         lib.oracle_gdr2_fwd.argtypes = [i, i, i, i, i] + [dp] * 9
         lib.oracle_gdr2_bwd.argtypes = [i, i, i, i, i] + [dp] * 16
+        lib.oracle_short_conv.argtypes = [i] * 5 + [dp] * 4 + [i, ctypes.c_double, dp, dp]
+        lib.oracle_rmsnorm_gate.argtypes = [i] * 4 + [dp] * 3 + [ctypes.c_double, dp]
         lib.oracle_num_threads.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -123,3 +125,28 @@ def gdr2_bwd(q, k, v, log_alpha, b, w, S0, dO, dS_T=None):
                             _p(out["dv"]), _p(out["dlog_alpha"]), _p(out["db"]), _p(out["dw"]),
                             _p(out["dS0"]))
     return out
+
+
+def short_conv(x, w, bias=None, state=None, l2=False, eps=0.0):
+    """Block prologue for one stream: depthwise causal ShortConv of width K,
+    SiLU, and (l2=True) L2 normalisation per (token, head).  x [B,T,H,d],
+    w [H*d, K], bias [H*d] or None, state [B, K-1, H*d] or None (zeros).
+    Returns (y [B,T,H,d], state_out [B, K-1, H*d]) as float64."""
+    x, w, bias, state = map(_in, (x, w, bias, state))
+    B, T, H, d = x.shape
+    K = w.shape[-1]
+    y = np.zeros_like(x)
+    st = np.zeros((B, K - 1, H * d))
+    _load().oracle_short_conv(B, T, H, d, K, _p(x), _p(w), _p(bias), _p(state), int(l2),
+                              float(eps), _p(y), _p(st) if K > 1 else None)
+    return y, st
+
+
+def rmsnorm_gate(o, g, weight, eps=0.0):
+    """Block epilogue: RMSNorm over dv per (token, head) with a per-channel
+    weight, times SiLU(g) (g None: no gate).  o, g [B,T,H,dv], weight [dv]."""
+    o, g, weight = map(_in, (o, g, weight))
+    B, T, H, dv = o.shape
+    y = np.zeros_like(o)
+    _load().oracle_rmsnorm_gate(B, T, H, dv, _p(o), _p(g), _p(weight), float(eps), _p(y))
+    return y

@@ -8,16 +8,16 @@ import subprocess
 import sys
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-SRC = os.path.join(HERE, "gdr_oracle.c")
+SRCS = [os.path.join(HERE, "gdr_oracle.c"), os.path.join(HERE, "block_oracle.c")]
 LIB = os.path.join(HERE, "liboracle.so")
 
 
 def build(force: bool = False) -> str:
-    if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= os.path.getmtime(SRC):
+    if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= max(map(os.path.getmtime, SRCS)):
         return LIB
     tmp = LIB + ".tmp%d" % os.getpid()
     cmd = ["gcc", "-O2", "-std=c99", "-fopenmp", "-fPIC", "-shared",
-           "-o", tmp, SRC, "-lm"]
+           "-o", tmp] + SRCS + ["-lm"]
     subprocess.check_call(cmd)
     os.replace(tmp, LIB)
     return LIB
