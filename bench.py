@@ -128,6 +128,18 @@ def gdr2_bytes(B, T, H, dk, dv, esize=2):
     return B * T * H * per + 2 * B * H * dv * dk * 4
 
 
+def prologue_bytes(B, T, H, dk, dv, K, esize=2):
+    """Block prologue: read xq, xk, xv and write q, k, v once, plus the fp32
+    conv taps and biases (the conv state is not used on this workload)."""
+    elems = B * T * H * (2 * dk + dv)
+    return 2 * elems * esize + H * (2 * dk + dv) * (K + 1) * 4
+
+
+def epilogue_bytes(B, T, H, dv, esize=2):
+    """Block epilogue: read o and g, write y; the fp32 norm weight."""
+    return 3 * B * T * H * dv * esize + dv * 4
+
+
 # ---------------------------------------------------------------------------
 # clocks sampled during the timed region
 # ---------------------------------------------------------------------------
@@ -419,6 +431,60 @@ def secondary(pk):
                            "kernels": "tensor-core recompute; CUDA-core reverse chunk pass and reduce"}
     except Exception as e:
         out["gdn2_fwd"] = {"unavailable": str(e).splitlines()[0][:200]}
+    del d, x
+    out.update(block_lines(pk))
+    return out
+
+
+def block_lines(pk):
+    """The block's prologue (ShortConv, SiLU, q/k L2) and epilogue (RMSNorm,
+    SiLU gate) on the layer workload, alone and around the forward."""
+    import gated_delta_rule_91_b200 as gdr
+    out = {}
+    B, T, H, d, K = 4, 4096, 16, 128, 4
+    px = {n: (t.cuda() if t is not None else None)
+          for n, t in synth.block_prologue_inputs(B, T, H, d, d, K, "bf16", seed=21, state=False).items()}
+    ex = {n: (t.cuda() if t is not None else None)
+          for n, t in synth.block_epilogue_inputs(B, T, H, d, "bf16", seed=22).items()}
+    gx = {n: (t.cuda() if t is not None else None)
+          for n, t in synth.gdr_inputs(B, T, H, d, d, "bf16", seed=23).items()}
+    q, k, v = (torch.empty(B, T, H, d, dtype=torch.bfloat16, device="cuda") for _ in range(3))
+    o = torch.empty_like(q)
+    y = torch.empty_like(q)
+    pro = lambda: gdr.gdr_block_prologue(px["xq"], px["xk"], px["xv"], px["wq"], px["wk"], px["wv"],
+                                         px["bq"], px["bk"], px["bv"], eps=1e-6, q=q, k=k, v=v)
+    epi = lambda oo: gdr.gdr_block_epilogue(oo, ex["g"], ex["weight"], 1e-6, y=y)
+    mix = lambda: gdr.gdr_fwd(q, k, v, gx["log_alpha"], gx["beta"], gx["S0"], o=o)
+
+    def timed(fn, reps=20):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    us_p = timed(pro) * 1e3
+    gbs_p = prologue_bytes(B, T, H, d, d, K) / (us_p * 1e-6) / 1e9
+    out["block_prologue"] = {"workload": "B=4 T=4096 H=16 dk=dv=128 bf16, ShortConv K=4 + SiLU + q/k L2",
+                             "us": us_p, "achieved_gbs": gbs_p, "hbm_frac": gbs_p / pk["hbm_gbs"]}
+    us_e = timed(lambda: epi(ex["o"])) * 1e3
+    gbs_e = epilogue_bytes(B, T, H, d) / (us_e * 1e-6) / 1e9
+    out["block_epilogue"] = {"workload": "B=4 T=4096 H=16 dv=128 bf16, RMSNorm + SiLU gate",
+                             "us": us_e, "achieved_gbs": gbs_e, "hbm_frac": gbs_e / pk["hbm_gbs"]}
+
+    def chain():
+        pro()
+        mix()
+        epi(o)
+
+    ms = timed(chain, reps=10)
+    out["block_mixer_fwd"] = {"workload": "B=4 T=4096 H=16 d=128 bf16: prologue -> gdr_fwd -> epilogue",
+                              "ms": ms, "mtok_per_s": B * T / (ms * 1e-3) / 1e6}
     return out
 
 

@@ -10,6 +10,9 @@ Functions (same names as the C entry points):
     gdr_step(q, k, v, log_alpha, beta, S)                -> o  (S advanced in place)
     gdr_bwd(q, k, v, log_alpha, beta, S0, dO, dS_T=None) -> dict of gradients
     gdr2_fwd(q, k, v, log_alpha, b, w, S0=None)          -> (o, S_T)
+    gdr2_bwd(q, k, v, log_alpha, b, w, S0, dO, dS_T=None) -> dict of gradients
+    gdr_block_prologue(xq, xk, xv, wq, wk, wv, ...)       -> (q, k, v)
+    gdr_block_epilogue(o, g, weight, eps)                 -> y
 """
 import ctypes
 import os
@@ -38,6 +41,8 @@ SIGNATURES = {
     "gdr2_fwd_workspace_bytes": (_SZ, [_I] * 6),
     "gdr2_bwd": (_I, [_I] * 6 + [_P] * 16 + [_P, _SZ, _P]),
     "gdr2_bwd_workspace_bytes": (_SZ, [_I] * 6),
+    "gdr_block_prologue": (_I, [_I] * 7 + [_P] * 11 + [ctypes.c_float] + [_P] * 3 + [_P]),
+    "gdr_block_epilogue": (_I, [_I] * 5 + [_P] * 3 + [ctypes.c_float, _P, _P]),
     "gdr_check_status": (_I, [_P]),
     "gdr_debug_wait_timeout": (_I, [_I, _P]),
     "gdr_last_error_string": (ctypes.c_char_p, []),
@@ -203,3 +208,39 @@ def gdr2_bwd(q, k, v, log_alpha, b, w, S0, dO, dS_T=None, *, want_dS0=True, work
                      _ptr(out["dlog_alpha"]), _ptr(out["db"]), _ptr(out["dw"]), _ptr(out["dS0"]),
                      _ptr(ws), ws_bytes, _stream(q)))
     return out
+
+
+def gdr_block_prologue(xq, xk, xv, wq, wk, wv, bq=None, bk=None, bv=None, *, conv_state=None,
+                       conv_state_out=None, eps=1e-6, q=None, k=None, v=None):
+    """The block's q/k/v paths after the input projections: depthwise causal
+    ShortConv (taps w* [H*d, K] fp32, biases b* [H*d] or None), SiLU, and L2
+    normalisation of q and k per (token, head).  xq, xk [B,T,H,dk]; xv
+    [B,T,H,dv].  conv_state [B, K-1, H*(2dk+dv)] (dtype of x, channels q, k,
+    v) carries the inputs before token 0; conv_state_out receives the last
+    K-1 inputs and may be conv_state itself.  Returns (q, k, v)."""
+    B, T, H, dk = xq.shape
+    dv = xv.shape[-1]
+    K = wq.shape[-1]
+    dt = _dt(xq)
+    for name, t in (("wq", wq), ("wk", wk), ("wv", wv), ("bq", bq), ("bk", bk), ("bv", bv)):
+        _f32(t, name)
+    q = torch.empty_like(xq) if q is None else q
+    k = torch.empty_like(xk) if k is None else k
+    v = torch.empty_like(xv) if v is None else v
+    check(lib().gdr_block_prologue(B, T, H, dk, dv, K, dt, _ptr(xq), _ptr(xk), _ptr(xv), _ptr(wq),
+                                   _ptr(wk), _ptr(wv), _ptr(bq), _ptr(bk), _ptr(bv),
+                                   _ptr(conv_state), _ptr(conv_state_out), float(eps), _ptr(q),
+                                   _ptr(k), _ptr(v), _stream(xq)))
+    return q, k, v
+
+
+def gdr_block_epilogue(o, g, weight, eps=1e-6, *, y=None):
+    """RMSNorm of the recurrent output over dv per (token, head), times the
+    per-channel weight [dv] fp32 and SiLU(g) (g None: no gate).  o, g
+    [B,T,H,dv].  Returns y."""
+    B, T, H, dv = o.shape
+    _f32(weight, "weight")
+    y = torch.empty_like(o) if y is None else y
+    check(lib().gdr_block_epilogue(B, T, H, dv, _dt(o), _ptr(o), _ptr(g), _ptr(weight), float(eps),
+                                   _ptr(y), _stream(o)))
+    return y

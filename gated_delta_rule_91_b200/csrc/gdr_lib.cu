@@ -14,6 +14,7 @@
 #include "step_kernel.cuh"
 #include "fwd_simt.cuh"
 #include "bwd_simt.cuh"
+#include "block.cuh"
 #include "gdr2_simt.cuh"
 #include "fwd_tc.cuh"
 #include "fwd_tc2.cuh"
@@ -352,6 +353,64 @@ gdr_status gdr2_bwd(int B, int T, int H, int dk, int dv, gdr_dtype dt, const voi
         e = dk == 128 ? launch_bwd2_simt<__nv_bfloat16, 128>(GDR2_BWD_ARGS)
                       : launch_bwd2_simt<__nv_bfloat16, 64>(GDR2_BWD_ARGS);
 #undef GDR2_BWD_ARGS
+    if (e != cudaSuccess) return cuda_fail(e, fn);
+    return GDR_OK;
+}
+
+gdr_status gdr_block_prologue(int B, int T, int H, int dk, int dv, int K, gdr_dtype dt, const void *xq,
+                              const void *xk, const void *xv, const float *wq, const float *wk,
+                              const float *wv, const float *bq, const float *bk, const float *bv,
+                              const void *conv_state_in, void *conv_state_out, float eps, void *q, void *k,
+                              void *v, gdr_stream_t stream) {
+    const char *fn = "gdr_block_prologue";
+    gdr_status st = check_dims(fn, B, T, H, dk, dv, dt);
+    if (st != GDR_OK) return st;
+    if (K < 1 || K > kConvMax)
+        return fail(GDR_ERR_UNSUPPORTED, "%s: conv width K=%d (supported: 1..%d)", fn, K, kConvMax);
+    if (!(eps >= 0.f) || eps > 1e30f) return fail(GDR_ERR_INVALID_ARGUMENT, "%s: eps=%g", fn, (double)eps);
+    GDR_REQUIRE_PTR(xq);
+    GDR_REQUIRE_PTR(xk);
+    GDR_REQUIRE_PTR(xv);
+    GDR_REQUIRE_PTR(wq);
+    GDR_REQUIRE_PTR(wk);
+    GDR_REQUIRE_PTR(wv);
+    GDR_OPTIONAL_PTR(bq);
+    GDR_OPTIONAL_PTR(bk);
+    GDR_OPTIONAL_PTR(bv);
+    GDR_OPTIONAL_PTR(conv_state_in);
+    GDR_OPTIONAL_PTR(conv_state_out);
+    GDR_REQUIRE_PTR(q);
+    GDR_REQUIRE_PTR(k);
+    GDR_REQUIRE_PTR(v);
+    PrologueArgs a{};
+    a.B = B; a.T = T; a.H = H; a.dk = dk; a.dv = dv; a.K = K;
+    a.x[0] = xq; a.x[1] = xk; a.x[2] = xv;
+    a.w[0] = wq; a.w[1] = wk; a.w[2] = wv;
+    a.bias[0] = bq; a.bias[1] = bk; a.bias[2] = bv;
+    a.state_in = K > 1 ? conv_state_in : nullptr;
+    a.state_out = K > 1 ? conv_state_out : nullptr;
+    a.eps = eps;
+    a.y[0] = q; a.y[1] = k; a.y[2] = v;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = dt == GDR_F32 ? launch_prologue<float>(a, s) : launch_prologue<__nv_bfloat16>(a, s);
+    if (e != cudaSuccess) return cuda_fail(e, fn);
+    return GDR_OK;
+}
+
+gdr_status gdr_block_epilogue(int B, int T, int H, int dv, gdr_dtype dt, const void *o, const void *g,
+                              const float *weight, float eps, void *y, gdr_stream_t stream) {
+    const char *fn = "gdr_block_epilogue";
+    gdr_status st = check_dims(fn, B, T, H, 64, dv, dt);
+    if (st != GDR_OK) return st;
+    if (!(eps >= 0.f) || eps > 1e30f) return fail(GDR_ERR_INVALID_ARGUMENT, "%s: eps=%g", fn, (double)eps);
+    GDR_REQUIRE_PTR(o);
+    GDR_OPTIONAL_PTR(g);
+    GDR_REQUIRE_PTR(weight);
+    GDR_REQUIRE_PTR(y);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const long long rows = (long long)B * T * H;
+    cudaError_t e = dt == GDR_F32 ? launch_epilogue<float>(rows, dv, o, g, weight, eps, y, s)
+                                  : launch_epilogue<__nv_bfloat16>(rows, dv, o, g, weight, eps, y, s);
     if (e != cudaSuccess) return cuda_fail(e, fn);
     return GDR_OK;
 }

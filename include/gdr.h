@@ -197,6 +197,59 @@ GDR_API gdr_status gdr2_bwd(int B, int T, int H, int dk, int dv, gdr_dtype dt,
                     void *workspace, size_t workspace_bytes, gdr_stream_t stream);
 GDR_API size_t gdr2_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, gdr_dtype dt);
 
+/*
+ * Block prologue: the q/k/v paths of a Gated DeltaNet block between the input
+ * projections and the recurrence, one pass over HBM.
+ *     q = L2(SiLU(ShortConv(xq))),  k = L2(SiLU(ShortConv(xk))),
+ *     v = SiLU(ShortConv(xv))
+ * Source: the Gated DeltaNet review (meaningful96.github.io/nr/GDN), section
+ * 3.8 "Gated DeltaNet Block", and the block-design paragraph of "Gated
+ * DeltaNet-2: Decoupling Erase and Write in Linear Attention"
+ * (agihunt.info/papers/2605.22791).  The pages fix no widths or epsilons:
+ *   * ShortConv is a depthwise causal convolution along time of width K
+ *     (1..8), in a framework Conv1d's cross-correlation convention:
+ *         z[t, c] = bias[c] + sum_{j<K} w[c, j] * x[t-K+1+j, c],
+ *     tokens before the first coming from the carried conv state;
+ *   * SiLU(z) = z / (1 + exp(-z));
+ *   * L2(y) = y / sqrt(sum y^2 + eps) over each head's d channels, per token.
+ *   in : xq, xk [B,T,H,dk]; xv [B,T,H,dv] (dtype dt): the projected inputs.
+ *        wq, wk [H*dk, K]; wv [H*dv, K] fp32 conv taps (row = channel h*d+i).
+ *        bq, bk [H*dk]; bv [H*dv] fp32 conv biases; each may be NULL (zero).
+ *        conv_state_in [B, K-1, H*(2*dk+dv)] (dtype dt; channels ordered q,
+ *        k, v): the K-1 inputs before token 0, oldest first; NULL = zeros.
+ *        eps >= 0 (0 is the plain definition; an all-zero head then gives NaN).
+ *   out: q, k [B,T,H,dk]; v [B,T,H,dv] (dtype dt).
+ *        conv_state_out (layout of conv_state_in, may be NULL): the last K-1
+ *        inputs of the concatenation (conv_state_in, x), for the next segment
+ *        or decode token.  It MAY equal conv_state_in (in-place update).
+ *   Both states are ignored when K = 1.  Other outputs must not alias inputs.
+ *   Errors: K outside 1..8 or the common size rules -> GDR_ERR_UNSUPPORTED;
+ *   negative or non-finite eps -> GDR_ERR_INVALID_ARGUMENT.
+ */
+GDR_API gdr_status gdr_block_prologue(int B, int T, int H, int dk, int dv, int K, gdr_dtype dt,
+                              const void *xq, const void *xk, const void *xv,
+                              const float *wq, const float *wk, const float *wv,
+                              const float *bq, const float *bk, const float *bv,
+                              const void *conv_state_in, void *conv_state_out, float eps,
+                              void *q, void *k, void *v, gdr_stream_t stream);
+
+/*
+ * Block epilogue: the recurrent output's normalisation and output gate, one
+ * pass over HBM (same sources as gdr_block_prologue):
+ *     y = o / sqrt(mean_i o_i^2 + eps) * weight * SiLU(g)
+ * per (token, head) over the dv channels.  The output projection that follows
+ * is a plain matrix product and not part of this library.
+ *   in : o [B,T,H,dv] (dtype dt, the output of gdr_fwd / gdr2_fwd);
+ *        g [B,T,H,dv] (dtype dt) the output-gate projection, or NULL for a
+ *        plain RMSNorm; weight [dv] fp32, shared by all heads; eps >= 0.
+ *   out: y [B,T,H,dv] (dtype dt); must not alias o or g.
+ *   Errors: dv not 64 or 128 and the common size rules -> GDR_ERR_UNSUPPORTED;
+ *   negative or non-finite eps -> GDR_ERR_INVALID_ARGUMENT.
+ */
+GDR_API gdr_status gdr_block_epilogue(int B, int T, int H, int dv, gdr_dtype dt, const void *o,
+                              const void *g, const float *weight, float eps, void *y,
+                              gdr_stream_t stream);
+
 /* Synchronise `stream`, then read and clear the device status word that
  * kernels set when a bounded wait gives up (GDR_ERR_TIMEOUT) or when
  * gdr2_bwd meets a chunk it does not handle (GDR_ERR_UNSUPPORTED).  Returns

@@ -17,6 +17,15 @@ distributions:
   b = sigmoid(N(0,1)) per key channel, write gate w = sigmoid(N(0,1)) per
   value channel, all fp32.
 
+* Block prologue/epilogue (the pre- and post-processing of the Gated
+  DeltaNet block): projected inputs xq, xk, xv ~ N(0,1) in the storage dtype;
+  ShortConv taps ~ U(-1/sqrt(K), 1/sqrt(K)) fp32 (the usual fan-in bound of a
+  depthwise convolution), biases ~ U(-1/sqrt(K), 1/sqrt(K)) fp32 or none, conv
+  state ~ N(0,1) in the storage dtype or none; recurrent output o ~ N(0, 0.1^2)
+  and gate projection g ~ N(0,1) in the storage dtype, norm weight
+  1 + N(0, 0.1^2) fp32.  Draw order: xq, xk, xv, wq, wk, wv, bq, bk, bv,
+  state; and o, g, weight.
+
 Draw order from one torch CPU Generator seeded with `seed`:
 q, k, v, x_alpha, x_beta, S0, dO for the scalar-gate rule;
 q, k, v, x_alpha (per channel), S0, b, w for Gated DeltaNet-2.
@@ -102,6 +111,35 @@ def gdr2_inputs(B: int, T: int, H: int, dk: int, dv: int, dtype: str = "bf16",
     b = b_max * torch.sigmoid(torch.randn(B, T, H, dk, generator=g))
     w = torch.sigmoid(torch.randn(B, T, H, dv, generator=g))
     return dict(q=q, k=k, v=v, log_alpha=log_alpha, b=b, w=w, S0=S0)
+
+
+def block_prologue_inputs(B: int, T: int, H: int, dk: int, dv: int, K: int, dtype: str = "bf16",
+                          seed: int = 0, bias: bool = True, state: bool = True) -> dict:
+    """Inputs of the block prologue (see the module docstring)."""
+    g = torch.Generator().manual_seed(seed)
+    dt = DTYPES[dtype]
+    bound = 1.0 / K ** 0.5
+    out = {}
+    for n, d in (("xq", dk), ("xk", dk), ("xv", dv)):
+        out[n] = torch.randn(B, T, H, d, generator=g).to(dt)
+    for n, d in (("wq", dk), ("wk", dk), ("wv", dv)):
+        out[n] = (torch.rand(H * d, K, generator=g) * 2 - 1) * bound
+    for n, d in (("bq", dk), ("bk", dk), ("bv", dv)):
+        out[n] = (torch.rand(H * d, generator=g) * 2 - 1) * bound if bias else None
+    out["conv_state"] = (torch.randn(B, K - 1, H * (2 * dk + dv), generator=g).to(dt)
+                         if state and K > 1 else None)
+    return out
+
+
+def block_epilogue_inputs(B: int, T: int, H: int, dv: int, dtype: str = "bf16", seed: int = 0,
+                          gate: bool = True) -> dict:
+    """Inputs of the block epilogue (see the module docstring)."""
+    g = torch.Generator().manual_seed(seed)
+    dt = DTYPES[dtype]
+    o = (0.1 * torch.randn(B, T, H, dv, generator=g)).to(dt)
+    gg = torch.randn(B, T, H, dv, generator=g).to(dt)
+    weight = 1.0 + 0.1 * torch.randn(dv, generator=g)
+    return {"o": o, "g": gg if gate else None, "weight": weight}
 
 
 def decode_state(B: int, H: int, dk: int, dv: int, seed: int, std: float = 0.02) -> torch.Tensor:

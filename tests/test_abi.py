@@ -78,3 +78,49 @@ def test_python_binding_refuses_cpu_tensors():
 def test_valid_arguments_without_gpu_report_cuda_error():
     # arguments pass validation; the launch then fails cleanly with no device
     assert _fwd() == gdr.GDR_ERR_CUDA
+
+
+def _prologue(B=1, T=4, H=1, dk=64, dv=64, K=4, dt=gdr.GDR_BF16, x=FAKE, w=FAKE, bias=None,
+              st=None, so=None, eps=1e-6, y=FAKE):
+    P = ctypes.c_void_p
+    return gdr.lib().gdr_block_prologue(B, T, H, dk, dv, K, dt, P(x), P(x), P(x), P(w), P(w), P(w),
+                                        P(bias), P(bias), P(bias), P(st), P(so), eps, P(y), P(y),
+                                        P(y), None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(B=0), gdr.GDR_ERR_INVALID_ARGUMENT),
+    (dict(K=0), gdr.GDR_ERR_UNSUPPORTED),
+    (dict(K=9), gdr.GDR_ERR_UNSUPPORTED),
+    (dict(dk=96), gdr.GDR_ERR_UNSUPPORTED),
+    (dict(dt=3), gdr.GDR_ERR_UNSUPPORTED),
+    (dict(eps=-1.0), gdr.GDR_ERR_INVALID_ARGUMENT),
+    (dict(eps=float("nan")), gdr.GDR_ERR_INVALID_ARGUMENT),
+    (dict(eps=float("inf")), gdr.GDR_ERR_INVALID_ARGUMENT),
+    (dict(x=None), gdr.GDR_ERR_INVALID_ARGUMENT),
+    (dict(w=None), gdr.GDR_ERR_INVALID_ARGUMENT),
+    (dict(y=FAKE + 2), gdr.GDR_ERR_INVALID_ARGUMENT),
+    (dict(st=FAKE + 8), gdr.GDR_ERR_INVALID_ARGUMENT),
+    (dict(bias=FAKE + 4), gdr.GDR_ERR_INVALID_ARGUMENT),
+])
+def test_prologue_rejects_bad_arguments(kw, status):
+    assert _prologue(**kw) == status
+    assert gdr.lib().gdr_last_error_string().decode().startswith("gdr_block_prologue")
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(T=0), gdr.GDR_ERR_INVALID_ARGUMENT),
+    (dict(dv=256), gdr.GDR_ERR_UNSUPPORTED),
+    (dict(eps=-0.5), gdr.GDR_ERR_INVALID_ARGUMENT),
+    (dict(o=None), gdr.GDR_ERR_INVALID_ARGUMENT),
+    (dict(weight=None), gdr.GDR_ERR_INVALID_ARGUMENT),
+    (dict(g=FAKE + 8), gdr.GDR_ERR_INVALID_ARGUMENT),
+])
+def test_epilogue_rejects_bad_arguments(kw, status):
+    a = dict(B=1, T=4, H=1, dv=64, dt=gdr.GDR_BF16, o=FAKE, g=None, weight=FAKE, eps=1e-6, y=FAKE)
+    a.update(kw)
+    P = ctypes.c_void_p
+    st = gdr.lib().gdr_block_epilogue(a["B"], a["T"], a["H"], a["dv"], a["dt"], P(a["o"]),
+                                      P(a["g"]), P(a["weight"]), a["eps"], P(a["y"]), None)
+    assert st == status
+    assert gdr.lib().gdr_last_error_string().decode().startswith("gdr_block_epilogue")

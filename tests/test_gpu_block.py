@@ -1,0 +1,193 @@
+"""GPU parity of the block prologue (ShortConv -> SiLU -> L2 on q, k; ShortConv
+-> SiLU on v) and epilogue (RMSNorm * weight * SiLU(g)) against the fp64
+oracle, through the C ABI.
+
+Tolerance (elementwise; the pages state none for these steps): the kernels
+compute in fp32 from the stored inputs and round once to the output dtype, so
+|gpu - ref| <= 2^-8 |ref| + 2^-12 max|ref| for bf16 outputs (half an ulp of
+bf16 is 2^-9 relative) and 1e-5 |ref| + 1e-6 max|ref| for fp32 outputs.  The
+carried conv state is a copy of inputs and must match bit for bit."""
+import numpy as np
+import pytest
+import torch
+
+import gated_delta_rule_91_b200 as gdr
+import oracle
+import synth
+from gpu_common import dev, np64
+
+pytestmark = pytest.mark.gpu
+
+
+def assert_close(got, ref, dtype):
+    got = np64(got) if isinstance(got, torch.Tensor) else np.asarray(got)
+    ref = np.asarray(ref, dtype=np.float64)
+    scale = max(float(np.max(np.abs(ref))), 1e-30)
+    if dtype == "bf16":
+        bound = 2.0 ** -8 * np.abs(ref) + 2.0 ** -12 * scale
+    else:
+        bound = 1e-5 * np.abs(ref) + 1e-6 * scale
+    err = np.abs(got - ref)
+    bad = err > bound
+    assert not bad.any(), "%d of %d elements off; worst %.3e at %s (ref %.3e)" % (
+        bad.sum(), bad.size, err.max(), np.unravel_index(np.argmax(err - bound), err.shape),
+        ref.flat[np.argmax(err - bound)])
+
+
+def oracle_prologue(x, eps):
+    """Per-stream oracle results and the concatenated next conv state."""
+    H, dk = x["xq"].shape[2], x["xq"].shape[3]
+    st = x["conv_state"]
+    outs, states = [], []
+    off = 0
+    for s, (xn, wn, bn) in enumerate((("xq", "wq", "bq"), ("xk", "wk", "bk"), ("xv", "wv", "bv"))):
+        d = x[xn].shape[-1]
+        sl = None if st is None else np64(st[:, :, off:off + H * d])
+        y, so = oracle.short_conv(np64(x[xn]), np64(x[wn]), np64(x[bn]), sl, l2=s < 2, eps=eps)
+        outs.append(y)
+        states.append(so)
+        off += H * d
+    return outs, np.concatenate(states, axis=-1)
+
+
+def run_prologue(x, eps, state_out=None, inplace=False):
+    d = {k: dev(v) for k, v in x.items()}
+    st = d["conv_state"]
+    if inplace:
+        state_out = st
+    q, k, v = gdr.gdr_block_prologue(d["xq"], d["xk"], d["xv"], d["wq"], d["wk"], d["wv"], d["bq"],
+                                     d["bk"], d["bv"], conv_state=st, conv_state_out=state_out,
+                                     eps=eps)
+    gdr.check_status()
+    return q, k, v
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("dk,dv", [(128, 128), (64, 64), (64, 128), (128, 64)])
+@pytest.mark.parametrize("T", [1, 3, 64, 130])
+def test_prologue_small(dtype, dk, dv, T):
+    B, H, K = 2, 3, 4
+    x = synth.block_prologue_inputs(B, T, H, dk, dv, K, dtype, seed=T + dk + 7 * dv)
+    ref, ref_state = oracle_prologue(x, 1e-6)
+    so = torch.empty(B, K - 1, H * (2 * dk + dv), dtype=x["xq"].dtype, device="cuda")
+    outs = run_prologue(x, 1e-6, state_out=so)
+    for got, r in zip(outs, ref):
+        assert_close(got, r, dtype)
+    np.testing.assert_array_equal(np64(so), ref_state)
+
+
+@pytest.mark.parametrize("K", [1, 2, 3, 5, 8])
+@pytest.mark.parametrize("bias,state", [(True, True), (False, False), (True, False)])
+def test_prologue_conv_widths(K, bias, state):
+    B, T, H, dk, dv = 2, 70, 2, 128, 128
+    x = synth.block_prologue_inputs(B, T, H, dk, dv, K, "bf16", seed=K, bias=bias, state=state)
+    ref, ref_state = oracle_prologue(x, 0.0)
+    so = (torch.empty(B, K - 1, H * (2 * dk + dv), dtype=torch.bfloat16, device="cuda")
+          if K > 1 else None)
+    outs = run_prologue(x, 0.0, state_out=so)
+    for got, r in zip(outs, ref):
+        assert_close(got, r, "bf16")
+    if K > 1:
+        np.testing.assert_array_equal(np64(so), ref_state)
+
+
+@pytest.mark.parametrize("T", [1, 2, 200])
+def test_prologue_in_place_state(T):
+    # conv_state_out == conv_state: decode (T = 1), T < K-1, and a long segment
+    B, H, dk, dv, K = 3, 2, 128, 64, 4
+    x = synth.block_prologue_inputs(B, T, H, dk, dv, K, "bf16", seed=100 + T)
+    ref, ref_state = oracle_prologue(x, 1e-6)
+    d = {k: dev(v) for k, v in x.items()}
+    st = d["conv_state"]
+    q, k, v = gdr.gdr_block_prologue(d["xq"], d["xk"], d["xv"], d["wq"], d["wk"], d["wv"], d["bq"],
+                                     d["bk"], d["bv"], conv_state=st, conv_state_out=st, eps=1e-6)
+    gdr.check_status()
+    for got, r in zip((q, k, v), ref):
+        assert_close(got, r, "bf16")
+    np.testing.assert_array_equal(np64(st), ref_state)
+
+
+def test_prologue_decode_chain_matches_one_pass():
+    # A prefill of 37 tokens then 5 decode tokens through the carried state is
+    # bit-identical to one pass over 42 tokens.
+    B, H, dk, dv, K, T = 2, 4, 128, 128, 4, 42
+    x = synth.block_prologue_inputs(B, T, H, dk, dv, K, "bf16", seed=5)
+    d = {k: dev(v) for k, v in x.items()}
+    full = gdr.gdr_block_prologue(d["xq"], d["xk"], d["xv"], d["wq"], d["wk"], d["wv"], d["bq"],
+                                  d["bk"], d["bv"], conv_state=d["conv_state"], eps=1e-6)
+    st = d["conv_state"].clone()
+    pieces = [[], [], []]
+    for a, b in [(0, 37)] + [(t, t + 1) for t in range(37, 42)]:
+        xs = [d[n][:, a:b].contiguous() for n in ("xq", "xk", "xv")]
+        outs = gdr.gdr_block_prologue(*xs, d["wq"], d["wk"], d["wv"], d["bq"], d["bk"], d["bv"],
+                                      conv_state=st, conv_state_out=st, eps=1e-6)
+        for i in range(3):
+            pieces[i].append(outs[i])
+    gdr.check_status()
+    for i in range(3):
+        assert torch.equal(torch.cat(pieces[i], dim=1), full[i])
+
+
+def test_prologue_zero_input_gives_zero():
+    B, T, H, d, K = 1, 5, 2, 128, 4
+    z = torch.zeros(B, T, H, d, dtype=torch.bfloat16, device="cuda")
+    w = torch.ones(H * d, K, device="cuda")
+    q, k, v = gdr.gdr_block_prologue(z, z, z, w, w, w, eps=1e-6)
+    gdr.check_status()
+    for t in (q, k, v):
+        assert torch.count_nonzero(t) == 0
+
+
+def test_prologue_workload_sampled_windows():
+    # The full block shape (B4 T4096 H16 d128 bf16, K = 4) in the launch the
+    # bench times; the oracle checks windows of tokens, each fed the K-1
+    # preceding inputs as its carried state.
+    B, T, H, dk, dv, K = 4, 4096, 16, 128, 128, 4
+    x = synth.block_prologue_inputs(B, T, H, dk, dv, K, "bf16", seed=11, state=False)
+    outs = run_prologue(x, 1e-6)
+    for t0, L in ((0, 70), (1000, 40), (4096 - 67, 67)):
+        for s, (xn, wn, bn) in enumerate((("xq", "wq", "bq"), ("xk", "wk", "bk"),
+                                           ("xv", "wv", "bv"))):
+            xs = np64(x[xn])
+            st = None
+            if t0 > 0:
+                st = xs[:, t0 - (K - 1):t0].reshape(B, K - 1, -1)
+            y, _ = oracle.short_conv(xs[:, t0:t0 + L], np64(x[wn]), np64(x[bn]), st, l2=s < 2,
+                                     eps=1e-6)
+            assert_close(outs[s][:, t0:t0 + L], y, "bf16")
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("dv", [64, 128])
+@pytest.mark.parametrize("gate", [True, False])
+@pytest.mark.parametrize("T", [1, 77])
+def test_epilogue_small(dtype, dv, gate, T):
+    x = synth.block_epilogue_inputs(2, T, 3, dv, dtype, seed=dv + T, gate=gate)
+    ref = oracle.rmsnorm_gate(np64(x["o"]), np64(x["g"]), np64(x["weight"]), 1e-6)
+    y = gdr.gdr_block_epilogue(dev(x["o"]), dev(x["g"]), dev(x["weight"]), 1e-6)
+    gdr.check_status()
+    assert_close(y, ref, dtype)
+
+
+def test_epilogue_workload_full():
+    x = synth.block_epilogue_inputs(4, 4096, 16, 128, "bf16", seed=3)
+    ref = oracle.rmsnorm_gate(np64(x["o"]), np64(x["g"]), np64(x["weight"]), 1e-6)
+    y = gdr.gdr_block_epilogue(dev(x["o"]), dev(x["g"]), dev(x["weight"]), 1e-6)
+    gdr.check_status()
+    assert_close(y, ref, "bf16")
+
+
+def test_epilogue_zero_rows():
+    o = torch.zeros(1, 3, 2, 128, dtype=torch.bfloat16, device="cuda")
+    y = gdr.gdr_block_epilogue(o, torch.ones_like(o), torch.ones(128, device="cuda"), 1e-6)
+    gdr.check_status()
+    assert torch.count_nonzero(y) == 0
+
+
+def test_block_kernels_count_launches():
+    x = synth.block_prologue_inputs(1, 10, 1, 64, 64, 4, "bf16", seed=1)
+    before = gdr.launch_count()
+    run_prologue(x, 1e-6)
+    e = synth.block_epilogue_inputs(1, 10, 1, 64, "bf16", seed=1)
+    gdr.gdr_block_epilogue(dev(e["o"]), dev(e["g"]), dev(e["weight"]))
+    assert gdr.launch_count() - before == 2
