@@ -58,7 +58,30 @@ def parse_args():
                         "(a short command for profilers) and exit")
     p.add_argument("--profile-gdn2", metavar="B,T,H", default=None,
                    help="only run gdr2_fwd twice on seeded bf16 d=128 inputs of this shape and exit")
+    p.add_argument("--profile-block", metavar="B,T,H", default=None,
+                   help="only run the block prologue (K=4) and epilogue twice each on seeded bf16 "
+                        "d=128 inputs of this shape and exit")
     return p.parse_args()
+
+
+def profile_block(shape):
+    """Two block prologue calls (ShortConv K=4, SiLU, q/k L2) and two block
+    epilogue calls (RMSNorm, SiLU gate) on the seeded block recipe, bf16,
+    d = 128, then a status check."""
+    import gated_delta_rule_91_b200 as gdr
+    B, T, H = (int(x) for x in shape.split(","))
+    px = {n: (t.cuda() if t is not None else None)
+          for n, t in synth.block_prologue_inputs(B, T, H, 128, 128, 4, "bf16", seed=21, state=False).items()}
+    ex = {n: (t.cuda() if t is not None else None)
+          for n, t in synth.block_epilogue_inputs(B, T, H, 128, "bf16", seed=22).items()}
+    for _ in range(2):
+        gdr.gdr_block_prologue(px["xq"], px["xk"], px["xv"], px["wq"], px["wk"], px["wv"], px["bq"],
+                               px["bk"], px["bv"], eps=1e-6)
+    for _ in range(2):
+        gdr.gdr_block_epilogue(ex["o"], ex["g"], ex["weight"], 1e-6)
+    torch.cuda.synchronize()
+    gdr.check_status()
+    print(json.dumps({"profile_block": shape, "status": "ok"}))
 
 
 def profile_gdn2(shape):
@@ -495,6 +518,9 @@ def main():
         return
     if args.profile_gdn2:
         profile_gdn2(args.profile_gdn2)
+        return
+    if args.profile_block:
+        profile_block(args.profile_block)
         return
     rank, world, local = dist_init(args)
     if args.impl == "reference":

@@ -26,13 +26,13 @@
 
 #include "common.cuh"
 #include "sm100.cuh"
+#include "fwd_tc.cuh"  // encode_tiled_fn
 
 namespace gdr {
 
 constexpr int kBlkThreads = 256;  // 8 warps
 constexpr int kConvMax = 8;       // widest ShortConv handled
 constexpr int kPrologueRun = 64;  // tokens per prologue work unit
-constexpr int kEpilogueRows = 8;    // rows per epilogue work unit
 
 // ---- CPL consecutive elements per lane ---------------------------------------
 template <int CPL> __device__ __forceinline__ void ld_row(const float *p, float *o) {
@@ -75,36 +75,9 @@ template <int CPL> __device__ __forceinline__ void st_row(__nv_bfloat16 *p, cons
     }
 }
 
-// A row slice kept packed in its storage type until it is used, so a batch of
-// bf16 rows in flight costs half the registers of the converted floats.
-template <typename Tio, int CPL> struct RawRow;
-template <> struct RawRow<float, 4> { float4 v; };
-template <> struct RawRow<float, 2> { float2 v; };
-template <> struct RawRow<__nv_bfloat16, 4> { uint2 v; };
-template <> struct RawRow<__nv_bfloat16, 2> { uint32_t v; };
-
-template <typename Tio, int CPL> __device__ __forceinline__ RawRow<Tio, CPL> ld_raw(const Tio *p) {
-    RawRow<Tio, CPL> r;
-    r.v = *reinterpret_cast<const decltype(r.v) *>(p);
-    return r;
-}
-__device__ __forceinline__ void unpack(const RawRow<float, 4> &r, float *o) {
-    o[0] = r.v.x; o[1] = r.v.y; o[2] = r.v.z; o[3] = r.v.w;
-}
-__device__ __forceinline__ void unpack(const RawRow<float, 2> &r, float *o) { o[0] = r.v.x; o[1] = r.v.y; }
-__device__ __forceinline__ void unpack(const RawRow<__nv_bfloat16, 4> &r, float *o) {
-    uint2 raw = r.v;
-    float2 a = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&raw.x));
-    float2 b = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&raw.y));
-    o[0] = a.x; o[1] = a.y; o[2] = b.x; o[3] = b.y;
-}
-__device__ __forceinline__ void unpack(const RawRow<__nv_bfloat16, 2> &r, float *o) {
-    uint32_t raw = r.v;
-    float2 a = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&raw));
-    o[0] = a.x; o[1] = a.y;
-}
-
-__device__ __forceinline__ float silu_f(float z) { return z / (1.f + __expf(-z)); }
+// SiLU with the fast divide: for z -> -inf the denominator overflows to +inf
+// and the quotient is -0, the limit of z / (1 + e^-z).
+__device__ __forceinline__ float silu_f(float z) { return __fdividef(z, 1.f + __expf(-z)); }
 
 // ---- prologue -------------------------------------------------------------------
 struct PrologueArgs {
@@ -118,31 +91,27 @@ struct PrologueArgs {
     void *y[3];          // q, k, v outputs, [B, T, H, d_s]
 };
 
-// A unit is one (stream, batch, head) and a run of kPrologueRun tokens.  Its
-// rows -- the K-1 tokens before the run, then the run -- are staged in shared
-// memory: row r holds token t0 - (K-1) + r, so output token t0 + i reads rows
-// i .. i+K-1.  Two stages: the next unit's bulk copies fly while this one is
-// computed.
+// Work split.  A block owns one (stream, head) pair -- its conv taps and
+// biases stay in registers -- and walks the (batch, run) units of that pair
+// with a stride; unit = kPrologueRun tokens of one batch.  The grid is the
+// 3H pairs times G blocks each; blocks with the same index on neighbouring
+// heads read the same tokens at about the same time (whole HBM rows).
+//
+// A unit's rows -- the K-1 tokens before the run, then the run -- arrive by
+// one tiled TMA load into a ring stage: row r holds token t0 - (K-1) + r, so
+// output token t0 + i reads rows i .. i+K-1.  Tokens before 0 or past T read
+// as zero; rows from a carried conv state are patched in after the load.
 constexpr int kPrologueRows = kPrologueRun + kConvMax - 1;
+constexpr int kBlkStages = 3;  // bulk-copy ring depth of the staged kernels
 
-struct PrologueUnit {
-    int s, b, h, t0, len, d;
-};
-
-__device__ __forceinline__ PrologueUnit prologue_decode(const PrologueArgs &a, long long u) {
-    const int runs = (a.T + kPrologueRun - 1) / kPrologueRun;
-    const long long per_stream = (long long)a.B * a.H * runs;
-    PrologueUnit p;
-    p.s = (int)(u / per_stream);
-    long long r = u - p.s * per_stream;
-    const int run = (int)(r % runs);
-    r /= runs;
-    p.h = (int)(r % a.H);
-    p.b = (int)(r / a.H);
-    p.t0 = run * kPrologueRun;
-    p.len = min(kPrologueRun, a.T - p.t0);
-    p.d = p.s < 2 ? a.dk : a.dv;
-    return p;
+// After a wait gave up at unit k (stage st): wait, with a short bound, for the
+// copies already issued into the other stages so that none lands after the
+// block has exited.
+__device__ __forceinline__ void blk_drain(uint64_t *bars, int st, int k, long long u, long long units,
+                                          long long stride) {
+    for (int m = 1; m < kBlkStages; ++m)
+        if (u + (long long)m * stride < units)
+            sm100::mbar_wait(&bars[(st + m) % kBlkStages], (uint32_t)((k + m) / kBlkStages) & 1u, 100000000ull);
 }
 
 // Stream pointers by selects (a runtime index into the parameter block would
@@ -156,201 +125,259 @@ __device__ __forceinline__ int prologue_state_col(const PrologueArgs &a, int s) 
     return s == 0 ? 0 : s == 1 ? a.H * a.dk : 2 * a.H * a.dk;
 }
 
-// Warp 0 stages unit p into `stage` (row bytes = d * sizeof(Tio), a multiple
-// of 128): bulk copies for tokens read from x or the old conv state, plain
-// zero stores for tokens before the start with no state.
-template <typename Tio>
-__device__ __forceinline__ void prologue_stage(const PrologueArgs &a, const PrologueUnit &p, uint8_t *stage,
-                                               uint64_t *bar, int lane) {
-    using namespace sm100;
-    const int K = a.K, rows = p.len + K - 1;
-    const uint32_t rb = (uint32_t)p.d * sizeof(Tio);
-    const int first = p.t0 - (K - 1);  // token of row 0
-    // bytes arriving by bulk copy
-    int zero_rows = 0;
-    if (first < 0 && a.state_in == nullptr) zero_rows = -first;
-    if (lane == 0) mbar_expect_tx(bar, (uint32_t)(rows - zero_rows) * rb);
-    __syncwarp();
-    const Tio *x = prologue_x<Tio>(a, p.s);
-    const int Ctot = a.H * (2 * a.dk + a.dv);
-    for (int r = lane; r < rows; r += 32) {
-        const int t = first + r;
-        uint8_t *dst = stage + (size_t)r * rb;
-        if (t >= 0) {
-            bulk_load_g2s(dst, x + (((size_t)p.b * a.T + t) * a.H + p.h) * p.d, rb, bar);
-        } else if (a.state_in) {
-            const Tio *st = static_cast<const Tio *>(a.state_in) +
-                            ((size_t)p.b * (K - 1) + (K - 1 + t)) * Ctot + prologue_state_col(a, p.s) + p.h * p.d;
-            bulk_load_g2s(dst, st, rb, bar);
-        } else {
-            for (uint32_t o = 0; o < rb; o += 16) *reinterpret_cast<uint4 *>(dst + o) = make_uint4(0, 0, 0, 0);
-        }
-    }
+__device__ __forceinline__ void store8(float *p, const float *v) {
+    reinterpret_cast<float4 *>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
+    reinterpret_cast<float4 *>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
+}
+__device__ __forceinline__ void store8(__nv_bfloat16 *p, const float *v) {
+    uint4 raw;
+    __nv_bfloat162 h0 = __floats2bfloat162_rn(v[0], v[1]), h1 = __floats2bfloat162_rn(v[2], v[3]);
+    __nv_bfloat162 h2 = __floats2bfloat162_rn(v[4], v[5]), h3 = __floats2bfloat162_rn(v[6], v[7]);
+    raw.x = *reinterpret_cast<uint32_t *>(&h0);
+    raw.y = *reinterpret_cast<uint32_t *>(&h1);
+    raw.z = *reinterpret_cast<uint32_t *>(&h2);
+    raw.w = *reinterpret_cast<uint32_t *>(&h3);
+    *reinterpret_cast<uint4 *>(p) = raw;
 }
 
-// Output rows of a staged unit: warp w takes rows w, w+8, ...; lane owns
-// CPL = d/32 channels.  KW (4 or 8) is the register window, K <= KW.
-template <typename Tio, int CPL, int KW>
-__device__ __forceinline__ void prologue_compute(const PrologueArgs &a, const PrologueUnit &p, const uint8_t *stage,
-                                                 int warp, int lane) {
-    constexpr int D = CPL * 32;
-    const int K = a.K;
-    const int c0 = p.h * D + lane * CPL;  // first channel of this lane in the stream
-    const float *wsel = p.s == 0 ? a.w[0] : p.s == 1 ? a.w[1] : a.w[2];
-    const float *bsel = p.s == 0 ? a.bias[0] : p.s == 1 ? a.bias[1] : a.bias[2];
-    Tio *y = static_cast<Tio *>(p.s == 0 ? a.y[0] : p.s == 1 ? a.y[1] : a.y[2]);
-    float wt[CPL][KW], bias[CPL];  // wt[c][j] multiplies row i + j
+// The block's part of the prologue for stream s, head h (D channels).  A lane
+// owns 8 channels and a group of D/8 lanes one row (the L2 norm is a
+// reduction inside the group); the groups of the block take consecutive row
+// blocks of the run and slide a K-row window down theirs, so each staged row
+// is read about once.  The window holds KW (4 or 8) rows with the taps
+// right-aligned: win[m] is row i + K - KW + m and taps m < KW - K are zero.
+// Every lane runs the same trip count (rows past the run are computed from
+// in-bounds stage memory and not stored), so the group shuffles always have
+// the full warp.
+template <typename Tio, int D, int KW>
+__device__ __forceinline__ void prologue_block(const PrologueArgs &a, const CUtensorMap *map, int s, int h, int idx,
+                                               int G, uint8_t *smem, int stage_bytes, uint64_t *bars) {
+    using namespace sm100;
+    constexpr int CPL = 8, LPR = D / CPL, GPW = 32 / LPR;
+    constexpr int RPG = kPrologueRun / ((kBlkThreads / 32) * GPW);  // rows per group
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int K = a.K, T = a.T;
+    const int runs = (T + kPrologueRun - 1) / kPrologueRun;
+    const int units = a.B * runs;  // (batch, run) units of this pair; B*T*H*d < 2^31 on the host
+    const int sl = lane % LPR, i0 = (warp * GPW + lane / LPR) * RPG;
+    const int c0 = h * D + sl * CPL;  // first channel of this lane in the stream
+    const uint32_t box_bytes = (uint32_t)(kPrologueRun + K - 1) * D * (uint32_t)sizeof(Tio);
+
+    // taps (right-aligned in the window) and biases of this lane's channels
+    const float *wsel = s == 0 ? a.w[0] : s == 1 ? a.w[1] : a.w[2];
+    const float *bsel = s == 0 ? a.bias[0] : s == 1 ? a.bias[1] : a.bias[2];
+    float wt[CPL][KW], bias[CPL];
 #pragma unroll
     for (int c = 0; c < CPL; ++c) {
 #pragma unroll
-        for (int j = 0; j < KW; ++j) wt[c][j] = j < K ? __ldg(wsel + (size_t)(c0 + c) * K + j) : 0.f;
+        for (int m = 0; m < KW; ++m) {
+            const int j = m - (KW - K);  // tap index
+            wt[c][m] = j >= 0 ? __ldg(wsel + (size_t)(c0 + c) * K + j) : 0.f;
+        }
         bias[c] = bsel ? __ldg(bsel + c0 + c) : 0.f;
     }
-    const Tio *sm = reinterpret_cast<const Tio *>(stage) + lane * CPL;
-    const bool l2 = p.s < 2;
+
+    // the ring: unit k of this block is (batch, run) idx + k*G, in stage
+    // k % kBlkStages with phase parity (k / kBlkStages) & 1
+    auto issue = [&](int k, int sidx) {  // one thread
+        const int j = idx + k * G, b = j / runs, t0 = (j % runs) * kPrologueRun;
+        mbar_expect_tx(&bars[sidx], box_bytes);
+        tma_load_4d(smem + sidx * stage_bytes, map, &bars[sidx], 0, h, t0 - (K - 1), b);
+    };
+    if (threadIdx.x == 0)
+        for (int k = 0; k < kBlkStages - 1; ++k)
+            if (idx + k * G < units) issue(k, k);
+    const bool l2 = s < 2;
+    const size_t ystride = (size_t)a.H * D;
+    Tio *ybase = static_cast<Tio *>(s == 0 ? a.y[0] : s == 1 ? a.y[1] : a.y[2]);
+    int st = 0;
 #pragma unroll 1
-    for (int i = warp; i < p.len; i += kBlkThreads / 32) {
-        float acc[CPL];
+    for (int k = 0;; ++k) {
+        const int j = idx + k * G;
+        if (j >= units) break;
+        const int b = j / runs, t0 = (j % runs) * kPrologueRun, len = min(kPrologueRun, T - t0);
+        // stage unit k + kBlkStages - 1 into the slot unit k - 1 used (its
+        // readers finished at the barrier that ended the previous iteration)
+        if (threadIdx.x == 0 && j + (kBlkStages - 1) * G < units) {
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            issue(k + kBlkStages - 1, st == 0 ? kBlkStages - 1 : st - 1);
+        }
+        if (!mbar_wait(&bars[st], (uint32_t)(k / kBlkStages) & 1u)) {
+            record_status(GDR_ERR_TIMEOUT);
+            blk_drain(bars, st, k, j, units, G);
+            return;
+        }
+        uint8_t *stage = smem + st * stage_bytes;
+        const int Ctot = a.H * (2 * a.dk + a.dv);
+        if (t0 == 0 && a.state_in != nullptr && K > 1) {
+            // rows 0 .. K-2 (read as zero by the TMA) take the old state's rows
+            constexpr int kPieces = D * (int)sizeof(Tio) / 16;
+            for (int i = threadIdx.x; i < (K - 1) * kPieces; i += kBlkThreads) {
+                const int r = i / kPieces, q = i % kPieces;
+                const Tio *src = static_cast<const Tio *>(a.state_in) + ((size_t)b * (K - 1) + r) * Ctot +
+                                 prologue_state_col(a, s) + h * D;
+                reinterpret_cast<uint4 *>(stage + (size_t)r * D * sizeof(Tio))[q] =
+                    reinterpret_cast<const uint4 *>(src)[q];
+            }
+            __syncthreads();
+        }
+
+        const Tio *sx = reinterpret_cast<const Tio *>(stage) + sl * CPL;
+        float win[KW][CPL];
 #pragma unroll
-        for (int c = 0; c < CPL; ++c) acc[c] = bias[c];
+        for (int m = 0; m < KW - 1; ++m) {
+            const int row = i0 + K - KW + m;
+            if (row >= 0)
+                load8(sx + row * D, win[m]);
+            else
 #pragma unroll
-        for (int j = 0; j < KW; ++j) {
-            if (j < K) {
-                float xv[CPL];
-                ld_row<CPL>(sm + (size_t)(i + j) * D, xv);
+                for (int c = 0; c < CPL; ++c) win[m][c] = 0.f;
+        }
+        Tio *y = ybase + (((size_t)b * T + t0 + i0) * a.H) * D + c0;
 #pragma unroll
-                for (int c = 0; c < CPL; ++c) acc[c] = fmaf(wt[c][j], xv[c], acc[c]);
+        for (int r = 0; r < RPG; ++r) {
+            load8(sx + (i0 + r + K - 1) * D, win[KW - 1]);
+            float acc[CPL], ss = 0.f;
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) {
+                float z = bias[c];
+#pragma unroll
+                for (int m = 0; m < KW; ++m) z = fmaf(wt[c][m], win[m][c], z);
+                acc[c] = silu_f(z);
+                ss = fmaf(acc[c], acc[c], ss);
+            }
+#pragma unroll
+            for (int m = 0; m < KW - 1; ++m)
+#pragma unroll
+                for (int c = 0; c < CPL; ++c) win[m][c] = win[m + 1][c];
+            if (l2) {
+#pragma unroll
+                for (int off = LPR / 2; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+                const float inv = rsqrtf(ss + a.eps);
+#pragma unroll
+                for (int c = 0; c < CPL; ++c) acc[c] *= inv;
+            }
+            if (i0 + r < len) store8(y + r * ystride, acc);
+        }
+
+        // The carried state of (stream, batch, head): the last K-1 inputs,
+        // written by the run-0 unit after its stage (holding the old state
+        // rows) is complete, so an in-place state is safe: no other unit reads
+        // the old state.
+        if (t0 == 0 && a.state_out != nullptr && K > 1) {
+            const Tio *x = prologue_x<Tio>(a, s);
+            Tio *so = static_cast<Tio *>(a.state_out) + (size_t)b * (K - 1) * Ctot + prologue_state_col(a, s) + h * D;
+            constexpr int kPieces = D * (int)sizeof(Tio) / 16;
+            for (int i = threadIdx.x; i < (K - 1) * kPieces; i += kBlkThreads) {
+                const int jr = i / kPieces, q = i % kPieces;
+                const int t = T - (K - 1) + jr;  // token held by state row jr
+                const uint4 *src = t < len ? reinterpret_cast<const uint4 *>(stage + (size_t)(t + K - 1) * D * sizeof(Tio))
+                                           : reinterpret_cast<const uint4 *>(x + (((size_t)b * T + t) * a.H + h) * D);
+                reinterpret_cast<uint4 *>(so + (size_t)jr * Ctot)[q] = src[q];
             }
         }
-        float ss = 0.f;
-#pragma unroll
-        for (int c = 0; c < CPL; ++c) {
-            acc[c] = silu_f(acc[c]);
-            ss = fmaf(acc[c], acc[c], ss);
-        }
-        if (l2) {
-            const float inv = rsqrtf(warp_sum(ss, 32) + a.eps);
-#pragma unroll
-            for (int c = 0; c < CPL; ++c) acc[c] *= inv;
-        }
-        st_row<CPL>(y + (((size_t)p.b * a.T + p.t0 + i) * a.H) * D + c0, acc);
+        __syncthreads();
+        st = st == kBlkStages - 1 ? 0 : st + 1;
     }
 }
 
-// The carried state of (stream, batch, head): the last K-1 inputs.  Written by
-// the run-0 unit after its stage (which holds the old state rows) is complete,
-// so an in-place state is safe: no other unit reads the old state.
-template <typename Tio, int CPL>
-__device__ __forceinline__ void prologue_state_out(const PrologueArgs &a, const PrologueUnit &p,
-                                                   const uint8_t *stage, int warp, int lane) {
-    constexpr int D = CPL * 32;
-    const int K = a.K, Ctot = a.H * (2 * a.dk + a.dv);
-    const Tio *sm = reinterpret_cast<const Tio *>(stage) + lane * CPL;
-    const Tio *x = prologue_x<Tio>(a, p.s);
-    Tio *so = static_cast<Tio *>(a.state_out) + (size_t)p.b * (K - 1) * Ctot + prologue_state_col(a, p.s) + p.h * D +
-              lane * CPL;
-    for (int j = warp; j < K - 1; j += kBlkThreads / 32) {
-        const int t = a.T - (K - 1) + j;  // token held by state row j
-        float v[CPL];
-        if (t < p.len)  // staged: row t + K - 1 (t >= -(K-1) always)
-            ld_row<CPL>(sm + (size_t)(t + K - 1) * D, v);
-        else
-            ld_row<CPL>(x + (((size_t)p.b * a.T + t) * a.H + p.h) * D + lane * CPL, v);
-        st_row<CPL>(so + (size_t)j * Ctot, v);
-    }
-}
-
-template <typename Tio, int CPLQK, int CPLV, int KW>
-__global__ void __launch_bounds__(kBlkThreads) gdr_prologue_kernel(const PrologueArgs a, int stage_bytes) {
+template <typename Tio, int DQK, int DV, int KW>
+__global__ void __launch_bounds__(kBlkThreads)
+    gdr_prologue_kernel(const PrologueArgs a, int stage_bytes, const __grid_constant__ CUtensorMap tm_q,
+                        const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v) {
     using namespace sm100;
     extern __shared__ __align__(128) uint8_t blk_smem[];
     uint8_t *smem = blk_smem;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + 2 * stage_bytes);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const long long units = 3LL * a.B * a.H * ((a.T + kPrologueRun - 1) / kPrologueRun);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kBlkStages * stage_bytes);
+    const int P = 3 * a.H, pair = blockIdx.x % P, idx = blockIdx.x / P, G = gridDim.x / P;
+    const int s = pair / a.H, h = pair % a.H;
     if (threadIdx.x == 0) {
-        mbar_init(&bars[0], 1);
-        mbar_init(&bars[1], 1);
+        for (int i = 0; i < kBlkStages; ++i) mbar_init(&bars[i], 1);
         fence_mbar_init();
     }
     __syncthreads();
-    long long u = blockIdx.x;
-    if (u < units && warp == 0) prologue_stage<Tio>(a, prologue_decode(a, u), smem, &bars[0], lane);
-    __syncthreads();  // zero-filled rows are plain stores: publish them to all warps
-#pragma unroll 1
-    for (int k = 0; u < units; ++k, u += gridDim.x) {
-        const int st = k & 1;
-        const PrologueUnit p = prologue_decode(a, u);
-        // stage the next unit into the other buffer (its readers finished at
-        // the barrier that ended the previous iteration)
-        const long long un = u + gridDim.x;
-        if (un < units && warp == 0) {
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            prologue_stage<Tio>(a, prologue_decode(a, un), smem + (st ^ 1) * stage_bytes, &bars[st ^ 1], lane);
-        }
-        if (!mbar_wait(&bars[st], (uint32_t)(k >> 1) & 1u)) {
-            record_status(GDR_ERR_TIMEOUT);
-            // let the copies already issued for the next unit land before the
-            // block exits
-            if (un < units) mbar_wait(&bars[st ^ 1], (uint32_t)((k + 1) >> 1) & 1u, 100000000ull);
-            return;
-        }
-        const uint8_t *stage = smem + st * stage_bytes;
-        if (p.s < 2)
-            prologue_compute<Tio, CPLQK, KW>(a, p, stage, warp, lane);
-        else
-            prologue_compute<Tio, CPLV, KW>(a, p, stage, warp, lane);
-        if (p.t0 == 0 && a.state_out != nullptr) {
-            if (p.s < 2)
-                prologue_state_out<Tio, CPLQK>(a, p, stage, warp, lane);
-            else
-                prologue_state_out<Tio, CPLV>(a, p, stage, warp, lane);
-        }
-        __syncthreads();
-    }
+    if (s == 0)
+        prologue_block<Tio, DQK, KW>(a, &tm_q, s, h, idx, G, smem, stage_bytes, bars);
+    else if (s == 1)
+        prologue_block<Tio, DQK, KW>(a, &tm_k, s, h, idx, G, smem, stage_bytes, bars);
+    else
+        prologue_block<Tio, DV, KW>(a, &tm_v, s, h, idx, G, smem, stage_bytes, bars);
 }
 
 // ---- epilogue ---------------------------------------------------------------------
 // y = o / sqrt(mean(o^2) + eps) * weight * SiLU(g) per row of dv channels;
-// g == nullptr leaves out the gate.  Rows are the B*T*H (token, head) pairs.
+// g == nullptr leaves out the gate.  Rows are the B*T*H (token, head) pairs,
+// contiguous in memory, so a unit of 64 rows of o (and of g) arrives by one
+// bulk copy each; a ring of kBlkStages units per block keeps copies in flight
+// while warps compute (warp w: rows 8w .. 8w+7 of the unit).
+constexpr int kEpilogueRows = 64;
+
 template <typename Tio, int CPL>
 __global__ void __launch_bounds__(kBlkThreads)
     gdr_epilogue_kernel(long long rows, const Tio *__restrict__ o, const Tio *__restrict__ g,
                         const float *__restrict__ weight, float eps, Tio *__restrict__ y) {
+    using namespace sm100;
     constexpr int D = CPL * 32;
-    const int lane = threadIdx.x & 31;
+    constexpr int kTile = kEpilogueRows * D * (int)sizeof(Tio);  // one tensor's unit
+    constexpr int kRowsPerWarp = kEpilogueRows / (kBlkThreads / 32);
+    extern __shared__ __align__(128) uint8_t blk_smem[];
+    uint8_t *smem = blk_smem;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kBlkStages * 2 * kTile);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long units = (rows + kEpilogueRows - 1) / kEpilogueRows;
+    auto issue = [&](long long uu, int sidx) {  // one thread
+        const long long r0 = uu * kEpilogueRows;
+        const uint32_t bytes = (uint32_t)min((long long)kEpilogueRows, rows - r0) * D * (uint32_t)sizeof(Tio);
+        mbar_expect_tx(&bars[sidx], g ? 2 * bytes : bytes);
+        bulk_load_g2s(smem + sidx * 2 * kTile, o + r0 * D, bytes, &bars[sidx]);
+        if (g) bulk_load_g2s(smem + sidx * 2 * kTile + kTile, g + r0 * D, bytes, &bars[sidx]);
+    };
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kBlkStages; ++i) mbar_init(&bars[i], 1);
+        fence_mbar_init();
+        for (int k = 0; k < kBlkStages - 1; ++k)
+            if (blockIdx.x + (long long)k * gridDim.x < units) issue(blockIdx.x + (long long)k * gridDim.x, k);
+    }
+    __syncthreads();
     float wl[CPL];
 #pragma unroll
     for (int c = 0; c < CPL; ++c) wl[c] = __ldg(weight + lane * CPL + c);
-    const long long units = (rows + kEpilogueRows - 1) / kEpilogueRows;
-    const long long nw = (long long)gridDim.x * (kBlkThreads / 32);
+    int st = 0;
 #pragma unroll 1
-    for (long long u = (blockIdx.x * (long long)kBlkThreads + threadIdx.x) >> 5; u < units; u += nw) {
+    for (int k = 0;; ++k) {
+        const long long u = blockIdx.x + (long long)k * gridDim.x;
+        if (u >= units) break;
+        const long long un = u + (long long)(kBlkStages - 1) * gridDim.x;
+        if (threadIdx.x == 0 && un < units) {
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            issue(un, st == 0 ? kBlkStages - 1 : st - 1);
+        }
+        if (!mbar_wait(&bars[st], (uint32_t)(k / kBlkStages) & 1u)) {
+            record_status(GDR_ERR_TIMEOUT);
+            blk_drain(bars, st, k, u, units, gridDim.x);
+            return;
+        }
+        const Tio *so = reinterpret_cast<const Tio *>(smem + st * 2 * kTile) + lane * CPL;
+        const Tio *sg = so + kTile / sizeof(Tio);
         const long long r0 = u * kEpilogueRows;
         const int n = (int)min((long long)kEpilogueRows, rows - r0);
-        const size_t base = (size_t)r0 * D + lane * CPL;
-        RawRow<Tio, CPL> orow[kEpilogueRows], grow[kEpilogueRows];
 #pragma unroll
-        for (int i = 0; i < kEpilogueRows; ++i) {
-            if (i < n) {
-                orow[i] = ld_raw<Tio, CPL>(o + base + (size_t)i * D);
-                if (g) grow[i] = ld_raw<Tio, CPL>(g + base + (size_t)i * D);
-            }
-        }
-#pragma unroll
-        for (int i = 0; i < kEpilogueRows; ++i) {
+        for (int r = 0; r < kRowsPerWarp; ++r) {
+            const int i = warp * kRowsPerWarp + r;
             if (i >= n) break;
             float ov[CPL], gv[CPL], ss = 0.f;
-            unpack(orow[i], ov);
-            if (g) unpack(grow[i], gv);
+            ld_row<CPL>(so + i * D, ov);
+            if (g) ld_row<CPL>(sg + i * D, gv);
 #pragma unroll
             for (int c = 0; c < CPL; ++c) ss = fmaf(ov[c], ov[c], ss);
             const float inv = rsqrtf(warp_sum(ss, 32) * (1.f / D) + eps);
             float out[CPL];
 #pragma unroll
             for (int c = 0; c < CPL; ++c) out[c] = ov[c] * inv * wl[c] * (g ? silu_f(gv[c]) : 1.f);
-            st_row<CPL>(y + base + (size_t)i * D, out);
+            st_row<CPL>(y + (size_t)(r0 + i) * D + lane * CPL, out);
         }
+        __syncthreads();
+        st = st == kBlkStages - 1 ? 0 : st + 1;
     }
 }
 
@@ -372,41 +399,72 @@ template <typename Kern> inline int resident_grid(Kern kernel, long long warps_n
     return (int)std::min<long long>(blocks, (long long)sms * per_sm);
 }
 
-template <typename Tio, int CPLQK, int CPLV>
+// 4-D map over one projected stream [B, T, H, d]: box = d channels x 1 head x
+// `rows` tokens x 1 batch, no swizzle (the stage is row-major [rows][d]);
+// coordinates outside the tensor read as zero.
+template <typename Tio>
+inline bool make_prologue_map(CUtensorMap *map, const void *base, int B, int T, int H, int d, int rows) {
+    EncodeTiledFn enc = encode_tiled_fn();
+    if (!enc) return false;
+    const cuuint64_t es = sizeof(Tio);
+    const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+    const cuuint64_t strides[3] = {(cuuint64_t)d * es, (cuuint64_t)H * d * es, (cuuint64_t)T * H * d * es};
+    const cuuint32_t box[4] = {(cuuint32_t)d, 1, (cuuint32_t)rows, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    const CUtensorMapDataType dt = sizeof(Tio) == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    return enc(map, dt, 4, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename Tio, int DQK, int DV>
 inline cudaError_t launch_prologue_t(const PrologueArgs &a, cudaStream_t stream) {
-    auto kern = a.K <= 4 ? gdr_prologue_kernel<Tio, CPLQK, CPLV, 4> : gdr_prologue_kernel<Tio, CPLQK, CPLV, kConvMax>;
-    const int stage_bytes = kPrologueRows * 32 * (CPLQK > CPLV ? CPLQK : CPLV) * (int)sizeof(Tio);
-    const int smem = 2 * stage_bytes + 16;
+    auto kern = a.K <= 4 ? gdr_prologue_kernel<Tio, DQK, DV, 4> : gdr_prologue_kernel<Tio, DQK, DV, kConvMax>;
+    constexpr int DMAX = DQK > DV ? DQK : DV;
+    const int stage_bytes = kPrologueRows * DMAX * (int)sizeof(Tio);
+    const int smem = kBlkStages * (stage_bytes + 8);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    const long long units = 3LL * a.B * a.H * ((a.T + kPrologueRun - 1) / kPrologueRun);
-    const int grid = resident_grid(kern, units * (kBlkThreads / 32), smem);
-    if (grid <= 0) return cudaErrorInvalidConfiguration;
-    kern<<<grid, kBlkThreads, smem, stream>>>(a, stage_bytes);
+    CUtensorMap mq, mk, mv;
+    if (!make_prologue_map<Tio>(&mq, a.x[0], a.B, a.T, a.H, a.dk, kPrologueRun + a.K - 1) ||
+        !make_prologue_map<Tio>(&mk, a.x[1], a.B, a.T, a.H, a.dk, kPrologueRun + a.K - 1) ||
+        !make_prologue_map<Tio>(&mv, a.x[2], a.B, a.T, a.H, a.dv, kPrologueRun + a.K - 1))
+        return cudaErrorInvalidValue;
+    // 3H (stream, head) pairs x G blocks each, G filling the resident slots
+    const long long pairs = 3LL * a.H, units = (long long)a.B * ((a.T + kPrologueRun - 1) / kPrologueRun);
+    const long long slots = resident_grid(kern, 1LL << 40, smem);
+    if (slots <= 0) return cudaErrorInvalidConfiguration;
+    const long long G = std::max(1LL, std::min(units, slots / pairs));
+    if (pairs * G >= (1LL << 31)) return cudaErrorInvalidConfiguration;
+    kern<<<(unsigned)(pairs * G), kBlkThreads, smem, stream>>>(a, stage_bytes, mq, mk, mv);
     g_launches.fetch_add(1, std::memory_order_relaxed);
     return cudaGetLastError();
 }
 
 template <typename Tio>
 inline cudaError_t launch_prologue(const PrologueArgs &a, cudaStream_t stream) {
-    if (a.dk == 128 && a.dv == 128) return launch_prologue_t<Tio, 4, 4>(a, stream);
-    if (a.dk == 128 && a.dv == 64) return launch_prologue_t<Tio, 4, 2>(a, stream);
-    if (a.dk == 64 && a.dv == 128) return launch_prologue_t<Tio, 2, 4>(a, stream);
-    return launch_prologue_t<Tio, 2, 2>(a, stream);
+    if (a.dk == 128 && a.dv == 128) return launch_prologue_t<Tio, 128, 128>(a, stream);
+    if (a.dk == 128 && a.dv == 64) return launch_prologue_t<Tio, 128, 64>(a, stream);
+    if (a.dk == 64 && a.dv == 128) return launch_prologue_t<Tio, 64, 128>(a, stream);
+    return launch_prologue_t<Tio, 64, 64>(a, stream);
 }
 
 template <typename Tio>
 inline cudaError_t launch_epilogue(long long rows, int dv, const void *o, const void *g, const float *weight,
                                    float eps, void *y, cudaStream_t stream) {
-    auto run = [&](auto kern) -> cudaError_t {
-        const int grid = resident_grid(kern, (rows + kEpilogueRows - 1) / kEpilogueRows);
+    auto run = [&](auto kern, int d) -> cudaError_t {
+        const int smem = kBlkStages * 2 * kEpilogueRows * d * (int)sizeof(Tio) + 8 * kBlkStages;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        const long long units = (rows + kEpilogueRows - 1) / kEpilogueRows;
+        const int grid = resident_grid(kern, units * (kBlkThreads / 32), smem);
         if (grid <= 0) return cudaErrorInvalidConfiguration;
-        kern<<<grid, kBlkThreads, 0, stream>>>(rows, static_cast<const Tio *>(o), static_cast<const Tio *>(g), weight,
-                                               eps, static_cast<Tio *>(y));
+        kern<<<grid, kBlkThreads, smem, stream>>>(rows, static_cast<const Tio *>(o), static_cast<const Tio *>(g),
+                                                  weight, eps, static_cast<Tio *>(y));
         g_launches.fetch_add(1, std::memory_order_relaxed);
         return cudaGetLastError();
     };
-    return dv == 128 ? run(gdr_epilogue_kernel<Tio, 4>) : run(gdr_epilogue_kernel<Tio, 2>);
+    return dv == 128 ? run(gdr_epilogue_kernel<Tio, 4>, 128) : run(gdr_epilogue_kernel<Tio, 2>, 64);
 }
 
 }  // namespace gdr
