@@ -32,7 +32,7 @@ namespace gdr {
 
 constexpr int kBlkThreads = 256;  // 8 warps
 constexpr int kConvMax = 8;       // widest ShortConv handled
-constexpr int kPrologueRun = 64;  // tokens per prologue work unit
+constexpr int kPrologueRun = 128;  // tokens per prologue work unit
 
 // ---- CPL consecutive elements per lane ---------------------------------------
 template <int CPL> __device__ __forceinline__ void ld_row(const float *p, float *o) {
@@ -75,9 +75,47 @@ template <int CPL> __device__ __forceinline__ void st_row(__nv_bfloat16 *p, cons
     }
 }
 
-// SiLU with the fast divide: for z -> -inf the denominator overflows to +inf
-// and the quotient is -0, the limit of z / (1 + e^-z).
-__device__ __forceinline__ float silu_f(float z) { return __fdividef(z, 1.f + __expf(-z)); }
+// Special-function-unit approximations with denormals flushed (ex2.approx,
+// rcp.approx, rsqrt.approx of the PTX ISA).
+__device__ __forceinline__ float ex2_ftz(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float rcp_ftz(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float rsqrt_ftz(float x) {
+    float y;
+    asm("rsqrt.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+// SiLU(z) = z / (1 + e^-z), with e^-z = 2^(-z log2 e).  For z -> -inf the
+// denominator overflows to +inf, its reciprocal is 0 and the result -0, the
+// limit; for z -> +inf the result is z.
+constexpr float kLog2e = 1.4426950408889634f;
+__device__ __forceinline__ float silu_f(float z) { return z * rcp_ftz(1.f + ex2_ftz(-kLog2e * z)); }
+
+// Packed fp32 pair arithmetic (fma.rn.f32x2 / mul.rn.f32x2): one instruction
+// for two lanes' worth of FMAs, each rounded as the scalar one.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("{\n .reg .b64 ra, rb, rc, rd;\n mov.b64 ra, {%2, %3};\n mov.b64 rb, {%4, %5};\n"
+        " mov.b64 rc, {%6, %7};\n fma.rn.f32x2 rd, ra, rb, rc;\n mov.b64 {%0, %1}, rd;\n}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n .reg .b64 ra, rb, rd;\n mov.b64 ra, {%2, %3};\n mov.b64 rb, {%4, %5};\n"
+        " mul.rn.f32x2 rd, ra, rb;\n mov.b64 {%0, %1}, rd;\n}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
 
 // ---- prologue -------------------------------------------------------------------
 struct PrologueArgs {
@@ -103,15 +141,17 @@ struct PrologueArgs {
 // as zero; rows from a carried conv state are patched in after the load.
 constexpr int kPrologueRows = kPrologueRun + kConvMax - 1;
 constexpr int kBlkStages = 3;  // bulk-copy ring depth of the staged kernels
+constexpr int kProStages = 3;  // ring depth of the prologue
 
 // After a wait gave up at unit k (stage st): wait, with a short bound, for the
 // copies already issued into the other stages so that none lands after the
 // block has exited.
+template <int NS>
 __device__ __forceinline__ void blk_drain(uint64_t *bars, int st, int k, long long u, long long units,
                                           long long stride) {
-    for (int m = 1; m < kBlkStages; ++m)
+    for (int m = 1; m < NS; ++m)
         if (u + (long long)m * stride < units)
-            sm100::mbar_wait(&bars[(st + m) % kBlkStages], (uint32_t)((k + m) / kBlkStages) & 1u, 100000000ull);
+            sm100::mbar_wait(&bars[(st + m) % NS], (uint32_t)((k + m) / NS) & 1u, 100000000ull);
 }
 
 // Stream pointers by selects (a runtime index into the parameter block would
@@ -178,14 +218,14 @@ __device__ __forceinline__ void prologue_block(const PrologueArgs &a, const CUte
     }
 
     // the ring: unit k of this block is (batch, run) idx + k*G, in stage
-    // k % kBlkStages with phase parity (k / kBlkStages) & 1
+    // k % kProStages with phase parity (k / kProStages) & 1
     auto issue = [&](int k, int sidx) {  // one thread
         const int j = idx + k * G, b = j / runs, t0 = (j % runs) * kPrologueRun;
         mbar_expect_tx(&bars[sidx], box_bytes);
         tma_load_4d(smem + sidx * stage_bytes, map, &bars[sidx], 0, h, t0 - (K - 1), b);
     };
     if (threadIdx.x == 0)
-        for (int k = 0; k < kBlkStages - 1; ++k)
+        for (int k = 0; k < kProStages - 1; ++k)
             if (idx + k * G < units) issue(k, k);
     const bool l2 = s < 2;
     const size_t ystride = (size_t)a.H * D;
@@ -196,15 +236,15 @@ __device__ __forceinline__ void prologue_block(const PrologueArgs &a, const CUte
         const int j = idx + k * G;
         if (j >= units) break;
         const int b = j / runs, t0 = (j % runs) * kPrologueRun, len = min(kPrologueRun, T - t0);
-        // stage unit k + kBlkStages - 1 into the slot unit k - 1 used (its
+        // stage unit k + kProStages - 1 into the slot unit k - 1 used (its
         // readers finished at the barrier that ended the previous iteration)
-        if (threadIdx.x == 0 && j + (kBlkStages - 1) * G < units) {
+        if (threadIdx.x == 0 && j + (kProStages - 1) * G < units) {
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            issue(k + kBlkStages - 1, st == 0 ? kBlkStages - 1 : st - 1);
+            issue(k + kProStages - 1, st == 0 ? kProStages - 1 : st - 1);
         }
-        if (!mbar_wait(&bars[st], (uint32_t)(k / kBlkStages) & 1u)) {
+        if (!mbar_wait(&bars[st], (uint32_t)(k / kProStages) & 1u)) {
             record_status(GDR_ERR_TIMEOUT);
-            blk_drain(bars, st, k, j, units, G);
+            blk_drain<kProStages>(bars, st, k, j, units, G);
             return;
         }
         uint8_t *stage = smem + st * stage_bytes;
@@ -234,30 +274,51 @@ __device__ __forceinline__ void prologue_block(const PrologueArgs &a, const CUte
                 for (int c = 0; c < CPL; ++c) win[m][c] = 0.f;
         }
         Tio *y = ybase + (((size_t)b * T + t0 + i0) * a.H) * D + c0;
+        // batches of NB rows: conv + SiLU for each, then their norm
+        // reductions interleaved (independent shuffle chains), then stores
+        constexpr int NB = RPG < 4 ? RPG : 4;
 #pragma unroll
-        for (int r = 0; r < RPG; ++r) {
-            load8(sx + (i0 + r + K - 1) * D, win[KW - 1]);
-            float acc[CPL], ss = 0.f;
+        for (int r0 = 0; r0 < RPG; r0 += NB) {
+            float acc[NB][CPL], ss[NB];
 #pragma unroll
-            for (int c = 0; c < CPL; ++c) {
-                float z = bias[c];
+            for (int q = 0; q < NB; ++q) {
+                load8(sx + (i0 + r0 + q + K - 1) * D, win[KW - 1]);
+                float2 ss2 = make_float2(0.f, 0.f);
 #pragma unroll
-                for (int m = 0; m < KW; ++m) z = fmaf(wt[c][m], win[m][c], z);
-                acc[c] = silu_f(z);
-                ss = fmaf(acc[c], acc[c], ss);
+                for (int c = 0; c < CPL; c += 2) {  // channel pairs on the packed FMA
+                    float2 z = make_float2(bias[c], bias[c + 1]);
+#pragma unroll
+                    for (int m = 0; m < KW; ++m)
+                        z = ffma2(make_float2(wt[c][m], wt[c + 1][m]), make_float2(win[m][c], win[m][c + 1]), z);
+                    acc[q][c] = silu_f(z.x);
+                    acc[q][c + 1] = silu_f(z.y);
+                    ss2 = ffma2(make_float2(acc[q][c], acc[q][c + 1]), make_float2(acc[q][c], acc[q][c + 1]), ss2);
+                }
+                ss[q] = ss2.x + ss2.y;
+#pragma unroll
+                for (int m = 0; m < KW - 1; ++m)
+#pragma unroll
+                    for (int c = 0; c < CPL; ++c) win[m][c] = win[m + 1][c];
             }
-#pragma unroll
-            for (int m = 0; m < KW - 1; ++m)
-#pragma unroll
-                for (int c = 0; c < CPL; ++c) win[m][c] = win[m + 1][c];
             if (l2) {
 #pragma unroll
-                for (int off = LPR / 2; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-                const float inv = rsqrtf(ss + a.eps);
+                for (int off = LPR / 2; off > 0; off >>= 1)
 #pragma unroll
-                for (int c = 0; c < CPL; ++c) acc[c] *= inv;
+                    for (int q = 0; q < NB; ++q) ss[q] += __shfl_xor_sync(0xffffffffu, ss[q], off);
+#pragma unroll
+                for (int q = 0; q < NB; ++q) {
+                    const float inv = rsqrt_ftz(ss[q] + a.eps);
+#pragma unroll
+                    for (int c = 0; c < CPL; c += 2) {
+                        const float2 t = fmul2(make_float2(acc[q][c], acc[q][c + 1]), make_float2(inv, inv));
+                        acc[q][c] = t.x;
+                        acc[q][c + 1] = t.y;
+                    }
+                }
             }
-            if (i0 + r < len) store8(y + r * ystride, acc);
+#pragma unroll
+            for (int q = 0; q < NB; ++q)
+                if (i0 + r0 + q < len) store8(y + (r0 + q) * ystride, acc[q]);
         }
 
         // The carried state of (stream, batch, head): the last K-1 inputs,
@@ -277,7 +338,7 @@ __device__ __forceinline__ void prologue_block(const PrologueArgs &a, const CUte
             }
         }
         __syncthreads();
-        st = st == kBlkStages - 1 ? 0 : st + 1;
+        st = st == kProStages - 1 ? 0 : st + 1;
     }
 }
 
@@ -288,11 +349,11 @@ __global__ void __launch_bounds__(kBlkThreads)
     using namespace sm100;
     extern __shared__ __align__(128) uint8_t blk_smem[];
     uint8_t *smem = blk_smem;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kBlkStages * stage_bytes);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kProStages * stage_bytes);
     const int P = 3 * a.H, pair = blockIdx.x % P, idx = blockIdx.x / P, G = gridDim.x / P;
     const int s = pair / a.H, h = pair % a.H;
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kBlkStages; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < kProStages; ++i) mbar_init(&bars[i], 1);
         fence_mbar_init();
     }
     __syncthreads();
@@ -354,7 +415,7 @@ __global__ void __launch_bounds__(kBlkThreads)
         }
         if (!mbar_wait(&bars[st], (uint32_t)(k / kBlkStages) & 1u)) {
             record_status(GDR_ERR_TIMEOUT);
-            blk_drain(bars, st, k, u, units, gridDim.x);
+            blk_drain<kBlkStages>(bars, st, k, u, units, gridDim.x);
             return;
         }
         const Tio *so = reinterpret_cast<const Tio *>(smem + st * 2 * kTile) + lane * CPL;
@@ -370,7 +431,7 @@ __global__ void __launch_bounds__(kBlkThreads)
             if (g) ld_row<CPL>(sg + i * D, gv);
 #pragma unroll
             for (int c = 0; c < CPL; ++c) ss = fmaf(ov[c], ov[c], ss);
-            const float inv = rsqrtf(warp_sum(ss, 32) * (1.f / D) + eps);
+            const float inv = rsqrt_ftz(warp_sum(ss, 32) * (1.f / D) + eps);
             float out[CPL];
 #pragma unroll
             for (int c = 0; c < CPL; ++c) out[c] = ov[c] * inv * wl[c] * (g ? silu_f(gv[c]) : 1.f);
@@ -422,7 +483,7 @@ inline cudaError_t launch_prologue_t(const PrologueArgs &a, cudaStream_t stream)
     auto kern = a.K <= 4 ? gdr_prologue_kernel<Tio, DQK, DV, 4> : gdr_prologue_kernel<Tio, DQK, DV, kConvMax>;
     constexpr int DMAX = DQK > DV ? DQK : DV;
     const int stage_bytes = kPrologueRows * DMAX * (int)sizeof(Tio);
-    const int smem = kBlkStages * (stage_bytes + 8);
+    const int smem = kProStages * (stage_bytes + 8);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     CUtensorMap mq, mk, mv;
