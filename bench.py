@@ -456,7 +456,43 @@ def secondary(pk):
         out["gdn2_fwd"] = {"unavailable": str(e).splitlines()[0][:200]}
     del d, x
     out.update(block_lines(pk))
+    out.update(seq_split_line())
     return out
+
+
+def seq_split_line(R=8):
+    """One rank's share of the long sequence (B1 T65536 H16 d128 bf16) split
+    into R segments: both forward passes of its 8192-token segment, the
+    combine as the last rank (R - 1 segment maps) and the output correction.
+    The all-gather of (M, N) is not timed on one GPU; its size is reported."""
+    import gated_delta_rule_91_b200 as gdr
+    x = synth.workload_inputs("long_fwd_bwd")
+    T = x["q"].shape[1]
+    Ts = T // R
+    d = {n: x[n][:, :Ts].contiguous().cuda() for n in ("q", "k", "v", "log_alpha", "beta")}
+    B, _, H, dk = d["q"].shape
+    dv = d["v"].shape[-1]
+    M_all = torch.zeros(R, B, H, dk, dk, device="cuda")
+    N_all = torch.zeros(R, B, H, dv, dk, device="cuda")
+
+    def rank_work():
+        o0, qt, N, M = gdr.gdr_seg_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"])
+        S_in, _ = gdr.gdr_seg_combine(M_all, N_all, R - 1, None, want_final=True)
+        gdr.gdr_seg_fixup(qt, S_in, o0)
+
+    for _ in range(2):
+        rank_work()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(3):
+        rank_work()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / 3
+    return {"seq_split_8": {"workload": "B=1 T=65536 H=16 d=128 bf16 split into %d segments of %d tokens" % (R, Ts),
+                            "rank_ms": ms, "exchange_bytes_per_rank": (dk * dk + dv * dk) * 4 * B * H,
+                            "note": "per-rank device time without the all-gather; the unsplit forward is long_fwd_bwd.fwd_ms"}}
 
 
 def block_lines(pk):

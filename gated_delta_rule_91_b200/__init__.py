@@ -13,6 +13,7 @@ Functions (same names as the C entry points):
     gdr2_bwd(q, k, v, log_alpha, b, w, S0, dO, dS_T=None) -> dict of gradients
     gdr_block_prologue(xq, xk, xv, wq, wk, wv, ...)       -> (q, k, v)
     gdr_block_epilogue(o, g, weight, eps)                 -> y
+    gdr_seg_fwd / gdr_seg_combine / gdr_seg_fixup         (sequence split; see seq_split)
 """
 import ctypes
 import os
@@ -43,6 +44,10 @@ SIGNATURES = {
     "gdr2_bwd_workspace_bytes": (_SZ, [_I] * 6),
     "gdr_block_prologue": (_I, [_I] * 7 + [_P] * 11 + [ctypes.c_float] + [_P] * 3 + [_P]),
     "gdr_block_epilogue": (_I, [_I] * 5 + [_P] * 3 + [ctypes.c_float, _P, _P]),
+    "gdr_seg_fwd": (_I, [_I] * 6 + [_P] * 9 + [_P, _SZ, _P]),
+    "gdr_seg_fwd_workspace_bytes": (_SZ, [_I] * 6),
+    "gdr_seg_combine": (_I, [_I] * 6 + [_P] * 5 + [_P]),
+    "gdr_seg_fixup": (_I, [_I] * 6 + [_P] * 3 + [_P]),
     "gdr_check_status": (_I, [_P]),
     "gdr_debug_wait_timeout": (_I, [_I, _P]),
     "gdr_last_error_string": (ctypes.c_char_p, []),
@@ -244,3 +249,44 @@ def gdr_block_epilogue(o, g, weight, eps=1e-6, *, y=None):
     check(lib().gdr_block_epilogue(B, T, H, dv, _dt(o), _ptr(o), _ptr(g), _ptr(weight), float(eps),
                                    _ptr(y), _stream(o)))
     return y
+
+
+def gdr_seg_fwd(q, k, v, log_alpha, beta, *, workspace=None):
+    """Both forward passes of one segment of a split sequence: returns
+    (o0 [B,T,H,dv] from S_in = 0, qt [B,T,H,dk] = M_<=t q_t,
+     N [B,H,dv,dk], M [B,H,dk,dk])."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = _dt(q)
+    o0 = torch.empty(B, T, H, dv, dtype=q.dtype, device=q.device)
+    qt = torch.empty(B, T, H, dk, dtype=q.dtype, device=q.device)
+    N = torch.empty(B, H, dv, dk, dtype=torch.float32, device=q.device)
+    M = torch.empty(B, H, dk, dk, dtype=torch.float32, device=q.device)
+    L = lib()
+    ws, ws_bytes = _workspace(L.gdr_seg_fwd_workspace_bytes(B, T, H, dk, dv, dt), q.device, workspace)
+    check(L.gdr_seg_fwd(B, T, H, dk, dv, dt, _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+                        _ptr(o0), _ptr(qt), _ptr(N), _ptr(M), _ptr(ws), ws_bytes, _stream(q)))
+    return o0, qt, N, M
+
+
+def gdr_seg_combine(M_all, N_all, r, S0=None, *, want_final=True):
+    """Sequential combine of the segment maps: M_all [R,B,H,dk,dk], N_all
+    [R,B,H,dv,dk] in segment order.  Returns (S_in of segment r, state after
+    the last segment or None)."""
+    R, B, H, dk, _ = M_all.shape
+    dv = N_all.shape[3]
+    _f32(M_all, "M_all"), _f32(N_all, "N_all"), _f32(S0, "S0")
+    S_in = torch.empty(B, H, dv, dk, dtype=torch.float32, device=M_all.device)
+    S_T = torch.empty_like(S_in) if want_final else None
+    check(lib().gdr_seg_combine(R, r, B, H, dk, dv, _ptr(M_all), _ptr(N_all), _ptr(S0), _ptr(S_in),
+                                _ptr(S_T), _stream(M_all)))
+    return S_in, S_T
+
+
+def gdr_seg_fixup(qt, S_in, o):
+    """o += S_in q~ per token (in place); returns o."""
+    B, T, H, dk = qt.shape
+    dv = o.shape[-1]
+    _f32(S_in, "S_in")
+    check(lib().gdr_seg_fixup(B, T, H, dk, dv, _dt(qt), _ptr(qt), _ptr(S_in), _ptr(o), _stream(qt)))
+    return o

@@ -15,6 +15,7 @@
 #include "fwd_simt.cuh"
 #include "bwd_simt.cuh"
 #include "block.cuh"
+#include "seg_split.cuh"
 #include "gdr2_simt.cuh"
 #include "fwd_tc.cuh"
 #include "fwd_tc2.cuh"
@@ -411,6 +412,83 @@ gdr_status gdr_block_epilogue(int B, int T, int H, int dv, gdr_dtype dt, const v
     const long long rows = (long long)B * T * H;
     cudaError_t e = dt == GDR_F32 ? launch_epilogue<float>(rows, dv, o, g, weight, eps, y, s)
                                   : launch_epilogue<__nv_bfloat16>(rows, dv, o, g, weight, eps, y, s);
+    if (e != cudaSuccess) return cuda_fail(e, fn);
+    return GDR_OK;
+}
+
+size_t gdr_seg_fwd_workspace_bytes(int B, int T, int H, int dk, int dv, gdr_dtype dt) {
+    if (B < 1 || T < 1 || H < 1 || (dk != 64 && dk != 128) || (dv != 64 && dv != 128) ||
+        (dt != GDR_F32 && dt != GDR_BF16))
+        return 0;
+    const size_t es = dt == GDR_F32 ? 4 : 2;
+    const size_t zero_v = ((size_t)B * T * H * dk * es + 255) & ~(size_t)255;
+    return zero_v + (size_t)B * H * dk * dk * 4;
+}
+
+gdr_status gdr_seg_fwd(int B, int T, int H, int dk, int dv, gdr_dtype dt, const void *q, const void *k,
+                       const void *v, const float *log_alpha, const float *beta, void *o0, void *qt, float *N,
+                       float *M, void *workspace, size_t workspace_bytes, gdr_stream_t stream) {
+    const char *fn = "gdr_seg_fwd";
+    gdr_status st = check_dims(fn, B, T, H, dk, dv, dt);
+    if (st != GDR_OK) return st;
+    GDR_REQUIRE_PTR(q);
+    GDR_REQUIRE_PTR(k);
+    GDR_REQUIRE_PTR(v);
+    GDR_REQUIRE_PTR(log_alpha);
+    GDR_REQUIRE_PTR(beta);
+    GDR_REQUIRE_PTR(o0);
+    GDR_REQUIRE_PTR(qt);
+    GDR_REQUIRE_PTR(N);
+    GDR_REQUIRE_PTR(M);
+    GDR_REQUIRE_PTR(workspace);
+    const size_t need = gdr_seg_fwd_workspace_bytes(B, T, H, dk, dv, dt);
+    if (workspace_bytes < need)
+        return fail(GDR_ERR_WORKSPACE, "%s: workspace of %zu bytes needed, %zu given", fn, need, workspace_bytes);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // pass 1: from S_in = 0 -> o(0) and N
+    st = gdr_fwd(B, T, H, dk, dv, dt, q, k, v, log_alpha, beta, nullptr, o0, N, nullptr, 0, stream);
+    if (st != GDR_OK) return st;
+    // pass 2: v = 0 from S_in = I (dv = dk) -> q~ and M
+    const size_t es = dt == GDR_F32 ? 4 : 2;
+    const size_t zero_v = ((size_t)B * T * H * dk * es + 255) & ~(size_t)255;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    float *eye = reinterpret_cast<float *>(ws + zero_v);
+    cudaError_t e = cudaMemsetAsync(ws, 0, (size_t)B * T * H * dk * es, s);
+    if (e == cudaSuccess) e = launch_seg_identity(eye, B * H, dk, s);
+    if (e != cudaSuccess) return cuda_fail(e, fn);
+    return gdr_fwd(B, T, H, dk, dk, dt, q, k, ws, log_alpha, beta, eye, qt, M, nullptr, 0, stream);
+}
+
+gdr_status gdr_seg_combine(int R, int r, int B, int H, int dk, int dv, const float *M, const float *N,
+                           const float *S0, float *S_in, float *S_T, gdr_stream_t stream) {
+    const char *fn = "gdr_seg_combine";
+    gdr_status st = check_dims(fn, B, 1, H, dk, dv, GDR_F32);
+    if (st != GDR_OK) return st;
+    if (R < 1 || r < 0 || r >= R)
+        return fail(GDR_ERR_INVALID_ARGUMENT, "%s: segment %d of %d", fn, r, R);
+    if (S_in == nullptr && S_T == nullptr)
+        return fail(GDR_ERR_INVALID_ARGUMENT, "%s: S_in and S_T are both NULL", fn);
+    GDR_REQUIRE_PTR(M);
+    GDR_REQUIRE_PTR(N);
+    GDR_OPTIONAL_PTR(S0);
+    GDR_OPTIONAL_PTR(S_in);
+    GDR_OPTIONAL_PTR(S_T);
+    cudaError_t e = launch_seg_combine(R, r, B * H, dk, dv, M, N, S0, S_in, S_T, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, fn);
+    return GDR_OK;
+}
+
+gdr_status gdr_seg_fixup(int B, int T, int H, int dk, int dv, gdr_dtype dt, const void *qt, const float *S_in,
+                         void *o, gdr_stream_t stream) {
+    const char *fn = "gdr_seg_fixup";
+    gdr_status st = check_dims(fn, B, T, H, dk, dv, dt);
+    if (st != GDR_OK) return st;
+    GDR_REQUIRE_PTR(qt);
+    GDR_REQUIRE_PTR(S_in);
+    GDR_REQUIRE_PTR(o);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = dt == GDR_F32 ? launch_seg_fixup<float>(B, T, H, dk, dv, qt, S_in, o, s)
+                                  : launch_seg_fixup<__nv_bfloat16>(B, T, H, dk, dv, qt, S_in, o, s);
     if (e != cudaSuccess) return cuda_fail(e, fn);
     return GDR_OK;
 }

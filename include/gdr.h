@@ -40,7 +40,8 @@
  *  * A launch failure returns GDR_ERR_CUDA.  Kernels that wait on on-chip
  *    barriers give up after a bounded number of polls and record
  *    GDR_ERR_TIMEOUT in a device status word, read by gdr_check_status().
- *  * Outputs must not alias inputs (except S in gdr_step, which is in-out).
+ *  * Outputs must not alias inputs (except S in gdr_step, o in gdr_seg_fixup
+ *    and the conv state in gdr_block_prologue, which are in-out).
  *  * gdr_last_error_string() describes the last non-OK status returned on the
  *    calling thread.
  */
@@ -249,6 +250,61 @@ GDR_API gdr_status gdr_block_prologue(int B, int T, int H, int dk, int dv, int K
 GDR_API gdr_status gdr_block_epilogue(int B, int T, int H, int dv, gdr_dtype dt, const void *o,
                               const void *g, const float *weight, float eps, void *y,
                               gdr_stream_t stream);
+
+/*
+ * Sequence split: one sequence divided into R consecutive segments, one per
+ * process/GPU, each run by its owner, with one exchange of small matrices.
+ * For one (b, h) the rule over a segment maps the incoming state affinely,
+ *     S_out = S_in M + N,
+ * N (dv x dk) being the segment's final state from S_in = 0 and M (dk x dk)
+ * the product of the per-token factors alpha_t (I - beta_t k_t k_t^T) in
+ * token order; in the chunkwise form of the Gated DeltaNet review
+ * (meaningful96.github.io/nr/GDN, section 3.7) it is the product of the
+ * chunks' (gamma_C I - W^T K) factors.  The readout is affine too:
+ *     o_t = o_t(S_in = 0) + S_in q~_t,   q~_t = M_<=t q_t,
+ * and the rule run with v = 0 from S_in = I (dv = dk) returns q~ as its
+ * outputs and M as its final state.  Per rank r of R:
+ *   1. gdr_seg_fwd on the segment -> o(0), q~, N, M;
+ *   2. all-gather (M, N) of every segment in order (the caller's collective);
+ *   3. gdr_seg_combine(R, r, ...) -> S_in of segment r (and the final state);
+ *   4. gdr_seg_fixup -> o = o(0) + S_in q~.
+ * The result equals gdr_fwd over the whole sequence up to rounding.
+ */
+
+/* Both forward passes of one segment (tokens of this segment only, T of
+ * them, inputs laid out as for gdr_fwd; S_in is not an input).
+ *   out: o0 [B,T,H,dv] (dtype dt) outputs from S_in = 0;
+ *        qt [B,T,H,dk] (dtype dt) q~_t = M_<=t q_t;
+ *        N [B,H,dv,dk] fp32; M [B,H,dk,dk] fp32.
+ * workspace (>= gdr_seg_fwd_workspace_bytes) holds a zero value tensor and the
+ * identity state of the second pass.  Errors as for gdr_fwd, plus
+ * GDR_ERR_WORKSPACE. */
+GDR_API gdr_status gdr_seg_fwd(int B, int T, int H, int dk, int dv, gdr_dtype dt,
+                       const void *q, const void *k, const void *v,
+                       const float *log_alpha, const float *beta,
+                       void *o0, void *qt, float *N, float *M,
+                       void *workspace, size_t workspace_bytes, gdr_stream_t stream);
+GDR_API size_t gdr_seg_fwd_workspace_bytes(int B, int T, int H, int dk, int dv, gdr_dtype dt);
+
+/* The sequential combine of the segment maps, fp32: S = S0 (NULL: zeros);
+ * for j = 0 .. R-1: S = S M_j + N_j.
+ *   in : M [R,B,H,dk,dk], N [R,B,H,dv,dk] (segment j's gdr_seg_fwd outputs at
+ *        index j); S0 [B,H,dv,dk] or NULL; 0 <= r < R.
+ *   out: S_in [B,H,dv,dk] = S before segment r (may be NULL);
+ *        S_T [B,H,dv,dk] = S after segment R-1, the state after the whole
+ *        sequence (may be NULL; not both).
+ *   Errors: r outside 0..R-1 or both outputs NULL -> GDR_ERR_INVALID_ARGUMENT;
+ *   sizes as for gdr_fwd. */
+GDR_API gdr_status gdr_seg_combine(int R, int r, int B, int H, int dk, int dv,
+                           const float *M, const float *N, const float *S0,
+                           float *S_in, float *S_T, gdr_stream_t stream);
+
+/* The correction of one segment's outputs: o[b,t,h,:] += S_in[b,h] qt[b,t,h,:]
+ * in fp32, rounded once to dtype dt.
+ *   in : qt [B,T,H,dk] (gdr_seg_fwd's q~), S_in [B,H,dv,dk] fp32.
+ *   in/out: o [B,T,H,dv] (gdr_seg_fwd's o0 on entry).  Sizes as gdr_fwd. */
+GDR_API gdr_status gdr_seg_fixup(int B, int T, int H, int dk, int dv, gdr_dtype dt,
+                         const void *qt, const float *S_in, void *o, gdr_stream_t stream);
 
 /* Synchronise `stream`, then read and clear the device status word that
  * kernels set when a bounded wait gives up (GDR_ERR_TIMEOUT) or when

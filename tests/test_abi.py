@@ -124,3 +124,35 @@ def test_epilogue_rejects_bad_arguments(kw, status):
                                       P(a["g"]), P(a["weight"]), a["eps"], P(a["y"]), None)
     assert st == status
     assert gdr.lib().gdr_last_error_string().decode().startswith("gdr_block_epilogue")
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(R=0), gdr.GDR_ERR_INVALID_ARGUMENT),
+    (dict(r=-1), gdr.GDR_ERR_INVALID_ARGUMENT),
+    (dict(r=3), gdr.GDR_ERR_INVALID_ARGUMENT),
+    (dict(S_in=None, S_T=None), gdr.GDR_ERR_INVALID_ARGUMENT),
+    (dict(M=None), gdr.GDR_ERR_INVALID_ARGUMENT),
+    (dict(dk=32), gdr.GDR_ERR_UNSUPPORTED),
+    (dict(S0=FAKE + 4), gdr.GDR_ERR_INVALID_ARGUMENT),
+])
+def test_seg_combine_rejects_bad_arguments(kw, status):
+    a = dict(R=3, r=1, B=1, H=2, dk=64, dv=64, M=FAKE, N=FAKE, S0=None, S_in=FAKE, S_T=None)
+    a.update(kw)
+    P = ctypes.c_void_p
+    st = gdr.lib().gdr_seg_combine(a["R"], a["r"], a["B"], a["H"], a["dk"], a["dv"], P(a["M"]),
+                                   P(a["N"]), P(a["S0"]), P(a["S_in"]), P(a["S_T"]), None)
+    assert st == status
+    assert gdr.lib().gdr_last_error_string().decode().startswith("gdr_seg_combine")
+
+
+def test_seg_fwd_checks_workspace_and_pointers():
+    L, P = gdr.lib(), ctypes.c_void_p
+    need = L.gdr_seg_fwd_workspace_bytes(1, 100, 2, 128, 64, gdr.GDR_BF16)
+    assert need >= 1 * 100 * 2 * 128 * 2 + 2 * 128 * 128 * 4
+    args = [1, 100, 2, 128, 64, gdr.GDR_BF16] + [P(FAKE)] * 9
+    assert L.gdr_seg_fwd(*args, P(FAKE), need - 1, None) == gdr.GDR_ERR_WORKSPACE
+    assert L.gdr_seg_fwd(*args, None, need, None) == gdr.GDR_ERR_INVALID_ARGUMENT
+    bad = [1, 100, 2, 128, 64, gdr.GDR_BF16] + [P(FAKE)] * 7 + [None, P(FAKE)]
+    assert L.gdr_seg_fwd(*bad, P(FAKE), need, None) == gdr.GDR_ERR_INVALID_ARGUMENT
+    assert L.gdr_seg_fixup(1, 4, 1, 64, 64, gdr.GDR_F32, P(FAKE), None, P(FAKE), None) == \
+        gdr.GDR_ERR_INVALID_ARGUMENT
