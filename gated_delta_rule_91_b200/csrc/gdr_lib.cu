@@ -416,6 +416,17 @@ gdr_status gdr_block_epilogue(int B, int T, int H, int dv, gdr_dtype dt, const v
     return GDR_OK;
 }
 
+// The two passes of gdr_seg_fwd are independent; the second runs on an
+// auxiliary stream of the device (created on first use, with a fork and a
+// join event), so the two small grids share the GPU.  The enqueue sequence is
+// serialised by a mutex so the events can be reused.
+struct SegAux {
+    cudaStream_t stream = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+};
+std::mutex g_seg_mu;
+SegAux g_seg_aux[64];
+
 size_t gdr_seg_fwd_workspace_bytes(int B, int T, int H, int dk, int dv, gdr_dtype dt) {
     if (B < 1 || T < 1 || H < 1 || (dk != 64 && dk != 128) || (dv != 64 && dv != 128) ||
         (dt != GDR_F32 && dt != GDR_BF16))
@@ -445,18 +456,42 @@ gdr_status gdr_seg_fwd(int B, int T, int H, int dk, int dv, gdr_dtype dt, const 
     if (workspace_bytes < need)
         return fail(GDR_ERR_WORKSPACE, "%s: workspace of %zu bytes needed, %zu given", fn, need, workspace_bytes);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    // pass 1: from S_in = 0 -> o(0) and N
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, fn);
+    if (dev < 0 || dev >= 64) return fail(GDR_ERR_UNSUPPORTED, "%s: device ordinal %d out of range", fn, dev);
+    std::lock_guard<std::mutex> lock(g_seg_mu);
+    SegAux &aux = g_seg_aux[dev];
+    if (aux.stream == nullptr) {
+        e = cudaStreamCreateWithFlags(&aux.stream, cudaStreamNonBlocking);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&aux.fork, cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&aux.join, cudaEventDisableTiming);
+        if (e != cudaSuccess) return cuda_fail(e, fn);
+    }
+    e = cudaEventRecord(aux.fork, s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(aux.stream, aux.fork, 0);
+    if (e != cudaSuccess) return cuda_fail(e, fn);
+    // pass 1 (caller's stream): from S_in = 0 -> o(0) and N
     st = gdr_fwd(B, T, H, dk, dv, dt, q, k, v, log_alpha, beta, nullptr, o0, N, nullptr, 0, stream);
-    if (st != GDR_OK) return st;
-    // pass 2: v = 0 from S_in = I (dv = dk) -> q~ and M
+    // pass 2 (auxiliary stream): v = 0 from S_in = I (dv = dk) -> q~ and M
     const size_t es = dt == GDR_F32 ? 4 : 2;
     const size_t zero_v = ((size_t)B * T * H * dk * es + 255) & ~(size_t)255;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     float *eye = reinterpret_cast<float *>(ws + zero_v);
-    cudaError_t e = cudaMemsetAsync(ws, 0, (size_t)B * T * H * dk * es, s);
-    if (e == cudaSuccess) e = launch_seg_identity(eye, B * H, dk, s);
+    gdr_status st2 = GDR_OK;
+    e = cudaMemsetAsync(ws, 0, (size_t)B * T * H * dk * es, aux.stream);
+    if (e == cudaSuccess) e = launch_seg_identity(eye, B * H, dk, aux.stream);
+    if (e == cudaSuccess)
+        st2 = gdr_fwd(B, T, H, dk, dk, dt, q, k, ws, log_alpha, beta, eye, qt, M, nullptr, 0,
+                      reinterpret_cast<gdr_stream_t>(aux.stream));
+    // join (always, so the caller's stream never runs ahead of pass 2)
+    cudaError_t ej = cudaEventRecord(aux.join, aux.stream);
+    if (ej == cudaSuccess) ej = cudaStreamWaitEvent(s, aux.join, 0);
+    if (st != GDR_OK) return st;
     if (e != cudaSuccess) return cuda_fail(e, fn);
-    return gdr_fwd(B, T, H, dk, dk, dt, q, k, ws, log_alpha, beta, eye, qt, M, nullptr, 0, stream);
+    if (st2 != GDR_OK) return st2;
+    if (ej != cudaSuccess) return cuda_fail(ej, fn);
+    return GDR_OK;
 }
 
 gdr_status gdr_seg_combine(int R, int r, int B, int H, int dk, int dv, const float *M, const float *N,

@@ -21,7 +21,9 @@
  *  * Pointers are DEVICE pointers (cudaMalloc / torch CUDA memory) on the
  *    current device unless stated otherwise.  The caller owns every buffer;
  *    the library never allocates device memory and keeps no state between
- *    calls other than a per-device table of kernel attributes.
+ *    calls other than a per-device table of kernel attributes and, once
+ *    gdr_seg_fwd has run on a device, one auxiliary stream and two events
+ *    there.
  *  * All tensors are dense, row-major, contiguous:
  *      q, k          [B, T, H, dk]      v, o, dO        [B, T, H, dv]
  *      log_alpha     [B, T, H] fp32     beta            [B, T, H] fp32
@@ -277,7 +279,10 @@ GDR_API gdr_status gdr_block_epilogue(int B, int T, int H, int dv, gdr_dtype dt,
  *        qt [B,T,H,dk] (dtype dt) q~_t = M_<=t q_t;
  *        N [B,H,dv,dk] fp32; M [B,H,dk,dk] fp32.
  * workspace (>= gdr_seg_fwd_workspace_bytes) holds a zero value tensor and the
- * identity state of the second pass.  Errors as for gdr_fwd, plus
+ * identity state of the second pass.  The two passes are independent: the
+ * second runs on the library's auxiliary stream of the device, forked from and
+ * joined back into `stream` with events, so both small grids share the GPU
+ * and `stream` sees the call complete as usual.  Errors as for gdr_fwd, plus
  * GDR_ERR_WORKSPACE. */
 GDR_API gdr_status gdr_seg_fwd(int B, int T, int H, int dk, int dv, gdr_dtype dt,
                        const void *q, const void *k, const void *v,
