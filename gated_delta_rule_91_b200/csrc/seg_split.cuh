@@ -20,6 +20,26 @@ namespace gdr {
 
 constexpr int kSegThreads = 256;
 
+// Four consecutive elements of a row (16-byte aligned for fp32, 8 for bf16).
+__device__ __forceinline__ void ld_row4(const float *p, float *v) {
+    const float4 f = *reinterpret_cast<const float4 *>(p);
+    v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
+}
+__device__ __forceinline__ void ld_row4(const __nv_bfloat16 *p, float *v) {
+    const float4 f = load4(p);
+    v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
+}
+__device__ __forceinline__ void st_row4(float *p, const float *v) {
+    *reinterpret_cast<float4 *>(p) = make_float4(v[0], v[1], v[2], v[3]);
+}
+__device__ __forceinline__ void st_row4(__nv_bfloat16 *p, const float *v) {
+    __nv_bfloat162 a = __floats2bfloat162_rn(v[0], v[1]), b = __floats2bfloat162_rn(v[2], v[3]);
+    uint2 raw;
+    raw.x = *reinterpret_cast<uint32_t *>(&a);
+    raw.y = *reinterpret_cast<uint32_t *>(&b);
+    *reinterpret_cast<uint2 *>(p) = raw;
+}
+
 // S[bh] = I (dk x dk) for every (batch, head).
 __global__ void __launch_bounds__(kSegThreads) seg_identity_kernel(float *S, int dk, long long n) {
     for (long long i = blockIdx.x * (long long)kSegThreads + threadIdx.x; i < n;
@@ -29,78 +49,98 @@ __global__ void __launch_bounds__(kSegThreads) seg_identity_kernel(float *S, int
     }
 }
 
-// One block per (batch, head): S = S0 (or 0); for segment j = 0 .. R-1:
-// S = S M_j + N_j, writing S_in = S before segment r and S_T = S after the
-// last one.  M: [R, B*H, dk, dk]; N: [R, B*H, dv, dk]; S0, S_in, S_T:
-// [B*H, dv, dk].  A thread owns DV/16 rows x DK/16 columns of the product
-// (rows ty + 16a, columns tx + 16c), read from S and M staged in shared
-// memory.
-template <int DK, int DV>
+// The combine.  S = S0 (or 0); for segment j = 0 .. R-1: S = S M_j + N_j,
+// writing S_in = S before segment r and S_T = S after the last one.  Rows of
+// S are independent, so block (bh, rb) carries rows [32 rb, 32 rb + 32) of
+// one (batch, head) through all the steps, staging M_j in shared memory.
+// M: [R, B*H, dk, dk]; N: [R, B*H, dv, dk]; S0, S_in, S_T: [B*H, dv, dk].
+// A thread owns RPT rows (2 for dk = 128, 1 for dk = 64) x 8 columns (two
+// float4 of M per k step).
+constexpr int kCombRows = 32;
+
+template <int DK>
 __global__ void __launch_bounds__(kSegThreads)
-    seg_combine_kernel(int R, int r, int BH, const float *__restrict__ M, const float *__restrict__ N,
+    seg_combine_kernel(int R, int r, int BH, int DV, const float *__restrict__ M, const float *__restrict__ N,
                        const float *__restrict__ S0, float *__restrict__ S_in, float *__restrict__ S_T) {
     extern __shared__ __align__(16) float seg_smem[];
-    float *sS = seg_smem;            // [DV][DK]
-    float *sM = seg_smem + DV * DK;  // [DK][DK]
-    constexpr int RA = DV / 16, CA = DK / 16;
-    const int bh = blockIdx.x, tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+    float *sM = seg_smem;             // [DK][DK]
+    float *sS = seg_smem + DK * DK;   // [kCombRows][DK]
+    constexpr int CG = DK / 8;               // column groups (8 columns each)
+    constexpr int RG = kSegThreads / CG;     // row groups
+    constexpr int RPT = kCombRows / RG;      // rows per thread
+    static_assert(RPT * RG == kCombRows && RPT >= 1, "row split");
+    const int bh = blockIdx.x, row0 = blockIdx.y * kCombRows;
+    const int cg = threadIdx.x % CG, rg = threadIdx.x / CG;
+    // columns of this thread: 4 cg .. 4 cg + 3 and DK/2 + 4 cg .. + 3
+    const int c0 = 4 * cg, c1 = DK / 2 + 4 * cg;
     const size_t sz = (size_t)DV * DK, mz = (size_t)DK * DK;
-    for (int i = threadIdx.x; i < DV * DK; i += kSegThreads) sS[i] = S0 ? S0[bh * sz + i] : 0.f;
+    for (int i = threadIdx.x; i < kCombRows * DK; i += kSegThreads)
+        sS[i] = S0 ? S0[bh * sz + (size_t)row0 * DK + i] : 0.f;
     __syncthreads();
-    if (r == 0 && S_in)
-        for (int i = threadIdx.x; i < DV * DK; i += kSegThreads) S_in[bh * sz + i] = sS[i];
+    auto write_rows = [&](float *dst) {
+        for (int i = threadIdx.x; i < kCombRows * DK; i += kSegThreads) dst[bh * sz + (size_t)row0 * DK + i] = sS[i];
+    };
+    if (r == 0 && S_in) write_rows(S_in);
     const int last = S_T ? R : r;  // segments whose map is applied
     for (int j = 0; j < last; ++j) {
         const float *Mj = M + ((size_t)j * BH + bh) * mz;
-        const float *Nj = N + ((size_t)j * BH + bh) * sz;
+        const float *Nj = N + ((size_t)j * BH + bh) * sz + (size_t)row0 * DK;
         for (int i = threadIdx.x; i < DK * DK / 4; i += kSegThreads)
             reinterpret_cast<float4 *>(sM)[i] = reinterpret_cast<const float4 *>(Mj)[i];
-        __syncthreads();
-        float acc[RA][CA];
+        float acc[RPT][8];
 #pragma unroll
-        for (int a = 0; a < RA; ++a)
-#pragma unroll
-            for (int c = 0; c < CA; ++c) acc[a][c] = Nj[(size_t)(ty + 16 * a) * DK + tx + 16 * c];
+        for (int a = 0; a < RPT; ++a) {
+            const float *nr = Nj + (size_t)(rg + RG * a) * DK;
+            const float4 n0 = *reinterpret_cast<const float4 *>(nr + c0);
+            const float4 n1 = *reinterpret_cast<const float4 *>(nr + c1);
+            acc[a][0] = n0.x; acc[a][1] = n0.y; acc[a][2] = n0.z; acc[a][3] = n0.w;
+            acc[a][4] = n1.x; acc[a][5] = n1.y; acc[a][6] = n1.z; acc[a][7] = n1.w;
+        }
+        __syncthreads();  // sM staged
 #pragma unroll 4
         for (int l = 0; l < DK; ++l) {
-            float sv[RA], mv[CA];
+            const float4 m0 = *reinterpret_cast<const float4 *>(sM + l * DK + c0);
+            const float4 m1 = *reinterpret_cast<const float4 *>(sM + l * DK + c1);
+            const float mv[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
 #pragma unroll
-            for (int a = 0; a < RA; ++a) sv[a] = sS[(ty + 16 * a) * DK + l];
+            for (int a = 0; a < RPT; ++a) {
+                const float sv = sS[(rg + RG * a) * DK + l];
 #pragma unroll
-            for (int c = 0; c < CA; ++c) mv[c] = sM[l * DK + tx + 16 * c];
-#pragma unroll
-            for (int a = 0; a < RA; ++a)
-#pragma unroll
-                for (int c = 0; c < CA; ++c) acc[a][c] = fmaf(sv[a], mv[c], acc[a][c]);
+                for (int c = 0; c < 8; ++c) acc[a][c] = fmaf(sv, mv[c], acc[a][c]);
+            }
         }
         __syncthreads();  // every thread is done reading sS and sM
 #pragma unroll
-        for (int a = 0; a < RA; ++a)
-#pragma unroll
-            for (int c = 0; c < CA; ++c) sS[(ty + 16 * a) * DK + tx + 16 * c] = acc[a][c];
+        for (int a = 0; a < RPT; ++a) {
+            float *sr = sS + (rg + RG * a) * DK;
+            *reinterpret_cast<float4 *>(sr + c0) = make_float4(acc[a][0], acc[a][1], acc[a][2], acc[a][3]);
+            *reinterpret_cast<float4 *>(sr + c1) = make_float4(acc[a][4], acc[a][5], acc[a][6], acc[a][7]);
+        }
         __syncthreads();
-        if (j + 1 == r && S_in)
-            for (int i = threadIdx.x; i < DV * DK; i += kSegThreads) S_in[bh * sz + i] = sS[i];
+        if (j + 1 == r && S_in) write_rows(S_in);
     }
-    if (S_T)
-        for (int i = threadIdx.x; i < DV * DK; i += kSegThreads) S_T[bh * sz + i] = sS[i];
+    if (S_T) write_rows(S_T);
 }
 
 // o[b, t, h, :] += S_in[b, h] q~[b, t, h, :] for the tokens of a segment.
-// Block (bh, g) keeps S_in^T in shared memory and walks 32-token tiles
-// g, g + G, ...; a thread owns 4 tokens (tt + 8a) x DV/32 outputs (ti + 32c).
-constexpr int kFixTok = 32;
+// Block (bh, g) keeps S_in^T in shared memory and walks 64-token tiles
+// g, g + G, ...; a thread owns 4 tokens (tg + 16a) x 8 outputs (4 og .. +3
+// and DV/2 + 4 og .. +3), read as float4 rows of S_in^T.  q~ rows are padded
+// by one float so the token groups of a warp hit different banks.
+constexpr int kFixTok = 64;
 
 template <typename Tio, int DK, int DV>
 __global__ void __launch_bounds__(kSegThreads)
     seg_fixup_kernel(int T, int H, const Tio *__restrict__ qt, const float *__restrict__ S_in, Tio *__restrict__ o) {
     extern __shared__ __align__(16) float seg_smem[];
+    constexpr int LDQ = DK + 1;
     float *sSt = seg_smem;            // [DK][DV]: S_in transposed
-    float *sQ = seg_smem + DK * DV;   // [kFixTok][DK]
-    constexpr int CO = DV / 32;
+    float *sQ = seg_smem + DK * DV;   // [kFixTok][LDQ]
+    constexpr int OG = DV / 8, TG = kSegThreads / OG, TA = kFixTok / TG;  // TA tokens per thread
     const int head = blockIdx.x, g = blockIdx.y, G = gridDim.y;
     const int b = head / H, h = head % H;
-    const int ti = threadIdx.x % 32, tt = threadIdx.x / 32;
+    const int og = threadIdx.x % OG, tg = threadIdx.x / OG;
+    const int c0 = 4 * og, c1 = DV / 2 + 4 * og;
     const float *S = S_in + (size_t)head * DV * DK;
     for (int i = threadIdx.x; i < DV * DK; i += kSegThreads) {
         const int col = i / DV, row = i % DV;  // St[col][row] = S[row][col]
@@ -110,37 +150,48 @@ __global__ void __launch_bounds__(kSegThreads)
     for (int tile = g; tile < tiles; tile += G) {
         const int t0 = tile * kFixTok, n = min(kFixTok, T - t0);
         __syncthreads();  // sSt written / previous tile's sQ consumed
-        for (int i = threadIdx.x; i < kFixTok * DK; i += kSegThreads) {
-            const int t = i / DK, j = i % DK;
-            sQ[i] = t < n ? to_f32(qt[(((size_t)b * T + t0 + t) * H + h) * DK + j]) : 0.f;
+        for (int i = threadIdx.x; i < kFixTok * DK / 8; i += kSegThreads) {  // 8 elements per piece
+            const int t = i / (DK / 8), j8 = (i % (DK / 8)) * 8;
+            float v[8];
+            if (t < n)
+                load8(qt + (((size_t)b * T + t0 + t) * H + h) * DK + j8, v);
+            else
+#pragma unroll
+                for (int e = 0; e < 8; ++e) v[e] = 0.f;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) sQ[t * LDQ + j8 + e] = v[e];
         }
         __syncthreads();
-        float acc[4][CO];
+        float acc[TA][8];
 #pragma unroll
-        for (int a = 0; a < 4; ++a)
+        for (int a = 0; a < TA; ++a)
 #pragma unroll
-            for (int c = 0; c < CO; ++c) acc[a][c] = 0.f;
+            for (int c = 0; c < 8; ++c) acc[a][c] = 0.f;
 #pragma unroll 4
         for (int j = 0; j < DK; ++j) {
-            float qv[4], sv[CO];
+            const float4 s0 = *reinterpret_cast<const float4 *>(sSt + j * DV + c0);
+            const float4 s1 = *reinterpret_cast<const float4 *>(sSt + j * DV + c1);
+            const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
 #pragma unroll
-            for (int a = 0; a < 4; ++a) qv[a] = sQ[(tt + 8 * a) * DK + j];
+            for (int a = 0; a < TA; ++a) {
+                const float qv = sQ[(tg + TG * a) * LDQ + j];
 #pragma unroll
-            for (int c = 0; c < CO; ++c) sv[c] = sSt[j * DV + ti + 32 * c];
-#pragma unroll
-            for (int a = 0; a < 4; ++a)
-#pragma unroll
-                for (int c = 0; c < CO; ++c) acc[a][c] = fmaf(qv[a], sv[c], acc[a][c]);
+                for (int c = 0; c < 8; ++c) acc[a][c] = fmaf(qv, sv[c], acc[a][c]);
+            }
         }
 #pragma unroll
-        for (int a = 0; a < 4; ++a) {
-            const int t = tt + 8 * a;
+        for (int a = 0; a < TA; ++a) {
+            const int t = tg + TG * a;
             if (t >= n) continue;
             Tio *orow = o + (((size_t)b * T + t0 + t) * H + h) * DV;
 #pragma unroll
-            for (int c = 0; c < CO; ++c) {
-                const int i = ti + 32 * c;
-                orow[i] = from_f32<Tio>(to_f32(orow[i]) + acc[a][c]);
+            for (int half = 0; half < 2; ++half) {
+                const int cc = half ? c1 : c0;
+                float cur[4];
+                ld_row4(orow + cc, cur);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) cur[e] += acc[a][4 * half + e];
+                st_row4(orow + cc, cur);
             }
         }
     }
@@ -154,29 +205,27 @@ inline cudaError_t launch_seg_identity(float *S, int BH, int dk, cudaStream_t st
     return cudaGetLastError();
 }
 
-template <int DK, int DV>
-inline cudaError_t launch_seg_combine_t(int R, int r, int BH, const float *M, const float *N, const float *S0,
+template <int DK>
+inline cudaError_t launch_seg_combine_t(int R, int r, int BH, int dv, const float *M, const float *N, const float *S0,
                                         float *S_in, float *S_T, cudaStream_t stream) {
-    const int smem = (DV * DK + DK * DK) * 4;
-    cudaError_t e = cudaFuncSetAttribute(seg_combine_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    const int smem = (DK * DK + kCombRows * DK) * 4;
+    cudaError_t e = cudaFuncSetAttribute(seg_combine_kernel<DK>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    seg_combine_kernel<DK, DV><<<BH, kSegThreads, smem, stream>>>(R, r, BH, M, N, S0, S_in, S_T);
+    seg_combine_kernel<DK><<<dim3(BH, dv / kCombRows), kSegThreads, smem, stream>>>(R, r, BH, dv, M, N, S0, S_in, S_T);
     g_launches.fetch_add(1, std::memory_order_relaxed);
     return cudaGetLastError();
 }
 
 inline cudaError_t launch_seg_combine(int R, int r, int BH, int dk, int dv, const float *M, const float *N,
                                       const float *S0, float *S_in, float *S_T, cudaStream_t stream) {
-    if (dk == 128 && dv == 128) return launch_seg_combine_t<128, 128>(R, r, BH, M, N, S0, S_in, S_T, stream);
-    if (dk == 128 && dv == 64) return launch_seg_combine_t<128, 64>(R, r, BH, M, N, S0, S_in, S_T, stream);
-    if (dk == 64 && dv == 128) return launch_seg_combine_t<64, 128>(R, r, BH, M, N, S0, S_in, S_T, stream);
-    return launch_seg_combine_t<64, 64>(R, r, BH, M, N, S0, S_in, S_T, stream);
+    return dk == 128 ? launch_seg_combine_t<128>(R, r, BH, dv, M, N, S0, S_in, S_T, stream)
+                     : launch_seg_combine_t<64>(R, r, BH, dv, M, N, S0, S_in, S_T, stream);
 }
 
 template <typename Tio, int DK, int DV>
 inline cudaError_t launch_seg_fixup_t(int B, int T, int H, const void *qt, const float *S_in, void *o,
                                       cudaStream_t stream) {
-    const int smem = (DK * DV + kFixTok * DK) * 4;
+    const int smem = (DK * DV + kFixTok * (DK + 1)) * 4;
     auto kern = seg_fixup_kernel<Tio, DK, DV>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
