@@ -522,7 +522,12 @@ gdr_status gdr_seg_fixup(int B, int T, int H, int dk, int dv, gdr_dtype dt, cons
     GDR_REQUIRE_PTR(S_in);
     GDR_REQUIRE_PTR(o);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    cudaError_t e = dt == GDR_F32 ? launch_seg_fixup<float>(B, T, H, dk, dv, qt, S_in, o, s)
+    // bf16 with dk = dv = 128 on the tensor cores (GDR_SEG_FIXUP=simt selects
+    // the CUDA-core kernel, used to cross-check it)
+    const char *sel = getenv("GDR_SEG_FIXUP");
+    const bool tc = dt == GDR_BF16 && dk == 128 && dv == 128 && !(sel && strcmp(sel, "simt") == 0);
+    cudaError_t e = tc ? launch_seg_fixup_tc(B, T, H, qt, S_in, o, s)
+                  : dt == GDR_F32 ? launch_seg_fixup<float>(B, T, H, dk, dv, qt, S_in, o, s)
                                   : launch_seg_fixup<__nv_bfloat16>(B, T, H, dk, dv, qt, S_in, o, s);
     if (e != cudaSuccess) return cuda_fail(e, fn);
     return GDR_OK;

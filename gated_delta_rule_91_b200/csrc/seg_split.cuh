@@ -15,6 +15,8 @@
 #pragma once
 
 #include "common.cuh"
+#include "sm100.cuh"
+#include "fwd_tc.cuh"  // make_token_map
 
 namespace gdr {
 
@@ -195,6 +197,149 @@ __global__ void __launch_bounds__(kSegThreads)
             }
         }
     }
+}
+
+// Tensor-core correction for bf16 with dk = dv = 128: per 128-token tile,
+// D[t, i] = sum_j q~[t, j] S_in[i, j] is one M128 N128 K128 tcgen05 product
+// (A = the q~ tile, B = S_in as bf16, both K-major with 128-byte swizzle, D in
+// TMEM); the epilogue adds D into the o tile staged by TMA and stores it back
+// with TMA.  Block (bh, g) converts S_in once and walks tiles g, g + G, ...
+// 128 threads: thread t of the epilogue owns token row t of the tile (its
+// warp's TMEM lane quarter).
+constexpr int kFixTcThreads = 128;
+struct FixTcLayout {
+    static constexpr int S = 0;           // S_in bf16: 2 K-halves x [128][64], 16 KB each
+    static constexpr int Q = 32768;       // q~ tile: 2 K-halves x [128][64]
+    static constexpr int O = 65536;       // o tile: 2 channel halves x 2 token halves x [64][64]
+    static constexpr int BAR = 98304;     // 2 mbarriers + TMEM address
+    static constexpr int kBytes = BAR + 64;
+    static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024
+};
+
+__global__ void __launch_bounds__(kFixTcThreads)
+    seg_fixup_tc_kernel(const __grid_constant__ CUtensorMap tm_qt, const __grid_constant__ CUtensorMap tm_o, int T,
+                        int H, const float *__restrict__ S_in) {
+    using namespace sm100;
+    using L = FixTcLayout;
+    extern __shared__ uint8_t fix_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(fix_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bar_tma = reinterpret_cast<uint64_t *>(sm + L::BAR);
+    uint64_t *bar_mma = bar_tma + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_tma + 2);
+    const int head = blockIdx.x, g = blockIdx.y, G = gridDim.y;
+    const int b = head / H, h = head % H;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    if (tid == 0) {
+        mbar_init(bar_tma, 1);
+        mbar_init(bar_mma, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) tmem_alloc(tmem_slot, 128);
+    // S_in (fp32 [128][128]) -> bf16 B operand: row i, column j in K-half j / 64
+    const float *S = S_in + (size_t)head * 128 * 128;
+    for (int p = tid; p < 128 * 64; p += kFixTcThreads) {
+        const int i = p / 64, j = (p % 64) * 2;
+        const float2 v = *reinterpret_cast<const float2 *>(S + (size_t)i * 128 + j);
+        st_sw_bf16x2(sm + L::S + (j >> 6) * 16384, i, j & 63, v.x, v.y);
+    }
+    fence_async_smem();
+    tc_before_sync();
+    __syncthreads();
+    tc_after_sync();
+    const uint32_t tl = *tmem_slot;
+    const int tiles = (T + 127) / 128;
+    bool ok = true;
+    uint32_t ph = 0;
+    for (int tile = g; tile < tiles; tile += G, ph ^= 1u) {
+        const int t0 = tile * 128;
+        if (tid == 0) {
+            mbar_expect_tx(bar_tma, 65536);
+#pragma unroll
+            for (int kh = 0; kh < 2; ++kh)
+#pragma unroll
+                for (int th = 0; th < 2; ++th) {
+                    tma_load_4d(sm + L::Q + kh * 16384 + th * 8192, &tm_qt, bar_tma, kh * 64, h, t0 + th * 64, b);
+                    tma_load_4d(sm + L::O + kh * 16384 + th * 8192, &tm_o, bar_tma, kh * 64, h, t0 + th * 64, b);
+                }
+        }
+        if (!__syncthreads_and(mbar_wait(bar_tma, ph))) {  // the block agrees before leaving
+            ok = false;
+            break;
+        }
+        if (tid == 0) {
+            tc_after_sync();
+            const uint32_t sq = smem_u32(sm + L::Q), ss = smem_u32(sm + L::S);
+#pragma unroll
+            for (int kh = 0; kh < 2; ++kh)
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16(tl, smem_desc_sw128(sq + kh * 16384 + kk * 32, 16, 1024),
+                             smem_desc_sw128(ss + kh * 16384 + kk * 32, 16, 1024), idesc_bf16(128, 128, false, false),
+                             (kh | kk) != 0);
+            mma_commit(bar_mma);
+        }
+        if (!__syncthreads_and(mbar_wait(bar_mma, ph))) {
+            ok = false;
+            break;
+        }
+        tc_after_sync();
+        // epilogue: row t of the tile (token t0 + t) += D[t, :]
+        const int t = tid, th = t >> 6, r = t & 63;
+#pragma unroll
+        for (int c32 = 0; c32 < 4; ++c32) {
+            float d[32];
+            tmem_ld32(tl + ((uint32_t)(warp * 32) << 16) + c32 * 32, d);
+            uint8_t *tileo = sm + L::O + (c32 >> 1) * 16384 + th * 8192;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int chunk = (c32 & 1) * 4 + q;  // 16-byte chunk of the 128-byte row
+                uint4 *pc = reinterpret_cast<uint4 *>(tileo + sw128_offset(r, chunk));
+                uint4 raw = *pc;
+                __nv_bfloat162 *hv = reinterpret_cast<__nv_bfloat162 *>(&raw);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = __bfloat1622float2(hv[e]);
+                    hv[e] = __floats2bfloat162_rn(f.x + d[q * 8 + 2 * e], f.y + d[q * 8 + 2 * e + 1]);
+                }
+                *pc = raw;
+            }
+        }
+        fence_async_smem();
+        tc_before_sync();
+        __syncthreads();
+        if (tid == 0) {
+#pragma unroll
+            for (int kh = 0; kh < 2; ++kh)
+#pragma unroll
+                for (int th2 = 0; th2 < 2; ++th2)
+                    tma_store_4d(&tm_o, sm + L::O + kh * 16384 + th2 * 8192, kh * 64, h, t0 + th2 * 64, b);
+            bulk_commit();
+            bulk_wait_read_all();  // the o tile is reused by the next load
+        }
+        __syncthreads();
+    }
+    if (!ok) record_status(GDR_ERR_TIMEOUT);
+    if (tid == 0) bulk_wait_all();
+    tc_before_sync();
+    __syncthreads();
+    tc_after_sync();
+    if (warp == 0) tmem_dealloc(tl, 128);
+}
+
+inline cudaError_t launch_seg_fixup_tc(int B, int T, int H, const void *qt, const float *S_in, void *o,
+                                       cudaStream_t stream) {
+    CUtensorMap mq, mo;
+    if (!make_token_map(&mq, qt, B, T, H, 128) || !make_token_map(&mo, o, B, T, H, 128)) return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(seg_fixup_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         FixTcLayout::kAlloc);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int tiles = (T + 127) / 128;
+    const int G = std::max(1, std::min(tiles, (2 * sms + B * H - 1) / (B * H)));
+    seg_fixup_tc_kernel<<<dim3(B * H, G), kFixTcThreads, FixTcLayout::kAlloc, stream>>>(mq, mo, T, H, S_in);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return cudaGetLastError();
 }
 
 inline cudaError_t launch_seg_identity(float *S, int BH, int dk, cudaStream_t stream) {

@@ -126,3 +126,20 @@ def test_orchestrator_over_one_rank_nccl_group():
         assert fro_rel(np64(S_T), np64(S1)) <= TOL_S
     finally:
         dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("T", [1, 100, 128, 1000])
+def test_tensor_core_fixup_matches_cuda_core_fixup(T, monkeypatch):
+    rng = np.random.default_rng(T)
+    B, H = 2, 3
+    qt = torch.from_numpy(rng.standard_normal((B, T, H, 128)).astype(np.float32)).to(torch.bfloat16).cuda()
+    o = torch.from_numpy(rng.standard_normal((B, T, H, 128)).astype(np.float32)).to(torch.bfloat16).cuda()
+    S = torch.from_numpy(rng.standard_normal((B, H, 128, 128)).astype(np.float32) * 0.1).cuda()
+    ref = np64(o) + np.einsum("bhij,bthj->bthi", np64(S), np64(qt))
+    o_tc = gdr.gdr_seg_fixup(qt, S, o.clone())
+    monkeypatch.setenv("GDR_SEG_FIXUP", "simt")
+    o_simt = gdr.gdr_seg_fixup(qt, S, o.clone())
+    gdr.check_status()
+    # the tensor-core product rounds S_in to bf16 (relative 2^-9 per term)
+    assert max_rel(np64(o_tc), ref) <= 1e-2
+    assert max_rel(np64(o_simt), ref) <= 8e-3
