@@ -155,7 +155,117 @@ gdr_status gdr_debug_wait_timeout(int timeout_ms, gdr_stream_t stream) {
     return GDR_OK;
 }
 
-size_t gdr_fwd_workspace_bytes(int, int, int, int, int, gdr_dtype) { return 0; }
+// The two passes of gdr_seg_fwd are independent; the second runs on an
+// auxiliary stream of the device (created on first use, with a fork and a
+// join event), so the two small grids share the GPU.  The enqueue sequence is
+// serialised by a mutex so the events can be reused.
+struct SegAux {
+    cudaStream_t stream = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+};
+std::mutex g_seg_mu;
+SegAux g_seg_aux[64];
+
+// The device's auxiliary stream and events (created on first use); call with
+// g_seg_mu held.
+cudaError_t seg_aux(SegAux **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    SegAux &aux = g_seg_aux[dev];
+    if (aux.stream == nullptr) {
+        e = cudaStreamCreateWithFlags(&aux.stream, cudaStreamNonBlocking);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&aux.fork, cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&aux.join, cudaEventDisableTiming);
+        if (e != cudaSuccess) return e;
+    }
+    *out = &aux;
+    return cudaSuccess;
+}
+
+// One sequence on one GPU as R segments (gdr_fwd for bf16, dk = dv = 128):
+// a B-batch sequence viewed as [B*R, T/R, H, d] runs both passes of the
+// sequence split concurrently -- pass 1 from S_in = 0 into o and N, pass 2
+// with v = 0 from S_in = I into q~ and M -- then the scan of the segment
+// maps and the tensor-core correction o += S_in q~.  Used when the two
+// passes still fit the SMs in one wave (4 B H R <= SMs: each (b, h) of the
+// forward is a cluster of two CTAs) and every segment has at least
+// kSplitMinTokens tokens.
+constexpr int kSplitMinTokens = 2048;
+
+int fwd_split_r(int B, int T, int H, int dk, int dv, gdr_dtype dt) {
+    if (dt != GDR_BF16 || dk != 128 || dv != 128) return 1;
+    const char *sel = getenv("GDR_FWD_SPLIT");
+    if (sel != nullptr && strcmp(sel, "off") == 0) return 1;
+    const char *ksel = getenv("GDR_FWD_KERNEL");
+    if (ksel != nullptr) return 1;  // a forced kernel runs unsplit
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return 1;
+    for (int R = sms / (4 * B * H); R >= 2; --R)
+        if (T % R == 0 && T / R >= kSplitMinTokens) return R;
+    return 1;
+}
+
+struct SplitWs {
+    size_t zero_v, eye, qt, N, M, S_in, total;
+};
+SplitWs split_ws(int B, int T, int H, int R) {
+    auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    SplitWs w;
+    const size_t tok = (size_t)B * T * H * 128 * 2, st = (size_t)B * R * H * 128 * 128 * 4;
+    w.zero_v = 0;
+    w.eye = al(tok);
+    w.qt = w.eye + al(st);
+    w.N = w.qt + al(tok);
+    w.M = w.N + al(st);
+    w.S_in = w.M + al(st);
+    w.total = w.S_in + al(st);
+    return w;
+}
+
+size_t gdr_fwd_workspace_bytes(int B, int T, int H, int dk, int dv, gdr_dtype dt) {
+    if (B < 1 || T < 1 || H < 1) return 0;
+    const int R = fwd_split_r(B, T, H, dk, dv, dt);
+    return R > 1 ? split_ws(B, T, H, R).total : 0;
+}
+
+// The split forward (see fwd_split_r); o, S_T as for gdr_fwd.
+gdr_status run_fwd_split(int B, int T, int H, int R, const void *q, const void *k, const void *v,
+                         const float *la, const float *beta, const float *S0, void *o, float *S_T, void *workspace,
+                         cudaStream_t s) {
+    const char *fn = "gdr_fwd";
+    const SplitWs w = split_ws(B, T, H, R);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    void *zero_v = ws + w.zero_v, *qt = ws + w.qt;
+    float *eye = reinterpret_cast<float *>(ws + w.eye), *N = reinterpret_cast<float *>(ws + w.N);
+    float *M = reinterpret_cast<float *>(ws + w.M), *S_in = reinterpret_cast<float *>(ws + w.S_in);
+    const int Bs = B * R, Ts = T / R;
+    std::lock_guard<std::mutex> lock(g_seg_mu);
+    SegAux *aux = nullptr;
+    cudaError_t e = seg_aux(&aux);
+    if (e == cudaSuccess) e = cudaEventRecord(aux->fork, s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(aux->stream, aux->fork, 0);
+    if (e != cudaSuccess) return cuda_fail(e, fn);
+    // pass 1 (caller's stream) and pass 2 (auxiliary stream)
+    cudaError_t e1 = launch_fwd_tc2(Bs, Ts, H, q, k, v, la, beta, nullptr, o, N, s);
+    cudaError_t e2 = cudaMemsetAsync(zero_v, 0, (size_t)B * T * H * 128 * 2, aux->stream);
+    if (e2 == cudaSuccess) e2 = launch_seg_identity(eye, Bs * H, 128, aux->stream);
+    if (e2 == cudaSuccess) e2 = launch_fwd_tc2(Bs, Ts, H, q, k, zero_v, la, beta, eye, qt, M, aux->stream);
+    cudaError_t ej = cudaEventRecord(aux->join, aux->stream);
+    if (ej == cudaSuccess) ej = cudaStreamWaitEvent(s, aux->join, 0);
+    if (e1 != cudaSuccess) return cuda_fail(e1, fn);
+    if (e2 != cudaSuccess) return cuda_fail(e2, fn);
+    if (ej != cudaSuccess) return cuda_fail(ej, fn);
+    // scan of the segment maps, then o += S_in q~ (segment 0 of a batch with
+    // S0 = 0 adds zero)
+    e = launch_seg_scan(B, R, H, 128, 128, M, N, S0, S_in, S_T, s);
+    if (e == cudaSuccess) e = launch_seg_fixup_tc(Bs, Ts, H, qt, S_in, o, s);
+    if (e != cudaSuccess) return cuda_fail(e, fn);
+    return GDR_OK;
+}
+
 
 gdr_status gdr_fwd(int B, int T, int H, int dk, int dv, gdr_dtype dt, const void *q, const void *k,
                    const void *v, const float *log_alpha, const float *beta, const float *S0,
@@ -173,12 +283,17 @@ gdr_status gdr_fwd(int B, int T, int H, int dk, int dv, gdr_dtype dt, const void
     GDR_OPTIONAL_PTR(S0);
     GDR_OPTIONAL_PTR(S_T);
     GDR_OPTIONAL_PTR(workspace);
+    // The workspace is optional: with at least gdr_fwd_workspace_bytes a long
+    // sequence over few heads runs as parallel segments, otherwise unsplit.
     const size_t need = gdr_fwd_workspace_bytes(B, T, H, dk, dv, dt);
-    if (need > 0 && (workspace == nullptr || workspace_bytes < need))
-        return fail(GDR_ERR_WORKSPACE, "%s: workspace of %zu bytes needed, %zu given", fn, need,
-                    workspace ? workspace_bytes : (size_t)0);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e;
+    // a long sequence over few (b, h): segments of the sequence in parallel
+    // (only with the workspace gdr_fwd_workspace_bytes asks for)
+    if (need > 0 && workspace != nullptr && workspace_bytes >= need) {
+        const int R = fwd_split_r(B, T, H, dk, dv, dt);
+        if (R > 1) return run_fwd_split(B, T, H, R, q, k, v, log_alpha, beta, S0, o, S_T, workspace, s);
+    }
     // bf16 with dk = dv = 128 runs on the tensor cores (the two-SM cluster
     // kernel); GDR_FWD_KERNEL=tc1 selects the single-CTA tensor-core kernel and
     // GDR_FWD_KERNEL=simt the CUDA-core kernel (used to cross-check them).
@@ -416,17 +531,6 @@ gdr_status gdr_block_epilogue(int B, int T, int H, int dv, gdr_dtype dt, const v
     return GDR_OK;
 }
 
-// The two passes of gdr_seg_fwd are independent; the second runs on an
-// auxiliary stream of the device (created on first use, with a fork and a
-// join event), so the two small grids share the GPU.  The enqueue sequence is
-// serialised by a mutex so the events can be reused.
-struct SegAux {
-    cudaStream_t stream = nullptr;
-    cudaEvent_t fork = nullptr, join = nullptr;
-};
-std::mutex g_seg_mu;
-SegAux g_seg_aux[64];
-
 size_t gdr_seg_fwd_workspace_bytes(int B, int T, int H, int dk, int dv, gdr_dtype dt) {
     if (B < 1 || T < 1 || H < 1 || (dk != 64 && dk != 128) || (dv != 64 && dv != 128) ||
         (dt != GDR_F32 && dt != GDR_BF16))
@@ -456,18 +560,11 @@ gdr_status gdr_seg_fwd(int B, int T, int H, int dk, int dv, gdr_dtype dt, const 
     if (workspace_bytes < need)
         return fail(GDR_ERR_WORKSPACE, "%s: workspace of %zu bytes needed, %zu given", fn, need, workspace_bytes);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return cuda_fail(e, fn);
-    if (dev < 0 || dev >= 64) return fail(GDR_ERR_UNSUPPORTED, "%s: device ordinal %d out of range", fn, dev);
     std::lock_guard<std::mutex> lock(g_seg_mu);
-    SegAux &aux = g_seg_aux[dev];
-    if (aux.stream == nullptr) {
-        e = cudaStreamCreateWithFlags(&aux.stream, cudaStreamNonBlocking);
-        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&aux.fork, cudaEventDisableTiming);
-        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&aux.join, cudaEventDisableTiming);
-        if (e != cudaSuccess) return cuda_fail(e, fn);
-    }
+    SegAux *auxp = nullptr;
+    cudaError_t e = seg_aux(&auxp);
+    if (e != cudaSuccess) return cuda_fail(e, fn);
+    SegAux &aux = *auxp;
     e = cudaEventRecord(aux.fork, s);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(aux.stream, aux.fork, 0);
     if (e != cudaSuccess) return cuda_fail(e, fn);

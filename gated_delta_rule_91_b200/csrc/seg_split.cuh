@@ -124,6 +124,82 @@ __global__ void __launch_bounds__(kSegThreads)
     if (S_T) write_rows(S_T);
 }
 
+// The same combine for R segments of every batch on one GPU (a sequence
+// viewed as [B*R, T/R, H, d]): M, N: [B*R, H, ...] with segment r of batch b
+// at head index (b R + r) H + h.  Block (b*H + h, rb) walks r = 0 .. R-1,
+// writing S_in of every segment ([B*R, H, dv, dk]) and the final state S_T
+// ([B, H, dv, dk], may be null).
+template <int DK>
+__global__ void __launch_bounds__(kSegThreads)
+    seg_scan_kernel(int R, int H, int DV, const float *__restrict__ M, const float *__restrict__ N,
+                    const float *__restrict__ S0, float *__restrict__ S_in, float *__restrict__ S_T) {
+    extern __shared__ __align__(16) float seg_smem[];
+    float *sM = seg_smem;             // [DK][DK]
+    float *sS = seg_smem + DK * DK;   // [kCombRows][DK]
+    constexpr int CG = DK / 8, RG = kSegThreads / CG, RPT = kCombRows / RG;
+    const int bh = blockIdx.x, b = bh / H, h = bh % H, row0 = blockIdx.y * kCombRows;
+    const int cg = threadIdx.x % CG, rg = threadIdx.x / CG;
+    const int c0 = 4 * cg, c1 = DK / 2 + 4 * cg;
+    const size_t sz = (size_t)DV * DK, mz = (size_t)DK * DK;
+    for (int i = threadIdx.x; i < kCombRows * DK; i += kSegThreads)
+        sS[i] = S0 ? S0[bh * sz + (size_t)row0 * DK + i] : 0.f;
+    __syncthreads();
+    for (int j = 0; j < R; ++j) {
+        const size_t seg = ((size_t)b * R + j) * H + h;
+        for (int i = threadIdx.x; i < kCombRows * DK; i += kSegThreads) S_in[seg * sz + (size_t)row0 * DK + i] = sS[i];
+        if (j + 1 == R && S_T == nullptr) break;
+        const float *Mj = M + seg * mz;
+        const float *Nj = N + seg * sz + (size_t)row0 * DK;
+        for (int i = threadIdx.x; i < DK * DK / 4; i += kSegThreads)
+            reinterpret_cast<float4 *>(sM)[i] = reinterpret_cast<const float4 *>(Mj)[i];
+        float acc[RPT][8];
+#pragma unroll
+        for (int a = 0; a < RPT; ++a) {
+            const float *nr = Nj + (size_t)(rg + RG * a) * DK;
+            const float4 n0 = *reinterpret_cast<const float4 *>(nr + c0);
+            const float4 n1 = *reinterpret_cast<const float4 *>(nr + c1);
+            acc[a][0] = n0.x; acc[a][1] = n0.y; acc[a][2] = n0.z; acc[a][3] = n0.w;
+            acc[a][4] = n1.x; acc[a][5] = n1.y; acc[a][6] = n1.z; acc[a][7] = n1.w;
+        }
+        __syncthreads();  // sM staged; sS copied out
+#pragma unroll 4
+        for (int l = 0; l < DK; ++l) {
+            const float4 m0 = *reinterpret_cast<const float4 *>(sM + l * DK + c0);
+            const float4 m1 = *reinterpret_cast<const float4 *>(sM + l * DK + c1);
+            const float mv[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+#pragma unroll
+            for (int a = 0; a < RPT; ++a) {
+                const float sv = sS[(rg + RG * a) * DK + l];
+#pragma unroll
+                for (int c = 0; c < 8; ++c) acc[a][c] = fmaf(sv, mv[c], acc[a][c]);
+            }
+        }
+        __syncthreads();
+#pragma unroll
+        for (int a = 0; a < RPT; ++a) {
+            float *sr = sS + (rg + RG * a) * DK;
+            *reinterpret_cast<float4 *>(sr + c0) = make_float4(acc[a][0], acc[a][1], acc[a][2], acc[a][3]);
+            *reinterpret_cast<float4 *>(sr + c1) = make_float4(acc[a][4], acc[a][5], acc[a][6], acc[a][7]);
+        }
+        __syncthreads();
+    }
+    if (S_T)
+        for (int i = threadIdx.x; i < kCombRows * DK; i += kSegThreads) S_T[bh * sz + (size_t)row0 * DK + i] = sS[i];
+}
+
+inline cudaError_t launch_seg_scan(int B, int R, int H, int dk, int dv, const float *M, const float *N,
+                                   const float *S0, float *S_in, float *S_T, cudaStream_t stream) {
+    auto run = [&](auto kern, int DK) -> cudaError_t {
+        const int smem = (DK * DK + kCombRows * DK) * 4;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        kern<<<dim3(B * H, dv / kCombRows), kSegThreads, smem, stream>>>(R, H, dv, M, N, S0, S_in, S_T);
+        g_launches.fetch_add(1, std::memory_order_relaxed);
+        return cudaGetLastError();
+    };
+    return dk == 128 ? run(seg_scan_kernel<128>, 128) : run(seg_scan_kernel<64>, 64);
+}
+
 // o[b, t, h, :] += S_in[b, h] q~[b, t, h, :] for the tokens of a segment.
 // Block (bh, g) keeps S_in^T in shared memory and walks 64-token tiles
 // g, g + G, ...; a thread owns 4 tokens (tg + 16a) x 8 outputs (4 og .. +3

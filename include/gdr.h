@@ -83,8 +83,15 @@ typedef enum { GDR_F32 = 0, GDR_BF16 = 1 } gdr_dtype;
  *   in : q, k [B,T,H,dk]; v [B,T,H,dv] (dtype dt); log_alpha, beta [B,T,H]
  *        fp32; S0 [B,H,dv,dk] fp32 or NULL (zero initial state).
  *   out: o [B,T,H,dv] (dtype dt); S_T [B,H,dv,dk] fp32, or NULL to skip.
- *   workspace: device scratch of at least gdr_fwd_workspace_bytes(...) bytes
- *        (may be NULL when that is 0).
+ *   workspace: optional device scratch.  gdr_fwd_workspace_bytes(...) is
+ *        nonzero only for a long sequence over few heads (bf16, dk = dv =
+ *        128, T/R >= 2048 tokens and 4*B*H*R <= the SM count for some R >= 2;
+ *        GDR_FWD_SPLIT=off in the environment turns it off).  Given at
+ *        least that many bytes, the call runs R segments of the sequence in
+ *        parallel (the sequence split below, inside one GPU: both passes on
+ *        two streams, the scan of the segment maps and the correction);
+ *        with less, or NULL, it runs the sequence as one chain.  The
+ *        results agree up to rounding.
  */
 GDR_API gdr_status gdr_fwd(int B, int T, int H, int dk, int dv, gdr_dtype dt,
                    const void *q, const void *k, const void *v,

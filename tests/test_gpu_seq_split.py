@@ -143,3 +143,32 @@ def test_tensor_core_fixup_matches_cuda_core_fixup(T, monkeypatch):
     # the tensor-core product rounds S_in to bf16 (relative 2^-9 per term)
     assert max_rel(np64(o_tc), ref) <= 1e-2
     assert max_rel(np64(o_simt), ref) <= 8e-3
+
+
+@pytest.mark.parametrize("B,T,H,R", [(1, 16384, 16, 2), (1, 8192, 8, 4), (2, 8192, 4, 4)])
+def test_gdr_fwd_runs_long_sequences_as_parallel_segments(B, T, H, R, monkeypatch):
+    # few (b, h) and a long T: gdr_fwd asks for a workspace and runs R
+    # segments of the sequence in parallel on this GPU; it must agree with the
+    # unsplit kernel and with the oracle
+    L = gdr.lib()
+    assert L.gdr_fwd_workspace_bytes(B, T, H, 128, 128, gdr.GDR_BF16) > 0
+    x = synth.gdr_inputs(B, T, H, 128, 128, "bf16", seed=R + B, s0_std=0.02)
+    d = {n: dev(t) for n, t in x.items() if t is not None}
+    o, S_T = gdr.gdr_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["S0"])
+    monkeypatch.setenv("GDR_FWD_SPLIT", "off")
+    assert L.gdr_fwd_workspace_bytes(B, T, H, 128, 128, gdr.GDR_BF16) == 0
+    o1, S1 = gdr.gdr_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["S0"])
+    gdr.check_status()
+    assert max_rel(np64(o), np64(o1)) <= TOL_O["bf16"]
+    assert fro_rel(np64(S_T), np64(S1)) <= TOL_S
+    h = H - 1
+    sl = lambda n: np64(x[n][:, :, h:h + 1])
+    o_ref, S_ref = oracle.gdr_fwd(sl("q"), sl("k"), sl("v"), sl("log_alpha"), sl("beta"),
+                                  np64(x["S0"][:, h:h + 1]))
+    assert max_rel(np64(o[:, :, h:h + 1]), o_ref) <= TOL_O["bf16"]
+    assert fro_rel(np64(S_T[:, h:h + 1]), S_ref) <= TOL_S
+
+
+def test_gdr_fwd_does_not_split_the_layer_workload():
+    assert gdr.lib().gdr_fwd_workspace_bytes(4, 4096, 16, 128, 128, gdr.GDR_BF16) == 0
+    assert gdr.lib().gdr_fwd_workspace_bytes(1, 1000, 16, 128, 128, gdr.GDR_BF16) == 0
