@@ -58,10 +58,27 @@ def parse_args():
                         "(a short command for profilers) and exit")
     p.add_argument("--profile-gdn2", metavar="B,T,H", default=None,
                    help="only run gdr2_fwd twice on seeded bf16 d=128 inputs of this shape and exit")
+    p.add_argument("--profile-gdn2-bwd", metavar="B,T,H", default=None,
+                   help="only run gdr2_bwd twice on seeded bf16 d=128 inputs of this shape and exit")
     p.add_argument("--profile-block", metavar="B,T,H", default=None,
                    help="only run the block prologue (K=4) and epilogue twice each on seeded bf16 "
                         "d=128 inputs of this shape and exit")
     return p.parse_args()
+
+
+def profile_gdn2_bwd(shape):
+    """Two Gated DeltaNet-2 backward calls on the seeded GDN-2 recipe (bf16,
+    d = 128, S0 ~ N(0, 0.02), dO ~ N(0, 1) seeded 7), then a status check."""
+    import gated_delta_rule_91_b200 as gdr
+    B, T, H = (int(x) for x in shape.split(","))
+    x = synth.gdr2_inputs(B, T, H, 128, 128, "bf16", seed=4, s0_std=0.02)
+    d = {n: (x[n].cuda() if x[n] is not None else None) for n in ("q", "k", "v", "log_alpha", "b", "w", "S0")}
+    dO = torch.randn(d["q"].shape, generator=torch.Generator().manual_seed(7)).to(d["q"].dtype).cuda()
+    for _ in range(2):
+        gdr.gdr2_bwd(d["q"], d["k"], d["v"], d["log_alpha"], d["b"], d["w"], d["S0"], dO)
+    torch.cuda.synchronize()
+    gdr.check_status()
+    print(json.dumps({"profile_gdn2_bwd": shape, "status": "ok"}))
 
 
 def profile_block(shape):
@@ -557,6 +574,9 @@ def main():
         return
     if args.profile_block:
         profile_block(args.profile_block)
+        return
+    if args.profile_gdn2_bwd:
+        profile_gdn2_bwd(args.profile_gdn2_bwd)
         return
     rank, world, local = dist_init(args)
     if args.impl == "reference":
