@@ -141,7 +141,8 @@ def peaks():
 
 
 # ---------------------------------------------------------------------------
-# workload arithmetic (algorithmic bytes and FLOPs)
+# workload arithmetic: algorithmic bytes and FLOPs per launch -- what the
+# algorithm must read, write and compute, the units the roofline divides by
 # ---------------------------------------------------------------------------
 def fwd_bytes(B, T, H, dk, dv, esize=2, with_s0=True, with_st=True):
     per_tok_head = 2 * dk * esize + dv * esize + 8 + dv * esize   # q,k,v in; gates; o out
