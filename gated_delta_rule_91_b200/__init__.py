@@ -14,6 +14,10 @@ Functions (same names as the C entry points):
     gdr_block_prologue(xq, xk, xv, wq, wk, wv, ...)       -> (q, k, v)
     gdr_block_epilogue(o, g, weight, eps)                 -> y
     gdr_seg_fwd / gdr_seg_combine / gdr_seg_fixup         (sequence split; see seq_split)
+
+The calls take the current CUDA stream and allocate nothing inside the
+library, so they can be captured in CUDA graphs.  `autograd` wraps the
+forward/backward pairs as torch.autograd Functions.
 """
 import ctypes
 import os

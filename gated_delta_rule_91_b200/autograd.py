@@ -1,0 +1,61 @@
+"""torch.autograd bindings of the library's forward/backward pairs.
+
+`gated_delta_rule(q, k, v, log_alpha, beta, S0=None)` returns (o, S_T) and
+differentiates through gdr_bwd; `gated_delta_rule2(q, k, v, log_alpha, b, w,
+S0=None)` does the same for Gated DeltaNet-2 through gdr2_bwd.  The forward
+and the backward are the library's CUDA calls: these classes only save the
+inputs and hand the incoming gradients over (the backward recomputes the
+forward's states itself, so nothing else is kept).  Unused outputs arrive as
+zero gradients.
+"""
+import torch
+
+from . import gdr2_bwd, gdr2_fwd, gdr_bwd, gdr_fwd
+
+
+def _c(x):
+    return None if x is None else x.contiguous()
+
+
+class GatedDeltaRule(torch.autograd.Function):
+    """o_t = S_t q_t with S_t = S_{t-1} alpha_t (I - beta_t k_t k_t^T) + beta_t v_t k_t^T."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, log_alpha, beta, S0):
+        q, k, v, log_alpha, beta, S0 = map(_c, (q, k, v, log_alpha, beta, S0))
+        o, S_T = gdr_fwd(q, k, v, log_alpha, beta, S0)
+        ctx.save_for_backward(q, k, v, log_alpha, beta, S0)
+        return o, S_T
+
+    @staticmethod
+    def backward(ctx, dO, dS_T):
+        q, k, v, log_alpha, beta, S0 = ctx.saved_tensors
+        g = gdr_bwd(q, k, v, log_alpha, beta, S0, _c(dO), _c(dS_T), want_dS0=S0 is not None)
+        return g["dq"], g["dk"], g["dv"], g["dlog_alpha"], g["dbeta"], g["dS0"]
+
+
+class GatedDeltaRule2(torch.autograd.Function):
+    """Gated Delta Rule-2: per-channel decay alpha, erase gate b, write gate w."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, log_alpha, b, w, S0):
+        q, k, v, log_alpha, b, w, S0 = map(_c, (q, k, v, log_alpha, b, w, S0))
+        o, S_T = gdr2_fwd(q, k, v, log_alpha, b, w, S0)
+        ctx.save_for_backward(q, k, v, log_alpha, b, w, S0)
+        return o, S_T
+
+    @staticmethod
+    def backward(ctx, dO, dS_T):
+        q, k, v, log_alpha, b, w, S0 = ctx.saved_tensors
+        g = gdr2_bwd(q, k, v, log_alpha, b, w, S0, _c(dO), _c(dS_T), want_dS0=S0 is not None)
+        return g["dq"], g["dk"], g["dv"], g["dlog_alpha"], g["db"], g["dw"], g["dS0"]
+
+
+def gated_delta_rule(q, k, v, log_alpha, beta, S0=None):
+    """Differentiable gdr_fwd: returns (o, S_T)."""
+    return GatedDeltaRule.apply(q, k, v, log_alpha, beta, S0)
+
+
+def gated_delta_rule2(q, k, v, log_alpha, b, w, S0=None):
+    """Differentiable gdr2_fwd: returns (o, S_T)."""
+    return GatedDeltaRule2.apply(q, k, v, log_alpha, b, w, S0)
