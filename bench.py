@@ -169,6 +169,13 @@ def gdr2_bytes(B, T, H, dk, dv, esize=2):
     return B * T * H * per + 2 * B * H * dv * dk * 4
 
 
+def step2_bytes(B, H, dk, dv, esize=2):
+    """Gated DeltaNet-2 decode step: the fp32 state read and written, q, k,
+    v and o, and the per-channel gates log alpha, b (dk) and w (dv) in fp32."""
+    return (2 * B * H * dv * dk * 4 + (2 * dk + 2 * dv) * B * H * esize
+            + (2 * dk + dv) * B * H * 4)
+
+
 def prologue_bytes(B, T, H, dk, dv, K, esize=2):
     """Block prologue: read xq, xk, xv and write q, k, v once, plus the fp32
     conv taps and biases (the conv state is not used on this workload)."""
@@ -394,6 +401,26 @@ def secondary(pk):
                      "tok_per_s": w.B / (us * 1e-6), "achieved_gbs": gbs,
                      "hbm_frac": gbs / pk["hbm_gbs"]}
     del S, xs
+
+    # Gated DeltaNet-2 decode on the same shape (per-channel gates, b in (0, 1))
+    S = synth.decode_state(w.B, w.H, w.dk, w.dv, w.seed).cuda()
+    x2 = synth.gdr2_inputs(w.B, 8, w.H, w.dk, w.dv, "bf16", seed=w.seed)
+    xs2 = [{n: x2[n][:, t].contiguous().cuda() for n in ("q", "k", "v", "log_alpha", "b", "w")} for t in range(8)]
+    call2 = lambda x: gdr.gdr2_step(x["q"], x["k"], x["v"], x["log_alpha"], x["b"], x["w"], S, o=o)
+    for i in range(5):
+        call2(xs2[i % 8])
+    e0, e1 = ev(), ev()
+    torch.cuda.synchronize()
+    e0.record()
+    for i in range(n):
+        call2(xs2[i % 8])
+    e1.record()
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / n
+    gbs = step2_bytes(w.B, w.H, w.dk, w.dv) / (us * 1e-6) / 1e9
+    out["gdn2_decode"] = {"workload": "GDN-2 decode B=256 H=16 d=128 bf16", "us_per_step": us,
+                          "tok_per_s": w.B / (us * 1e-6), "achieved_gbs": gbs, "hbm_frac": gbs / pk["hbm_gbs"]}
+    del S, xs2
 
     # backward at full length T=65536 (timed only when the backward is built)
     w = synth.WORKLOADS["long_fwd_bwd"]

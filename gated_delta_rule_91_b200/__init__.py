@@ -11,6 +11,7 @@ Functions (same names as the C entry points):
     gdr_bwd(q, k, v, log_alpha, beta, S0, dO, dS_T=None) -> dict of gradients
     gdr2_fwd(q, k, v, log_alpha, b, w, S0=None)          -> (o, S_T)
     gdr2_bwd(q, k, v, log_alpha, b, w, S0, dO, dS_T=None) -> dict of gradients
+    gdr2_step(q, k, v, log_alpha, b, w, S)               -> o  (S advanced in place)
     gdr_block_prologue(xq, xk, xv, wq, wk, wv, ...)       -> (q, k, v)
     gdr_block_epilogue(o, g, weight, eps)                 -> y
     gdr_seg_fwd / gdr_seg_combine / gdr_seg_fixup         (sequence split; see seq_split)
@@ -46,6 +47,7 @@ SIGNATURES = {
     "gdr2_fwd_workspace_bytes": (_SZ, [_I] * 6),
     "gdr2_bwd": (_I, [_I] * 6 + [_P] * 16 + [_P, _SZ, _P]),
     "gdr2_bwd_workspace_bytes": (_SZ, [_I] * 6),
+    "gdr2_step": (_I, [_I] * 5 + [_P] * 8 + [_P]),
     "gdr_block_prologue": (_I, [_I] * 7 + [_P] * 11 + [ctypes.c_float] + [_P] * 3 + [_P]),
     "gdr_block_epilogue": (_I, [_I] * 5 + [_P] * 3 + [ctypes.c_float, _P, _P]),
     "gdr_seg_fwd": (_I, [_I] * 6 + [_P] * 9 + [_P, _SZ, _P]),
@@ -200,6 +202,20 @@ def gdr2_fwd(q, k, v, log_alpha, b, w, S0=None, *, o=None, S_T=None, return_stat
     check(L.gdr2_fwd(B, T, H, dk, dv, dt, _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b),
                      _ptr(w), _ptr(S0), _ptr(o), _ptr(S_T), _ptr(ws), ws_bytes, _stream(q)))
     return o, S_T
+
+
+def gdr2_step(q, k, v, log_alpha, b, w, S, *, o=None):
+    """One Gated DeltaNet-2 decode token.  q, k [B,H,dk]; v [B,H,dv];
+    log_alpha, b [B,H,dk] fp32; w [B,H,dv] fp32; S [B,H,dv,dk] fp32 updated in
+    place.  Returns o [B,H,dv]."""
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    _f32(log_alpha, "log_alpha"), _f32(b, "b"), _f32(w, "w"), _f32(S, "S")
+    if o is None:
+        o = torch.empty(B, H, dv, dtype=q.dtype, device=q.device)
+    check(lib().gdr2_step(B, H, dk, dv, _dt(q), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w),
+                          _ptr(S), _ptr(o), _stream(q)))
+    return o
 
 
 def gdr2_bwd(q, k, v, log_alpha, b, w, S0, dO, dS_T=None, *, want_dS0=True, workspace=None):

@@ -342,6 +342,32 @@ gdr_status gdr_step(int B, int H, int dk, int dv, gdr_dtype dt, const void *q, c
     return GDR_OK;
 }
 
+gdr_status gdr2_step(int B, int H, int dk, int dv, gdr_dtype dt, const void *q, const void *k,
+                     const void *v, const float *log_alpha, const float *b, const float *w, float *S, void *o,
+                     gdr_stream_t stream) {
+    const char *fn = "gdr2_step";
+    gdr_status st = check_dims(fn, B, 1, H, dk, dv, dt);
+    if (st != GDR_OK) return st;
+    GDR_REQUIRE_PTR(q);
+    GDR_REQUIRE_PTR(k);
+    GDR_REQUIRE_PTR(v);
+    GDR_REQUIRE_PTR(log_alpha);
+    GDR_REQUIRE_PTR(b);
+    GDR_REQUIRE_PTR(w);
+    GDR_REQUIRE_PTR(S);
+    GDR_REQUIRE_PTR(o);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    if (dt == GDR_F32)
+        e = dk == 128 ? launch_step2<float, 128>(B, H, dv, q, k, v, log_alpha, b, w, S, o, s)
+                      : launch_step2<float, 64>(B, H, dv, q, k, v, log_alpha, b, w, S, o, s);
+    else
+        e = dk == 128 ? launch_step2<__nv_bfloat16, 128>(B, H, dv, q, k, v, log_alpha, b, w, S, o, s)
+                      : launch_step2<__nv_bfloat16, 64>(B, H, dv, q, k, v, log_alpha, b, w, S, o, s);
+    if (e != cudaSuccess) return cuda_fail(e, fn);
+    return GDR_OK;
+}
+
 size_t gdr_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, gdr_dtype dt) {
     if (B < 1 || T < 1 || H < 1 || (dk != 64 && dk != 128) || (dv != 64 && dv != 128)) return 0;
     return bwd_scratch_bytes(B, T, H, dk, dv, dt);

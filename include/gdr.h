@@ -42,7 +42,7 @@
  *  * A launch failure returns GDR_ERR_CUDA.  Kernels that wait on on-chip
  *    barriers give up after a bounded number of polls and record
  *    GDR_ERR_TIMEOUT in a device status word, read by gdr_check_status().
- *  * Outputs must not alias inputs (except S in gdr_step, o in gdr_seg_fixup
+ *  * Outputs must not alias inputs (except S in gdr_step and gdr2_step, o in gdr_seg_fixup
  *    and the conv state in gdr_block_prologue, which are in-out).
  *  * gdr_last_error_string() describes the last non-OK status returned on the
  *    calling thread.
@@ -206,6 +206,22 @@ GDR_API gdr_status gdr2_bwd(int B, int T, int H, int dk, int dv, gdr_dtype dt,
                     float *dlog_alpha, float *db, float *dw, float *dS0,
                     void *workspace, size_t workspace_bytes, gdr_stream_t stream);
 GDR_API size_t gdr2_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, gdr_dtype dt);
+
+/*
+ * Gated DeltaNet-2 single-token decode, state updated in place:
+ *     S' = S Diag(alpha),  S <- S' - (S'(b*k) - w*v) k^T,  o = S q
+ * (the Gated Delta Rule-2 paragraph of "Gated DeltaNet-2: Decoupling Erase
+ * and Write in Linear Attention", agihunt.info/papers/2605.22791; the same
+ * step gdr2_fwd takes per token).
+ *   in : q, k [B,H,dk]; v [B,H,dv] (dtype dt); log_alpha, b [B,H,dk] fp32
+ *        (per key channel); w [B,H,dv] fp32 (per value channel).
+ *   in/out: S [B,H,dv,dk] fp32.   out: o [B,H,dv] (dtype dt).
+ *   Errors: the common size rules (T = 1).
+ */
+GDR_API gdr_status gdr2_step(int B, int H, int dk, int dv, gdr_dtype dt,
+                     const void *q, const void *k, const void *v,
+                     const float *log_alpha, const float *b, const float *w,
+                     float *S, void *o, gdr_stream_t stream);
 
 /*
  * Block prologue: the q/k/v paths of a Gated DeltaNet block between the input

@@ -156,3 +156,20 @@ def test_seg_fwd_checks_workspace_and_pointers():
     assert L.gdr_seg_fwd(*bad, P(FAKE), need, None) == gdr.GDR_ERR_INVALID_ARGUMENT
     assert L.gdr_seg_fixup(1, 4, 1, 64, 64, gdr.GDR_F32, P(FAKE), None, P(FAKE), None) == \
         gdr.GDR_ERR_INVALID_ARGUMENT
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(B=0), gdr.GDR_ERR_INVALID_ARGUMENT),
+    (dict(dk=96), gdr.GDR_ERR_UNSUPPORTED),
+    (dict(w=None), gdr.GDR_ERR_INVALID_ARGUMENT),
+    (dict(S=FAKE + 4), gdr.GDR_ERR_INVALID_ARGUMENT),
+])
+def test_gdr2_step_rejects_bad_arguments(kw, status):
+    a = dict(B=1, H=2, dk=64, dv=64, dt=gdr.GDR_BF16, q=FAKE, k=FAKE, v=FAKE, la=FAKE, b=FAKE, w=FAKE, S=FAKE,
+             o=FAKE)
+    a.update(kw)
+    P = ctypes.c_void_p
+    st = gdr.lib().gdr2_step(a["B"], a["H"], a["dk"], a["dv"], a["dt"], P(a["q"]), P(a["k"]), P(a["v"]),
+                             P(a["la"]), P(a["b"]), P(a["w"]), P(a["S"]), P(a["o"]), None)
+    assert st == status
+    assert gdr.lib().gdr_last_error_string().decode().startswith("gdr2_step")
