@@ -58,12 +58,29 @@ def parse_args():
                         "(a short command for profilers) and exit")
     p.add_argument("--profile-gdn2", metavar="B,T,H", default=None,
                    help="only run gdr2_fwd twice on seeded bf16 d=128 inputs of this shape and exit")
+    p.add_argument("--profile-fwd", metavar="B,T,H", default=None,
+                   help="only run gdr_fwd twice on seeded bf16 d=128 inputs of this shape and exit "
+                        "(long sequences over few heads take the parallel-segment path)")
     p.add_argument("--profile-gdn2-bwd", metavar="B,T,H", default=None,
                    help="only run gdr2_bwd twice on seeded bf16 d=128 inputs of this shape and exit")
     p.add_argument("--profile-block", metavar="B,T,H", default=None,
                    help="only run the block prologue (K=4) and epilogue twice each on seeded bf16 "
                         "d=128 inputs of this shape and exit")
     return p.parse_args()
+
+
+def profile_fwd(shape):
+    """Two gdr_fwd calls on the seeded layer recipe (bf16, d = 128, S0 = 0),
+    then a status check."""
+    import gated_delta_rule_91_b200 as gdr
+    B, T, H = (int(x) for x in shape.split(","))
+    x = synth.gdr_inputs(B, T, H, 128, 128, "bf16", seed=1)
+    d = {n: x[n].cuda() for n in ("q", "k", "v", "log_alpha", "beta")}
+    for _ in range(2):
+        gdr.gdr_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], None)
+    torch.cuda.synchronize()
+    gdr.check_status()
+    print(json.dumps({"profile_fwd": shape, "status": "ok"}))
 
 
 def profile_gdn2_bwd(shape):
@@ -605,6 +622,9 @@ def main():
         return
     if args.profile_gdn2_bwd:
         profile_gdn2_bwd(args.profile_gdn2_bwd)
+        return
+    if args.profile_fwd:
+        profile_fwd(args.profile_fwd)
         return
     rank, world, local = dist_init(args)
     if args.impl == "reference":

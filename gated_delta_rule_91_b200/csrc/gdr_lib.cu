@@ -250,18 +250,26 @@ gdr_status run_fwd_split(int B, int T, int H, int R, const void *q, const void *
     if (e != cudaSuccess) return cuda_fail(e, fn);
     // pass 1 (caller's stream) and pass 2 (auxiliary stream)
     cudaError_t e1 = launch_fwd_tc2(Bs, Ts, H, q, k, v, la, beta, nullptr, o, N, s);
-    cudaError_t e2 = cudaMemsetAsync(zero_v, 0, (size_t)B * T * H * 128 * 2, aux->stream);
-    if (e2 == cudaSuccess) e2 = launch_seg_identity(eye, Bs * H, 128, aux->stream);
-    if (e2 == cudaSuccess) e2 = launch_fwd_tc2(Bs, Ts, H, q, k, zero_v, la, beta, eye, qt, M, aux->stream);
+    // With S0 = 0 and one batch, segment 0 needs neither q~ (its S_in is 0)
+    // nor M (segment 1 starts from N_0): pass 2 covers segments 1 .. R-1.
+    const int m0 = (S0 == nullptr && B == 1) ? 1 : 0;
+    const size_t tok_seg = (size_t)Ts * H * 128;  // elements of one segment
+    cudaError_t e2 = cudaMemsetAsync(zero_v, 0, (size_t)(Bs - m0) * tok_seg * 2, aux->stream);
+    if (e2 == cudaSuccess) e2 = launch_seg_identity(eye, (Bs - m0) * H, 128, aux->stream);
+    if (e2 == cudaSuccess)
+        e2 = launch_fwd_tc2(Bs - m0, Ts, H, static_cast<const __nv_bfloat16 *>(q) + m0 * tok_seg,
+                            static_cast<const __nv_bfloat16 *>(k) + m0 * tok_seg, zero_v, la + m0 * (size_t)Ts * H,
+                            beta + m0 * (size_t)Ts * H, eye, static_cast<__nv_bfloat16 *>(qt) + m0 * tok_seg,
+                            M + m0 * (size_t)H * 128 * 128, aux->stream);
     cudaError_t ej = cudaEventRecord(aux->join, aux->stream);
     if (ej == cudaSuccess) ej = cudaStreamWaitEvent(s, aux->join, 0);
     if (e1 != cudaSuccess) return cuda_fail(e1, fn);
     if (e2 != cudaSuccess) return cuda_fail(e2, fn);
     if (ej != cudaSuccess) return cuda_fail(ej, fn);
-    // scan of the segment maps, then o += S_in q~ (segment 0 of a batch with
-    // S0 = 0 adds zero)
+    // scan of the segment maps, then o += S_in q~
     e = launch_seg_scan(B, R, H, 128, 128, M, N, S0, S_in, S_T, s);
-    if (e == cudaSuccess) e = launch_seg_fixup_tc(Bs, Ts, H, qt, S_in, o, s);
+    // with S0 = 0 the first segment of every batch has S_in = 0: skip it
+    if (e == cudaSuccess) e = launch_seg_fixup_tc(B, Ts, H, qt, S_in, o, s, R, S0 == nullptr ? 1 : 0);
     if (e != cudaSuccess) return cuda_fail(e, fn);
     return GDR_OK;
 }

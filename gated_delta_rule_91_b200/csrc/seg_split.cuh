@@ -128,7 +128,8 @@ __global__ void __launch_bounds__(kSegThreads)
 // viewed as [B*R, T/R, H, d]): M, N: [B*R, H, ...] with segment r of batch b
 // at head index (b R + r) H + h.  Block (b*H + h, rb) walks r = 0 .. R-1,
 // writing S_in of every segment ([B*R, H, dv, dk]) and the final state S_T
-// ([B, H, dv, dk], may be null).
+// ([B, H, dv, dk], may be null).  With S0 null the first segment's M is
+// never read (S is zero there).
 template <int DK>
 __global__ void __launch_bounds__(kSegThreads)
     seg_scan_kernel(int R, int H, int DV, const float *__restrict__ M, const float *__restrict__ N,
@@ -148,6 +149,13 @@ __global__ void __launch_bounds__(kSegThreads)
         const size_t seg = ((size_t)b * R + j) * H + h;
         for (int i = threadIdx.x; i < kCombRows * DK; i += kSegThreads) S_in[seg * sz + (size_t)row0 * DK + i] = sS[i];
         if (j + 1 == R && S_T == nullptr) break;
+        if (j == 0 && S0 == nullptr) {  // S = 0: the map of segment 0 is N_0 alone (M_0 is not read)
+            __syncthreads();
+            for (int i = threadIdx.x; i < kCombRows * DK; i += kSegThreads)
+                sS[i] = N[seg * sz + (size_t)row0 * DK + i];
+            __syncthreads();
+            continue;
+        }
         const float *Mj = M + seg * mz;
         const float *Nj = N + seg * sz + (size_t)row0 * DK;
         for (int i = threadIdx.x; i < DK * DK / 4; i += kSegThreads)
@@ -279,40 +287,49 @@ __global__ void __launch_bounds__(kSegThreads)
 // D[t, i] = sum_j q~[t, j] S_in[i, j] is one M128 N128 K128 tcgen05 product
 // (A = the q~ tile, B = S_in as bf16, both K-major with 128-byte swizzle, D in
 // TMEM); the epilogue adds D into the o tile staged by TMA and stores it back
-// with TMA.  Block (bh, g) converts S_in once and walks tiles g, g + G, ...
-// 128 threads: thread t of the epilogue owns token row t of the tile (its
-// warp's TMEM lane quarter).
+// with TMA.  Two stages: the next tile's loads fly while this one is
+// multiplied and finished.  128 threads: thread t of the epilogue owns token
+// row t of the tile (its warp's TMEM lane quarter).
+//
+// The heads are the segments r0 .. R-1 of every batch of a [B*R, T, H, 128]
+// view (a plain [B, T, H, 128] tensor is R = 1, r0 = 0): block (x, g) takes
+// batch x / ((R - r0) H), segment r0 + (x / H) % (R - r0), head x % H, and
+// walks tiles g, g + G, ...
 constexpr int kFixTcThreads = 128;
 struct FixTcLayout {
     static constexpr int S = 0;           // S_in bf16: 2 K-halves x [128][64], 16 KB each
-    static constexpr int Q = 32768;       // q~ tile: 2 K-halves x [128][64]
-    static constexpr int O = 65536;       // o tile: 2 channel halves x 2 token halves x [64][64]
-    static constexpr int BAR = 98304;     // 2 mbarriers + TMEM address
+    static constexpr int ST0 = 32768;     // stage s at ST0 + s * 65536: q~ tile (2 K-halves x [128][64]),
+    static constexpr int QOFF = 0;        //   then the o tile (2 channel halves x 2 token halves x [64][64])
+    static constexpr int OOFF = 32768;
+    static constexpr int BAR = ST0 + 2 * 65536;  // 2 load barriers, 1 MMA barrier, TMEM address
     static constexpr int kBytes = BAR + 64;
     static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024
 };
 
 __global__ void __launch_bounds__(kFixTcThreads)
     seg_fixup_tc_kernel(const __grid_constant__ CUtensorMap tm_qt, const __grid_constant__ CUtensorMap tm_o, int T,
-                        int H, const float *__restrict__ S_in) {
+                        int H, int R, int r0, const float *__restrict__ S_in) {
     using namespace sm100;
     using L = FixTcLayout;
     extern __shared__ uint8_t fix_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(fix_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t *bar_tma = reinterpret_cast<uint64_t *>(sm + L::BAR);
-    uint64_t *bar_mma = bar_tma + 1;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_tma + 2);
-    const int head = blockIdx.x, g = blockIdx.y, G = gridDim.y;
-    const int b = head / H, h = head % H;
+    uint64_t *bar_tma = reinterpret_cast<uint64_t *>(sm + L::BAR);  // [2]
+    uint64_t *bar_mma = bar_tma + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_tma + 3);
+    const int nseg = R - r0;
+    const int b = blockIdx.x / (nseg * H), r = r0 + (blockIdx.x / H) % nseg, h = blockIdx.x % H;
+    const int bs = b * R + r;  // batch index in the [B*R, T, H, 128] view
+    const int g = blockIdx.y, G = gridDim.y;
     const int tid = threadIdx.x, warp = tid >> 5;
     if (tid == 0) {
-        mbar_init(bar_tma, 1);
+        mbar_init(&bar_tma[0], 1);
+        mbar_init(&bar_tma[1], 1);
         mbar_init(bar_mma, 1);
         fence_mbar_init();
     }
     if (warp == 0) tmem_alloc(tmem_slot, 128);
     // S_in (fp32 [128][128]) -> bf16 B operand: row i, column j in K-half j / 64
-    const float *S = S_in + (size_t)head * 128 * 128;
+    const float *S = S_in + ((size_t)bs * H + h) * 128 * 128;
     for (int p = tid; p < 128 * 64; p += kFixTcThreads) {
         const int i = p / 64, j = (p % 64) * 2;
         const float2 v = *reinterpret_cast<const float2 *>(S + (size_t)i * 128 + j);
@@ -324,27 +341,31 @@ __global__ void __launch_bounds__(kFixTcThreads)
     tc_after_sync();
     const uint32_t tl = *tmem_slot;
     const int tiles = (T + 127) / 128;
-    bool ok = true;
-    uint32_t ph = 0;
-    for (int tile = g; tile < tiles; tile += G, ph ^= 1u) {
+    auto issue_loads = [&](int tile, int st) {  // one thread
+        uint8_t *stage = sm + L::ST0 + st * 65536;
         const int t0 = tile * 128;
-        if (tid == 0) {
-            mbar_expect_tx(bar_tma, 65536);
+        mbar_expect_tx(&bar_tma[st], 65536);
 #pragma unroll
-            for (int kh = 0; kh < 2; ++kh)
+        for (int kh = 0; kh < 2; ++kh)
 #pragma unroll
-                for (int th = 0; th < 2; ++th) {
-                    tma_load_4d(sm + L::Q + kh * 16384 + th * 8192, &tm_qt, bar_tma, kh * 64, h, t0 + th * 64, b);
-                    tma_load_4d(sm + L::O + kh * 16384 + th * 8192, &tm_o, bar_tma, kh * 64, h, t0 + th * 64, b);
-                }
-        }
-        if (!__syncthreads_and(mbar_wait(bar_tma, ph))) {  // the block agrees before leaving
+            for (int th = 0; th < 2; ++th) {
+                tma_load_4d(stage + L::QOFF + kh * 16384 + th * 8192, &tm_qt, &bar_tma[st], kh * 64, h, t0 + th * 64, bs);
+                tma_load_4d(stage + L::OOFF + kh * 16384 + th * 8192, &tm_o, &bar_tma[st], kh * 64, h, t0 + th * 64, bs);
+            }
+    };
+    if (tid == 0 && g < tiles) issue_loads(g, 0);
+    bool ok = true;
+    int k = 0;
+    for (int tile = g; tile < tiles; tile += G, ++k) {
+        const int st = k & 1;
+        uint8_t *stage = sm + L::ST0 + st * 65536;
+        if (!__syncthreads_and(mbar_wait(&bar_tma[st], (uint32_t)(k >> 1) & 1u))) {  // the block agrees
             ok = false;
             break;
         }
         if (tid == 0) {
             tc_after_sync();
-            const uint32_t sq = smem_u32(sm + L::Q), ss = smem_u32(sm + L::S);
+            const uint32_t sq = smem_u32(stage + L::QOFF), ss = smem_u32(sm + L::S);
 #pragma unroll
             for (int kh = 0; kh < 2; ++kh)
 #pragma unroll
@@ -353,23 +374,29 @@ __global__ void __launch_bounds__(kFixTcThreads)
                              smem_desc_sw128(ss + kh * 16384 + kk * 32, 16, 1024), idesc_bf16(128, 128, false, false),
                              (kh | kk) != 0);
             mma_commit(bar_mma);
+            // the next tile into the other stage, once its previous o tile has
+            // been read out by the TMA store
+            if (tile + G < tiles) {
+                bulk_wait_read_all();
+                issue_loads(tile + G, st ^ 1);
+            }
         }
-        if (!__syncthreads_and(mbar_wait(bar_mma, ph))) {
+        if (!__syncthreads_and(mbar_wait(bar_mma, (uint32_t)k & 1u))) {
             ok = false;
             break;
         }
         tc_after_sync();
         // epilogue: row t of the tile (token t0 + t) += D[t, :]
-        const int t = tid, th = t >> 6, r = t & 63;
+        const int t = tid, th = t >> 6, rr = t & 63;
 #pragma unroll
         for (int c32 = 0; c32 < 4; ++c32) {
             float d[32];
             tmem_ld32(tl + ((uint32_t)(warp * 32) << 16) + c32 * 32, d);
-            uint8_t *tileo = sm + L::O + (c32 >> 1) * 16384 + th * 8192;
+            uint8_t *tileo = stage + L::OOFF + (c32 >> 1) * 16384 + th * 8192;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const int chunk = (c32 & 1) * 4 + q;  // 16-byte chunk of the 128-byte row
-                uint4 *pc = reinterpret_cast<uint4 *>(tileo + sw128_offset(r, chunk));
+                uint4 *pc = reinterpret_cast<uint4 *>(tileo + sw128_offset(rr, chunk));
                 uint4 raw = *pc;
                 __nv_bfloat162 *hv = reinterpret_cast<__nv_bfloat162 *>(&raw);
 #pragma unroll
@@ -382,17 +409,16 @@ __global__ void __launch_bounds__(kFixTcThreads)
         }
         fence_async_smem();
         tc_before_sync();
-        __syncthreads();
+        __syncthreads();  // o tile complete; TMEM free for the next product
         if (tid == 0) {
+            const int t0 = tile * 128;
 #pragma unroll
             for (int kh = 0; kh < 2; ++kh)
 #pragma unroll
                 for (int th2 = 0; th2 < 2; ++th2)
-                    tma_store_4d(&tm_o, sm + L::O + kh * 16384 + th2 * 8192, kh * 64, h, t0 + th2 * 64, b);
+                    tma_store_4d(&tm_o, stage + L::OOFF + kh * 16384 + th2 * 8192, kh * 64, h, t0 + th2 * 64, bs);
             bulk_commit();
-            bulk_wait_read_all();  // the o tile is reused by the next load
         }
-        __syncthreads();
     }
     if (!ok) record_status(GDR_ERR_TIMEOUT);
     if (tid == 0) bulk_wait_all();
@@ -402,18 +428,22 @@ __global__ void __launch_bounds__(kFixTcThreads)
     if (warp == 0) tmem_dealloc(tl, 128);
 }
 
+// o [B*R, T, H, 128] += S_in q~ for the segments r0 .. R-1 of every batch
+// (R = 1, r0 = 0: a plain [B, T, H, 128] tensor).
 inline cudaError_t launch_seg_fixup_tc(int B, int T, int H, const void *qt, const float *S_in, void *o,
-                                       cudaStream_t stream) {
+                                       cudaStream_t stream, int R = 1, int r0 = 0) {
     CUtensorMap mq, mo;
-    if (!make_token_map(&mq, qt, B, T, H, 128) || !make_token_map(&mo, o, B, T, H, 128)) return cudaErrorInvalidValue;
+    if (!make_token_map(&mq, qt, B * R, T, H, 128) || !make_token_map(&mo, o, B * R, T, H, 128))
+        return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(seg_fixup_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          FixTcLayout::kAlloc);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int heads = B * (R - r0) * H;
     const int tiles = (T + 127) / 128;
-    const int G = std::max(1, std::min(tiles, (2 * sms + B * H - 1) / (B * H)));
-    seg_fixup_tc_kernel<<<dim3(B * H, G), kFixTcThreads, FixTcLayout::kAlloc, stream>>>(mq, mo, T, H, S_in);
+    const int G = std::max(1, std::min(tiles, (sms + heads - 1) / heads));
+    seg_fixup_tc_kernel<<<dim3(heads, G), kFixTcThreads, FixTcLayout::kAlloc, stream>>>(mq, mo, T, H, R, r0, S_in);
     g_launches.fetch_add(1, std::memory_order_relaxed);
     return cudaGetLastError();
 }

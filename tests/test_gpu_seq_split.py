@@ -172,3 +172,39 @@ def test_gdr_fwd_runs_long_sequences_as_parallel_segments(B, T, H, R, monkeypatc
 def test_gdr_fwd_does_not_split_the_layer_workload():
     assert gdr.lib().gdr_fwd_workspace_bytes(4, 4096, 16, 128, 128, gdr.GDR_BF16) == 0
     assert gdr.lib().gdr_fwd_workspace_bytes(1, 1000, 16, 128, 128, gdr.GDR_BF16) == 0
+
+
+@pytest.mark.parametrize("B,want_state", [(1, True), (1, False), (2, True)])
+def test_split_forward_without_initial_state(B, want_state, monkeypatch):
+    # S0 = 0: the first segment needs no correction, and with one batch no
+    # identity pass either; outputs and the final state must still agree
+    T, H = 8192, 8 if B == 1 else 4
+    x = synth.gdr_inputs(B, T, H, 128, 128, "bf16", seed=20 + B)
+    d = {n: dev(t) for n, t in x.items() if t is not None}
+    assert gdr.lib().gdr_fwd_workspace_bytes(B, T, H, 128, 128, gdr.GDR_BF16) > 0
+    o, S_T = gdr.gdr_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], None, return_state=want_state)
+    monkeypatch.setenv("GDR_FWD_SPLIT", "off")
+    o1, S1 = gdr.gdr_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], None)
+    gdr.check_status()
+    assert max_rel(np64(o), np64(o1)) <= TOL_O["bf16"]
+    if want_state:
+        assert fro_rel(np64(S_T), np64(S1)) <= TOL_S
+    else:
+        assert S_T is None
+    sl = lambda n: np64(x[n][:, :, 1:2])
+    o_ref, _ = oracle.gdr_fwd(sl("q"), sl("k"), sl("v"), sl("log_alpha"), sl("beta"), None)
+    assert max_rel(np64(o[:, :, 1:2]), o_ref) <= TOL_O["bf16"]
+
+
+def test_long_workload_forward_sampled_heads():
+    # B1 T65536 H16 d128 bf16, S0 = 0: gdr_fwd runs it as two parallel
+    # segments; the oracle follows two heads over all 65,536 tokens
+    x = synth.workload_inputs("long_fwd_bwd")
+    d = {n: dev(x[n]) for n in ("q", "k", "v", "log_alpha", "beta")}
+    o, S_T = gdr.gdr_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], None)
+    gdr.check_status()
+    for h in (0, 9):
+        sl = lambda n: np64(x[n][:, :, h:h + 1])
+        o_ref, S_ref = oracle.gdr_fwd(sl("q"), sl("k"), sl("v"), sl("log_alpha"), sl("beta"), None)
+        assert max_rel(np64(o[:, :, h:h + 1]), o_ref) <= TOL_O["bf16"]
+        assert fro_rel(np64(S_T[:, h:h + 1]), S_ref) <= TOL_S
