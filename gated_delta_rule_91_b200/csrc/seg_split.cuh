@@ -442,7 +442,8 @@ inline cudaError_t launch_seg_fixup_tc(int B, int T, int H, const void *qt, cons
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int heads = B * (R - r0) * H;
     const int tiles = (T + 127) / 128;
-    const int G = std::max(1, std::min(tiles, (sms + heads - 1) / heads));
+    // one block per SM (its shared memory): G blocks per head in one wave
+    const int G = std::max(1, std::min(tiles, sms / heads));
     seg_fixup_tc_kernel<<<dim3(heads, G), kFixTcThreads, FixTcLayout::kAlloc, stream>>>(mq, mo, T, H, R, r0, S_in);
     g_launches.fetch_add(1, std::memory_order_relaxed);
     return cudaGetLastError();
