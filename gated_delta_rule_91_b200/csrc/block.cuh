@@ -372,15 +372,16 @@ __global__ void __launch_bounds__(kBlkThreads)
 // bulk copy each; a ring of kBlkStages units per block keeps copies in flight
 // while warps compute (warp w: rows 8w .. 8w+7 of the unit).
 constexpr int kEpilogueRows = 64;
+constexpr int kEpiThreads = 512;  // 16 warps: 4 rows of a unit each
 
 template <typename Tio, int CPL>
-__global__ void __launch_bounds__(kBlkThreads)
+__global__ void __launch_bounds__(kEpiThreads)
     gdr_epilogue_kernel(long long rows, const Tio *__restrict__ o, const Tio *__restrict__ g,
                         const float *__restrict__ weight, float eps, Tio *__restrict__ y) {
     using namespace sm100;
     constexpr int D = CPL * 32;
     constexpr int kTile = kEpilogueRows * D * (int)sizeof(Tio);  // one tensor's unit
-    constexpr int kRowsPerWarp = kEpilogueRows / (kBlkThreads / 32);
+    constexpr int kRowsPerWarp = kEpilogueRows / (kEpiThreads / 32);
     extern __shared__ __align__(128) uint8_t blk_smem[];
     uint8_t *smem = blk_smem;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kBlkStages * 2 * kTile);
@@ -445,18 +446,19 @@ __global__ void __launch_bounds__(kBlkThreads)
 // Grid = SMs x resident blocks of the kernel (capped by the work), so the
 // stride loop covers the units in whole waves.
 // (One cached figure per kernel instantiation: the library runs on B200s only.)
-template <typename Kern> inline int resident_grid(Kern kernel, long long warps_needed, int smem = 0) {
+template <typename Kern>
+inline int resident_grid(Kern kernel, long long warps_needed, int smem = 0, int threads = kBlkThreads) {
     static int per_sm = 0, sms = 0;
     if (per_sm == 0) {
         int dev = 0, nb = 0, ns = 0;
         if (cudaGetDevice(&dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&ns, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kernel, kBlkThreads, smem) != cudaSuccess)
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kernel, threads, smem) != cudaSuccess)
             return 0;
         sms = ns;
         per_sm = nb > 0 ? nb : 1;
     }
-    const long long blocks = (warps_needed + kBlkThreads / 32 - 1) / (kBlkThreads / 32);
+    const long long blocks = (warps_needed + threads / 32 - 1) / (threads / 32);
     return (int)std::min<long long>(blocks, (long long)sms * per_sm);
 }
 
@@ -518,9 +520,9 @@ inline cudaError_t launch_epilogue(long long rows, int dv, const void *o, const 
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
         const long long units = (rows + kEpilogueRows - 1) / kEpilogueRows;
-        const int grid = resident_grid(kern, units * (kBlkThreads / 32), smem);
+        const int grid = resident_grid(kern, units * (kEpiThreads / 32), smem, kEpiThreads);
         if (grid <= 0) return cudaErrorInvalidConfiguration;
-        kern<<<grid, kBlkThreads, smem, stream>>>(rows, static_cast<const Tio *>(o), static_cast<const Tio *>(g),
+        kern<<<grid, kEpiThreads, smem, stream>>>(rows, static_cast<const Tio *>(o), static_cast<const Tio *>(g),
                                                   weight, eps, static_cast<Tio *>(y));
         g_launches.fetch_add(1, std::memory_order_relaxed);
         return cudaGetLastError();
