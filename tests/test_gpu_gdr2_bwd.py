@@ -109,3 +109,15 @@ def test_gdr2_bwd_reports_a_chunk_it_does_not_handle():
         gdr.check_status()
     assert e.value.status == gdr.GDR_ERR_UNSUPPORTED
     gdr.check_status()  # the status word was cleared
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_gdr2_bwd_negative_eigenvalue_erase_gate(dtype):
+    # b in (0, 2): the erase factor can reflect; the gradients must still
+    # match the oracle's reverse mode
+    x = _inputs(2, 200, 2, 128, 128, dtype, seed=41, b_max=2.0)
+    assert float(x["b"].max()) > 1.0
+    dST = torch.randn(2, 2, 128, 128, generator=torch.Generator().manual_seed(3)) * 0.1
+    got = _gpu(x, dST)
+    gdr.check_status()
+    _compare(got, _oracle(x, dST), dtype)
