@@ -33,6 +33,7 @@ def _load():
         lib.oracle_gdr2_bwd.argtypes = [i, i, i, i, i] + [dp] * 16
         lib.oracle_short_conv.argtypes = [i] * 5 + [dp] * 4 + [i, ctypes.c_double, dp, dp]
         lib.oracle_rmsnorm_gate.argtypes = [i] * 4 + [dp] * 3 + [ctypes.c_double, dp]
+        lib.oracle_rmsnorm_gate_bwd.argtypes = [i] * 4 + [dp] * 3 + [ctypes.c_double] + [dp] * 4
         lib.oracle_num_threads.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -150,3 +151,14 @@ def rmsnorm_gate(o, g, weight, eps=0.0):
     y = np.zeros_like(o)
     _load().oracle_rmsnorm_gate(B, T, H, dv, _p(o), _p(g), _p(weight), float(eps), _p(y))
     return y
+
+
+def rmsnorm_gate_bwd(o, g, weight, dy, eps=0.0):
+    """Reverse mode of rmsnorm_gate: returns dict(do, dg (None without a
+    gate), dweight [dv])."""
+    o, g, weight, dy = map(_in, (o, g, weight, dy))
+    B, T, H, dv = o.shape
+    out = dict(do=np.zeros_like(o), dg=None if g is None else np.zeros_like(o), dweight=np.zeros(dv))
+    _load().oracle_rmsnorm_gate_bwd(B, T, H, dv, _p(o), _p(g), _p(weight), float(eps), _p(dy),
+                                    _p(out["do"]), _p(out["dg"]), _p(out["dweight"]))
+    return out

@@ -122,3 +122,50 @@ void oracle_rmsnorm_gate(int B, int T, int H, int dv, const double *o,
         }
     }
 }
+
+/* Reverse mode of oracle_rmsnorm_gate (the chain rule of the epilogue's
+ * definition above): with r = 1/sqrt(mean o^2 + eps), a = o r, s = SiLU(g)
+ * (s = 1 without a gate) and y = a * weight * s,
+ *     dg = dy a weight SiLU'(g),   SiLU'(z) = sigma(z) (1 + z (1 - sigma(z)))
+ *     da = dy weight s,            do = r (da - a mean(da a))
+ *     dweight = sum over rows of dy a s.
+ * dg may be NULL (no gate); every output is overwritten. */
+void oracle_rmsnorm_gate_bwd(int B, int T, int H, int dv, const double *o,
+                             const double *g, const double *weight, double eps,
+                             const double *dy, double *dO, double *dg,
+                             double *dweight) {
+    size_t rows = (size_t)B * T * H;
+    for (int i = 0; i < dv; ++i) dweight[i] = 0.0;
+    for (size_t r = 0; r < rows; ++r) {
+        const double *orow = o + r * dv, *dyr = dy + r * dv;
+        double ms = 0.0;
+        for (int i = 0; i < dv; ++i) ms += orow[i] * orow[i];
+        ms /= dv;
+        const double inv = 1.0 / sqrt(ms + eps);
+        double dot = 0.0; /* sum_i da_i a_i */
+        for (int i = 0; i < dv; ++i) {
+            const double a = orow[i] * inv;
+            double s = 1.0;
+            if (g) {
+                const double z = g[r * dv + i];
+                const double sig = 1.0 / (1.0 + exp(-z));
+                s = z * sig;
+                dg[r * dv + i] = dyr[i] * a * weight[i] * sig * (1.0 + z * (1.0 - sig));
+            }
+            const double da = dyr[i] * weight[i] * s;
+            dot += da * a;
+            dweight[i] += dyr[i] * a * s;
+        }
+        dot /= dv;
+        for (int i = 0; i < dv; ++i) {
+            const double a = orow[i] * inv;
+            double s = 1.0;
+            if (g) {
+                const double z = g[r * dv + i];
+                s = z / (1.0 + exp(-z));
+            }
+            const double da = dyr[i] * weight[i] * s;
+            dO[r * dv + i] = inv * (da - a * dot);
+        }
+    }
+}

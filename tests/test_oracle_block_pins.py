@@ -190,3 +190,40 @@ def test_output_gate_closed_forms():
                                rtol=1e-14)
     g = rng.standard_normal(o.shape)                                      # library SiLU
     np.testing.assert_allclose(oracle.rmsnorm_gate(o, g, wgt), plain * _silu_lib(g), rtol=1e-13)
+
+
+def _fd(f, x, eps=1e-6):
+    """Central finite differences of the scalar f at x (array), elementwise."""
+    gr = np.zeros_like(x)
+    it = np.nditer(x, flags=["multi_index"])
+    for _ in it:
+        idx = it.multi_index
+        xp = x.copy(); xp[idx] += eps
+        xm = x.copy(); xm[idx] -= eps
+        gr[idx] = (f(xp) - f(xm)) / (2 * eps)
+    return gr
+
+
+@pytest.mark.parametrize("gate,eps", [(True, 1e-6), (False, 0.0), (True, 0.3)])
+def test_rmsnorm_gate_bwd_matches_finite_differences(gate, eps):
+    rng = np.random.default_rng(30 + int(gate))
+    o = rng.standard_normal((1, 2, 2, 6))
+    g = rng.standard_normal(o.shape) if gate else None
+    wgt = rng.uniform(0.5, 1.5, 6)
+    dy = rng.standard_normal(o.shape)
+    loss = lambda o_, g_, w_: float((oracle.rmsnorm_gate(o_, g_, w_, eps) * dy).sum())
+    got = oracle.rmsnorm_gate_bwd(o, g, wgt, dy, eps)
+    np.testing.assert_allclose(got["do"], _fd(lambda v: loss(v, g, wgt), o), rtol=1e-6, atol=1e-8)
+    np.testing.assert_allclose(got["dweight"], _fd(lambda v: loss(o, g, v), wgt), rtol=1e-6, atol=1e-8)
+    if gate:
+        np.testing.assert_allclose(got["dg"], _fd(lambda v: loss(o, v, wgt), g), rtol=1e-6, atol=1e-8)
+    else:
+        assert got["dg"] is None
+
+
+def test_rmsnorm_bwd_is_orthogonal_to_the_row():
+    # with eps = 0 the norm is scale-invariant, so do . o = 0 per row
+    rng = np.random.default_rng(4)
+    o = rng.standard_normal((2, 3, 2, 16))
+    got = oracle.rmsnorm_gate_bwd(o, rng.standard_normal(o.shape), np.ones(16), rng.standard_normal(o.shape))
+    np.testing.assert_allclose((got["do"] * o).sum(-1), 0.0, atol=1e-12)
