@@ -205,6 +205,12 @@ def epilogue_bytes(B, T, H, dv, esize=2):
     return 3 * B * T * H * dv * esize + dv * 4
 
 
+def epilogue_bwd_bytes(B, T, H, dv, esize=2):
+    """Block epilogue backward: read o, g and dy, write do and dg; the fp32
+    weight in and dweight out."""
+    return 5 * B * T * H * dv * esize + 2 * dv * 4
+
+
 # ---------------------------------------------------------------------------
 # clocks sampled during the timed region
 # ---------------------------------------------------------------------------
@@ -597,6 +603,13 @@ def block_lines(pk):
     gbs_e = epilogue_bytes(B, T, H, d) / (us_e * 1e-6) / 1e9
     out["block_epilogue"] = {"workload": "B=4 T=4096 H=16 dv=128 bf16, RMSNorm + SiLU gate",
                              "us": us_e, "achieved_gbs": gbs_e, "hbm_frac": gbs_e / pk["hbm_gbs"]}
+    dy = torch.randn(B, T, H, d, generator=torch.Generator().manual_seed(24)).to(torch.bfloat16).cuda()
+    ws = torch.empty(gdr.lib().gdr_block_epilogue_bwd_workspace_bytes(d), dtype=torch.uint8, device="cuda")
+    us_b = timed(lambda: gdr.gdr_block_epilogue_bwd(ex["o"], ex["g"], ex["weight"], dy, 1e-6, workspace=ws)) * 1e3
+    gbs_b = epilogue_bwd_bytes(B, T, H, d) / (us_b * 1e-6) / 1e9
+    out["block_epilogue_bwd"] = {"workload": "B=4 T=4096 H=16 dv=128 bf16, backward of RMSNorm + SiLU gate "
+                                             "(do, dg, dweight; 2 launches)",
+                                 "us": us_b, "achieved_gbs": gbs_b, "hbm_frac": gbs_b / pk["hbm_gbs"]}
 
     def chain():
         pro()

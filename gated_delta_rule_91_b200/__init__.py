@@ -14,6 +14,7 @@ Functions (same names as the C entry points):
     gdr2_step(q, k, v, log_alpha, b, w, S)               -> o  (S advanced in place)
     gdr_block_prologue(xq, xk, xv, wq, wk, wv, ...)       -> (q, k, v)
     gdr_block_epilogue(o, g, weight, eps)                 -> y
+    gdr_block_epilogue_bwd(o, g, weight, dy, eps)         -> (do, dg, dweight)
     gdr_seg_fwd / gdr_seg_combine / gdr_seg_fixup         (sequence split; see seq_split)
 
 The calls take the current CUDA stream and allocate nothing inside the
@@ -50,6 +51,8 @@ SIGNATURES = {
     "gdr2_step": (_I, [_I] * 5 + [_P] * 8 + [_P]),
     "gdr_block_prologue": (_I, [_I] * 7 + [_P] * 11 + [ctypes.c_float] + [_P] * 3 + [_P]),
     "gdr_block_epilogue": (_I, [_I] * 5 + [_P] * 3 + [ctypes.c_float, _P, _P]),
+    "gdr_block_epilogue_bwd": (_I, [_I] * 5 + [_P] * 3 + [ctypes.c_float] + [_P] * 5 + [_SZ, _P]),
+    "gdr_block_epilogue_bwd_workspace_bytes": (_SZ, [_I]),
     "gdr_seg_fwd": (_I, [_I] * 6 + [_P] * 9 + [_P, _SZ, _P]),
     "gdr_seg_fwd_workspace_bytes": (_SZ, [_I] * 6),
     "gdr_seg_combine": (_I, [_I] * 6 + [_P] * 5 + [_P]),
@@ -269,6 +272,21 @@ def gdr_block_epilogue(o, g, weight, eps=1e-6, *, y=None):
     check(lib().gdr_block_epilogue(B, T, H, dv, _dt(o), _ptr(o), _ptr(g), _ptr(weight), float(eps),
                                    _ptr(y), _stream(o)))
     return y
+
+
+def gdr_block_epilogue_bwd(o, g, weight, dy, eps=1e-6, *, workspace=None):
+    """Backward of gdr_block_epilogue for an incoming dy [B,T,H,dv]: returns
+    (do, dg or None without a gate, dweight [dv] fp32)."""
+    B, T, H, dv = o.shape
+    _f32(weight, "weight")
+    do = torch.empty_like(o)
+    dg = None if g is None else torch.empty_like(g)
+    dweight = torch.empty(dv, dtype=torch.float32, device=o.device)
+    L = lib()
+    ws, ws_bytes = _workspace(L.gdr_block_epilogue_bwd_workspace_bytes(dv), o.device, workspace)
+    check(L.gdr_block_epilogue_bwd(B, T, H, dv, _dt(o), _ptr(o), _ptr(g), _ptr(weight), float(eps), _ptr(dy),
+                                   _ptr(do), _ptr(dg), _ptr(dweight), _ptr(ws), ws_bytes, _stream(o)))
+    return do, dg, dweight
 
 
 def gdr_seg_fwd(q, k, v, log_alpha, beta, *, workspace=None):

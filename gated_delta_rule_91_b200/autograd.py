@@ -6,11 +6,12 @@ S0=None)` does the same for Gated DeltaNet-2 through gdr2_bwd.  The forward
 and the backward are the library's CUDA calls: these classes only save the
 inputs and hand the incoming gradients over (the backward recomputes the
 forward's states itself, so nothing else is kept).  Unused outputs arrive as
-zero gradients.
+zero gradients.  `block_epilogue(o, g, weight, eps)` is the block's output
+normalisation and gate, differentiated through gdr_block_epilogue_bwd.
 """
 import torch
 
-from . import gdr2_bwd, gdr2_fwd, gdr_bwd, gdr_fwd
+from . import gdr2_bwd, gdr2_fwd, gdr_block_epilogue, gdr_block_epilogue_bwd, gdr_bwd, gdr_fwd
 
 
 def _c(x):
@@ -59,3 +60,25 @@ def gated_delta_rule(q, k, v, log_alpha, beta, S0=None):
 def gated_delta_rule2(q, k, v, log_alpha, b, w, S0=None):
     """Differentiable gdr2_fwd: returns (o, S_T)."""
     return GatedDeltaRule2.apply(q, k, v, log_alpha, b, w, S0)
+
+
+class BlockEpilogue(torch.autograd.Function):
+    """y = RMSNorm(o) * weight * SiLU(g) over dv per (token, head)."""
+
+    @staticmethod
+    def forward(ctx, o, g, weight, eps):
+        o, g = _c(o), _c(g)
+        ctx.eps = eps
+        ctx.save_for_backward(o, g, weight)
+        return gdr_block_epilogue(o, g, weight, eps)
+
+    @staticmethod
+    def backward(ctx, dy):
+        o, g, weight = ctx.saved_tensors
+        do, dg, dweight = gdr_block_epilogue_bwd(o, g, weight, _c(dy), ctx.eps)
+        return do, dg, dweight, None
+
+
+def block_epilogue(o, g, weight, eps=1e-6):
+    """Differentiable gdr_block_epilogue: returns y."""
+    return BlockEpilogue.apply(o, g, weight, eps)

@@ -443,6 +443,138 @@ __global__ void __launch_bounds__(kEpiThreads)
     }
 }
 
+// ---- epilogue backward ------------------------------------------------------------
+// Reverse mode of y = a * weight * s, a = o * r, r = 1/sqrt(mean(o^2) + eps),
+// s = SiLU(g) (s = 1 without a gate), for an incoming dy:
+//   dg      = dy a weight sig (1 + g (1 - sig)),   sig = 1/(1 + e^-g)
+//   da      = dy weight s
+//   do      = r (da - a mean(da a))
+//   dweight = sum over rows of dy a s.
+// Same unit walk as the forward (64 rows, one bulk copy per tensor: o, g, dy),
+// NS stages deep.  Each lane keeps its channels' dweight partial sums over its
+// rows in registers; at the end the block sums its 16 warps in warp order and
+// writes one row of `partial` [gridDim.x, D], which a second launch sums over
+// blocks in block order -- the result is independent of timing.
+constexpr int kEpiBwdMaxBlocks = 1024;  // partial rows: the workspace bound
+
+template <typename Tio, int CPL, int NS>
+__global__ void __launch_bounds__(kEpiThreads)
+    gdr_epilogue_bwd_kernel(long long rows, const Tio *__restrict__ o, const Tio *__restrict__ g,
+                            const Tio *__restrict__ dy, const float *__restrict__ weight, float eps,
+                            Tio *__restrict__ dO, Tio *__restrict__ dg, float *__restrict__ partial) {
+    using namespace sm100;
+    constexpr int D = CPL * 32;
+    constexpr int kTile = kEpilogueRows * D * (int)sizeof(Tio);
+    constexpr int kWarps = kEpiThreads / 32;
+    constexpr int kRowsPerWarp = kEpilogueRows / kWarps;
+    extern __shared__ __align__(128) uint8_t blk_smem[];
+    uint8_t *smem = blk_smem;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + NS * 3 * kTile);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long units = (rows + kEpilogueRows - 1) / kEpilogueRows;
+    auto issue = [&](long long uu, int sidx) {  // one thread
+        const long long r0 = uu * kEpilogueRows;
+        const uint32_t bytes = (uint32_t)min((long long)kEpilogueRows, rows - r0) * D * (uint32_t)sizeof(Tio);
+        uint8_t *dst = smem + sidx * 3 * kTile;
+        mbar_expect_tx(&bars[sidx], g ? 3 * bytes : 2 * bytes);
+        bulk_load_g2s(dst, o + r0 * D, bytes, &bars[sidx]);
+        bulk_load_g2s(dst + 2 * kTile, dy + r0 * D, bytes, &bars[sidx]);
+        if (g) bulk_load_g2s(dst + kTile, g + r0 * D, bytes, &bars[sidx]);
+    };
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < NS; ++i) mbar_init(&bars[i], 1);
+        fence_mbar_init();
+        for (int k = 0; k < NS - 1; ++k)
+            if (blockIdx.x + (long long)k * gridDim.x < units) issue(blockIdx.x + (long long)k * gridDim.x, k);
+    }
+    __syncthreads();
+    float wl[CPL], dwp[CPL];
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) {
+        wl[c] = __ldg(weight + lane * CPL + c);
+        dwp[c] = 0.f;
+    }
+    int st = 0;
+#pragma unroll 1
+    for (int k = 0;; ++k) {
+        const long long u = blockIdx.x + (long long)k * gridDim.x;
+        if (u >= units) break;
+        const long long un = u + (long long)(NS - 1) * gridDim.x;
+        if (threadIdx.x == 0 && un < units) {
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            issue(un, st == 0 ? NS - 1 : st - 1);
+        }
+        if (!mbar_wait(&bars[st], (uint32_t)(k / NS) & 1u)) {
+            record_status(GDR_ERR_TIMEOUT);
+            blk_drain<NS>(bars, st, k, u, units, gridDim.x);
+            return;
+        }
+        const Tio *so = reinterpret_cast<const Tio *>(smem + st * 3 * kTile) + lane * CPL;
+        const Tio *sg = so + kTile / sizeof(Tio);
+        const Tio *sd = so + 2 * (kTile / sizeof(Tio));
+        const long long r0 = u * kEpilogueRows;
+        const int n = (int)min((long long)kEpilogueRows, rows - r0);
+#pragma unroll
+        for (int r = 0; r < kRowsPerWarp; ++r) {
+            const int i = warp * kRowsPerWarp + r;
+            if (i >= n) break;
+            float ov[CPL], gv[CPL], dv_[CPL], ss = 0.f;
+            ld_row<CPL>(so + i * D, ov);
+            ld_row<CPL>(sd + i * D, dv_);
+            if (g) ld_row<CPL>(sg + i * D, gv);
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) ss = fmaf(ov[c], ov[c], ss);
+            const float inv = rsqrt_ftz(warp_sum(ss, 32) * (1.f / D) + eps);
+            float a[CPL], da[CPL], dgo[CPL], dot = 0.f;
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) {
+                a[c] = ov[c] * inv;
+                float s = 1.f;
+                if (g) {
+                    const float z = gv[c];
+                    const float sig = rcp_ftz(1.f + ex2_ftz(-kLog2e * z));
+                    s = z * sig;
+                    dgo[c] = dv_[c] * a[c] * wl[c] * sig * fmaf(z, 1.f - sig, 1.f);
+                }
+                const float dys = dv_[c] * s;
+                da[c] = dys * wl[c];
+                dwp[c] = fmaf(dys, a[c], dwp[c]);
+                dot = fmaf(da[c], a[c], dot);
+            }
+            dot = warp_sum(dot, 32) * (1.f / D);
+            float out[CPL];
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) out[c] = inv * fmaf(-a[c], dot, da[c]);
+            const size_t off = (size_t)(r0 + i) * D + lane * CPL;
+            st_row<CPL>(dO + off, out);
+            if (g) st_row<CPL>(dg + off, dgo);
+        }
+        __syncthreads();
+        st = st == NS - 1 ? 0 : st + 1;
+    }
+    // every issued copy has been waited on: the stages are free for the sums
+    float *red = reinterpret_cast<float *>(smem);
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) red[warp * D + lane * CPL + c] = dwp[c];
+    __syncthreads();
+    if (threadIdx.x < D) {
+        float acc = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) acc += red[w * D + threadIdx.x];
+        partial[(size_t)blockIdx.x * D + threadIdx.x] = acc;
+    }
+}
+
+// dweight[c] = sum over b < nblk of partial[b, c], in block order.
+__global__ void epilogue_dweight_sum_kernel(int nblk, int D, const float *__restrict__ partial,
+                                            float *__restrict__ dweight) {
+    const int c = threadIdx.x;
+    if (c >= D) return;
+    float acc = 0.f;
+    for (int b = 0; b < nblk; ++b) acc += partial[(size_t)b * D + c];
+    dweight[c] = acc;
+}
+
 // Grid = SMs x resident blocks of the kernel (capped by the work), so the
 // stride loop covers the units in whole waves.
 // (One cached figure per kernel instantiation: the library runs on B200s only.)
@@ -528,6 +660,31 @@ inline cudaError_t launch_epilogue(long long rows, int dv, const void *o, const 
         return cudaGetLastError();
     };
     return dv == 128 ? run(gdr_epilogue_kernel<Tio, 4>, 128) : run(gdr_epilogue_kernel<Tio, 2>, 64);
+}
+
+template <typename Tio>
+inline cudaError_t launch_epilogue_bwd(long long rows, int dv, const void *o, const void *g, const void *dy,
+                                       const float *weight, float eps, void *dO, void *dg, float *dweight,
+                                       float *partial, cudaStream_t stream) {
+    // 3 tensors x NS stages x 64 rows: 3 stages for bf16 (144 KB), 2 for fp32
+    constexpr int NS = sizeof(Tio) == 2 ? 3 : 2;
+    auto run = [&](auto kern, int d) -> cudaError_t {
+        const int smem = NS * 3 * kEpilogueRows * d * (int)sizeof(Tio) + 8 * NS;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        const long long units = (rows + kEpilogueRows - 1) / kEpilogueRows;
+        const int grid = std::min(resident_grid(kern, units * (kEpiThreads / 32), smem, kEpiThreads), kEpiBwdMaxBlocks);
+        if (grid <= 0) return cudaErrorInvalidConfiguration;
+        kern<<<grid, kEpiThreads, smem, stream>>>(rows, static_cast<const Tio *>(o), static_cast<const Tio *>(g),
+                                                  static_cast<const Tio *>(dy), weight, eps, static_cast<Tio *>(dO),
+                                                  static_cast<Tio *>(dg), partial);
+        g_launches.fetch_add(1, std::memory_order_relaxed);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        epilogue_dweight_sum_kernel<<<1, d, 0, stream>>>(grid, d, partial, dweight);
+        g_launches.fetch_add(1, std::memory_order_relaxed);
+        return cudaGetLastError();
+    };
+    return dv == 128 ? run(gdr_epilogue_bwd_kernel<Tio, 4, NS>, 128) : run(gdr_epilogue_bwd_kernel<Tio, 2, NS>, 64);
 }
 
 }  // namespace gdr

@@ -565,6 +565,40 @@ gdr_status gdr_block_epilogue(int B, int T, int H, int dv, gdr_dtype dt, const v
     return GDR_OK;
 }
 
+size_t gdr_block_epilogue_bwd_workspace_bytes(int dv) {
+    return (dv == 64 || dv == 128) ? (size_t)kEpiBwdMaxBlocks * dv * sizeof(float) : 0;
+}
+
+gdr_status gdr_block_epilogue_bwd(int B, int T, int H, int dv, gdr_dtype dt, const void *o, const void *g,
+                                  const float *weight, float eps, const void *dy, void *dO, void *dg,
+                                  float *dweight, void *workspace, size_t workspace_bytes, gdr_stream_t stream) {
+    const char *fn = "gdr_block_epilogue_bwd";
+    gdr_status st = check_dims(fn, B, T, H, 64, dv, dt);
+    if (st != GDR_OK) return st;
+    if (!(eps >= 0.f) || eps > 1e30f) return fail(GDR_ERR_INVALID_ARGUMENT, "%s: eps=%g", fn, (double)eps);
+    GDR_REQUIRE_PTR(o);
+    GDR_OPTIONAL_PTR(g);
+    GDR_REQUIRE_PTR(weight);
+    GDR_REQUIRE_PTR(dy);
+    GDR_REQUIRE_PTR(dO);
+    GDR_REQUIRE_PTR(dweight);
+    if ((g == nullptr) != (dg == nullptr))
+        return fail(GDR_ERR_INVALID_ARGUMENT, "%s: g and dg must both be given or both NULL", fn);
+    GDR_OPTIONAL_PTR(dg);
+    const size_t need = gdr_block_epilogue_bwd_workspace_bytes(dv);
+    if (workspace == nullptr || workspace_bytes < need)
+        return fail(GDR_ERR_WORKSPACE, "%s: workspace %zu bytes, need %zu", fn, workspace_bytes, need);
+    if (!aligned16(workspace)) return fail(GDR_ERR_INVALID_ARGUMENT, "%s: workspace is not 16-byte aligned", fn);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const long long rows = (long long)B * T * H;
+    float *partial = static_cast<float *>(workspace);
+    cudaError_t e = dt == GDR_F32
+                        ? launch_epilogue_bwd<float>(rows, dv, o, g, dy, weight, eps, dO, dg, dweight, partial, s)
+                        : launch_epilogue_bwd<__nv_bfloat16>(rows, dv, o, g, dy, weight, eps, dO, dg, dweight, partial, s);
+    if (e != cudaSuccess) return cuda_fail(e, fn);
+    return GDR_OK;
+}
+
 size_t gdr_seg_fwd_workspace_bytes(int B, int T, int H, int dk, int dv, gdr_dtype dt) {
     if (B < 1 || T < 1 || H < 1 || (dk != 64 && dk != 128) || (dv != 64 && dv != 128) ||
         (dt != GDR_F32 && dt != GDR_BF16))

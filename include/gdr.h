@@ -277,6 +277,31 @@ GDR_API gdr_status gdr_block_epilogue(int B, int T, int H, int dv, gdr_dtype dt,
                               gdr_stream_t stream);
 
 /*
+ * Backward of gdr_block_epilogue (the same normalised, gated output of the
+ * Gated DeltaNet block: the Gated DeltaNet review, meaningful96.github.io/nr/GDN,
+ * section 3.8).  With a = o r, r = 1/sqrt(mean_i o_i^2 + eps), s = SiLU(g)
+ * (s = 1 without a gate), sig = 1/(1 + e^-g) and an incoming dy:
+ *     dg      = dy a weight sig (1 + g (1 - sig))
+ *     do      = r (dy weight s - a mean_i(dy_i weight_i s_i a_i))
+ *     dweight = sum over all B*T*H rows of dy a s.
+ *   in:  o, g (or NULL), dy [B,T,H,dv] dtype dt; weight [dv] fp32; eps >= 0
+ *        as in the forward.
+ *   out: dO [B,T,H,dv] dtype dt; dg likewise (NULL exactly when g is NULL);
+ *        dweight [dv] fp32, overwritten (not accumulated).
+ *   workspace: device scratch of gdr_block_epilogue_bwd_workspace_bytes(dv)
+ *        bytes (per-block partial sums of dweight, which a second launch adds
+ *        in a fixed order, so repeated calls give identical bits).
+ *   Errors: as gdr_block_epilogue; g and dg not both given or both NULL ->
+ *   GDR_ERR_INVALID_ARGUMENT; workspace NULL or short -> GDR_ERR_WORKSPACE.
+ */
+GDR_API gdr_status gdr_block_epilogue_bwd(int B, int T, int H, int dv, gdr_dtype dt, const void *o,
+                                  const void *g, const float *weight, float eps, const void *dy,
+                                  void *dO, void *dg, float *dweight, void *workspace,
+                                  size_t workspace_bytes, gdr_stream_t stream);
+/* 0 for an unsupported dv. */
+GDR_API size_t gdr_block_epilogue_bwd_workspace_bytes(int dv);
+
+/*
  * Sequence split: one sequence divided into R consecutive segments, one per
  * process/GPU, each run by its owner, with one exchange of small matrices.
  * For one (b, h) the rule over a segment maps the incoming state affinely,

@@ -142,6 +142,15 @@ def block_epilogue_inputs(B: int, T: int, H: int, dv: int, dtype: str = "bf16", 
     return {"o": o, "g": gg if gate else None, "weight": weight}
 
 
+def block_epilogue_bwd_inputs(B: int, T: int, H: int, dv: int, dtype: str = "bf16", seed: int = 0,
+                              gate: bool = True) -> dict:
+    """Epilogue inputs plus an incoming gradient dy ~ N(0, 1) [B,T,H,dv] in dtype."""
+    x = block_epilogue_inputs(B, T, H, dv, dtype, seed, gate)
+    g = torch.Generator().manual_seed(seed * 7919 + 1)
+    x["dy"] = torch.randn(B, T, H, dv, generator=g).to(DTYPES[dtype])
+    return x
+
+
 def decode_state(B: int, H: int, dk: int, dv: int, seed: int, std: float = 0.02) -> torch.Tensor:
     """Initial decode state S [B,H,dv,dk] fp32 ~ N(0, std^2)."""
     g = torch.Generator().manual_seed(seed)

@@ -127,6 +127,37 @@ def test_epilogue_rejects_bad_arguments(kw, status):
 
 
 @pytest.mark.parametrize("kw,status", [
+    (dict(T=0), gdr.GDR_ERR_INVALID_ARGUMENT),
+    (dict(dv=32), gdr.GDR_ERR_UNSUPPORTED),
+    (dict(eps=float("nan")), gdr.GDR_ERR_INVALID_ARGUMENT),
+    (dict(dy=None), gdr.GDR_ERR_INVALID_ARGUMENT),
+    (dict(dO=FAKE + 4), gdr.GDR_ERR_INVALID_ARGUMENT),
+    (dict(dweight=None), gdr.GDR_ERR_INVALID_ARGUMENT),
+    (dict(g=FAKE), gdr.GDR_ERR_INVALID_ARGUMENT),            # g without dg
+    (dict(dg=FAKE), gdr.GDR_ERR_INVALID_ARGUMENT),           # dg without g
+    (dict(ws=None), gdr.GDR_ERR_WORKSPACE),
+    (dict(ws_bytes=1024 * 64 * 4 - 1), gdr.GDR_ERR_WORKSPACE),
+    (dict(ws=FAKE + 8), gdr.GDR_ERR_INVALID_ARGUMENT),
+])
+def test_epilogue_bwd_rejects_bad_arguments(kw, status):
+    a = dict(B=1, T=4, H=1, dv=64, dt=gdr.GDR_BF16, o=FAKE, g=None, weight=FAKE, eps=1e-6, dy=FAKE,
+             dO=FAKE, dg=None, dweight=FAKE, ws=FAKE, ws_bytes=1 << 20)
+    a.update(kw)
+    P = ctypes.c_void_p
+    st = gdr.lib().gdr_block_epilogue_bwd(a["B"], a["T"], a["H"], a["dv"], a["dt"], P(a["o"]), P(a["g"]),
+                                          P(a["weight"]), a["eps"], P(a["dy"]), P(a["dO"]), P(a["dg"]),
+                                          P(a["dweight"]), P(a["ws"]), a["ws_bytes"], None)
+    assert st == status
+    assert gdr.lib().gdr_last_error_string().decode().startswith("gdr_block_epilogue_bwd")
+
+
+def test_epilogue_bwd_workspace_bytes():
+    assert gdr.lib().gdr_block_epilogue_bwd_workspace_bytes(128) == 1024 * 128 * 4
+    assert gdr.lib().gdr_block_epilogue_bwd_workspace_bytes(64) == 1024 * 64 * 4
+    assert gdr.lib().gdr_block_epilogue_bwd_workspace_bytes(96) == 0
+
+
+@pytest.mark.parametrize("kw,status", [
     (dict(R=0), gdr.GDR_ERR_INVALID_ARGUMENT),
     (dict(r=-1), gdr.GDR_ERR_INVALID_ARGUMENT),
     (dict(r=3), gdr.GDR_ERR_INVALID_ARGUMENT),

@@ -9,7 +9,7 @@ import torch
 import gated_delta_rule_91_b200 as gdr
 import oracle
 import synth
-from gated_delta_rule_91_b200.autograd import gated_delta_rule, gated_delta_rule2
+from gated_delta_rule_91_b200.autograd import block_epilogue, gated_delta_rule, gated_delta_rule2
 from gpu_common import TOL_G, TOL_O, dtype_name, fro_rel, max_rel, np64
 
 pytestmark = pytest.mark.gpu
@@ -57,6 +57,20 @@ def test_autograd_without_initial_state():
     ref = oracle.gdr_bwd(np64(x["q"]), np64(x["k"]), np64(x["v"]), np64(x["log_alpha"]), np64(x["beta"]),
                          None, np.ones(o.shape), np.ones(S_T.shape))
     assert max_rel(np64(leaves["k"].grad), ref["dk"]) <= TOL_G["f32"]
+
+
+@pytest.mark.parametrize("gate", [True, False])
+def test_autograd_block_epilogue(gate):
+    x = synth.block_epilogue_bwd_inputs(2, 90, 3, 128, "bf16", seed=11, gate=gate)
+    o, w = _leaf(x["o"]), _leaf(x["weight"])
+    g = _leaf(x["g"])
+    y = block_epilogue(o, g, w, 1e-6)
+    (y.float() * x["dy"].cuda().float()).sum().backward()
+    ref = oracle.rmsnorm_gate_bwd(np64(x["o"]), np64(x["g"]), np64(x["weight"]), np64(x["dy"]), 1e-6)
+    assert max_rel(np64(o.grad), ref["do"]) <= TOL_O["bf16"]
+    assert max_rel(np64(w.grad), ref["dweight"]) <= 1e-4
+    if gate:
+        assert max_rel(np64(g.grad), ref["dg"]) <= TOL_O["bf16"]
 
 
 def test_captured_decode_loop_replays_like_eager():

@@ -184,6 +184,68 @@ def test_epilogue_zero_rows():
     assert torch.count_nonzero(y) == 0
 
 
+def _epi_bwd_ref(x, eps):
+    return oracle.rmsnorm_gate_bwd(np64(x["o"]), np64(x["g"]), np64(x["weight"]), np64(x["dy"]), eps)
+
+
+def _epi_bwd_gpu(x, eps):
+    return gdr.gdr_block_epilogue_bwd(dev(x["o"]), dev(x["g"]), dev(x["weight"]), dev(x["dy"]), eps)
+
+
+def _assert_dweight(got, ref, rows):
+    # fp32 sums over `rows` rows: a relative bound that grows with the count
+    scale = float(np.max(np.abs(ref)))
+    err = float(np.max(np.abs(np64(got) - ref)))
+    assert err <= (1e-5 + 2e-10 * rows) * scale, (err, scale)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("dv", [64, 128])
+@pytest.mark.parametrize("gate", [True, False])
+@pytest.mark.parametrize("T", [1, 77, 300])
+def test_epilogue_bwd_small(dtype, dv, gate, T):
+    x = synth.block_epilogue_bwd_inputs(2, T, 3, dv, dtype, seed=dv + T + 5, gate=gate)
+    ref = _epi_bwd_ref(x, 1e-6)
+    do, dg, dw = _epi_bwd_gpu(x, 1e-6)
+    gdr.check_status()
+    assert_close(do, ref["do"], dtype)
+    if gate:
+        assert_close(dg, ref["dg"], dtype)
+    else:
+        assert dg is None
+    _assert_dweight(dw, ref["dweight"], 2 * T * 3)
+
+
+def test_epilogue_bwd_workload_full():
+    # 262,144 rows: many 64-row units per block, every block's partial used
+    x = synth.block_epilogue_bwd_inputs(4, 4096, 16, 128, "bf16", seed=4)
+    ref = _epi_bwd_ref(x, 1e-6)
+    do, dg, dw = _epi_bwd_gpu(x, 1e-6)
+    gdr.check_status()
+    assert_close(do, ref["do"], "bf16")
+    assert_close(dg, ref["dg"], "bf16")
+    _assert_dweight(dw, ref["dweight"], 4 * 4096 * 16)
+
+
+def test_epilogue_bwd_is_deterministic():
+    x = synth.block_epilogue_bwd_inputs(2, 3000, 8, 128, "bf16", seed=9)
+    a = _epi_bwd_gpu(x, 1e-6)
+    b = _epi_bwd_gpu(x, 1e-6)
+    for u, v in zip(a, b):
+        assert torch.equal(u, v)
+
+
+def test_epilogue_bwd_zero_rows_and_large_eps():
+    # o = 0: a = 0, so dg = 0 and do = dy weight SiLU(g) / sqrt(eps)
+    x = synth.block_epilogue_bwd_inputs(1, 5, 2, 128, "f32", seed=2)
+    x["o"] = torch.zeros_like(x["o"])
+    ref = _epi_bwd_ref(x, 0.25)
+    do, dg, dw = _epi_bwd_gpu(x, 0.25)
+    gdr.check_status()
+    assert torch.count_nonzero(dg) == 0 and torch.count_nonzero(dw) == 0
+    assert_close(do, ref["do"], "f32")
+
+
 def test_block_kernels_count_launches():
     x = synth.block_prologue_inputs(1, 10, 1, 64, 64, 4, "bf16", seed=1)
     before = gdr.launch_count()
@@ -191,3 +253,6 @@ def test_block_kernels_count_launches():
     e = synth.block_epilogue_inputs(1, 10, 1, 64, "bf16", seed=1)
     gdr.gdr_block_epilogue(dev(e["o"]), dev(e["g"]), dev(e["weight"]))
     assert gdr.launch_count() - before == 2
+    e["dy"] = torch.ones_like(e["o"])
+    _epi_bwd_gpu(e, 1e-6)   # the backward and its fixed-order dweight sum
+    assert gdr.launch_count() - before == 4
