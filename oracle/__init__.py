@@ -34,6 +34,7 @@ def _load():
         lib.oracle_short_conv.argtypes = [i] * 5 + [dp] * 4 + [i, ctypes.c_double, dp, dp]
         lib.oracle_rmsnorm_gate.argtypes = [i] * 4 + [dp] * 3 + [ctypes.c_double, dp]
         lib.oracle_rmsnorm_gate_bwd.argtypes = [i] * 4 + [dp] * 3 + [ctypes.c_double] + [dp] * 4
+        lib.oracle_short_conv_bwd.argtypes = [i] * 5 + [dp] * 4 + [i, ctypes.c_double] + [dp] * 6
         lib.oracle_num_threads.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -141,6 +142,21 @@ def short_conv(x, w, bias=None, state=None, l2=False, eps=0.0):
     _load().oracle_short_conv(B, T, H, d, K, _p(x), _p(w), _p(bias), _p(state), int(l2),
                               float(eps), _p(y), _p(st) if K > 1 else None)
     return y, st
+
+
+def short_conv_bwd(x, w, dy, bias=None, state=None, dstate_out=None, l2=False, eps=0.0):
+    """Reverse mode of short_conv for an incoming dy [B,T,H,d] (and the
+    gradient of the returned state, dstate_out [B,K-1,H*d], or None).
+    Returns dict(dx [B,T,H,d], dw [H*d,K], dbias [H*d], dstate [B,K-1,H*d])."""
+    x, w, dy, bias, state, dso = map(_in, (x, w, dy, bias, state, dstate_out))
+    B, T, H, d = x.shape
+    K = w.shape[-1]
+    out = dict(dx=np.zeros_like(x), dw=np.zeros((H * d, K)), dbias=np.zeros(H * d),
+               dstate=np.zeros((B, K - 1, H * d)))
+    _load().oracle_short_conv_bwd(B, T, H, d, K, _p(x), _p(w), _p(bias), _p(state), int(l2), float(eps),
+                                  _p(dy), _p(dso) if K > 1 else None, _p(out["dx"]), _p(out["dw"]),
+                                  _p(out["dbias"]), _p(out["dstate"]) if K > 1 else None)
+    return out
 
 
 def rmsnorm_gate(o, g, weight, eps=0.0):

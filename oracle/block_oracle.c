@@ -45,10 +45,12 @@
  *
  * Parity status: pinned by tests/test_oracle_block_pins.py (numpy convolution
  * of the zero-state case, impulse response, state continuity across a split,
- * unit norm, closed forms of SiLU and RMSNorm).
+ * unit norm, closed forms of SiLU and RMSNorm; the reverse modes by central
+ * differences of the forward functions and by their invariants).
  */
 #include <math.h>
 #include <stddef.h>
+#include <stdlib.h>
 
 static double silu(double z) { return z / (1.0 + exp(-z)); }
 
@@ -168,4 +170,89 @@ void oracle_rmsnorm_gate_bwd(int B, int T, int H, int dv, const double *o,
             dO[r * dv + i] = inv * (da - a * dot);
         }
     }
+}
+
+/* Reverse mode of oracle_short_conv for an incoming dy [B,T,H,d] (and, if
+ * not NULL, dstate_out [B,K-1,H*d], the gradient of the returned state).
+ * Steps, each the chain rule of one forward step:
+ *   z = conv(x), u = SiLU(z), y = u / n with n = sqrt(sum_head u^2 + eps)
+ *   du = (dy - y (y . dy)) / n          (l2; du = dy without it)
+ *   dz = du sig(z) (1 + z (1 - sig(z)))
+ *   dx[s] = sum_j w[j] dz[s + K-1-j]    (+ dstate_out where x[s] was carried)
+ *   dw[c,j] = sum_t dz[t,c] x[t-K+1+j, c],  dbias[c] = sum_t dz[t,c]
+ * Tokens s < 0 are the carried state: their dx goes to dstate_in.
+ * Outputs dx [B,T,H,d], dw [H*d,K] and dbias [H*d] (may be NULL) are
+ * overwritten; dstate_in [B,K-1,H*d] is written if not NULL. */
+void oracle_short_conv_bwd(int B, int T, int H, int d, int K, const double *x,
+                           const double *w, const double *bias,
+                           const double *state_in, int l2, double eps,
+                           const double *dy, const double *dstate_out,
+                           double *dx, double *dw, double *dbias,
+                           double *dstate_in) {
+    const int C = H * d;
+    double *dz = (double *)malloc(sizeof(double) * ((size_t)T * C + 1));
+    double *ub = (double *)malloc(sizeof(double) * ((size_t)C + 1));
+    double *zb = (double *)malloc(sizeof(double) * ((size_t)C + 1));
+    for (int i = 0; i < C * K; ++i) dw[i] = 0.0;
+    if (dbias)
+        for (int c = 0; c < C; ++c) dbias[c] = 0.0;
+    for (int b = 0; b < B; ++b) {
+        const double *xb = x + (size_t)b * T * C;
+        const double *sb = state_in ? state_in + (size_t)b * (K - 1) * C : NULL;
+        const double *dyb = dy + (size_t)b * T * C;
+        /* x at token s (s < 0: carried state or zero) */
+#define XAT(s, c) ((s) >= 0 ? xb[(size_t)(s) * C + (c)] : (sb ? sb[(size_t)(K - 1 + (s)) * C + (c)] : 0.0))
+        for (int t = 0; t < T; ++t) {
+            for (int c = 0; c < C; ++c) {
+                double acc = bias ? bias[c] : 0.0;
+                for (int j = 0; j < K; ++j) acc += w[(size_t)c * K + j] * XAT(t - (K - 1) + j, c);
+                zb[c] = acc;
+                ub[c] = silu(acc);
+            }
+            for (int h = 0; h < H; ++h) {
+                const double *u = ub + (size_t)h * d, *g = dyb + (size_t)t * C + (size_t)h * d;
+                double *dzr = dz + (size_t)t * C + (size_t)h * d;
+                double n = 1.0, dot = 0.0;
+                if (l2) {
+                    double ss = 0.0;
+                    for (int i = 0; i < d; ++i) ss += u[i] * u[i];
+                    n = sqrt(ss + eps);
+                    for (int i = 0; i < d; ++i) dot += (u[i] / n) * g[i];
+                }
+                for (int i = 0; i < d; ++i) {
+                    const double du = l2 ? (g[i] - (u[i] / n) * dot) / n : g[i];
+                    const double z = zb[(size_t)h * d + i];
+                    const double sig = 1.0 / (1.0 + exp(-z));
+                    dzr[i] = du * sig * (1.0 + z * (1.0 - sig));
+                }
+            }
+        }
+        for (int t = 0; t < T; ++t)
+            for (int c = 0; c < C; ++c) {
+                const double g = dz[(size_t)t * C + c];
+                for (int j = 0; j < K; ++j) dw[(size_t)c * K + j] += g * XAT(t - (K - 1) + j, c);
+                if (dbias) dbias[c] += g;
+            }
+#undef XAT
+        /* dx[s] for s in [-(K-1), T): conv transpose plus the state gradient */
+        for (int s = -(K - 1); s < T; ++s) {
+            if (s < 0 && !dstate_in) continue;
+            for (int c = 0; c < C; ++c) {
+                double acc = 0.0;
+                for (int j = 0; j < K; ++j) {
+                    const int t = s + (K - 1) - j; /* output token that read x[s] via tap j */
+                    if (t >= 0 && t < T) acc += w[(size_t)c * K + j] * dz[(size_t)t * C + c];
+                }
+                const int m = s - (T - (K - 1)); /* slot of x[s] in the returned state */
+                if (dstate_out && m >= 0) acc += dstate_out[((size_t)b * (K - 1) + m) * C + c];
+                if (s >= 0)
+                    dx[((size_t)b * T + s) * C + c] = acc;
+                else
+                    dstate_in[((size_t)b * (K - 1) + (K - 1 + s)) * C + c] = acc;
+            }
+        }
+    }
+    free(dz);
+    free(ub);
+    free(zb);
 }

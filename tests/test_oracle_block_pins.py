@@ -227,3 +227,67 @@ def test_rmsnorm_bwd_is_orthogonal_to_the_row():
     o = rng.standard_normal((2, 3, 2, 16))
     got = oracle.rmsnorm_gate_bwd(o, rng.standard_normal(o.shape), np.ones(16), rng.standard_normal(o.shape))
     np.testing.assert_allclose((got["do"] * o).sum(-1), 0.0, atol=1e-12)
+
+
+def _conv_loss(x, w, bias, st, dy, dso, l2, eps):
+    y, so = oracle.short_conv(x, w, bias, st, l2=l2, eps=eps)
+    return float((y * dy).sum() + ((so * dso).sum() if dso is not None else 0.0))
+
+
+@pytest.mark.parametrize("K,T,l2,eps", [(4, 6, True, 1e-6), (4, 2, True, 0.3), (3, 5, False, 0.0),
+                                         (1, 4, True, 0.0), (2, 1, False, 0.0)])
+def test_short_conv_bwd_matches_finite_differences(K, T, l2, eps):
+    rng = np.random.default_rng(40 + K + T)
+    B, H, d = 2, 2, 3
+    x = rng.standard_normal((B, T, H, d))
+    w = rng.standard_normal((H * d, K))
+    bias = rng.standard_normal(H * d)
+    st = rng.standard_normal((B, K - 1, H * d))
+    dy = rng.standard_normal(x.shape)
+    dso = rng.standard_normal((B, K - 1, H * d))
+    got = oracle.short_conv_bwd(x, w, dy, bias, st, dso, l2=l2, eps=eps)
+    f = lambda **kw: _conv_loss(**{**dict(x=x, w=w, bias=bias, st=st, dy=dy, dso=dso, l2=l2, eps=eps), **kw})
+    np.testing.assert_allclose(got["dx"], _fd(lambda v: f(x=v), x), rtol=1e-6, atol=1e-8)
+    np.testing.assert_allclose(got["dw"], _fd(lambda v: f(w=v), w), rtol=1e-6, atol=1e-8)
+    np.testing.assert_allclose(got["dbias"], _fd(lambda v: f(bias=v), bias), rtol=1e-6, atol=1e-8)
+    if K > 1:
+        np.testing.assert_allclose(got["dstate"], _fd(lambda v: f(st=v), st), rtol=1e-6, atol=1e-8)
+
+
+@pytest.mark.parametrize("l2", [False, True])
+def test_short_conv_bwd_matches_torch_autograd(l2):
+    # torch's depthwise conv1d over [state, x], SiLU and F.normalize (eps
+    # inside the norm's clamp is 0 here), differentiated by torch autograd.
+    rng = np.random.default_rng(8)
+    B, T, H, d, K = 2, 9, 2, 8, 4
+    C = H * d
+    x = rng.standard_normal((B, T, H, d))
+    w = rng.standard_normal((C, K))
+    bias = rng.standard_normal(C)
+    st = rng.standard_normal((B, K - 1, C))
+    dy = rng.standard_normal(x.shape)
+    tx, tw, tb, ts = (torch.tensor(a, requires_grad=True) for a in (x, w, bias, st))
+    seq = torch.cat([ts, tx.reshape(B, T, C)], dim=1)
+    z = torch.nn.functional.conv1d(seq.transpose(1, 2), tw.unsqueeze(1), tb, groups=C).transpose(1, 2)
+    u = torch.nn.functional.silu(z).reshape(B, T, H, d)
+    y = torch.nn.functional.normalize(u, dim=-1, eps=0.0) if l2 else u
+    (y * torch.from_numpy(dy)).sum().backward()
+    got = oracle.short_conv_bwd(x, w, dy, bias, st, l2=l2)
+    np.testing.assert_allclose(got["dx"], tx.grad.numpy(), rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(got["dw"], tw.grad.numpy(), rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(got["dbias"], tb.grad.numpy(), rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(got["dstate"], ts.grad.numpy(), rtol=1e-11, atol=1e-12)
+
+
+def test_short_conv_bwd_l2_is_orthogonal_to_the_row():
+    # with eps = 0 the L2 output is scale-invariant in u: du . u = 0 per head
+    # row, so with an identity filter (last tap 1, no bias) dz / silu'(x) . silu(x) = 0
+    rng = np.random.default_rng(9)
+    B, T, H, d, K = 1, 4, 2, 8, 3
+    x = rng.standard_normal((B, T, H, d))
+    w = np.zeros((H * d, K))
+    w[:, K - 1] = 1.0
+    got = oracle.short_conv_bwd(x, w, rng.standard_normal(x.shape), l2=True)
+    sig = 1.0 / (1.0 + np.exp(-x))
+    du = got["dx"] / (sig * (1.0 + x * (1.0 - sig)))
+    np.testing.assert_allclose((du * x * sig).sum(-1), 0.0, atol=1e-12)
