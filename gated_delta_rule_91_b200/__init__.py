@@ -13,6 +13,7 @@ Functions (same names as the C entry points):
     gdr2_bwd(q, k, v, log_alpha, b, w, S0, dO, dS_T=None) -> dict of gradients
     gdr2_step(q, k, v, log_alpha, b, w, S)               -> o  (S advanced in place)
     gdr_block_prologue(xq, xk, xv, wq, wk, wv, ...)       -> (q, k, v)
+    gdr_block_prologue_bwd(xq, xk, xv, wq, wk, wv, dq, dk, dv, ...) -> dict of gradients
     gdr_block_epilogue(o, g, weight, eps)                 -> y
     gdr_block_epilogue_bwd(o, g, weight, dy, eps)         -> (do, dg, dweight)
     gdr_seg_fwd / gdr_seg_combine / gdr_seg_fixup         (sequence split; see seq_split)
@@ -50,6 +51,8 @@ SIGNATURES = {
     "gdr2_bwd_workspace_bytes": (_SZ, [_I] * 6),
     "gdr2_step": (_I, [_I] * 5 + [_P] * 8 + [_P]),
     "gdr_block_prologue": (_I, [_I] * 7 + [_P] * 11 + [ctypes.c_float] + [_P] * 3 + [_P]),
+    "gdr_block_prologue_bwd": (_I, [_I] * 7 + [_P] * 10 + [ctypes.c_float] + [_P] * 14 + [_P, _SZ, _P]),
+    "gdr_block_prologue_bwd_workspace_bytes": (_SZ, [_I] * 4),
     "gdr_block_epilogue": (_I, [_I] * 5 + [_P] * 3 + [ctypes.c_float, _P, _P]),
     "gdr_block_epilogue_bwd": (_I, [_I] * 5 + [_P] * 3 + [ctypes.c_float] + [_P] * 5 + [_SZ, _P]),
     "gdr_block_epilogue_bwd_workspace_bytes": (_SZ, [_I]),
@@ -260,6 +263,39 @@ def gdr_block_prologue(xq, xk, xv, wq, wk, wv, bq=None, bk=None, bv=None, *, con
                                    _ptr(conv_state), _ptr(conv_state_out), float(eps), _ptr(q),
                                    _ptr(k), _ptr(v), _stream(xq)))
     return q, k, v
+
+
+def gdr_block_prologue_bwd(xq, xk, xv, wq, wk, wv, dyq, dyk, dyv, bq=None, bk=None, bv=None, *,
+                           conv_state=None, dconv_state_out=None, eps=1e-6, want_dbias=None,
+                           want_dconv_state=None, workspace=None):
+    """Backward of gdr_block_prologue for incoming gradients dyq, dyk, dyv of
+    (q, k, v) and optionally of the returned conv state.  Returns dict(dxq,
+    dxk, dxv, dwq, dwk, dwv, dbq, dbk, dbv (None unless a bias was given or
+    want_dbias), dconv_state (None unless conv_state was given or
+    want_dconv_state))."""
+    B, T, H, dk = xq.shape
+    dv = xv.shape[-1]
+    K = wq.shape[-1]
+    for n, t in (("wq", wq), ("wk", wk), ("wv", wv), ("bq", bq), ("bk", bk), ("bv", bv)):
+        _f32(t, n)
+    want_db = (bq is not None) if want_dbias is None else want_dbias
+    want_ds = (conv_state is not None) if want_dconv_state is None else want_dconv_state
+    out = dict(dxq=torch.empty_like(xq), dxk=torch.empty_like(xk), dxv=torch.empty_like(xv))
+    for n, t in (("dwq", wq), ("dwk", wk), ("dwv", wv)):
+        out[n] = torch.empty_like(t)
+    for n, d in (("dbq", dk), ("dbk", dk), ("dbv", dv)):
+        out[n] = torch.empty(H * d, dtype=torch.float32, device=xq.device) if want_db else None
+    out["dconv_state"] = (torch.empty(B, max(K - 1, 0), H * (2 * dk + dv), dtype=xq.dtype, device=xq.device)
+                          if want_ds and K > 1 else None)
+    L = lib()
+    ws, ws_bytes = _workspace(L.gdr_block_prologue_bwd_workspace_bytes(H, dk, dv, K), xq.device, workspace)
+    check(L.gdr_block_prologue_bwd(
+        B, T, H, dk, dv, K, _dt(xq), _ptr(xq), _ptr(xk), _ptr(xv), _ptr(wq), _ptr(wk), _ptr(wv), _ptr(bq),
+        _ptr(bk), _ptr(bv), _ptr(conv_state), float(eps), _ptr(dyq), _ptr(dyk), _ptr(dyv), _ptr(dconv_state_out),
+        _ptr(out["dxq"]), _ptr(out["dxk"]), _ptr(out["dxv"]), _ptr(out["dwq"]), _ptr(out["dwk"]),
+        _ptr(out["dwv"]), _ptr(out["dbq"]), _ptr(out["dbk"]), _ptr(out["dbv"]), _ptr(out["dconv_state"]),
+        _ptr(ws), ws_bytes, _stream(xq)))
+    return out
 
 
 def gdr_block_epilogue(o, g, weight, eps=1e-6, *, y=None):

@@ -365,6 +365,275 @@ __global__ void __launch_bounds__(kBlkThreads)
         prologue_block<Tio, DV, KW>(a, &tm_v, s, h, idx, G, smem, stage_bytes, bars);
 }
 
+// ---- prologue backward ----------------------------------------------------------
+// Reverse mode of the prologue, per stream, for incoming dy (and optionally
+// the gradient of the returned conv state):
+//   recompute z = conv(x), u = SiLU(z), n = sqrt(sum_head u^2 + eps)
+//   du = (dy - y (y . dy)) / n   with y = u / n   (q, k; du = dy for v)
+//   dz = du sig(z) (1 + z (1 - sig(z)))
+//   dx[s] = sum_j w[j] dz[s + K-1-j] (+ dstate_out where x[s] is carried out;
+//           s < 0: dstate_in)
+//   dw[c, j] = sum_t dz[t, c] x[t-K+1+j, c],   dbias[c] = sum_t dz[t, c].
+// Same (stream, head) pair ownership as the forward.  A unit is 64 tokens
+// [t0, t0+64); its stage holds x for tokens t0-(K-1) .. t0+64+K-2 and dy for
+// t0 .. t0+64+K-2 (one tiled TMA load each, zero past T), because dx of the
+// unit's last tokens needs dz of the K-1 tokens after it.  Phase 1 (a warp per
+// row, D/32 channels per lane) recomputes dz for those 64+K-1 tokens into a
+// fp32 shared buffer and adds the unit's own 64 rows into the lane's dw and
+// dbias registers; phase 2 reads K rows of dz per output row.  At the end the
+// block adds its warps' sums in warp order into one row of `partial`, and a
+// second launch adds the G blocks of each pair in block order.
+constexpr int kProBwdRun = 64;
+constexpr int kProBwdStages = 2;
+constexpr int kProBwdMaxG = 32;  // blocks per (stream, head) pair: the workspace bound
+
+struct PrologueBwdArgs {
+    int B, T, H, dk, dv, K;
+    const void *x[3];
+    const float *w[3];
+    const float *bias[3];   // or null (zero)
+    const void *state_in;   // [B, K-1, H*(2dk+dv)] or null (zeros)
+    float eps;
+    const void *dy[3];      // incoming gradients of q, k, v
+    const void *dstate_out; // gradient of the returned conv state, or null
+    void *dx[3];
+    void *dstate_in;        // gradient of the carried-in state, or null (not written)
+    float *partial;         // [3H*G][DMAX*(KW+1)]: per-block dw (slots 0..K-1) and dbias (slot KW)
+    int partial_stride;     // DMAX*(KW+1)
+};
+
+template <typename Tio, int D, int KW>
+__device__ __forceinline__ void prologue_bwd_block(const PrologueBwdArgs &a, const CUtensorMap *mx,
+                                                   const CUtensorMap *mdy, int s, int h, int idx, int G,
+                                                   uint8_t *smem, int stage_bytes, int xalloc, float *dzs,
+                                                   uint64_t *bars) {
+    using namespace sm100;
+    constexpr int CPL = D / 32, NW = kBlkThreads / 32;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int K = a.K, T = a.T, H = a.H;
+    const int runs = (T + kProBwdRun - 1) / kProBwdRun;
+    const int units = a.B * runs;
+    const int c0 = h * D + lane * CPL;  // this lane's first channel in the stream
+    const uint32_t xbox = (uint32_t)(kProBwdRun + 2 * (K - 1)) * D * (uint32_t)sizeof(Tio);
+    const uint32_t dybox = (uint32_t)(kProBwdRun + K - 1) * D * (uint32_t)sizeof(Tio);
+    const int Ctot = H * (2 * a.dk + a.dv);
+    const int col = s == 0 ? 0 : s == 1 ? H * a.dk : 2 * H * a.dk;  // stream's columns in the state
+
+    const float *wsel = s == 0 ? a.w[0] : s == 1 ? a.w[1] : a.w[2];
+    const float *bsel = s == 0 ? a.bias[0] : s == 1 ? a.bias[1] : a.bias[2];
+    float wt[CPL][KW], bias[CPL], dwa[CPL][KW], dba[CPL];
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) {
+#pragma unroll
+        for (int m = 0; m < KW; ++m) {
+            wt[c][m] = m < K ? __ldg(wsel + (size_t)(c0 + c) * K + m) : 0.f;
+            dwa[c][m] = 0.f;
+        }
+        bias[c] = bsel ? __ldg(bsel + c0 + c) : 0.f;
+        dba[c] = 0.f;
+    }
+    auto issue = [&](int k, int sidx) {  // one thread
+        const int j = idx + k * G, b = j / runs, t0 = (j % runs) * kProBwdRun;
+        uint8_t *stg = smem + sidx * stage_bytes;
+        mbar_expect_tx(&bars[sidx], xbox + dybox);
+        tma_load_4d(stg, mx, &bars[sidx], 0, h, t0 - (K - 1), b);
+        tma_load_4d(stg + xalloc, mdy, &bars[sidx], 0, h, t0, b);
+    };
+    if (threadIdx.x == 0)
+        for (int k = 0; k < kProBwdStages - 1; ++k)
+            if (idx + k * G < units) issue(k, k);
+    const bool l2 = s < 2;
+    const Tio *dso = static_cast<const Tio *>(a.dstate_out);
+    Tio *dxb = static_cast<Tio *>(s == 0 ? a.dx[0] : s == 1 ? a.dx[1] : a.dx[2]);
+    Tio *dsi = static_cast<Tio *>(a.dstate_in);
+    int st = 0;
+#pragma unroll 1
+    for (int k = 0;; ++k) {
+        const int j = idx + k * G;
+        if (j >= units) break;
+        const int b = j / runs, t0 = (j % runs) * kProBwdRun, len = min(kProBwdRun, T - t0);
+        if (threadIdx.x == 0 && j + (kProBwdStages - 1) * G < units) {
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            issue(k + kProBwdStages - 1, st == 0 ? kProBwdStages - 1 : st - 1);
+        }
+        if (!mbar_wait(&bars[st], (uint32_t)(k / kProBwdStages) & 1u)) {
+            record_status(GDR_ERR_TIMEOUT);
+            blk_drain<kProBwdStages>(bars, st, k, j, units, G);
+            return;
+        }
+        uint8_t *stage = smem + st * stage_bytes;
+        if (t0 == 0 && a.state_in != nullptr && K > 1) {
+            constexpr int kPieces = D * (int)sizeof(Tio) / 16;
+            for (int i = threadIdx.x; i < (K - 1) * kPieces; i += kBlkThreads) {
+                const int r = i / kPieces, q = i % kPieces;
+                const Tio *src = static_cast<const Tio *>(a.state_in) + ((size_t)b * (K - 1) + r) * Ctot + col + h * D;
+                reinterpret_cast<uint4 *>(stage + (size_t)r * D * sizeof(Tio))[q] =
+                    reinterpret_cast<const uint4 *>(src)[q];
+            }
+            __syncthreads();
+        }
+        const Tio *sx = reinterpret_cast<const Tio *>(stage) + lane * CPL;
+        const Tio *sdy = reinterpret_cast<const Tio *>(stage + xalloc) + lane * CPL;
+
+        // phase 1: dz for tokens t0 .. t0+64+K-2 (row r = token t0 + r)
+        const int R1 = kProBwdRun + K - 1;
+#pragma unroll 1
+        for (int r = warp; r < R1; r += NW) {
+            float xv[KW][CPL], dyv[CPL], z[CPL], sg[CPL], u[CPL];
+#pragma unroll
+            for (int m = 0; m < KW; ++m) {
+                if (m < K)
+                    ld_row<CPL>(sx + (r + m) * D, xv[m]);
+                else
+#pragma unroll
+                    for (int c = 0; c < CPL; ++c) xv[m][c] = 0.f;
+            }
+            ld_row<CPL>(sdy + r * D, dyv);
+            float ss = 0.f;
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) {
+                float acc = bias[c];
+#pragma unroll
+                for (int m = 0; m < KW; ++m) acc = fmaf(wt[c][m], xv[m][c], acc);
+                z[c] = acc;
+                sg[c] = rcp_ftz(1.f + ex2_ftz(-kLog2e * acc));
+                u[c] = acc * sg[c];
+                ss = fmaf(u[c], u[c], ss);
+            }
+            float du[CPL];
+            if (l2) {
+                const float ninv = rsqrt_ftz(warp_sum(ss, 32) + a.eps);
+                float dot = 0.f;
+#pragma unroll
+                for (int c = 0; c < CPL; ++c) dot = fmaf(u[c] * ninv, dyv[c], dot);
+                dot = warp_sum(dot, 32);
+#pragma unroll
+                for (int c = 0; c < CPL; ++c) du[c] = fmaf(-u[c] * ninv, dot, dyv[c]) * ninv;
+            } else {
+#pragma unroll
+                for (int c = 0; c < CPL; ++c) du[c] = dyv[c];
+            }
+            const bool live = t0 + r < T;
+            float dz[CPL];
+#pragma unroll
+            for (int c = 0; c < CPL; ++c)
+                dz[c] = live ? du[c] * sg[c] * fmaf(z[c], 1.f - sg[c], 1.f) : 0.f;
+            st_row<CPL>(dzs + r * D + lane * CPL, dz);
+            if (r < kProBwdRun) {
+#pragma unroll
+                for (int c = 0; c < CPL; ++c) {
+#pragma unroll
+                    for (int m = 0; m < KW; ++m) dwa[c][m] = fmaf(dz[c], xv[m][c], dwa[c][m]);
+                    dba[c] += dz[c];
+                }
+            }
+        }
+        __syncthreads();
+
+        // phase 2: dx for the unit's tokens (and the carried-in state's rows)
+        const int rlo = (t0 == 0 && dsi != nullptr) ? -(K - 1) : 0;
+#pragma unroll 1
+        for (int i = rlo + warp; i < len; i += NW) {
+            float acc[CPL];
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) acc[c] = 0.f;
+#pragma unroll
+            for (int m = 0; m < KW; ++m) {
+                const int r = i + K - 1 - m;  // dz row that read this x through tap m
+                if (m < K && r >= 0) {
+                    float dzv[CPL];
+                    ld_row<CPL>(dzs + r * D + lane * CPL, dzv);
+#pragma unroll
+                    for (int c = 0; c < CPL; ++c) acc[c] = fmaf(wt[c][m], dzv[c], acc[c]);
+                }
+            }
+            const int ms = t0 + i - (T - (K - 1));  // slot of this x in the returned state
+            if (dso != nullptr && ms >= 0) {
+                float g[CPL];
+                ld_row<CPL>(dso + ((size_t)b * (K - 1) + ms) * Ctot + col + c0, g);
+#pragma unroll
+                for (int c = 0; c < CPL; ++c) acc[c] += g[c];
+            }
+            if (i >= 0)
+                st_row<CPL>(dxb + ((size_t)b * T + t0 + i) * H * D + c0, acc);
+            else
+                st_row<CPL>(dsi + ((size_t)b * (K - 1) + (K - 1 + i)) * Ctot + col + c0, acc);
+        }
+        __syncthreads();
+        st = st == kProBwdStages - 1 ? 0 : st + 1;
+    }
+    // every issued copy has been waited on: stage memory holds the warp sums
+    float *red = reinterpret_cast<float *>(smem);
+    constexpr int E = D * (KW + 1);
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) {
+#pragma unroll
+        for (int m = 0; m < KW; ++m) red[warp * E + (lane * CPL + c) * (KW + 1) + m] = dwa[c][m];
+        red[warp * E + (lane * CPL + c) * (KW + 1) + KW] = dba[c];
+    }
+    __syncthreads();
+    float *out = a.partial + (size_t)blockIdx.x * a.partial_stride;
+    for (int e = threadIdx.x; e < E; e += kBlkThreads) {
+        float acc = 0.f;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) acc += red[w * E + e];
+        out[e] = acc;
+    }
+}
+
+template <typename Tio, int DQK, int DV, int KW>
+__global__ void __launch_bounds__(kBlkThreads)
+    gdr_prologue_bwd_kernel(const PrologueBwdArgs a, int stage_bytes, int xalloc,
+                            const __grid_constant__ CUtensorMap tm_xq, const __grid_constant__ CUtensorMap tm_xk,
+                            const __grid_constant__ CUtensorMap tm_xv, const __grid_constant__ CUtensorMap tm_dq,
+                            const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv) {
+    using namespace sm100;
+    constexpr int DMAX = DQK > DV ? DQK : DV;
+    extern __shared__ __align__(128) uint8_t blk_smem[];
+    uint8_t *smem = blk_smem;
+    float *dzs = reinterpret_cast<float *>(smem + kProBwdStages * stage_bytes);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(dzs + (kProBwdRun + KW - 1) * DMAX);
+    const int P = 3 * a.H, pair = blockIdx.x % P, idx = blockIdx.x / P, G = gridDim.x / P;
+    const int s = pair / a.H, h = pair % a.H;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kProBwdStages; ++i) mbar_init(&bars[i], 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (s == 0)
+        prologue_bwd_block<Tio, DQK, KW>(a, &tm_xq, &tm_dq, s, h, idx, G, smem, stage_bytes, xalloc, dzs, bars);
+    else if (s == 1)
+        prologue_bwd_block<Tio, DQK, KW>(a, &tm_xk, &tm_dk, s, h, idx, G, smem, stage_bytes, xalloc, dzs, bars);
+    else
+        prologue_bwd_block<Tio, DV, KW>(a, &tm_xv, &tm_dv, s, h, idx, G, smem, stage_bytes, xalloc, dzs, bars);
+}
+
+// dw[s][(h*D + c)*K + j] and dbias[s][h*D + c]: the sums over the G blocks of
+// pair (s, h) in block order.  One block per pair.
+struct PrologueBwdSum {
+    int H, dk, dv, K, KW, G, stride;
+    const float *partial;
+    float *dw[3];
+    float *dbias[3];  // each may be null (not written)
+};
+
+__global__ void prologue_bwd_sum_kernel(const PrologueBwdSum p) {
+    const int P = 3 * p.H, pair = blockIdx.x, s = pair / p.H, h = pair % p.H;
+    const int D = s < 2 ? p.dk : p.dv;
+    float *dw = s == 0 ? p.dw[0] : s == 1 ? p.dw[1] : p.dw[2];
+    float *db = s == 0 ? p.dbias[0] : s == 1 ? p.dbias[1] : p.dbias[2];
+    for (int e = threadIdx.x; e < D * (p.K + 1); e += blockDim.x) {
+        const int c = e / (p.K + 1), m = e % (p.K + 1);
+        const int slot = c * (p.KW + 1) + (m < p.K ? m : p.KW);
+        float acc = 0.f;
+        for (int g = 0; g < p.G; ++g) acc += p.partial[(size_t)(g * P + pair) * p.stride + slot];
+        if (m < p.K)
+            dw[(size_t)(h * D + c) * p.K + m] = acc;
+        else if (db != nullptr)
+            db[h * D + c] = acc;
+    }
+}
+
 // ---- epilogue ---------------------------------------------------------------------
 // y = o / sqrt(mean(o^2) + eps) * weight * SiLU(g) per row of dv channels;
 // g == nullptr leaves out the gate.  Rows are the B*T*H (token, head) pairs,
@@ -686,6 +955,73 @@ inline cudaError_t launch_epilogue_bwd(long long rows, int dv, const void *o, co
         return cudaGetLastError();
     };
     return dv == 128 ? run(gdr_epilogue_bwd_kernel<Tio, 4, NS>, 128) : run(gdr_epilogue_bwd_kernel<Tio, 2, NS>, 64);
+}
+
+// Grid: 3H pairs x G blocks, G filling the resident slots (at most
+// kProBwdMaxG); then one block per pair for the fixed-order sums.
+template <typename Tio, int DQK, int DV, int KW>
+inline cudaError_t launch_prologue_bwd_kw(PrologueBwdArgs a, float *const dw[3], float *const dbias[3],
+                                          cudaStream_t stream) {
+    constexpr int DMAX = DQK > DV ? DQK : DV;
+    auto kern = gdr_prologue_bwd_kernel<Tio, DQK, DV, KW>;
+    const int xalloc = (kProBwdRun + 2 * (KW - 1)) * DMAX * (int)sizeof(Tio);
+    const int stage_bytes = xalloc + (kProBwdRun + KW - 1) * DMAX * (int)sizeof(Tio);
+    static_assert((kBlkThreads / 32) * DMAX * (KW + 1) * 4 <=
+                      kProBwdStages * ((kProBwdRun + 2 * (KW - 1)) + (kProBwdRun + KW - 1)) * DMAX * 2,
+                  "warp sums must fit in the stages");
+    const int smem = kProBwdStages * stage_bytes + (kProBwdRun + KW - 1) * DMAX * 4 + 8 * kProBwdStages;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    const int K = a.K;
+    CUtensorMap mx[3], mdy[3];
+    for (int s = 0; s < 3; ++s) {
+        const int d = s < 2 ? a.dk : a.dv;
+        if (!make_prologue_map<Tio>(&mx[s], a.x[s], a.B, a.T, a.H, d, kProBwdRun + 2 * (K - 1)) ||
+            !make_prologue_map<Tio>(&mdy[s], a.dy[s], a.B, a.T, a.H, d, kProBwdRun + K - 1))
+            return cudaErrorInvalidValue;
+    }
+    const long long pairs = 3LL * a.H, units = (long long)a.B * ((a.T + kProBwdRun - 1) / kProBwdRun);
+    const long long slots = resident_grid(kern, 1LL << 40, smem);
+    if (slots <= 0) return cudaErrorInvalidConfiguration;
+    const long long G = std::max(1LL, std::min({units, slots / pairs, (long long)kProBwdMaxG}));
+    if (pairs * G >= (1LL << 31)) return cudaErrorInvalidConfiguration;
+    a.partial_stride = DMAX * (KW + 1);
+    kern<<<(unsigned)(pairs * G), kBlkThreads, smem, stream>>>(a, stage_bytes, xalloc, mx[0], mx[1], mx[2], mdy[0],
+                                                              mdy[1], mdy[2]);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    PrologueBwdSum p{};
+    p.H = a.H; p.dk = a.dk; p.dv = a.dv; p.K = K; p.KW = KW; p.G = (int)G; p.stride = a.partial_stride;
+    p.partial = a.partial;
+    for (int s = 0; s < 3; ++s) {
+        p.dw[s] = dw[s];
+        p.dbias[s] = dbias[s];
+    }
+    prologue_bwd_sum_kernel<<<(unsigned)pairs, kBlkThreads, 0, stream>>>(p);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return cudaGetLastError();
+}
+
+// Workspace of the per-block partial sums.
+inline size_t prologue_bwd_workspace(int H, int dk, int dv, int K) {
+    const int KW = K <= 4 ? 4 : kConvMax;
+    return (size_t)3 * H * kProBwdMaxG * std::max(dk, dv) * (KW + 1) * sizeof(float);
+}
+
+template <typename Tio, int DQK, int DV>
+inline cudaError_t launch_prologue_bwd_t(const PrologueBwdArgs &a, float *const dw[3], float *const dbias[3],
+                                         cudaStream_t stream) {
+    return a.K <= 4 ? launch_prologue_bwd_kw<Tio, DQK, DV, 4>(a, dw, dbias, stream)
+                    : launch_prologue_bwd_kw<Tio, DQK, DV, kConvMax>(a, dw, dbias, stream);
+}
+
+template <typename Tio>
+inline cudaError_t launch_prologue_bwd(const PrologueBwdArgs &a, float *const dw[3], float *const dbias[3],
+                                       cudaStream_t stream) {
+    if (a.dk == 128 && a.dv == 128) return launch_prologue_bwd_t<Tio, 128, 128>(a, dw, dbias, stream);
+    if (a.dk == 128 && a.dv == 64) return launch_prologue_bwd_t<Tio, 128, 64>(a, dw, dbias, stream);
+    if (a.dk == 64 && a.dv == 128) return launch_prologue_bwd_t<Tio, 64, 128>(a, dw, dbias, stream);
+    return launch_prologue_bwd_t<Tio, 64, 64>(a, dw, dbias, stream);
 }
 
 }  // namespace gdr

@@ -547,6 +547,74 @@ gdr_status gdr_block_prologue(int B, int T, int H, int dk, int dv, int K, gdr_dt
     return GDR_OK;
 }
 
+size_t gdr_block_prologue_bwd_workspace_bytes(int H, int dk, int dv, int K) {
+    if (H < 1 || (dk != 64 && dk != 128) || (dv != 64 && dv != 128) || K < 1 || K > kConvMax) return 0;
+    return prologue_bwd_workspace(H, dk, dv, K);
+}
+
+gdr_status gdr_block_prologue_bwd(int B, int T, int H, int dk, int dv, int K, gdr_dtype dt, const void *xq,
+                                  const void *xk, const void *xv, const float *wq, const float *wk,
+                                  const float *wv, const float *bq, const float *bk, const float *bv,
+                                  const void *conv_state_in, float eps, const void *dyq, const void *dyk,
+                                  const void *dyv, const void *dconv_state_out, void *dxq, void *dxk, void *dxv,
+                                  float *dwq, float *dwk, float *dwv, float *dbq, float *dbk, float *dbv,
+                                  void *dconv_state_in, void *workspace, size_t workspace_bytes,
+                                  gdr_stream_t stream) {
+    const char *fn = "gdr_block_prologue_bwd";
+    gdr_status st = check_dims(fn, B, T, H, dk, dv, dt);
+    if (st != GDR_OK) return st;
+    if (K < 1 || K > kConvMax)
+        return fail(GDR_ERR_UNSUPPORTED, "%s: conv width K=%d (supported: 1..%d)", fn, K, kConvMax);
+    if (!(eps >= 0.f) || eps > 1e30f) return fail(GDR_ERR_INVALID_ARGUMENT, "%s: eps=%g", fn, (double)eps);
+    GDR_REQUIRE_PTR(xq);
+    GDR_REQUIRE_PTR(xk);
+    GDR_REQUIRE_PTR(xv);
+    GDR_REQUIRE_PTR(wq);
+    GDR_REQUIRE_PTR(wk);
+    GDR_REQUIRE_PTR(wv);
+    GDR_OPTIONAL_PTR(bq);
+    GDR_OPTIONAL_PTR(bk);
+    GDR_OPTIONAL_PTR(bv);
+    GDR_OPTIONAL_PTR(conv_state_in);
+    GDR_REQUIRE_PTR(dyq);
+    GDR_REQUIRE_PTR(dyk);
+    GDR_REQUIRE_PTR(dyv);
+    GDR_OPTIONAL_PTR(dconv_state_out);
+    GDR_REQUIRE_PTR(dxq);
+    GDR_REQUIRE_PTR(dxk);
+    GDR_REQUIRE_PTR(dxv);
+    GDR_REQUIRE_PTR(dwq);
+    GDR_REQUIRE_PTR(dwk);
+    GDR_REQUIRE_PTR(dwv);
+    GDR_OPTIONAL_PTR(dbq);
+    GDR_OPTIONAL_PTR(dbk);
+    GDR_OPTIONAL_PTR(dbv);
+    GDR_OPTIONAL_PTR(dconv_state_in);
+    const size_t need = prologue_bwd_workspace(H, dk, dv, K);
+    if (workspace == nullptr || workspace_bytes < need)
+        return fail(GDR_ERR_WORKSPACE, "%s: workspace %zu bytes, need %zu", fn, workspace_bytes, need);
+    if (!aligned16(workspace)) return fail(GDR_ERR_INVALID_ARGUMENT, "%s: workspace is not 16-byte aligned", fn);
+    PrologueBwdArgs a{};
+    a.B = B; a.T = T; a.H = H; a.dk = dk; a.dv = dv; a.K = K;
+    a.x[0] = xq; a.x[1] = xk; a.x[2] = xv;
+    a.w[0] = wq; a.w[1] = wk; a.w[2] = wv;
+    a.bias[0] = bq; a.bias[1] = bk; a.bias[2] = bv;
+    a.state_in = K > 1 ? conv_state_in : nullptr;
+    a.eps = eps;
+    a.dy[0] = dyq; a.dy[1] = dyk; a.dy[2] = dyv;
+    a.dstate_out = K > 1 ? dconv_state_out : nullptr;
+    a.dx[0] = dxq; a.dx[1] = dxk; a.dx[2] = dxv;
+    a.dstate_in = K > 1 ? dconv_state_in : nullptr;
+    a.partial = static_cast<float *>(workspace);
+    float *const dw[3] = {dwq, dwk, dwv};
+    float *const db[3] = {dbq, dbk, dbv};
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = dt == GDR_F32 ? launch_prologue_bwd<float>(a, dw, db, s)
+                                  : launch_prologue_bwd<__nv_bfloat16>(a, dw, db, s);
+    if (e != cudaSuccess) return cuda_fail(e, fn);
+    return GDR_OK;
+}
+
 gdr_status gdr_block_epilogue(int B, int T, int H, int dv, gdr_dtype dt, const void *o, const void *g,
                               const float *weight, float eps, void *y, gdr_stream_t stream) {
     const char *fn = "gdr_block_epilogue";

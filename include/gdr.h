@@ -260,6 +260,45 @@ GDR_API gdr_status gdr_block_prologue(int B, int T, int H, int dk, int dv, int K
                               void *q, void *k, void *v, gdr_stream_t stream);
 
 /*
+ * Backward of gdr_block_prologue (same page sections).  For each stream, with
+ * z = ShortConv(x), u = SiLU(z), n = sqrt(sum_head u^2 + eps), y = u / n
+ * (q, k) or y = u (v), and the incoming gradient dy of y:
+ *     du = (dy - y (y . dy)) / n   (q, k; per token and head)   du = dy (v)
+ *     dz = du sig(z) (1 + z (1 - sig(z))),  sig = 1/(1 + e^-z)
+ *     dx[s, c] = sum_j w[c, j] dz[s+K-1-j, c] over output tokens in [0, T)
+ *     dw[c, j] = sum_{b,t} dz[t, c] x[t-K+1+j, c]      dbias[c] = sum_{b,t} dz[t, c]
+ * where x at tokens -(K-1)..-1 is conv_state_in.  dconv_state_out, if given,
+ * is the gradient of the returned state: it adds to dx of the last K-1
+ * inputs (or to dconv_state_in where those were carried in, T < K-1).
+ *   in : the forward's inputs (xq, xk, xv, taps, biases, conv_state_in, eps);
+ *        dyq, dyk [B,T,H,dk]; dyv [B,T,H,dv] (dtype dt);
+ *        dconv_state_out [B, K-1, H*(2*dk+dv)] (dtype dt) or NULL (zero).
+ *   out: dxq, dxk [B,T,H,dk]; dxv [B,T,H,dv] (dtype dt);
+ *        dwq, dwk [H*dk, K]; dwv [H*dv, K] fp32, overwritten;
+ *        dbq, dbk, dbv fp32 or NULL (not written);
+ *        dconv_state_in [B, K-1, H*(2*dk+dv)] (dtype dt) or NULL (not written).
+ *   workspace: device scratch of gdr_block_prologue_bwd_workspace_bytes(H,
+ *        dk, dv, K) bytes: per-block partial sums of dw and dbias, which a
+ *        second launch adds in a fixed order (repeated calls give identical
+ *        bits).  No output may alias an input or another output.
+ *   Errors: as gdr_block_prologue; workspace NULL or short -> GDR_ERR_WORKSPACE.
+ */
+GDR_API gdr_status gdr_block_prologue_bwd(int B, int T, int H, int dk, int dv, int K, gdr_dtype dt,
+                                  const void *xq, const void *xk, const void *xv,
+                                  const float *wq, const float *wk, const float *wv,
+                                  const float *bq, const float *bk, const float *bv,
+                                  const void *conv_state_in, float eps,
+                                  const void *dyq, const void *dyk, const void *dyv,
+                                  const void *dconv_state_out,
+                                  void *dxq, void *dxk, void *dxv,
+                                  float *dwq, float *dwk, float *dwv,
+                                  float *dbq, float *dbk, float *dbv,
+                                  void *dconv_state_in, void *workspace, size_t workspace_bytes,
+                                  gdr_stream_t stream);
+/* 0 for unsupported sizes. */
+GDR_API size_t gdr_block_prologue_bwd_workspace_bytes(int H, int dk, int dv, int K);
+
+/*
  * Block epilogue: the recurrent output's normalisation and output gate, one
  * pass over HBM (same sources as gdr_block_prologue):
  *     y = o / sqrt(mean_i o_i^2 + eps) * weight * SiLU(g)

@@ -131,6 +131,22 @@ def block_prologue_inputs(B: int, T: int, H: int, dk: int, dv: int, K: int, dtyp
     return out
 
 
+def block_prologue_bwd_inputs(B: int, T: int, H: int, dk: int, dv: int, K: int, dtype: str = "bf16",
+                              seed: int = 0, bias: bool = True, state: bool = True,
+                              dstate: bool = False) -> dict:
+    """Prologue inputs plus incoming gradients dyq, dyk [B,T,H,dk], dyv
+    [B,T,H,dv] ~ N(0, 1) in dtype and, with dstate, a gradient of the returned
+    conv state dconv_state_out [B, K-1, H*(2dk+dv)] ~ N(0, 1)."""
+    x = block_prologue_inputs(B, T, H, dk, dv, K, dtype, seed, bias, state)
+    g = torch.Generator().manual_seed(seed * 7919 + 2)
+    dt = DTYPES[dtype]
+    for n, d in (("dyq", dk), ("dyk", dk), ("dyv", dv)):
+        x[n] = torch.randn(B, T, H, d, generator=g).to(dt)
+    x["dconv_state_out"] = (torch.randn(B, K - 1, H * (2 * dk + dv), generator=g).to(dt)
+                            if dstate and K > 1 else None)
+    return x
+
+
 def block_epilogue_inputs(B: int, T: int, H: int, dv: int, dtype: str = "bf16", seed: int = 0,
                           gate: bool = True) -> dict:
     """Inputs of the block epilogue (see the module docstring)."""

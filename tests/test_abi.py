@@ -151,6 +151,47 @@ def test_epilogue_bwd_rejects_bad_arguments(kw, status):
     assert gdr.lib().gdr_last_error_string().decode().startswith("gdr_block_epilogue_bwd")
 
 
+def _prologue_bwd(**kw):
+    a = dict(B=1, T=4, H=1, dk=64, dv=64, K=4, dt=gdr.GDR_BF16, x=FAKE, w=FAKE, bias=None, st=None,
+             eps=1e-6, dy=FAKE, dso=None, dx=FAKE, dw=FAKE, db=None, dsi=None, ws=FAKE, ws_bytes=1 << 24)
+    a.update(kw)
+    P = ctypes.c_void_p
+    return gdr.lib().gdr_block_prologue_bwd(
+        a["B"], a["T"], a["H"], a["dk"], a["dv"], a["K"], a["dt"], P(a["x"]), P(a["x"]), P(a["x"]), P(a["w"]),
+        P(a["w"]), P(a["w"]), P(a["bias"]), P(a["bias"]), P(a["bias"]), P(a["st"]), a["eps"], P(a["dy"]),
+        P(a["dy"]), P(a["dy"]), P(a["dso"]), P(a["dx"]), P(a["dx"]), P(a["dx"]), P(a["dw"]), P(a["dw"]),
+        P(a["dw"]), P(a["db"]), P(a["db"]), P(a["db"]), P(a["dsi"]), P(a["ws"]), a["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(K=0), gdr.GDR_ERR_UNSUPPORTED),
+    (dict(K=9), gdr.GDR_ERR_UNSUPPORTED),
+    (dict(dv=32), gdr.GDR_ERR_UNSUPPORTED),
+    (dict(eps=-1.0), gdr.GDR_ERR_INVALID_ARGUMENT),
+    (dict(x=None), gdr.GDR_ERR_INVALID_ARGUMENT),
+    (dict(dy=None), gdr.GDR_ERR_INVALID_ARGUMENT),
+    (dict(dx=None), gdr.GDR_ERR_INVALID_ARGUMENT),
+    (dict(dw=None), gdr.GDR_ERR_INVALID_ARGUMENT),
+    (dict(db=FAKE + 4), gdr.GDR_ERR_INVALID_ARGUMENT),
+    (dict(dso=FAKE + 2), gdr.GDR_ERR_INVALID_ARGUMENT),
+    (dict(dsi=FAKE + 8), gdr.GDR_ERR_INVALID_ARGUMENT),
+    (dict(ws=None), gdr.GDR_ERR_WORKSPACE),
+    (dict(ws_bytes=16), gdr.GDR_ERR_WORKSPACE),
+])
+def test_prologue_bwd_rejects_bad_arguments(kw, status):
+    assert _prologue_bwd(**kw) == status
+    assert gdr.lib().gdr_last_error_string().decode().startswith("gdr_block_prologue_bwd")
+
+
+def test_prologue_bwd_workspace_bytes():
+    L = gdr.lib()
+    # 3H pairs x 32 blocks x max(dk, dv) channels x (taps + bias) fp32
+    assert L.gdr_block_prologue_bwd_workspace_bytes(16, 128, 128, 4) == 3 * 16 * 32 * 128 * 5 * 4
+    assert L.gdr_block_prologue_bwd_workspace_bytes(2, 64, 128, 6) == 3 * 2 * 32 * 128 * 9 * 4
+    assert L.gdr_block_prologue_bwd_workspace_bytes(2, 64, 64, 9) == 0
+    assert L.gdr_block_prologue_bwd_workspace_bytes(0, 64, 64, 4) == 0
+
+
 def test_epilogue_bwd_workspace_bytes():
     assert gdr.lib().gdr_block_epilogue_bwd_workspace_bytes(128) == 1024 * 128 * 4
     assert gdr.lib().gdr_block_epilogue_bwd_workspace_bytes(64) == 1024 * 64 * 4

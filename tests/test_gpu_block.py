@@ -246,6 +246,87 @@ def test_epilogue_bwd_zero_rows_and_large_eps():
     assert_close(do, ref["do"], "f32")
 
 
+def _stream_cols(H, dk, dv):
+    return ((0, H * dk), (H * dk, 2 * H * dk), (2 * H * dk, H * (2 * dk + dv)))
+
+
+def _pro_bwd_ref(x, eps):
+    """Oracle reverse mode per stream; states split by column."""
+    H, dk, dv = x["xq"].shape[2], x["xq"].shape[3], x["xv"].shape[3]
+    st, dso = x["conv_state"], x["dconv_state_out"]
+    refs = []
+    for i, (s, (a_, b_)) in enumerate(zip("qkv", _stream_cols(H, dk, dv))):
+        refs.append(oracle.short_conv_bwd(
+            np64(x["x" + s]), np64(x["w" + s]), np64(x["dy" + s]), np64(x["b" + s]),
+            None if st is None else np64(st)[:, :, a_:b_], None if dso is None else np64(dso)[:, :, a_:b_],
+            l2=i < 2, eps=eps))
+    return refs
+
+
+def _pro_bwd_gpu(x, eps, want_dconv_state=None):
+    d = {k: dev(v) for k, v in x.items()}
+    out = gdr.gdr_block_prologue_bwd(d["xq"], d["xk"], d["xv"], d["wq"], d["wk"], d["wv"], d["dyq"], d["dyk"],
+                                     d["dyv"], d["bq"], d["bk"], d["bv"], conv_state=d["conv_state"],
+                                     dconv_state_out=d["dconv_state_out"], eps=eps,
+                                     want_dconv_state=want_dconv_state)
+    gdr.check_status()
+    return out
+
+
+def _check_pro_bwd(x, out, refs, dtype):
+    B, T, H, dk = x["xq"].shape
+    dv = x["xv"].shape[3]
+    for s, r, (a_, b_) in zip("qkv", refs, _stream_cols(H, dk, dv)):
+        assert_close(out["dx" + s], r["dx"], dtype)
+        _assert_dweight(out["dw" + s], r["dw"], B * T)
+        if out["db" + s] is not None:
+            _assert_dweight(out["db" + s], r["dbias"], B * T)
+        if out["dconv_state"] is not None:
+            assert_close(out["dconv_state"][:, :, a_:b_], r["dstate"], dtype)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("dk,dv", [(128, 128), (64, 64), (64, 128), (128, 64)])
+@pytest.mark.parametrize("T", [1, 3, 64, 130])
+def test_prologue_bwd_small(dtype, dk, dv, T):
+    x = synth.block_prologue_bwd_inputs(2, T, 3, dk, dv, 4, dtype, seed=T + dk + 5 * dv, dstate=True)
+    _check_pro_bwd(x, _pro_bwd_gpu(x, 1e-6), _pro_bwd_ref(x, 1e-6), dtype)
+
+
+@pytest.mark.parametrize("K", [1, 2, 3, 5, 8])
+@pytest.mark.parametrize("bias,state,dstate", [(True, True, True), (False, False, False), (True, False, True),
+                                              (False, True, False)])
+def test_prologue_bwd_widths_and_optional_inputs(K, bias, state, dstate):
+    x = synth.block_prologue_bwd_inputs(2, 97, 2, 128, 128, K, "bf16", seed=K * 11 + bias + 2 * state,
+                                        bias=bias, state=state, dstate=dstate)
+    _check_pro_bwd(x, _pro_bwd_gpu(x, 1e-6, want_dconv_state=K > 1), _pro_bwd_ref(x, 1e-6), "bf16")
+
+
+@pytest.mark.parametrize("T", [1, 2, 5])
+def test_prologue_bwd_shorter_than_the_window(T):
+    # T < K-1: part of the returned state is the carried-in state, so its
+    # gradient flows into dconv_state_in
+    x = synth.block_prologue_bwd_inputs(1, T, 2, 64, 64, 8, "f32", seed=T, dstate=True)
+    _check_pro_bwd(x, _pro_bwd_gpu(x, 0.0), _pro_bwd_ref(x, 0.0), "f32")
+
+
+def test_prologue_bwd_workload_full():
+    # B4 T4096 H16 d128 K4 bf16: every element of dx and the full sums
+    x = synth.block_prologue_bwd_inputs(4, 4096, 16, 128, 128, 4, "bf16", seed=31, state=False)
+    out = _pro_bwd_gpu(x, 1e-6)
+    refs = _pro_bwd_ref(x, 1e-6)
+    _check_pro_bwd(x, out, refs, "bf16")
+
+
+def test_prologue_bwd_is_deterministic():
+    x = synth.block_prologue_bwd_inputs(2, 1500, 8, 128, 128, 4, "bf16", seed=3, dstate=True)
+    a = _pro_bwd_gpu(x, 1e-6)
+    b = _pro_bwd_gpu(x, 1e-6)
+    for n in a:
+        if a[n] is not None:
+            assert torch.equal(a[n], b[n]), n
+
+
 def test_block_kernels_count_launches():
     x = synth.block_prologue_inputs(1, 10, 1, 64, 64, 4, "bf16", seed=1)
     before = gdr.launch_count()
@@ -256,3 +337,5 @@ def test_block_kernels_count_launches():
     e["dy"] = torch.ones_like(e["o"])
     _epi_bwd_gpu(e, 1e-6)   # the backward and its fixed-order dweight sum
     assert gdr.launch_count() - before == 4
+    _pro_bwd_gpu(synth.block_prologue_bwd_inputs(1, 10, 1, 64, 64, 4, "bf16", seed=1), 1e-6)
+    assert gdr.launch_count() - before == 6
