@@ -205,6 +205,13 @@ def epilogue_bytes(B, T, H, dv, esize=2):
     return 3 * B * T * H * dv * esize + dv * 4
 
 
+def prologue_bwd_bytes(B, T, H, dk, dv, K, esize=2):
+    """Block prologue backward: read x and dy of the three streams, write dx;
+    the fp32 taps and biases in, their gradients out."""
+    C = H * (2 * dk + dv)
+    return 3 * B * T * C * esize + 2 * C * (K + 1) * 4
+
+
 def epilogue_bwd_bytes(B, T, H, dv, esize=2):
     """Block epilogue backward: read o, g and dy, write do and dg; the fp32
     weight in and dweight out."""
@@ -599,6 +606,17 @@ def block_lines(pk):
     gbs_p = prologue_bytes(B, T, H, d, d, K) / (us_p * 1e-6) / 1e9
     out["block_prologue"] = {"workload": "B=4 T=4096 H=16 dk=dv=128 bf16, ShortConv K=4 + SiLU + q/k L2",
                              "us": us_p, "achieved_gbs": gbs_p, "hbm_frac": gbs_p / pk["hbm_gbs"]}
+    pg = torch.Generator().manual_seed(25)
+    dys = [torch.randn(B, T, H, d, generator=pg).to(torch.bfloat16).cuda() for _ in range(3)]
+    pws = torch.empty(gdr.lib().gdr_block_prologue_bwd_workspace_bytes(H, d, d, K), dtype=torch.uint8,
+                      device="cuda")
+    pro_bwd = lambda: gdr.gdr_block_prologue_bwd(px["xq"], px["xk"], px["xv"], px["wq"], px["wk"], px["wv"],
+                                                 *dys, px["bq"], px["bk"], px["bv"], eps=1e-6, workspace=pws)
+    us_pb = timed(pro_bwd) * 1e3
+    gbs_pb = prologue_bwd_bytes(B, T, H, d, d, K) / (us_pb * 1e-6) / 1e9
+    out["block_prologue_bwd"] = {"workload": "B=4 T=4096 H=16 dk=dv=128 bf16, backward of ShortConv K=4 + SiLU "
+                                             "+ q/k L2 (dx, dw, dbias; 2 launches)",
+                                 "us": us_pb, "achieved_gbs": gbs_pb, "hbm_frac": gbs_pb / pk["hbm_gbs"]}
     us_e = timed(lambda: epi(ex["o"])) * 1e3
     gbs_e = epilogue_bytes(B, T, H, d) / (us_e * 1e-6) / 1e9
     out["block_epilogue"] = {"workload": "B=4 T=4096 H=16 dv=128 bf16, RMSNorm + SiLU gate",

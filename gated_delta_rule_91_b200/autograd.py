@@ -6,12 +6,15 @@ S0=None)` does the same for Gated DeltaNet-2 through gdr2_bwd.  The forward
 and the backward are the library's CUDA calls: these classes only save the
 inputs and hand the incoming gradients over (the backward recomputes the
 forward's states itself, so nothing else is kept).  Unused outputs arrive as
-zero gradients.  `block_epilogue(o, g, weight, eps)` is the block's output
-normalisation and gate, differentiated through gdr_block_epilogue_bwd.
+zero gradients.  `block_prologue(...)` (ShortConv, SiLU, q/k L2) and
+`block_epilogue(o, g, weight, eps)` (RMSNorm, weight, SiLU gate) are the
+block's steps around the recurrence, differentiated through
+gdr_block_prologue_bwd and gdr_block_epilogue_bwd.
 """
 import torch
 
-from . import gdr2_bwd, gdr2_fwd, gdr_block_epilogue, gdr_block_epilogue_bwd, gdr_bwd, gdr_fwd
+from . import (gdr2_bwd, gdr2_fwd, gdr_block_epilogue, gdr_block_epilogue_bwd, gdr_block_prologue,
+               gdr_block_prologue_bwd, gdr_bwd, gdr_fwd)
 
 
 def _c(x):
@@ -82,3 +85,30 @@ class BlockEpilogue(torch.autograd.Function):
 def block_epilogue(o, g, weight, eps=1e-6):
     """Differentiable gdr_block_epilogue: returns y."""
     return BlockEpilogue.apply(o, g, weight, eps)
+
+
+class BlockPrologue(torch.autograd.Function):
+    """q = L2(SiLU(conv(xq))), k = L2(SiLU(conv(xk))), v = SiLU(conv(xv)),
+    the convolution reading the carried conv state before token 0."""
+
+    @staticmethod
+    def forward(ctx, xq, xk, xv, wq, wk, wv, bq, bk, bv, conv_state, eps):
+        xq, xk, xv, conv_state = map(_c, (xq, xk, xv, conv_state))
+        ctx.eps = eps
+        ctx.has_bias = bq is not None
+        ctx.save_for_backward(xq, xk, xv, wq, wk, wv, bq, bk, bv, conv_state)
+        return gdr_block_prologue(xq, xk, xv, wq, wk, wv, bq, bk, bv, conv_state=conv_state, eps=eps)
+
+    @staticmethod
+    def backward(ctx, dq, dk, dv):
+        xq, xk, xv, wq, wk, wv, bq, bk, bv, conv_state = ctx.saved_tensors
+        g = gdr_block_prologue_bwd(xq, xk, xv, wq, wk, wv, _c(dq), _c(dk), _c(dv), bq, bk, bv,
+                                   conv_state=conv_state, eps=ctx.eps, want_dbias=ctx.has_bias,
+                                   want_dconv_state=conv_state is not None)
+        return (g["dxq"], g["dxk"], g["dxv"], g["dwq"], g["dwk"], g["dwv"], g["dbq"], g["dbk"], g["dbv"],
+                g["dconv_state"], None)
+
+
+def block_prologue(xq, xk, xv, wq, wk, wv, bq=None, bk=None, bv=None, conv_state=None, eps=1e-6):
+    """Differentiable gdr_block_prologue: returns (q, k, v)."""
+    return BlockPrologue.apply(xq, xk, xv, wq, wk, wv, bq, bk, bv, conv_state, eps)

@@ -9,7 +9,7 @@ import torch
 import gated_delta_rule_91_b200 as gdr
 import oracle
 import synth
-from gated_delta_rule_91_b200.autograd import block_epilogue, gated_delta_rule, gated_delta_rule2
+from gated_delta_rule_91_b200.autograd import block_epilogue, block_prologue, gated_delta_rule, gated_delta_rule2
 from gpu_common import TOL_G, TOL_O, dtype_name, fro_rel, max_rel, np64
 
 pytestmark = pytest.mark.gpu
@@ -71,6 +71,39 @@ def test_autograd_block_epilogue(gate):
     assert max_rel(np64(w.grad), ref["dweight"]) <= 1e-4
     if gate:
         assert max_rel(np64(g.grad), ref["dg"]) <= TOL_O["bf16"]
+
+
+def test_autograd_block_prologue_into_the_rule():
+    # prologue -> gated delta rule, one loss: gradients reach the conv taps,
+    # biases, inputs and the carried conv state through both backward calls
+    B, T, H, d, K = 1, 80, 2, 128, 4
+    px = synth.block_prologue_inputs(B, T, H, d, d, K, "bf16", seed=12)
+    gx = synth.gdr_inputs(B, T, H, d, d, "bf16", seed=13)
+    leaves = {n: _leaf(t) for n, t in px.items()}
+    q, k, v = block_prologue(*(leaves[n] for n in ("xq", "xk", "xv", "wq", "wk", "wv", "bq", "bk", "bv",
+                                                   "conv_state")), eps=1e-6)
+    la, be = gx["log_alpha"].cuda(), gx["beta"].cuda()
+    o, _ = gated_delta_rule(q, k, v, la, be, None)
+    wo = torch.randn(o.shape, generator=torch.Generator().manual_seed(3)).to(o.dtype).cuda()
+    (o.float() * wo.float()).sum().backward()
+    # reference: the oracle's forward of both steps, then both reverse modes
+    cols = ((0, H * d), (H * d, 2 * H * d), (2 * H * d, 3 * H * d))
+    ys = []
+    for i, (s, (a_, b_)) in enumerate(zip("qkv", cols)):
+        y, _ = oracle.short_conv(np64(px["x" + s]), np64(px["w" + s]), np64(px["b" + s]),
+                                 np64(px["conv_state"])[:, :, a_:b_], l2=i < 2, eps=1e-6)
+        ys.append(y)
+    # the rule consumes bf16 q, k, v: round the oracle's prologue outputs the same way
+    ys = [torch.from_numpy(y).to(torch.bfloat16).double().numpy() for y in ys]
+    gr = oracle.gdr_bwd(ys[0], ys[1], ys[2], np64(gx["log_alpha"]), np64(gx["beta"]), None, np64(wo),
+                        np.zeros((B, H, d, d)))
+    for i, (s, (a_, b_)) in enumerate(zip("qkv", cols)):
+        ref = oracle.short_conv_bwd(np64(px["x" + s]), np64(px["w" + s]), gr["d" + s], np64(px["b" + s]),
+                                    np64(px["conv_state"])[:, :, a_:b_], l2=i < 2, eps=1e-6)
+        assert max_rel(np64(leaves["x" + s].grad), ref["dx"]) <= TOL_G["bf16"], s
+        assert max_rel(np64(leaves["w" + s].grad), ref["dw"]) <= TOL_G["bf16"], s
+        assert max_rel(np64(leaves["b" + s].grad), ref["dbias"]) <= TOL_G["bf16"], s
+        assert max_rel(np64(leaves["conv_state"].grad)[:, :, a_:b_], ref["dstate"]) <= TOL_G["bf16"], s
 
 
 def test_captured_decode_loop_replays_like_eager():
