@@ -63,6 +63,9 @@ def parse_args():
                         "(long sequences over few heads take the parallel-segment path)")
     p.add_argument("--profile-gdn2-bwd", metavar="B,T,H", default=None,
                    help="only run gdr2_bwd twice on seeded bf16 d=128 inputs of this shape and exit")
+    p.add_argument("--profile-step", action="store_true",
+                   help="only run gdr_step three times on the decode workload (B256 H16 d128 bf16, "
+                        "268 MB fp32 state) and exit")
     p.add_argument("--profile-block", metavar="B,T,H", default=None,
                    help="only run the block prologue (K=4) and epilogue twice each on seeded bf16 "
                         "d=128 inputs of this shape and exit")
@@ -81,6 +84,20 @@ def profile_fwd(shape):
     torch.cuda.synchronize()
     gdr.check_status()
     print(json.dumps({"profile_fwd": shape, "status": "ok"}))
+
+
+def profile_step():
+    """Three decode steps on the decode workload's state and first inputs,
+    then a status check."""
+    import gated_delta_rule_91_b200 as gdr
+    w = synth.WORKLOADS["decode"]
+    S = synth.decode_state(w.B, w.H, w.dk, w.dv, w.seed).cuda()
+    x = {n: t.cuda() for n, t in synth.decode_step_inputs(w.B, w.H, w.dk, w.dv, w.dtype, w.seed, 0).items()}
+    for _ in range(3):
+        gdr.gdr_step(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], S)
+    torch.cuda.synchronize()
+    gdr.check_status()
+    print(json.dumps({"profile_step": "decode", "status": "ok"}))
 
 
 def profile_gdn2_bwd(shape):
@@ -348,21 +365,90 @@ def traffic_from_profile(kernel_tag):
     return float(tb)
 
 
-def cpu_baseline(w):
-    import oracle
-    x = synth.workload_inputs(WORKLOAD)
-    a = {n: (x[n].double().numpy() if x[n] is not None else None) for n in x}
+def workload_config(world):
+    """The `config` object of both arms' JSON lines (identical by construction)."""
+    w = synth.WORKLOADS[WORKLOAD]
+    return {"workload": WORKLOAD, "B": w.B, "T": w.T, "H": w.H, "dk": w.dk, "dv": w.dv,
+            "io_dtype": "bf16", "gates_state_dtype": "f32", "S0": "N(0,0.02)",
+            "l2": "inputs_exceed_l2 (q,k,v 201 MB > 126 MB L2); no flush",
+            "parallelism": "dp%d (independent (b,h) shards, no collective)" % world}
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def _np(x):
+    return {n: (t.double().numpy() if t is not None else None) for n, t in x.items()}
+
+
+def _time_oracle(fn, min_s=0.0):
+    """Run fn once (at least once, repeated until min_s seconds); seconds per run."""
     reps, t0 = 0, time.time()
     while True:
-        oracle.gdr_fwd(a["q"], a["k"], a["v"], a["log_alpha"], a["beta"], a["S0"])
+        fn()
         reps += 1
-        if time.time() - t0 >= 10.0:
+        if time.time() - t0 >= min_s:
             break
-    dt = (time.time() - t0) / reps
+    return (time.time() - t0) / reps, reps
+
+
+def cpu_baseline(w):
+    """The fp64 oracle on the host cores: the headline workload (repeated for
+    10 s), and once each the other workloads' oracle work -- the tiny fp32
+    workload and the Gated DeltaNet-2 workload in full, all 1024 decode steps,
+    the long workload's forward at full length and its backward on the first
+    2048 tokens (tokens/s of that slice)."""
+    import oracle
+    a = _np(synth.workload_inputs(WORKLOAD))
+    dt, reps = _time_oracle(lambda: oracle.gdr_fwd(a["q"], a["k"], a["v"], a["log_alpha"], a["beta"], a["S0"]),
+                            10.0)
+    per = {}
+    wt = synth.WORKLOADS["tiny_f32"]
+    t = _np(synth.workload_inputs("tiny_f32"))
+    s, r = _time_oracle(lambda: oracle.gdr_fwd(t["q"], t["k"], t["v"], t["log_alpha"], t["beta"], t["S0"]), 1.0)
+    per["tiny_f32"] = {"tok_per_s": wt.B * wt.T / s, "s_per_run": s, "runs": r}
+    w4 = synth.WORKLOADS["gdn2_fwd"]
+    g = _np(synth.workload_inputs("gdn2_fwd"))
+    s, r = _time_oracle(lambda: oracle.gdr2_fwd(g["q"], g["k"], g["v"], g["log_alpha"], g["b"], g["w"], g["S0"]))
+    per["gdn2_fwd"] = {"tok_per_s": w4.B * w4.T / s, "s_per_run": s, "runs": r}
+    del g
+    # decode: the 1024 steps' inputs are drawn outside the timed loop, 64 at a time
+    wd = synth.WORKLOADS["decode"]
+    S = synth.decode_state(wd.B, wd.H, wd.dk, wd.dv, wd.seed).double().numpy()
+    spent = 0.0
+    for c0 in range(0, wd.steps, 64):
+        xs = [_np(synth.decode_step_inputs(wd.B, wd.H, wd.dk, wd.dv, wd.dtype, wd.seed, st))
+              for st in range(c0, min(c0 + 64, wd.steps))]
+        t0 = time.time()
+        for xx in xs:
+            oracle.gdr_step_inplace(xx["q"], xx["k"], xx["v"], xx["log_alpha"], xx["beta"], S)
+        spent += time.time() - t0
+    per["decode"] = {"tok_per_s": wd.B * wd.steps / spent, "s_total": spent, "steps": wd.steps}
+    del S
+    wl = synth.WORKLOADS["long_fwd_bwd"]
+    l = _np(synth.workload_inputs("long_fwd_bwd"))
+    s, r = _time_oracle(lambda: oracle.gdr_fwd(l["q"], l["k"], l["v"], l["log_alpha"], l["beta"], l["S0"]))
+    per["long_fwd"] = {"tok_per_s": wl.B * wl.T / s, "s_per_run": s, "runs": r}
+    Ts = 2048
+    sl = {n: (v[:, :Ts].copy() if v is not None and v.ndim >= 3 else v) for n, v in l.items()}
+    s, r = _time_oracle(lambda: oracle.gdr_bwd(sl["q"], sl["k"], sl["v"], sl["log_alpha"], sl["beta"], None,
+                                               sl["dO"], None))
+    per["long_bwd_T2048_slice"] = {"tok_per_s": wl.B * Ts / s, "s_per_run": s, "runs": r,
+                                   "note": "backward on the first 2048 tokens (all 16 heads); the full "
+                                           "65,536 tokens would take about 32x as long"}
     return {"value": w.B * w.T / dt / 1e6, "unit": "Mtok/s", "cores": oracle.num_threads(),
-            "kind": "oracle",
+            "cpu_model": cpu_model(), "kind": "oracle",
             "sample": "the full workload B=%d T=%d H=%d d=%d, run %d time(s) back to back, "
-                      "fp64 sequential recurrence, OpenMP over (b,h)" % (w.B, w.T, w.H, w.dk, reps)}
+                      "fp64 sequential recurrence, OpenMP over (b,h)" % (w.B, w.T, w.H, w.dk, reps),
+            "per_workload": per}
 
 
 def run_reference(args, rank, world):
@@ -393,9 +479,9 @@ def run_reference(args, rank, world):
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "B": w.B, "T": w.T, "H": w.H, "dk": w.dk, "dv": w.dv},
+            "config": workload_config(world),
             "cpu_baseline": {"value": value, "unit": "Mtok/s", "cores": oracle.num_threads(),
-                             "kind": "oracle", "sample": sample},
+                             "cpu_model": cpu_model(), "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "Mtok/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -657,6 +743,9 @@ def main():
     if args.profile_fwd:
         profile_fwd(args.profile_fwd)
         return
+    if args.profile_step:
+        profile_step()
+        return
     rank, world, local = dist_init(args)
     if args.impl == "reference":
         run_reference(args, rank, world)  # no process group: rank 0 alone works
@@ -777,10 +866,7 @@ def main():
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "bf16", "data": "synthetic",
-                "config": {"workload": WORKLOAD, "B": B, "T": T, "H": H, "dk": dk, "dv": dv,
-                           "io_dtype": "bf16", "gates_state_dtype": "f32", "S0": "N(0,0.02)",
-                           "l2": "inputs_exceed_l2 (q,k,v 201 MB > 126 MB L2); no flush",
-                           "parallelism": "dp%d (independent (b,h) shards, no collective)" % world},
+                "config": workload_config(world),
                 "roofline": roof, "e2e": e2e, "gpu_launches": launches, "clocks": clk,
                 "cpu_baseline": cpu, "secondary": extra}
         print(json.dumps(line), flush=True)

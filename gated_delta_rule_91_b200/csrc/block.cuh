@@ -639,7 +639,7 @@ __global__ void prologue_bwd_sum_kernel(const PrologueBwdSum p) {
 // g == nullptr leaves out the gate.  Rows are the B*T*H (token, head) pairs,
 // contiguous in memory, so a unit of 64 rows of o (and of g) arrives by one
 // bulk copy each; a ring of kBlkStages units per block keeps copies in flight
-// while warps compute (warp w: rows 8w .. 8w+7 of the unit).
+// while warps compute (warp w: rows kRowsPerWarp*w .. kRowsPerWarp*(w+1)-1 of the unit, four rows at 512 threads).
 constexpr int kEpilogueRows = 64;
 constexpr int kEpiThreads = 512;  // 16 warps: 4 rows of a unit each
 
@@ -846,19 +846,17 @@ __global__ void epilogue_dweight_sum_kernel(int nblk, int D, const float *__rest
 
 // Grid = SMs x resident blocks of the kernel (capped by the work), so the
 // stride loop covers the units in whole waves.
-// (One cached figure per kernel instantiation: the library runs on B200s only.)
+// (Queried on every launch: the occupancy call is a cheap host query, and a
+// cache keyed on the kernel's type would mix instantiations whose shared
+// memory differs.)
 template <typename Kern>
 inline int resident_grid(Kern kernel, long long warps_needed, int smem = 0, int threads = kBlkThreads) {
-    static int per_sm = 0, sms = 0;
-    if (per_sm == 0) {
-        int dev = 0, nb = 0, ns = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&ns, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kernel, threads, smem) != cudaSuccess)
-            return 0;
-        sms = ns;
-        per_sm = nb > 0 ? nb : 1;
-    }
+    int dev = 0, nb = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kernel, threads, smem) != cudaSuccess)
+        return 0;
+    const int per_sm = nb > 0 ? nb : 1;
     const long long blocks = (warps_needed + threads / 32 - 1) / (threads / 32);
     return (int)std::min<long long>(blocks, (long long)sms * per_sm);
 }

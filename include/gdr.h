@@ -152,7 +152,10 @@ GDR_API size_t gdr_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, gdr_
  *
  * The first call on each device resolves the array's device address
  * (cudaGetSymbolAddress) with that device current; make that first call
- * before any stream capture.  All calls share the one array and it keeps
+ * before any stream capture.  The library keeps that address for the rest
+ * of the process: after cudaDeviceReset on a device the module is loaded
+ * again and the array may move, so do not call this entry point on a device
+ * that has been reset.  All calls share the one array and it keeps
  * the last call's contents (nothing in it needs to start at zero: every
  * byte a call reads is written earlier in the same call), so calls whose
  * work overlaps on the GPU (different streams, or threads racing on one

@@ -84,6 +84,22 @@ def gdr_step(q, k, v, log_alpha, beta, S):
     return o, S
 
 
+def gdr_step_inplace(q, k, v, log_alpha, beta, S):
+    """One decode token applied to S in place (S: float64, C-contiguous
+    [B,H,dv,dk], as returned by an earlier call or built by the caller).
+    Returns o [B,H,dv].  Same arithmetic as gdr_step without the copy of S,
+    for long decode sequences over a large state."""
+    q, k, v, la, be = map(_in, (q, k, v, log_alpha, beta))
+    if S.dtype != np.float64 or not S.flags["C_CONTIGUOUS"]:
+        raise ValueError("S must be a C-contiguous float64 array")
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    o = np.zeros((B, H, dv))
+    _load().oracle_gdr_step(B, H, dk, dv, _p(q), _p(k), _p(v), _p(la), _p(be),
+                            _p(S), _p(o))
+    return o
+
+
 def gdr_bwd(q, k, v, log_alpha, beta, S0, dO, dS_T=None):
     """Hand-derived reverse mode of gdr_fwd.  Returns a dict with dq, dk, dv,
     dlog_alpha, dbeta, dS0 (float64)."""

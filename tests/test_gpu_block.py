@@ -302,12 +302,17 @@ def test_prologue_bwd_widths_and_optional_inputs(K, bias, state, dstate):
     _check_pro_bwd(x, _pro_bwd_gpu(x, 1e-6, want_dconv_state=K > 1), _pro_bwd_ref(x, 1e-6), "bf16")
 
 
+@pytest.mark.parametrize("K", [4, 8])
 @pytest.mark.parametrize("T", [1, 2, 5])
-def test_prologue_bwd_shorter_than_the_window(T):
-    # T < K-1: part of the returned state is the carried-in state, so its
-    # gradient flows into dconv_state_in
-    x = synth.block_prologue_bwd_inputs(1, T, 2, 64, 64, 8, "f32", seed=T, dstate=True)
-    _check_pro_bwd(x, _pro_bwd_gpu(x, 0.0), _pro_bwd_ref(x, 0.0), "f32")
+@pytest.mark.parametrize("dtype,d", [("f32", 64), ("bf16", 128)])
+def test_prologue_bwd_shorter_than_the_window(T, K, dtype, d):
+    # T < K-1 (and, at K = 4, T >= K-1 for T = 5): part of the returned state
+    # is the carried-in state, so the gradient of the returned state flows
+    # into dconv_state_in; both the carried state and that gradient are given
+    x = synth.block_prologue_bwd_inputs(1, T, 2, d, d, K, dtype, seed=T + 10 * K, state=True, dstate=True)
+    assert x["conv_state"] is not None and x["dconv_state_out"] is not None
+    eps = 0.0 if dtype == "f32" else 1e-6
+    _check_pro_bwd(x, _pro_bwd_gpu(x, eps), _pro_bwd_ref(x, eps), dtype)
 
 
 def test_prologue_bwd_workload_full():

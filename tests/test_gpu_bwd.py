@@ -77,15 +77,15 @@ def test_bwd_long_workload_T2048_slice():
     _compare(got, ref, "bf16")
 
 
-def test_bwd_long_workload_full_length_sampled_heads():
-    """Full T=65536 backward (the timed configuration), two heads checked
-    against the oracle's reverse mode over the whole sequence."""
+def test_bwd_long_workload_full_length_all_heads():
+    """Full T=65536 backward (the timed configuration): every gradient of all
+    16 heads against the oracle's reverse mode over the whole sequence
+    (about 20 s of fp64 on 8 host cores)."""
     x = synth.workload_inputs("long_fwd_bwd")
     got = _gpu(x, None)
     torch.cuda.synchronize()
-    heads = [(0, 3), (0, 11)]
-    ref = _oracle(x, None, heads)
-    _compare(got, ref, "bf16", heads)
+    ref = _oracle(x, None)
+    _compare(got, ref, "bf16")
     gdr.check_status()
 
 

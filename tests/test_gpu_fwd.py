@@ -3,8 +3,7 @@
 Small cases compare every output element and span several chunks and a
 ragged tail; the full-size workloads (tiny fp32 B1 H2 T128 d64, and the
 layer-shaped bf16 B4 T4096 H16 d128 with random S0) run in the same launch
-configuration as the bench and are compared on sampled (b, h) heads that the
-oracle computes on their own (heads are independent).
+configuration as the bench and are compared on every head.
 """
 import numpy as np
 import pytest
@@ -63,19 +62,21 @@ def test_fwd_tiny_f32_workload():
     assert fro_rel(np64(ST), ST_ref) <= 1e-4
 
 
-def test_fwd_layer_workload_sampled_heads():
+def test_fwd_layer_workload_all_heads():
+    """Layer workload B4 T4096 H16 d128 bf16 with random S0, in the bench's
+    launch configuration: every output and final state of all 64 heads
+    against the oracle (about 2 s of fp64 on 8 host cores)."""
     x = synth.workload_inputs("layer_fwd")
     o, ST = _run(x)
     torch.cuda.synchronize()
-    rng = np.random.default_rng(1)
-    flat = rng.choice(4 * 16, size=6, replace=False)
-    bsel, hsel = flat // 16, flat % 16
-    o_ref, ST_ref = _ref(x, bsel, hsel)
+    o_ref, ST_ref = _ref(x)
     o_np, ST_np = np64(o), np64(ST)
-    for i, (b, h) in enumerate(zip(bsel, hsel)):
-        assert max_rel(o_np[b, :, h], o_ref[i, :, 0]) <= TOL_O["bf16"], (b, h)
-        assert fro_rel(ST_np[b, h], ST_ref[i, 0]) <= TOL_S, (b, h)
     assert np.isfinite(o_np).all()
+    for b in range(4):
+        for h in range(16):
+            assert max_rel(o_np[b, :, h], o_ref[b, :, h]) <= TOL_O["bf16"], (b, h)
+            assert fro_rel(ST_np[b, h], ST_ref[b, h]) <= TOL_S, (b, h)
+    assert max_rel(o_np, o_ref) <= TOL_O["bf16"]
 
 
 def test_fwd_matches_repeated_steps():

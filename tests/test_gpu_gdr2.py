@@ -38,16 +38,19 @@ def test_gdr2_small(dtype, T, dk, dv):
     assert fro_rel(np64(ST), ST_ref) <= (TOL_O["f32"] if dtype == "f32" else TOL_S)
 
 
-def test_gdr2_workload_sampled_heads():
+def test_gdr2_workload_all_heads():
+    """Gated DeltaNet-2 workload B4 T4096 H16 d128 bf16: every head's outputs
+    and final state against the oracle."""
     x = synth.workload_inputs("gdn2_fwd")
     o, ST = _gpu(x)
     torch.cuda.synchronize()
-    heads = [(0, 0), (1, 7), (3, 15), (2, 9)]
-    o_ref, ST_ref = _oracle(x, heads)
+    o_ref, ST_ref = _oracle(x)
     o_np, ST_np = np64(o), np64(ST)
-    for i, (b, h) in enumerate(heads):
-        assert max_rel(o_np[b, :, h], o_ref[i, :, 0]) <= TOL_O["bf16"], (b, h)
-        assert fro_rel(ST_np[b, h], ST_ref[i, 0]) <= TOL_S, (b, h)
+    assert np.isfinite(o_np).all()
+    for b in range(4):
+        for h in range(16):
+            assert max_rel(o_np[b, :, h], o_ref[b, :, h]) <= TOL_O["bf16"], (b, h)
+            assert fro_rel(ST_np[b, h], ST_ref[b, h]) <= TOL_S, (b, h)
 
 
 def test_gdr2_collapses_to_gated_delta_rule_on_gpu():

@@ -30,31 +30,28 @@ def test_step_sequence_small(dtype, dk, dv):
     assert fro_rel(np64(S_dev), S_ref) <= (1e-5 if dtype == "f32" else TOL_S)
 
 
-def test_decode_workload_sampled_heads():
+def test_decode_workload_all_heads():
     """Decode workload B=256 H=16 d=128, bf16, 1024 consecutive steps on the
-    full state; o is checked at every step and S after the last step on 48
-    sampled (b, h) heads that the oracle follows."""
+    full state: o of all 4096 heads at every step and the whole state after
+    the last step against the oracle, which follows the full fp64 state in
+    place (about 45 ms per step on 8 host cores)."""
     w = synth.WORKLOADS["decode"]
     B, H, dk, dv = w.B, w.H, w.dk, w.dv
-    rng = np.random.default_rng(0)
-    flat = np.sort(rng.choice(B * H, size=48, replace=False))
-    bi, hi = flat // H, flat % H
     S = synth.decode_state(B, H, dk, dv, w.seed)
     S_dev = dev(S)
-    S_ref = np64(S)[bi, hi][:, None]          # [48, 1, dv, dk]
+    S_ref = np.ascontiguousarray(np64(S))
     worst = 0.0
     for t in range(w.steps):
         x = synth.decode_step_inputs(B, H, dk, dv, w.dtype, w.seed, t)
         o = gdr.gdr_step(dev(x["q"]), dev(x["k"]), dev(x["v"]), dev(x["log_alpha"]),
                          dev(x["beta"]), S_dev)
-        sel = lambda a: np64(a)[bi, hi][:, None]
-        o_ref, S_ref = oracle.gdr_step(sel(x["q"]), sel(x["k"]), sel(x["v"]),
-                                       sel(x["log_alpha"]), sel(x["beta"]), S_ref)
-        err = max_rel(np64(o)[bi, hi], o_ref[:, 0])
+        o_ref = oracle.gdr_step_inplace(np64(x["q"]), np64(x["k"]), np64(x["v"]),
+                                        np64(x["log_alpha"]), np64(x["beta"]), S_ref)
+        err = max_rel(np64(o), o_ref)
         worst = max(worst, err)
         assert err <= TOL_O["bf16"], (t, err)
     torch.cuda.synchronize()
-    assert fro_rel(np64(S_dev)[bi, hi], S_ref[:, 0]) <= TOL_S
+    assert fro_rel(np64(S_dev), S_ref) <= TOL_S
     gdr.check_status()
 
 
