@@ -25,8 +25,10 @@
 // dKiE and dE_C are sums over slices, written per slice and summed in a
 // fixed order by gdr2_bwd_reduce_kernel, which also applies the per-element
 // chain rule (deterministic, no atomics).  A chunk in which some channel
-// decays by more than e^80 (K/E would overflow) is not handled: the kernel
-// reports GDR_ERR_UNSUPPORTED through the status word.
+// decays by more than e^80 (where K/E would overflow) is walked token by
+// token instead, with the step's own reverse mode (gdr2_chunk_reverse_exact);
+// its per-token partials are summed by the same reduce kernel without the
+// E factors.
 #pragma once
 #include "common.cuh"
 #include "bwd_simt.cuh"
@@ -62,6 +64,138 @@ struct Bwd2Layout {
     static_assert(kBytes <= 232448, "shared memory budget");
 };
 
+// Reverse of one chunk for this CTA's slice of kBwd2Dvs state rows, token by
+// token, for a chunk whose factored operands would overflow.  Per token, with
+// S = S_{t-1}, P = S Diag(alpha), e = w*v - P(b*k) (so S_t = P + e k^T) and
+// G = dL/dS_t + do q^T, the step's reverse mode is
+//     gk = G k,  dv = w * gk,  dw = v * gk,  dL/dS_{t-1} = (G - gk (b*k)^T) Diag(alpha)
+// and the key-channel gradients are sums over the state rows:
+//     dq = S_t^T do,  dk = G^T e - b * X,  db = -k * X,
+//     dlog alpha_j = sum_i P_ij G_ij - b_j k_j X_j,   X = P^T gk.
+// This CTA writes its rows' dv, dw and its slice's partial sums of S_t^T do,
+// X, G^T e and sum_i P_ij G_ij per token; the reduce kernel adds the slices.
+// The states S_{t-1} of an 8-token block are recomputed from the chunk's entry
+// state (blocks from last to first) into `st` [8][kBwd2Dvs][DK]; D (dL/dS of
+// the slice) stays in registers.  Thread layout: row = tid / 8 of the slice,
+// DK / 8 channels from (tid % 8) * DK / 8; row dot products reduce over the
+// 8 lanes that share a row.
+template <typename Tio, int DK>
+__device__ void gdr2_chunk_reverse_exact(int n, size_t tok0, int H, int dv, int vcol0, const Tio *__restrict__ q,
+                                         const Tio *__restrict__ k, const Tio *__restrict__ v,
+                                         const float *__restrict__ log_alpha, const float *__restrict__ bgate,
+                                         const float *__restrict__ wgate, const Tio *__restrict__ dO, float *st,
+                                         float *red, const float *sS, float *sD, Tio *__restrict__ dv_out,
+                                         float *__restrict__ dw_out, float *__restrict__ part_qe,
+                                         float *__restrict__ part_kb, float *__restrict__ part_ki,
+                                         float *__restrict__ part_x, size_t pslice) {
+    constexpr int JW = DK / 8, LDK = DK + 1, R = kBwd2Dvs;
+    static_assert(R * 8 == kSimtThreads, "one row of the slice per 8 threads");
+    const int tid = threadIdx.x, row = tid >> 3, j0 = (tid & 7) * JW;
+    auto rowsum = [](float x) {
+        x += __shfl_xor_sync(0xffffffffu, x, 1);
+        x += __shfl_xor_sync(0xffffffffu, x, 2);
+        x += __shfl_xor_sync(0xffffffffu, x, 4);
+        return x;
+    };
+    auto ld = [&](const float *p, size_t t, float *out) {  // one token's JW key channels
+        const float *src = p + (tok0 + t * H) * DK + j0;
+#pragma unroll
+        for (int jj = 0; jj < JW; ++jj) out[jj] = src[jj];
+    };
+    auto ldt = [&](const Tio *p, size_t t, float *out) {
+        const Tio *src = p + (tok0 + t * H) * DK + j0;
+#pragma unroll
+        for (int jj = 0; jj < JW; ++jj) out[jj] = to_f32(src[jj]);
+    };
+    float d[JW];
+#pragma unroll
+    for (int jj = 0; jj < JW; ++jj) d[jj] = sD[row * LDK + j0 + jj];
+    const int nblk = (n + 7) / 8;
+#pragma unroll 1
+    for (int blk = nblk - 1; blk >= 0; --blk) {
+        const int ts = blk * 8, te = min(n, ts + 8);
+        {   // S_{t-1} for t = ts .. te-1, by the forward from the chunk's entry state
+            float s[JW];
+#pragma unroll
+            for (int jj = 0; jj < JW; ++jj) s[jj] = sS[row * LDK + j0 + jj];
+#pragma unroll 1
+            for (int t = 0; t < te; ++t) {
+                if (t >= ts) {
+#pragma unroll
+                    for (int jj = 0; jj < JW; ++jj) st[((t - ts) * R + row) * DK + j0 + jj] = s[jj];
+                }
+                if (t + 1 >= te) break;
+                float la[JW], bb[JW], kk[JW];
+                ld(log_alpha, t, la);
+                ld(bgate, t, bb);
+                ldt(k, t, kk);
+                float r = 0.f;
+#pragma unroll
+                for (int jj = 0; jj < JW; ++jj) {
+                    s[jj] *= expf(la[jj]);
+                    r = fmaf(s[jj], bb[jj] * kk[jj], r);
+                }
+                r = rowsum(r);
+                const size_t vo = (tok0 + (size_t)t * H) * dv + vcol0 + row;
+                const float e = wgate[vo] * to_f32(v[vo]) - r;
+#pragma unroll
+                for (int jj = 0; jj < JW; ++jj) s[jj] = fmaf(e, kk[jj], s[jj]);
+            }
+        }
+        __syncthreads();
+#pragma unroll 1
+        for (int t = te - 1; t >= ts; --t) {
+            float la[JW], bb[JW], kk[JW], qq[JW], p[JW], g[JW];
+            ld(log_alpha, t, la);
+            ld(bgate, t, bb);
+            ldt(k, t, kk);
+            ldt(q, t, qq);
+            const size_t vo = (tok0 + (size_t)t * H) * dv + vcol0 + row;
+            const float wv = wgate[vo], vv = to_f32(v[vo]), dov = to_f32(dO[vo]);
+            float r = 0.f, gk = 0.f;
+#pragma unroll
+            for (int jj = 0; jj < JW; ++jj) {
+                la[jj] = expf(la[jj]);  // alpha
+                p[jj] = st[((t - ts) * R + row) * DK + j0 + jj] * la[jj];
+                r = fmaf(p[jj], bb[jj] * kk[jj], r);
+                g[jj] = fmaf(dov, qq[jj], d[jj]);
+                gk = fmaf(g[jj], kk[jj], gk);
+            }
+            r = rowsum(r);
+            gk = rowsum(gk);
+            const float e = wv * vv - r;
+            if ((tid & 7) == 0) {
+                dv_out[vo] = from_f32<Tio>(wv * gk);
+                dw_out[vo] = vv * gk;
+            }
+            // the four row sums of this token, two at a time through `red` [2][R][DK]
+            const size_t prow = pslice * DK + (tok0 + (size_t)t * H) * DK;
+#pragma unroll
+            for (int pass = 0; pass < 2; ++pass) {
+#pragma unroll
+                for (int jj = 0; jj < JW; ++jj) {
+                    const float st_ = fmaf(e, kk[jj], p[jj]);  // S_t
+                    red[row * DK + j0 + jj] = pass == 0 ? st_ * dov : g[jj] * e;
+                    red[(R + row) * DK + j0 + jj] = pass == 0 ? p[jj] * gk : p[jj] * g[jj];
+                }
+                __syncthreads();
+                for (int c = tid; c < 2 * DK; c += kSimtThreads) {
+                    const int which = c / DK, j = c % DK;
+                    float acc = 0.f;
+                    for (int i = 0; i < R; ++i) acc += red[(which * R + i) * DK + j];
+                    float *dst = pass == 0 ? (which == 0 ? part_qe : part_ki) : (which == 0 ? part_kb : part_x);
+                    dst[prow + j] = acc;
+                }
+                __syncthreads();
+            }
+#pragma unroll
+            for (int jj = 0; jj < JW; ++jj) d[jj] = (g[jj] - gk * bb[jj] * kk[jj]) * la[jj];
+        }
+    }
+#pragma unroll
+    for (int jj = 0; jj < JW; ++jj) sD[row * LDK + j0 + jj] = d[jj];
+}
+
 template <typename Tio, int DK>
 __global__ void __launch_bounds__(kSimtThreads, 1)
 gdr2_bwd_simt_kernel(int T, int H, int dv, const Tio *__restrict__ q, const Tio *__restrict__ k,
@@ -70,7 +204,8 @@ gdr2_bwd_simt_kernel(int T, int H, int dv, const Tio *__restrict__ q, const Tio 
                      const Tio *__restrict__ dO, const float *__restrict__ dS_T,
                      const float *__restrict__ S_chunks, Tio *__restrict__ dv_out,
                      float *__restrict__ dw_out, float *__restrict__ dS0, float *__restrict__ part_kb,
-                     float *__restrict__ part_qe, float *__restrict__ part_ki, float *__restrict__ part_ec) {
+                     float *__restrict__ part_qe, float *__restrict__ part_ki, float *__restrict__ part_ec,
+                     float *__restrict__ part_x, int *__restrict__ exact_flags) {
     using L = Bwd2Layout<DK>;
     constexpr int NB = DK / 16;
     extern __shared__ float smem[];
@@ -134,7 +269,13 @@ gdr2_bwd_simt_kernel(int T, int H, int dv, const Tio *__restrict__ q, const Tio 
             if (-g > 80.f) *s_flag = 1;
         }
         __syncthreads();
-        if (*s_flag && tid == 0) record_status(GDR_ERR_UNSUPPORTED);
+        if (slice == 0 && tid == 0) exact_flags[(size_t)bh * nchunks + ch] = *s_flag;
+        if (*s_flag) {  // a channel decays past e^80 inside the chunk: token by token
+            gdr2_chunk_reverse_exact<Tio, DK>(n, tok0, H, dv, vcol0, q, k, v, log_alpha, bgate, wgate, dO, smem,
+                                              smem + L::odO, sS, sD, dv_out, dw_out, part_qe, part_kb, part_ki,
+                                              part_x, pslice);
+            continue;
+        }
 
         // ---- P1: A, P (C x C); R = W*V - KBE S^T -> sU
         {
@@ -427,6 +568,7 @@ gdr2_bwd_reduce_kernel(int T, int H, int nslice, const Tio *__restrict__ q, cons
                        const float *__restrict__ log_alpha, const float *__restrict__ bgate,
                        const float *__restrict__ part_kb, const float *__restrict__ part_qe,
                        const float *__restrict__ part_ki, const float *__restrict__ part_ec,
+                       const float *__restrict__ part_x, const int *__restrict__ exact_flags,
                        Tio *__restrict__ dq, Tio *__restrict__ dk, float *__restrict__ dlog_alpha,
                        float *__restrict__ db, size_t BTH) {
     __shared__ float sg[kChunk][DK];
@@ -438,6 +580,26 @@ gdr2_bwd_reduce_kernel(int T, int H, int nslice, const Tio *__restrict__ q, cons
     const size_t tok0 = ((size_t)b * T + c0) * H + h;
     const size_t nbh = BTH / T;
     const int j = threadIdx.x;
+    if (exact_flags[(size_t)bh * nchunks + ch]) {
+        // token-by-token partials: S_t^T do (part_qe), X = P^T gk (part_ki),
+        // G^T e (part_kb), sum_i P_ij G_ij (part_x)
+        for (int r = 0; r < n; ++r) {
+            const size_t off = (tok0 + (size_t)r * H) * DK + j;
+            float pq = 0.f, x = 0.f, y = 0.f, z = 0.f;
+            for (int s = 0; s < nslice; ++s) {
+                pq += part_qe[(size_t)s * BTH * DK + off];
+                x += part_ki[(size_t)s * BTH * DK + off];
+                y += part_kb[(size_t)s * BTH * DK + off];
+                z += part_x[(size_t)s * BTH * DK + off];
+            }
+            const float kv = to_f32(k[off]), bv = bgate[off];
+            dq[off] = from_f32<Tio>(pq);
+            dk[off] = from_f32<Tio>(fmaf(-bv, x, y));
+            db[off] = -kv * x;
+            dlog_alpha[off] = fmaf(-bv * kv, x, z);
+        }
+        return;
+    }
     float g = 0.f;
     for (int r = 0; r < n; ++r) {
         g += log_alpha[(tok0 + (size_t)r * H) * DK + j];
@@ -465,7 +627,8 @@ gdr2_bwd_reduce_kernel(int T, int H, int nslice, const Tio *__restrict__ q, cons
 }
 
 struct Bwd2Workspace {
-    float *states, *part_kb, *part_qe, *part_ki, *part_ec;
+    float *states, *part_kb, *part_qe, *part_ki, *part_ec, *part_x;
+    int *flags;
 };
 
 inline size_t bwd2_workspace_bytes(int B, int T, int H, int dk, int dv) {
@@ -473,7 +636,8 @@ inline size_t bwd2_workspace_bytes(int B, int T, int H, int dk, int dv) {
     const size_t ns = (size_t)dv / kBwd2Dvs;
     const size_t bth = (size_t)B * T * H;
     auto al = [](size_t x) { return (x + 255) / 256 * 256; };
-    return al((size_t)B * H * nch * dv * dk * 4) + 3 * al(ns * bth * dk * 4) + al(ns * B * H * nch * dk * 4);
+    return al((size_t)B * H * nch * dv * dk * 4) + 4 * al(ns * bth * dk * 4) + al(ns * B * H * nch * dk * 4) +
+           al((size_t)B * H * nch * 4);
 }
 
 inline Bwd2Workspace bwd2_carve(void *ws, int B, int T, int H, int dk, int dv) {
@@ -492,6 +656,10 @@ inline Bwd2Workspace bwd2_carve(void *ws, int B, int T, int H, int dk, int dv) {
     w.part_ki = reinterpret_cast<float *>(p);
     p += al(ns * bth * dk * 4);
     w.part_ec = reinterpret_cast<float *>(p);
+    p += al(ns * B * H * nch * dk * 4);
+    w.part_x = reinterpret_cast<float *>(p);
+    p += al(ns * bth * dk * 4);
+    w.flags = reinterpret_cast<int *>(p);
     return w;
 }
 
@@ -517,7 +685,7 @@ cudaError_t launch_bwd2_simt(int B, int T, int H, int dv, const void *q, const v
     kern<<<(unsigned)(B * H * nslice), kSimtThreads, L::kBytes, stream>>>(
         T, H, dv, static_cast<const Tio *>(q), static_cast<const Tio *>(k), static_cast<const Tio *>(v), la, bg,
         wg, static_cast<const Tio *>(dO), dS_T, w.states, static_cast<Tio *>(dv_out), dw, dS0, w.part_kb,
-        w.part_qe, w.part_ki, w.part_ec);
+        w.part_qe, w.part_ki, w.part_ec, w.part_x, w.flags);
     g_launches.fetch_add(1, std::memory_order_relaxed);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
@@ -525,7 +693,8 @@ cudaError_t launch_bwd2_simt(int B, int T, int H, int dv, const void *q, const v
     const int nch = (T + kChunk - 1) / kChunk;
     gdr2_bwd_reduce_kernel<Tio, DK><<<(unsigned)(B * H * nch), DK, 0, stream>>>(
         T, H, nslice, static_cast<const Tio *>(q), static_cast<const Tio *>(k), la, bg, w.part_kb, w.part_qe,
-        w.part_ki, w.part_ec, static_cast<Tio *>(dq), static_cast<Tio *>(dk_out), dla, db, (size_t)B * T * H);
+        w.part_ki, w.part_ec, w.part_x, w.flags, static_cast<Tio *>(dq), static_cast<Tio *>(dk_out), dla, db,
+        (size_t)B * T * H);
     g_launches.fetch_add(1, std::memory_order_relaxed);
     return cudaGetLastError();
 }

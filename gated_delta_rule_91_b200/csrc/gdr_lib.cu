@@ -128,7 +128,7 @@ gdr_status gdr_check_status(gdr_stream_t stream) {
         if (e != cudaSuccess) return cuda_fail(e, "gdr_check_status: clear status");
         return fail((gdr_status)host, "device status %d: %s", host,
                     host == GDR_ERR_TIMEOUT ? "a bounded on-chip wait gave up"
-                                            : "a chunk the kernel does not handle (gdr2_bwd: channel decay past e^80)");
+                                            : "a kernel reported an input it does not handle");
     }
     return GDR_OK;
 }

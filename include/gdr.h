@@ -196,10 +196,10 @@ GDR_API size_t gdr2_fwd_workspace_bytes(int B, int T, int H, int dk, int dv, gdr
  *        dlog_alpha, db [B,T,H,dk] fp32; dw [B,T,H,dv] fp32;
  *        dS0 [B,H,dv,dk] fp32 or NULL.
  * The caller-owned workspace (at least gdr2_bwd_workspace_bytes) holds the
- * recomputed forward's chunk-entry states and per-slice partial sums.  A
- * 64-token chunk in which some key channel decays by more than e^80 is not
- * handled: its gradients are not valid, and gdr_check_status then returns
- * GDR_ERR_UNSUPPORTED.
+ * recomputed forward's chunk-entry states and per-slice partial sums.  Any
+ * decay is handled: a 64-token chunk in which some key channel decays by more
+ * than e^80 (where the chunk form's per-channel factors would overflow) is
+ * differentiated token by token instead.
  */
 GDR_API gdr_status gdr2_bwd(int B, int T, int H, int dk, int dv, gdr_dtype dt,
                     const void *q, const void *k, const void *v,
@@ -402,8 +402,7 @@ GDR_API gdr_status gdr_seg_fixup(int B, int T, int H, int dk, int dv, gdr_dtype 
                          const void *qt, const float *S_in, void *o, gdr_stream_t stream);
 
 /* Synchronise `stream`, then read and clear the device status word that
- * kernels set when a bounded wait gives up (GDR_ERR_TIMEOUT) or when
- * gdr2_bwd meets a chunk it does not handle (GDR_ERR_UNSUPPORTED).  Returns
+ * kernels set when a bounded wait gives up (GDR_ERR_TIMEOUT).  Returns
  * GDR_OK, that status, or GDR_ERR_CUDA if the synchronisation itself failed. */
 GDR_API gdr_status gdr_check_status(gdr_stream_t stream);
 

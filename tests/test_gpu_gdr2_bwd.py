@@ -99,16 +99,29 @@ def test_gdr2_bwd_collapses_to_gdr_bwd_on_gpu():
     assert max_rel(np64(g2["db"].sum(-1) + g2["dw"].sum(-1)), np64(g1["dbeta"])) <= 1e-4
 
 
-def test_gdr2_bwd_reports_a_chunk_it_does_not_handle():
-    """A chunk in which some channel decays by more than e^80 is reported
-    through gdr_check_status as GDR_ERR_UNSUPPORTED (no fault)."""
-    x = _inputs(1, 100, 1, 128, 128, "bf16", seed=10)
-    x["log_alpha"][:, :, :, :8] = -3.0
-    _gpu(x, None)
-    with pytest.raises(gdr.GdrError) as e:
-        gdr.check_status()
-    assert e.value.status == gdr.GDR_ERR_UNSUPPORTED
-    gdr.check_status()  # the status word was cleared
+@pytest.mark.parametrize("dtype,dk,dv", [("f32", 64, 64), ("f32", 128, 128), ("bf16", 128, 128),
+                                          ("bf16", 64, 128)])
+def test_gdr2_bwd_strong_decay(dtype, dk, dv):
+    """Chunks in which some channel decays by more than e^80 (log alpha = -3
+    on 8 of the key channels: e^-192 over 64 tokens) go through the exact
+    token-by-token reverse; the others through the chunk form.  T = 229 mixes
+    both (the decay is applied from token 70 on) and ends in a ragged chunk."""
+    x = _inputs(2, 229, 2, dk, dv, dtype, seed=10 + dk + dv)
+    x["log_alpha"][:, 70:, :, :8] = -3.0
+    dST = torch.randn(2, 2, dv, dk, generator=torch.Generator().manual_seed(12)) * 0.1
+    got = _gpu(x, dST)
+    gdr.check_status()
+    _compare(got, _oracle(x, dST), dtype)
+
+
+def test_gdr2_bwd_strong_decay_every_channel():
+    """Every channel decays past e^80 in every chunk (log alpha = -2): the
+    whole sequence takes the exact path, with the erase gate in (0, 2)."""
+    x = _inputs(1, 150, 2, 128, 128, "bf16", seed=77, b_max=2.0)
+    x["log_alpha"][:] = -2.0
+    got = _gpu(x, None)
+    gdr.check_status()
+    _compare(got, _oracle(x, None), "bf16")
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
