@@ -34,11 +34,18 @@
 #include "bwd_simt.cuh"
 #include "gdr2_simt.cuh"
 #include "fwd2_tc.cuh"
+#include "bwd2_tc.cuh"
 #include <type_traits>
 
 namespace gdr {
 
 constexpr int kBwd2Dvs = 32;  // state rows per CTA
+// How a chunk is differentiated, from its largest per-channel decay span
+// -G_C: up to kBwd2TcSpan the products with dA and dP run on the tensor cores
+// (bf16 operands K/E, K*B*E, Q*E span e^span there), up to 80 in fp32 in the
+// reverse pass, beyond that token by token.
+constexpr float kBwd2TcSpan = 20.f;
+enum : int { kChunkTc = 0, kChunkExact = 1, kChunkF32 = 2 };
 
 template <int DK>
 struct Bwd2Layout {
@@ -205,7 +212,7 @@ gdr2_bwd_simt_kernel(int T, int H, int dv, const Tio *__restrict__ q, const Tio 
                      const float *__restrict__ S_chunks, Tio *__restrict__ dv_out,
                      float *__restrict__ dw_out, float *__restrict__ dS0, float *__restrict__ part_kb,
                      float *__restrict__ part_qe, float *__restrict__ part_ki, float *__restrict__ part_ec,
-                     float *__restrict__ part_x, int *__restrict__ exact_flags) {
+                     float *__restrict__ part_x, int *__restrict__ exact_flags, float *__restrict__ dAP) {
     using L = Bwd2Layout<DK>;
     constexpr int NB = DK / 16;
     extern __shared__ float smem[];
@@ -266,11 +273,14 @@ gdr2_bwd_simt_kernel(int T, int H, int dv, const Tio *__restrict__ q, const Tio 
                 sKI[r * L::LDK + j] = -g <= 80.f ? sKI[r * L::LDK + j] / e : 0.f;
             }
             sEC[j] = expf(g);
-            if (-g > 80.f) *s_flag = 1;
+            if (-g > 80.f) atomicMax(s_flag, kChunkExact + 1);
+            else if (-g > kBwd2TcSpan) atomicMax(s_flag, 1);
         }
         __syncthreads();
-        if (slice == 0 && tid == 0) exact_flags[(size_t)bh * nchunks + ch] = *s_flag;
-        if (*s_flag) {  // a channel decays past e^80 inside the chunk: token by token
+        // s_flag: 0 moderate decay, 1 past the tensor-core span, 2 past e^80
+        const int mode = *s_flag == 2 ? kChunkExact : (*s_flag == 1 || !dAP) ? kChunkF32 : kChunkTc;
+        if (slice == 0 && tid == 0) exact_flags[(size_t)bh * nchunks + ch] = mode;
+        if (mode == kChunkExact) {  // a channel decays past e^80 inside the chunk: token by token
             gdr2_chunk_reverse_exact<Tio, DK>(n, tok0, H, dv, vcol0, q, k, v, log_alpha, bgate, wgate, dO, smem,
                                               smem + L::odO, sS, sD, dv_out, dw_out, part_qe, part_kb, part_ki,
                                               part_x, pslice);
@@ -427,7 +437,17 @@ gdr2_bwd_simt_kernel(int T, int H, int dv, const Tio *__restrict__ q, const Tio 
         }
         __syncthreads();
 
-        // ---- P6: slice partials of dKBE, dQE, dKiE (C x DK) and of dE_C (DK)
+        // ---- P6: slice partials of dKBE, dQE, dKiE (C x DK) and of dE_C (DK).
+        // With dAP the products with dA and dP are left to the chunk kernel
+        // (bwd2_tc.cuh), which adds the slices' dA and dP first.
+        if (mode == kChunkTc) {
+            float *dst = dAP + (((size_t)slice * (BTH / T) + bh) * nchunks + ch) * 2 * kChunk * kChunk;
+            for (int idx = tid; idx < kChunk * kChunk; idx += blockDim.x) {
+                const int r = idx / kChunk, i = idx % kChunk;
+                dst[idx] = sdA[r * L::LDC + i];
+                dst[kChunk * kChunk + idx] = sdP[r * L::LDC + i];
+            }
+        }
         {
             float akb[4][NB] = {}, aqe[4][NB] = {}, aki[4][NB] = {}, ud[4][NB] = {};
             // -dR S (-> dKBE), dO S (-> dQE), U D (-> dKiE via Diag(E_C))
@@ -457,7 +477,7 @@ gdr2_bwd_simt_kernel(int T, int H, int dv, const Tio *__restrict__ q, const Tio 
             }
             // dA KiE (-> dKBE), dP KiE (-> dQE), dA^T KBE + dP^T QE (-> dKiE)
 #pragma unroll 2
-            for (int i = 0; i < kChunk; ++i) {
+            for (int i = 0; i < (mode == kChunkTc ? 0 : kChunk); ++i) {
                 float w_a[4], w_p[4], w_at[4], w_pt[4], ki[NB], kb[NB], qe[NB];
 #pragma unroll
                 for (int a = 0; a < 4; ++a) {
@@ -580,7 +600,7 @@ gdr2_bwd_reduce_kernel(int T, int H, int nslice, const Tio *__restrict__ q, cons
     const size_t tok0 = ((size_t)b * T + c0) * H + h;
     const size_t nbh = BTH / T;
     const int j = threadIdx.x;
-    if (exact_flags[(size_t)bh * nchunks + ch]) {
+    if (exact_flags[(size_t)bh * nchunks + ch] == kChunkExact) {
         // token-by-token partials: S_t^T do (part_qe), X = P^T gk (part_ki),
         // G^T e (part_kb), sum_i P_ij G_ij (part_x)
         for (int r = 0; r < n; ++r) {
@@ -627,17 +647,20 @@ gdr2_bwd_reduce_kernel(int T, int H, int nslice, const Tio *__restrict__ q, cons
 }
 
 struct Bwd2Workspace {
-    float *states, *part_kb, *part_qe, *part_ki, *part_ec, *part_x;
+    float *states, *part_kb, *part_qe, *part_ki, *part_ec, *part_x, *dAP;
     int *flags;
 };
 
-inline size_t bwd2_workspace_bytes(int B, int T, int H, int dk, int dv) {
+// bf16 with dk = 128 forms the chunk products on the tensor cores (bwd2_tc.cuh)
+inline bool bwd2_uses_tc(int dk, bool bf16) { return bf16 && dk == 128; }
+
+inline size_t bwd2_workspace_bytes(int B, int T, int H, int dk, int dv, bool bf16) {
     const size_t nch = (size_t)(T + kChunk - 1) / kChunk;
     const size_t ns = (size_t)dv / kBwd2Dvs;
     const size_t bth = (size_t)B * T * H;
     auto al = [](size_t x) { return (x + 255) / 256 * 256; };
     return al((size_t)B * H * nch * dv * dk * 4) + 4 * al(ns * bth * dk * 4) + al(ns * B * H * nch * dk * 4) +
-           al((size_t)B * H * nch * 4);
+           al((size_t)B * H * nch * 4) + (bwd2_uses_tc(dk, bf16) ? al(ns * B * H * nch * 2 * kChunk * kChunk * 4) : 0);
 }
 
 inline Bwd2Workspace bwd2_carve(void *ws, int B, int T, int H, int dk, int dv) {
@@ -660,6 +683,8 @@ inline Bwd2Workspace bwd2_carve(void *ws, int B, int T, int H, int dk, int dv) {
     w.part_x = reinterpret_cast<float *>(p);
     p += al(ns * bth * dk * 4);
     w.flags = reinterpret_cast<int *>(p);
+    p += al((size_t)B * H * nch * 4);
+    w.dAP = reinterpret_cast<float *>(p);  // used only with the tensor-core chunk kernel
     return w;
 }
 
@@ -677,6 +702,7 @@ cudaError_t launch_bwd2_simt(int B, int T, int H, int dv, const void *q, const v
                                                       w.states);
     if (err != cudaSuccess) return err;
     // 2) reverse chunk pass per (b, h, slice)
+    const bool tc = bwd2_uses_tc(DK, std::is_same<Tio, __nv_bfloat16>::value);
     using L = Bwd2Layout<DK>;
     auto kern = gdr2_bwd_simt_kernel<Tio, DK>;
     err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kBytes);
@@ -685,12 +711,24 @@ cudaError_t launch_bwd2_simt(int B, int T, int H, int dv, const void *q, const v
     kern<<<(unsigned)(B * H * nslice), kSimtThreads, L::kBytes, stream>>>(
         T, H, dv, static_cast<const Tio *>(q), static_cast<const Tio *>(k), static_cast<const Tio *>(v), la, bg,
         wg, static_cast<const Tio *>(dO), dS_T, w.states, static_cast<Tio *>(dv_out), dw, dS0, w.part_kb,
-        w.part_qe, w.part_ki, w.part_ec, w.part_x, w.flags);
+        w.part_qe, w.part_ki, w.part_ec, w.part_x, w.flags, tc ? w.dAP : nullptr);
     g_launches.fetch_add(1, std::memory_order_relaxed);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
-    // 3) sum the slices, chain rule through the gates, dlog alpha by reverse prefix sums
+    // 3) sum the slices (and, on the tensor cores, form the products with dA
+    //    and dP), chain rule through the gates, dlog alpha by reverse prefix sums
     const int nch = (T + kChunk - 1) / kChunk;
+    if (tc) {
+        auto ck = nslice == 4 ? gdr2_bwd_chunk_tc_kernel<Tio, 4> : gdr2_bwd_chunk_tc_kernel<Tio, 2>;
+        err = cudaFuncSetAttribute(ck, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Bwd2TcSmem::kAlloc);
+        if (err != cudaSuccess) return err;
+        ck<<<(unsigned)(B * H * nch), kBwd2TcThreads, Bwd2TcSmem::kAlloc, stream>>>(
+            T, H, static_cast<const Tio *>(q), static_cast<const Tio *>(k), la, bg, w.part_kb, w.part_qe,
+            w.part_ki, w.part_ec, w.part_x, w.flags, w.dAP, static_cast<Tio *>(dq), static_cast<Tio *>(dk_out), dla,
+            db, (size_t)B * T * H);
+        g_launches.fetch_add(1, std::memory_order_relaxed);
+        return cudaGetLastError();
+    }
     gdr2_bwd_reduce_kernel<Tio, DK><<<(unsigned)(B * H * nch), DK, 0, stream>>>(
         T, H, nslice, static_cast<const Tio *>(q), static_cast<const Tio *>(k), la, bg, w.part_kb, w.part_qe,
         w.part_ki, w.part_ec, w.part_x, w.flags, static_cast<Tio *>(dq), static_cast<Tio *>(dk_out), dla, db,

@@ -458,9 +458,9 @@ gdr_status gdr2_fwd(int B, int T, int H, int dk, int dv, gdr_dtype dt, const voi
     return GDR_OK;
 }
 
-size_t gdr2_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, gdr_dtype) {
+size_t gdr2_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, gdr_dtype dt) {
     if (B < 1 || T < 1 || H < 1 || (dk != 64 && dk != 128) || (dv != 64 && dv != 128)) return 0;
-    return bwd2_workspace_bytes(B, T, H, dk, dv);
+    return bwd2_workspace_bytes(B, T, H, dk, dv, dt == GDR_BF16);
 }
 
 gdr_status gdr2_bwd(int B, int T, int H, int dk, int dv, gdr_dtype dt, const void *q, const void *k,
@@ -487,7 +487,7 @@ gdr_status gdr2_bwd(int B, int T, int H, int dk, int dv, gdr_dtype dt, const voi
     GDR_OPTIONAL_PTR(S0);
     GDR_OPTIONAL_PTR(dS_T);
     GDR_OPTIONAL_PTR(dS0);
-    const size_t need = bwd2_workspace_bytes(B, T, H, dk, dv);
+    const size_t need = bwd2_workspace_bytes(B, T, H, dk, dv, dt == GDR_BF16);
     if (workspace == nullptr || workspace_bytes < need)
         return fail(GDR_ERR_WORKSPACE, "%s: workspace of %zu bytes needed, %zu given", fn, need,
                     workspace ? workspace_bytes : (size_t)0);

@@ -114,6 +114,19 @@ def test_gdr2_bwd_strong_decay(dtype, dk, dv):
     _compare(got, _oracle(x, dST), dtype)
 
 
+@pytest.mark.parametrize("la", [-0.3, -0.35])
+def test_gdr2_bwd_decay_near_the_tensor_core_span(la):
+    """A full chunk decays by e^-19.2 (log alpha = -0.3: products on the
+    tensor cores) or e^-22.4 (-0.35: products in fp32 in the reverse pass) on
+    every channel; both must match the oracle."""
+    x = _inputs(1, 200, 2, 128, 128, "bf16", seed=81)
+    x["log_alpha"][:] = la
+    dST = torch.randn(1, 2, 128, 128, generator=torch.Generator().manual_seed(13)) * 0.1
+    got = _gpu(x, dST)
+    gdr.check_status()
+    _compare(got, _oracle(x, dST), "bf16")
+
+
 def test_gdr2_bwd_strong_decay_every_channel():
     """Every channel decays past e^80 in every chunk (log alpha = -2): the
     whole sequence takes the exact path, with the erase gate in (0, 2)."""
