@@ -212,7 +212,8 @@ gdr2_bwd_simt_kernel(int T, int H, int dv, const Tio *__restrict__ q, const Tio 
                      const float *__restrict__ S_chunks, Tio *__restrict__ dv_out,
                      float *__restrict__ dw_out, float *__restrict__ dS0, float *__restrict__ part_kb,
                      float *__restrict__ part_qe, float *__restrict__ part_ki, float *__restrict__ part_ec,
-                     float *__restrict__ part_x, int *__restrict__ exact_flags, float *__restrict__ dAP) {
+                     float *__restrict__ part_x, int *__restrict__ exact_flags, float *__restrict__ dAP,
+                     const float *__restrict__ TP) {
     using L = Bwd2Layout<DK>;
     constexpr int NB = DK / 16;
     extern __shared__ float smem[];
@@ -287,11 +288,23 @@ gdr2_bwd_simt_kernel(int T, int H, int dv, const Tio *__restrict__ q, const Tio 
             continue;
         }
 
-        // ---- P1: A, P (C x C); R = W*V - KBE S^T -> sU
+        // ---- P1: A, P (C x C); R = W*V - KBE S^T -> sU.  With TP (tensor-core
+        // path, moderate decay) the recompute already formed T = (I + A)^{-1}
+        // and P: T goes where A would, and U = T R, dR = T^T dU replace the
+        // triangular solves below.
+        const bool have_t = TP != nullptr && mode == kChunkTc;
+        if (have_t) {
+            const float *src = TP + ((size_t)bh * nchunks + ch) * 2 * kChunk * kChunk;
+            for (int idx = tid; idx < kChunk * kChunk; idx += blockDim.x) {
+                const int r = idx >> 6, i = idx & 63;
+                sA[r * L::LDC + i] = src[idx];
+                sP[r * L::LDC + i] = src[kChunk * kChunk + idx];
+            }
+        }
         {
             float aa[4][4] = {}, pp[4][4] = {}, xs[4][2] = {};
 #pragma unroll 2
-            for (int j = 0; j < DK; ++j) {
+            for (int j = 0; j < (have_t ? 0 : DK); ++j) {
                 float kb[4], qe[4], ki[4], sc[2];
 #pragma unroll
                 for (int a = 0; a < 4; ++a) {
@@ -312,14 +325,30 @@ gdr2_bwd_simt_kernel(int T, int H, int dv, const Tio *__restrict__ q, const Tio 
                     for (int c = 0; c < 2; ++c) xs[a][c] = fmaf(kb[a], sc[c], xs[a][c]);
                 }
             }
+            if (have_t) {  // R alone
+#pragma unroll 2
+                for (int j = 0; j < DK; ++j) {
+                    float kb[4], sc[2];
+#pragma unroll
+                    for (int a = 0; a < 4; ++a) kb[a] = sKB[(ty + 16 * a) * L::LDK + j];
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) sc[c] = sS[(tx + 16 * c) * L::LDK + j];
+#pragma unroll
+                    for (int a = 0; a < 4; ++a)
+#pragma unroll
+                        for (int c = 0; c < 2; ++c) xs[a][c] = fmaf(kb[a], sc[c], xs[a][c]);
+                }
+            }
 #pragma unroll
             for (int a = 0; a < 4; ++a) {
                 const int r = ty + 16 * a;
+                if (!have_t) {
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const int i = tx + 16 * c;
-                    sA[r * L::LDC + i] = (i < r) ? aa[a][c] : 0.f;
-                    sP[r * L::LDC + i] = (i <= r) ? pp[a][c] : 0.f;
+                    for (int c = 0; c < 4; ++c) {
+                        const int i = tx + 16 * c;
+                        sA[r * L::LDC + i] = (i < r) ? aa[a][c] : 0.f;
+                        sP[r * L::LDC + i] = (i <= r) ? pp[a][c] : 0.f;
+                    }
                 }
 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
@@ -336,7 +365,28 @@ gdr2_bwd_simt_kernel(int T, int H, int dv, const Tio *__restrict__ q, const Tio 
         __syncthreads();
 
         // ---- P2: U = (I + A)^{-1} R
-        fwd_solve<L::LDC, L::LDV, kBwd2Dvs>(sA, sOne, sU);
+        if (have_t) {
+            float u[4][2] = {};
+            for (int i = 0; i < kChunk; ++i) {
+                float t[4], rr[2];
+#pragma unroll
+                for (int a = 0; a < 4; ++a) t[a] = sA[(ty + 16 * a) * L::LDC + i];
+#pragma unroll
+                for (int c = 0; c < 2; ++c) rr[c] = sU[i * L::LDV + tx + 16 * c];
+#pragma unroll
+                for (int a = 0; a < 4; ++a)
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) u[a][c] = fmaf(t[a], rr[c], u[a][c]);
+            }
+            __syncthreads();  // every read of R done
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int c = 0; c < 2; ++c) sU[(ty + 16 * a) * L::LDV + tx + 16 * c] = u[a][c];
+            __syncthreads();
+        } else {
+            fwd_solve<L::LDC, L::LDV, kBwd2Dvs>(sA, sOne, sU);
+        }
 
         // ---- P3: dU = Kt D^T + P^T dO -> sdR ; dP = dO U^T (i <= r) -> sdP
         {
@@ -397,7 +447,28 @@ gdr2_bwd_simt_kernel(int T, int H, int dv, const Tio *__restrict__ q, const Tio 
         __syncthreads();
 
         // ---- P4: dR = (I + A)^{-T} dU (in sdR)
-        back_solve<L::LDC, L::LDV, kBwd2Dvs>(sA, sOne, sdR);
+        if (have_t) {
+            float dr[4][2] = {};
+            for (int r = 0; r < kChunk; ++r) {
+                float t[4], du[2];
+#pragma unroll
+                for (int a = 0; a < 4; ++a) t[a] = sA[r * L::LDC + ty + 16 * a];
+#pragma unroll
+                for (int c = 0; c < 2; ++c) du[c] = sdR[r * L::LDV + tx + 16 * c];
+#pragma unroll
+                for (int a = 0; a < 4; ++a)
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) dr[a][c] = fmaf(t[a], du[c], dr[a][c]);
+            }
+            __syncthreads();  // every read of dU done
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int c = 0; c < 2; ++c) sdR[(ty + 16 * a) * L::LDV + tx + 16 * c] = dr[a][c];
+            __syncthreads();
+        } else {
+            back_solve<L::LDC, L::LDV, kBwd2Dvs>(sA, sOne, sdR);
+        }
 
         // ---- P5: dA = -dR U^T (i < r) -> sdA ; dV = W*dR, dW = V*dR
         {
@@ -647,7 +718,7 @@ gdr2_bwd_reduce_kernel(int T, int H, int nslice, const Tio *__restrict__ q, cons
 }
 
 struct Bwd2Workspace {
-    float *states, *part_kb, *part_qe, *part_ki, *part_ec, *part_x, *dAP;
+    float *states, *part_kb, *part_qe, *part_ki, *part_ec, *part_x, *dAP, *TP;
     int *flags;
 };
 
@@ -660,7 +731,10 @@ inline size_t bwd2_workspace_bytes(int B, int T, int H, int dk, int dv, bool bf1
     const size_t bth = (size_t)B * T * H;
     auto al = [](size_t x) { return (x + 255) / 256 * 256; };
     return al((size_t)B * H * nch * dv * dk * 4) + 4 * al(ns * bth * dk * 4) + al(ns * B * H * nch * dk * 4) +
-           al((size_t)B * H * nch * 4) + (bwd2_uses_tc(dk, bf16) ? al(ns * B * H * nch * 2 * kChunk * kChunk * 4) : 0);
+           al((size_t)B * H * nch * 4) +
+           (bwd2_uses_tc(dk, bf16) ? al(ns * B * H * nch * 2 * kChunk * kChunk * 4) +
+                                         al((size_t)B * H * nch * 2 * kChunk * kChunk * 4)
+                                   : 0);
 }
 
 inline Bwd2Workspace bwd2_carve(void *ws, int B, int T, int H, int dk, int dv) {
@@ -684,7 +758,9 @@ inline Bwd2Workspace bwd2_carve(void *ws, int B, int T, int H, int dk, int dv) {
     p += al(ns * bth * dk * 4);
     w.flags = reinterpret_cast<int *>(p);
     p += al((size_t)B * H * nch * 4);
-    w.dAP = reinterpret_cast<float *>(p);  // used only with the tensor-core chunk kernel
+    w.dAP = reinterpret_cast<float *>(p);  // these two only on the tensor-core path
+    p += al(ns * B * H * nch * 2 * kChunk * kChunk * 4);
+    w.TP = reinterpret_cast<float *>(p);
     return w;
 }
 
@@ -696,8 +772,11 @@ cudaError_t launch_bwd2_simt(int B, int T, int H, int dv, const void *q, const v
     Bwd2Workspace w = bwd2_carve(ws, B, T, H, DK, dv);
     // 1) forward recompute keeping every chunk's fp32 entry state (the
     //    tensor-core forward for bf16 with dk = dv = 128, else CUDA cores)
-    cudaError_t err = (std::is_same<Tio, __nv_bfloat16>::value && DK == 128 && dv == 128)
-                          ? launch_fwd2_tc(B, T, H, q, k, v, la, bg, wg, S0, nullptr, nullptr, stream, w.states)
+    // (the tensor-core forward also leaves every chunk's T and P for step 2)
+    const bool tc_fwd = std::is_same<Tio, __nv_bfloat16>::value && DK == 128 && dv == 128;
+    cudaError_t err = tc_fwd
+                          ? launch_fwd2_tc(B, T, H, q, k, v, la, bg, wg, S0, nullptr, nullptr, stream, w.states,
+                                           w.TP)
                           : launch_gdr2_simt<Tio, DK>(B, T, H, dv, q, k, v, la, bg, wg, S0, nullptr, nullptr, stream,
                                                       w.states);
     if (err != cudaSuccess) return err;
@@ -711,7 +790,7 @@ cudaError_t launch_bwd2_simt(int B, int T, int H, int dv, const void *q, const v
     kern<<<(unsigned)(B * H * nslice), kSimtThreads, L::kBytes, stream>>>(
         T, H, dv, static_cast<const Tio *>(q), static_cast<const Tio *>(k), static_cast<const Tio *>(v), la, bg,
         wg, static_cast<const Tio *>(dO), dS_T, w.states, static_cast<Tio *>(dv_out), dw, dS0, w.part_kb,
-        w.part_qe, w.part_ki, w.part_ec, w.part_x, w.flags, tc ? w.dAP : nullptr);
+        w.part_qe, w.part_ki, w.part_ec, w.part_x, w.flags, tc ? w.dAP : nullptr, tc_fwd ? w.TP : nullptr);
     g_launches.fetch_add(1, std::memory_order_relaxed);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;

@@ -165,7 +165,7 @@ gdr2_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                    int T, int H, const float *__restrict__ log_alpha, const float *__restrict__ bgate,
                    const float *__restrict__ wgate, const float *__restrict__ S0, float *__restrict__ S_T,
-                   int store_o, float *__restrict__ S_chunks) {
+                   int store_o, float *__restrict__ S_chunks, float *__restrict__ TP_chunks) {
     using L = G2Layout;
     using namespace sm100;
     constexpr int D = 128;
@@ -312,6 +312,13 @@ gdr2_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 for (int i = 0; i < 16; ++i) v[i] = (i0 + i <= r) ? v[i] : 0.f;
 #pragma unroll
                 for (int ch = 0; ch < 2; ++ch) st_bf16x8(sm + L::PB + sw128_offset(r, wc * 2 + ch), v + 8 * ch);
+                if (TP_chunks) {  // P in fp32 for the backward (second 64 x 64 block of the chunk)
+                    float4 *dst = reinterpret_cast<float4 *>(
+                        TP_chunks + (((size_t)bh * nch + n) * 2 + 1) * kChunk * kChunk + r * kChunk + i0);
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4)
+                        dst[k4] = make_float4(v[4 * k4], v[4 * k4 + 1], v[4 * k4 + 2], v[4 * k4 + 3]);
+                }
             }
         }
         __syncthreads();
@@ -380,6 +387,13 @@ gdr2_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                          smem_desc_sw128(tb + kk * 32, 16, 1024), idesc_bf16(128, 64, true, false), kk > 0);
             mma_commit(bar_mma);
             ++ncommit;
+        }
+        if (TP_chunks) {  // T in fp32 for the backward (its upper triangle as zeros)
+            float *dst = TP_chunks + ((size_t)bh * nch + n) * 2 * kChunk * kChunk;
+            for (int idx = tid; idx < kChunk * kChunk; idx += kG2Threads) {
+                const int r = idx >> 6, i = idx & 63;
+                dst[idx] = i <= r ? sT[r * kLdT + i] : 0.f;
+            }
         }
         if (!mma_wait_all()) break;
         {   // W^T (lane j, column r) -> W [j][r] bf16 over K/E
@@ -469,11 +483,14 @@ gdr2_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     }
 }
 
+// TP_chunks (nullable) receives every chunk's T = (I + A)^{-1} and P in fp32,
+// [B, H, nchunks, 2, 64, 64], for the backward's reverse pass.
 // o == nullptr runs without outputs (the backward's recompute); S_chunks
 // (nullable) receives every chunk's entry state, [B, H, nchunks, 128, 128] fp32.
 inline cudaError_t launch_fwd2_tc(int B, int T, int H, const void *q, const void *k, const void *v,
                                   const float *la, const float *bgate, const float *wgate, const float *S0,
-                                  void *o, float *S_T, cudaStream_t stream, float *S_chunks = nullptr) {
+                                  void *o, float *S_T, cudaStream_t stream, float *S_chunks = nullptr,
+                                  float *TP_chunks = nullptr) {
     CUtensorMap mq, mk, mv, mo;
     if (!make_token_map(&mq, q, B, T, H, 128) || !make_token_map(&mk, k, B, T, H, 128) ||
         !make_token_map(&mv, v, B, T, H, 128) || !make_token_map(&mo, o ? o : q, B, T, H, 128))
@@ -482,7 +499,7 @@ inline cudaError_t launch_fwd2_tc(int B, int T, int H, const void *q, const void
                                            (int)G2Layout::kAlloc);
     if (err != cudaSuccess) return err;
     gdr2_fwd_tc_kernel<<<(unsigned)(B * H), kG2Threads, G2Layout::kAlloc, stream>>>(
-        mq, mk, mv, mo, T, H, la, bgate, wgate, S0, S_T, o != nullptr ? 1 : 0, S_chunks);
+        mq, mk, mv, mo, T, H, la, bgate, wgate, S0, S_T, o != nullptr ? 1 : 0, S_chunks, TP_chunks);
     g_launches.fetch_add(1, std::memory_order_relaxed);
     return cudaGetLastError();
 }
