@@ -34,6 +34,7 @@
 #include "bwd_simt.cuh"
 #include "gdr2_simt.cuh"
 #include "fwd2_tc.cuh"
+#include "fwd2_tc2.cuh"
 #include "bwd2_tc.cuh"
 #include <type_traits>
 
@@ -775,8 +776,8 @@ cudaError_t launch_bwd2_simt(int B, int T, int H, int dv, const void *q, const v
     // (the tensor-core forward also leaves every chunk's T and P for step 2)
     const bool tc_fwd = std::is_same<Tio, __nv_bfloat16>::value && DK == 128 && dv == 128;
     cudaError_t err = tc_fwd
-                          ? launch_fwd2_tc(B, T, H, q, k, v, la, bg, wg, S0, nullptr, nullptr, stream, w.states,
-                                           w.TP)
+                          ? launch_fwd2_tc2(B, T, H, q, k, v, la, bg, wg, S0, nullptr, nullptr, stream, w.states,
+                                            w.TP)
                           : launch_gdr2_simt<Tio, DK>(B, T, H, dv, q, k, v, la, bg, wg, S0, nullptr, nullptr, stream,
                                                       w.states);
     if (err != cudaSuccess) return err;

@@ -21,6 +21,7 @@
 #include "fwd_tc2.cuh"
 #include "bwd_tc.cuh"
 #include "fwd2_tc.cuh"
+#include "fwd2_tc2.cuh"
 #include "bwd2_simt.cuh"
 
 namespace gdr {
@@ -439,11 +440,14 @@ gdr_status gdr2_fwd(int B, int T, int H, int dk, int dv, gdr_dtype dt, const voi
     (void)workspace_bytes;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e;
-    // bf16 with dk = dv = 128 runs on the tensor cores; GDR2_FWD_KERNEL=simt
-    // selects the CUDA-core kernel (used to cross-check it).
+    // bf16 with dk = dv = 128 runs on the tensor cores (the two-SM cluster
+    // kernel); GDR2_FWD_KERNEL=tc1 selects the single-CTA tensor-core kernel
+    // and GDR2_FWD_KERNEL=simt the CUDA-core kernel (used to cross-check them).
     const char *sel = getenv("GDR2_FWD_KERNEL");
     if (dt == GDR_BF16 && dk == 128 && dv == 128 && !(sel != nullptr && strcmp(sel, "simt") == 0)) {
-        e = launch_fwd2_tc(B, T, H, q, k, v, log_alpha, b, w, S0, o, S_T, s);
+        const bool tc1 = sel != nullptr && strcmp(sel, "tc1") == 0;
+        e = tc1 ? launch_fwd2_tc(B, T, H, q, k, v, log_alpha, b, w, S0, o, S_T, s)
+                : launch_fwd2_tc2(B, T, H, q, k, v, log_alpha, b, w, S0, o, S_T, s);
         if (e != cudaSuccess) return cuda_fail(e, fn);
         return GDR_OK;
     }

@@ -67,6 +67,42 @@ def test_gdr2_collapses_to_gated_delta_rule_on_gpu():
     assert fro_rel(np64(S2), np64(S1)) <= 1e-4
 
 
+@pytest.mark.parametrize("kernel", ["default", "tc1"])
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 130, 300])
+def test_gdr2_cluster_and_single_cta_kernels(kernel, T, monkeypatch):
+    """The default two-SM cluster kernel and the single-CTA tensor-core kernel
+    (GDR2_FWD_KERNEL=tc1) against the oracle: one token, a chunk less one, a
+    whole chunk, one past it, and ragged multi-chunk lengths."""
+    if kernel != "default":
+        monkeypatch.setenv("GDR2_FWD_KERNEL", kernel)
+    x = synth.gdr2_inputs(2, T, 3, 128, 128, "bf16", seed=400 + T, s0_std=0.02)
+    o, S = _gpu(x)
+    gdr.check_status()
+    o_ref, S_ref = _oracle(x)
+    assert max_rel(np64(o), o_ref) <= TOL_O["bf16"]
+    assert fro_rel(np64(S), S_ref) <= TOL_S
+
+
+@pytest.mark.parametrize("kernel", ["default", "tc1"])
+def test_gdr2_exact_chunks_between_ordinary_ones(kernel, monkeypatch):
+    """A decay spike (log alpha = -100 in four channels at one token) puts
+    chunks 1 and 3 past e^80: they take the exact path, the chunks around
+    them the tensor-core form, and the state must carry across both kinds.
+    T = 300 ends on a ragged chunk."""
+    if kernel != "default":
+        monkeypatch.setenv("GDR2_FWD_KERNEL", kernel)
+    x = synth.gdr2_inputs(2, 300, 2, 128, 128, "bf16", seed=88, s0_std=0.02)
+    la = x["log_alpha"].clone()
+    la[:, 70, :, 8:12] = -100.0
+    la[:, 200, :, 100:104] = -100.0
+    x["log_alpha"] = la
+    o, S = _gpu(x)
+    gdr.check_status()
+    o_ref, S_ref = _oracle(x)
+    assert max_rel(np64(o), o_ref) <= TOL_O["bf16"]
+    assert fro_rel(np64(S), S_ref) <= TOL_S
+
+
 @pytest.mark.parametrize("T", [64, 129, 1000])
 def test_tensor_core_gdr2_matches_cuda_core_gdr2(T, monkeypatch):
     """bf16 d=128 runs on tcgen05; the fp32 CUDA-core kernel
@@ -84,11 +120,14 @@ def test_tensor_core_gdr2_matches_cuda_core_gdr2(T, monkeypatch):
     assert fro_rel(np64(S_tc), S_ref) <= TOL_S
 
 
-def test_gdr2_strong_decay_takes_the_exact_path():
+@pytest.mark.parametrize("kernel", ["default", "tc1"])
+def test_gdr2_strong_decay_takes_the_exact_path(kernel, monkeypatch):
     """Channels that decay by e^-3 per token fall by e^-192 over a chunk, past
     what K/E can hold in a bf16 operand; those chunks evaluate A and P term
     by term.  Half the heads decay strongly in half the channels; all must
-    still match the oracle."""
+    still match the oracle, on the two-SM kernel and the single-CTA one."""
+    if kernel != "default":
+        monkeypatch.setenv("GDR2_FWD_KERNEL", kernel)
     x = synth.gdr2_inputs(1, 200, 4, 128, 128, "bf16", seed=77, s0_std=0.02)
     la = x["log_alpha"].clone()
     la[:, :, :2, :64] = -3.0
@@ -135,7 +174,7 @@ def test_gdr2_null_state_and_no_final_state():
     assert max_rel(np64(o), o_ref) <= TOL_O["bf16"]
 
 
-@pytest.mark.parametrize("kernel", ["default", "simt"])
+@pytest.mark.parametrize("kernel", ["default", "tc1", "simt"])
 def test_gdr2_negative_eigenvalue_erase_gate(kernel, monkeypatch):
     """Erase gate b in (0, 2) (the negative-eigenvalue range): the erase
     factor's eigenvalue along k reaches -1, and over 1000 tokens both
