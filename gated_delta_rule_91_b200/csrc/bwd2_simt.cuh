@@ -247,8 +247,26 @@ gdr2_bwd_simt_kernel(int T, int H, int dv, const Tio *__restrict__ q, const Tio 
         const int n = min(kChunk, T - c0);
         const size_t tok0 = ((size_t)b * T + c0) * H + h;
         __syncthreads();
+        if (ch > 0) {  // the previous chunk's inputs -> L2 while this one is reversed
+            const size_t tp = tok0 - (size_t)kChunk * H;  // its first token-head
+            constexpr int kRowLines = (DK * 4 + 127) / 128, kRowLinesIo = (DK * (int)sizeof(Tio) + 127) / 128;
+            for (int idx = tid; idx < kChunk * (2 * kRowLines + 2 * kRowLinesIo + 1); idx += blockDim.x) {
+                const int r = idx % kChunk, w = idx / kChunk;
+                const size_t row = tp + (size_t)r * H;
+                if (w < kRowLines) sm100::prefetch_l2(log_alpha + row * DK + 32 * w);
+                else if (w < 2 * kRowLines) sm100::prefetch_l2(bgate + row * DK + 32 * (w - kRowLines));
+                else if (w < 2 * kRowLines + kRowLinesIo)
+                    sm100::prefetch_l2(k + row * DK + (128 / sizeof(Tio)) * (w - 2 * kRowLines));
+                else if (w < 2 * kRowLines + 2 * kRowLinesIo)
+                    sm100::prefetch_l2(q + row * DK + (128 / sizeof(Tio)) * (w - 2 * kRowLines - kRowLinesIo));
+                else sm100::prefetch_l2(dO + row * dv + vcol0);
+            }
+            const float *sp = S_chunks + (((size_t)bh * nchunks + ch - 1) * dv + vcol0) * DK;
+            for (int l = tid; l < kBwd2Dvs * DK / 32; l += blockDim.x) sm100::prefetch_l2(sp + 32 * l);
+        }
         // ---- gates: G (per-channel cumulative log decay), E_C; K, Q, B, dO, S
         if (tid == 0) *s_flag = 0;
+#pragma unroll 8
         for (int idx = tid; idx < kChunk * DK; idx += blockDim.x) {
             const int r = idx / DK, j = idx % DK;
             const size_t off = (tok0 + (size_t)r * H) * DK + j;
