@@ -36,6 +36,7 @@
 #include "fwd2_tc.cuh"
 #include "fwd2_tc2.cuh"
 #include "bwd2_tc.cuh"
+#include "bwd2_ds.cuh"
 #include <type_traits>
 
 namespace gdr {
@@ -214,7 +215,7 @@ gdr2_bwd_simt_kernel(int T, int H, int dv, const Tio *__restrict__ q, const Tio 
                      float *__restrict__ dw_out, float *__restrict__ dS0, float *__restrict__ part_kb,
                      float *__restrict__ part_qe, float *__restrict__ part_ki, float *__restrict__ part_ec,
                      float *__restrict__ part_x, int *__restrict__ exact_flags, float *__restrict__ dAP,
-                     const float *__restrict__ TP) {
+                     const float *__restrict__ TP, const float *__restrict__ D_chunks) {
     using L = Bwd2Layout<DK>;
     constexpr int NB = DK / 16;
     extern __shared__ float smem[];
@@ -235,19 +236,29 @@ gdr2_bwd_simt_kernel(int T, int H, int dv, const Tio *__restrict__ q, const Tio 
     const size_t BTH = (size_t)gridDim.x / nslice * T;  // B*H*T token-heads
     const size_t pslice = (size_t)slice * BTH;
 
-    for (int idx = tid; idx < kBwd2Dvs * DK; idx += blockDim.x) {
-        const int r = idx / DK, c = idx % DK;
-        sD[r * L::LDK + c] = dS_T ? dS_T[((size_t)bh * dv + vcol0 + r) * DK + c] : 0.f;
-    }
+    // With D_chunks (every chunk's exit-state gradient, from the tensor-core dS
+    // pass) the CTA reverses the one chunk blockIdx.y; otherwise it carries D
+    // through all chunks, last to first.
+    const bool chunk_par = D_chunks != nullptr;
+    if (!chunk_par)
+        for (int idx = tid; idx < kBwd2Dvs * DK; idx += blockDim.x) {
+            const int r = idx / DK, c = idx % DK;
+            sD[r * L::LDK + c] = dS_T ? dS_T[((size_t)bh * dv + vcol0 + r) * DK + c] : 0.f;
+        }
     if (tid < kChunk) sOne[tid] = 1.f;
+    const int ch_first = chunk_par ? (int)blockIdx.y : nchunks - 1, ch_last = chunk_par ? (int)blockIdx.y : 0;
 
 #pragma unroll 1
-    for (int ch = nchunks - 1; ch >= 0; --ch) {
+    for (int ch = ch_first; ch >= ch_last; --ch) {
         const int c0 = ch * kChunk;
         const int n = min(kChunk, T - c0);
         const size_t tok0 = ((size_t)b * T + c0) * H + h;
         __syncthreads();
-        if (ch > 0) {  // the previous chunk's inputs -> L2 while this one is reversed
+        if (chunk_par) {
+            const float *src = D_chunks + (((size_t)bh * nchunks + ch) * dv + vcol0) * DK;
+            for (int idx = tid; idx < kBwd2Dvs * DK; idx += blockDim.x)
+                sD[(idx / DK) * L::LDK + idx % DK] = src[idx];
+        } else if (ch > 0) {  // the previous chunk's inputs -> L2 while this one is reversed
             const size_t tp = tok0 - (size_t)kChunk * H;  // its first token-head
             constexpr int kRowLines = (DK * 4 + 127) / 128, kRowLinesIo = (DK * (int)sizeof(Tio) + 127) / 128;
             for (int idx = tid; idx < kChunk * (2 * kRowLines + 2 * kRowLinesIo + 1); idx += blockDim.x) {
@@ -625,7 +636,7 @@ gdr2_bwd_simt_kernel(int T, int H, int dv, const Tio *__restrict__ q, const Tio 
         __syncthreads();
 
         // ---- P7: D <- D Diag(E_C) + dO^T QE - dR^T KBE (slice rows)
-        {
+        if (!chunk_par) {
             float dn[2][NB];
 #pragma unroll
             for (int a = 0; a < 2; ++a)
@@ -661,7 +672,7 @@ gdr2_bwd_simt_kernel(int T, int H, int dv, const Tio *__restrict__ q, const Tio 
         }
     }
     __syncthreads();
-    if (dS0) {
+    if (dS0 && !chunk_par) {
         for (int idx = tid; idx < kBwd2Dvs * DK; idx += blockDim.x) {
             const int r = idx / DK, c = idx % DK;
             dS0[((size_t)bh * dv + vcol0 + r) * DK + c] = sD[r * L::LDK + c];
@@ -737,9 +748,13 @@ gdr2_bwd_reduce_kernel(int T, int H, int nslice, const Tio *__restrict__ q, cons
 }
 
 struct Bwd2Workspace {
-    float *states, *part_kb, *part_qe, *part_ki, *part_ec, *part_x, *dAP, *TP;
+    float *states, *part_kb, *part_qe, *part_ki, *part_ec, *part_x, *dAP, *TP, *Dch;
     int *flags;
 };
+
+// bf16 with dk = dv = 128 recomputes on the cluster forward and carries dL/dS
+// on the tensor cores (bwd2_ds.cuh); the reverse pass then runs per chunk
+inline bool bwd2_uses_ds(int dk, int dv, bool bf16) { return bf16 && dk == 128 && dv == 128; }
 
 // bf16 with dk = 128 forms the chunk products on the tensor cores (bwd2_tc.cuh)
 inline bool bwd2_uses_tc(int dk, bool bf16) { return bf16 && dk == 128; }
@@ -753,7 +768,8 @@ inline size_t bwd2_workspace_bytes(int B, int T, int H, int dk, int dv, bool bf1
            al((size_t)B * H * nch * 4) +
            (bwd2_uses_tc(dk, bf16) ? al(ns * B * H * nch * 2 * kChunk * kChunk * 4) +
                                          al((size_t)B * H * nch * 2 * kChunk * kChunk * 4)
-                                   : 0);
+                                   : 0) +
+           (bwd2_uses_ds(dk, dv, bf16) ? al((size_t)B * H * nch * dv * dk * 4) : 0);
 }
 
 inline Bwd2Workspace bwd2_carve(void *ws, int B, int T, int H, int dk, int dv) {
@@ -780,6 +796,8 @@ inline Bwd2Workspace bwd2_carve(void *ws, int B, int T, int H, int dk, int dv) {
     w.dAP = reinterpret_cast<float *>(p);  // these two only on the tensor-core path
     p += al(ns * B * H * nch * 2 * kChunk * kChunk * 4);
     w.TP = reinterpret_cast<float *>(p);
+    p += al((size_t)B * H * nch * 2 * kChunk * kChunk * 4);
+    w.Dch = reinterpret_cast<float *>(p);  // only with the tensor-core dS pass
     return w;
 }
 
@@ -799,21 +817,29 @@ cudaError_t launch_bwd2_simt(int B, int T, int H, int dv, const void *q, const v
                           : launch_gdr2_simt<Tio, DK>(B, T, H, dv, q, k, v, la, bg, wg, S0, nullptr, nullptr, stream,
                                                       w.states);
     if (err != cudaSuccess) return err;
-    // 2) reverse chunk pass per (b, h, slice)
+    // 2) with the cluster recompute: every chunk's dL/dS and dS0 by the
+    //    tensor-core dS pass, so that step 3 runs per chunk
+    if (tc_fwd) {
+        err = launch_bwd2_ds(B, T, H, q, k, la, bg, dO, dS_T, dS0, w.Dch, stream);
+        if (err != cudaSuccess) return err;
+    }
+    // 3) reverse chunk pass per (b, h, slice), and per chunk with step 2
     const bool tc = bwd2_uses_tc(DK, std::is_same<Tio, __nv_bfloat16>::value);
     using L = Bwd2Layout<DK>;
     auto kern = gdr2_bwd_simt_kernel<Tio, DK>;
     err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kBytes);
     if (err != cudaSuccess) return err;
     const int nslice = dv / kBwd2Dvs;
-    kern<<<(unsigned)(B * H * nslice), kSimtThreads, L::kBytes, stream>>>(
+    const int nch_grid = tc_fwd ? (T + kChunk - 1) / kChunk : 1;
+    kern<<<dim3((unsigned)(B * H * nslice), (unsigned)nch_grid), kSimtThreads, L::kBytes, stream>>>(
         T, H, dv, static_cast<const Tio *>(q), static_cast<const Tio *>(k), static_cast<const Tio *>(v), la, bg,
-        wg, static_cast<const Tio *>(dO), dS_T, w.states, static_cast<Tio *>(dv_out), dw, dS0, w.part_kb,
-        w.part_qe, w.part_ki, w.part_ec, w.part_x, w.flags, tc ? w.dAP : nullptr, tc_fwd ? w.TP : nullptr);
+        wg, static_cast<const Tio *>(dO), dS_T, w.states, static_cast<Tio *>(dv_out), dw, tc_fwd ? nullptr : dS0,
+        w.part_kb, w.part_qe, w.part_ki, w.part_ec, w.part_x, w.flags, tc ? w.dAP : nullptr,
+        tc_fwd ? w.TP : nullptr, tc_fwd ? w.Dch : nullptr);
     g_launches.fetch_add(1, std::memory_order_relaxed);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
-    // 3) sum the slices (and, on the tensor cores, form the products with dA
+    // 4) sum the slices (and, on the tensor cores, form the products with dA
     //    and dP), chain rule through the gates, dlog alpha by reverse prefix sums
     const int nch = (T + kChunk - 1) / kChunk;
     if (tc) {

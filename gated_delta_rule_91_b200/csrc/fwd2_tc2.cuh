@@ -94,15 +94,17 @@ constexpr uint32_t kG2cBarKq = 0, kG2cBarLa = 2, kG2cBarEmpty = 4, kG2cBarLanded
 constexpr int kG2cScan0 = 256, kG2cScanThreads = 256, kG2cLoader = 32;
 
 // ------------------------------------------------------------------ prep CTA --
-// Per chunk n in staging slot s = n % 2: the raw K/Q tiles and b land in the
-// slot (one TMA barrier per slot, issued one chunk ahead once the copy of
-// chunk n-2 out of the slot has landed); log alpha lands in its own buffer
-// during the previous chunk and is scanned there while that chunk's inverse
+// Per step n in staging slot s = n % 2: the raw K/Q tiles and b land in the
+// slot (one TMA barrier per slot, issued one step ahead once the copy of
+// step n-2 out of the slot has landed); log alpha lands in its own buffer
+// during the previous step and is scanned there while that step's inverse
 // runs.  k, q and b are also read from global memory by the exact path.
+// Step n works on chunk n, or with `reverse` on chunk nch-1-n (the
+// backward's dS pass); slots, buffers and parities follow the step.
 __device__ __forceinline__ void g2c_prep(uint8_t *sm, const CUtensorMap *tm_q, const CUtensorMap *tm_k,
                                          const CUtensorMap *tm_la, const CUtensorMap *tm_bg, int T, int H, int b,
                                          int h, const __nv_bfloat16 *kg, const __nv_bfloat16 *qg,
-                                         const float *bgate, float *TP_chunks) {
+                                         const float *bgate, float *TP_chunks, bool reverse = false) {
     using L = G2cLayout;
     using namespace sm100;
     constexpr int D = 128;
@@ -125,6 +127,7 @@ __device__ __forceinline__ void g2c_prep(uint8_t *sm, const CUtensorMap *tm_q, c
     float *sg = reinterpret_cast<float *>(sm + L::P_LA);
     float *sA = reinterpret_cast<float *>(sm + L::P_A), *sT = reinterpret_cast<float *>(sm + L::P_T);
     auto ec_of = [&](int c) { return reinterpret_cast<float *>(sm + L::P_EC + (c & 3) * L::H_EC); };
+    auto chunk_of = [&](int n) { return reverse ? nch - 1 - n : n; };
     const uint32_t sbase = smem_u32(sm);
 
     if (tid == 0) {
@@ -151,24 +154,24 @@ __device__ __forceinline__ void g2c_prep(uint8_t *sm, const CUtensorMap *tm_q, c
 
     // raw K into the slot's K*exp(G_C - G) tile, raw Q into its Q*E rows, b
     // rows 16p .. 16p + 15 into piece p (K*B*E's two halves, T, P)
-    auto issue_kq = [&](int c) {
-        const int sl = c & 1;
+    auto issue_kq = [&](int n) {  // step n: slot n % 2, chunk chunk_of(n)
+        const int sl = n & 1, t0 = chunk_of(n) * kChunk;
         uint8_t *st = sm + L::P_STG + sl * L::H_TILES;
         uint64_t *bar = &tma_kq[sl];
         mbar_expect_tx(bar, 65536);
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
-            tma_load_4d(st + L::H_KTL + half * 8192, tm_k, bar, half * 64, h, c * kChunk, b);
-            tma_load_4d(st + L::H_KQE + half * 16384 + 8192, tm_q, bar, half * 64, h, c * kChunk, b);
+            tma_load_4d(st + L::H_KTL + half * 8192, tm_k, bar, half * 64, h, t0, b);
+            tma_load_4d(st + L::H_KQE + half * 16384 + 8192, tm_q, bar, half * 64, h, t0, b);
         }
         const uint32_t piece[4] = {L::H_KQE, L::H_KQE + 16384, L::H_TB, L::H_PB};
 #pragma unroll
-        for (int p = 0; p < 4; ++p) tma_load_4d(st + piece[p], tm_bg, bar, 0, h, c * kChunk + 16 * p, b);
+        for (int p = 0; p < 4; ++p) tma_load_4d(st + piece[p], tm_bg, bar, 0, h, t0 + 16 * p, b);
         kq_issued[sl] = kq_issued[sl] + 1;
     };
-    auto issue_la = [&](int c) {
+    auto issue_la = [&](int n) {
         mbar_expect_tx(tma_la, 32768);
-        tma_load_4d(sm + L::P_LA, tm_la, tma_la, 0, h, c * kChunk, b);
+        tma_load_4d(sm + L::P_LA, tm_la, tma_la, 0, h, chunk_of(n) * kChunk, b);
         *la_issued = *la_issued + 1;
     };
     // log alpha of chunk c (landed in P_LA) -> G in place, E_C, exact-path
@@ -211,8 +214,8 @@ __device__ __forceinline__ void g2c_prep(uint8_t *sm, const CUtensorMap *tm_q, c
 
 #pragma unroll 1
     for (int n = 0; n < nch; ++n) {
-        const int s = n & 1;
-        const int t0 = n * kChunk, nv = min(kChunk, T - t0);
+        const int s = n & 1, cn = chunk_of(n);
+        const int t0 = cn * kChunk, nv = min(kChunk, T - t0);
         const size_t tok0 = ((size_t)b * T + t0) * H + h;
         uint8_t *stg = sm + L::P_STG + s * L::H_TILES;
         const float *ec = ec_of(n);
@@ -305,7 +308,7 @@ __device__ __forceinline__ void g2c_prep(uint8_t *sm, const CUtensorMap *tm_q, c
         tc_after_sync();
         // K/E has been read: T's tile is cleared (the inverse writes only its lower triangle)
         *reinterpret_cast<uint4 *>(stg + L::H_TB + tid * 16) = make_uint4(0, 0, 0, 0);
-        float *tp = TP_chunks ? TP_chunks + ((size_t)bh * nch + n) * 2 * kChunk * kChunk : nullptr;
+        float *tp = TP_chunks ? TP_chunks + ((size_t)bh * nch + cn) * 2 * kChunk * kChunk : nullptr;
         if (!exact) {
             float v[16];
             tmem_ld16(tl + wc * 16, v);
