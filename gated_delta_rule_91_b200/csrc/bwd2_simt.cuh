@@ -37,17 +37,12 @@
 #include "fwd2_tc2.cuh"
 #include "bwd2_tc.cuh"
 #include "bwd2_ds.cuh"
+#include "bwd2_grad_tc.cuh"
 #include <type_traits>
 
 namespace gdr {
 
 constexpr int kBwd2Dvs = 32;  // state rows per CTA
-// How a chunk is differentiated, from its largest per-channel decay span
-// -G_C: up to kBwd2TcSpan the products with dA and dP run on the tensor cores
-// (bf16 operands K/E, K*B*E, Q*E span e^span there), up to 80 in fp32 in the
-// reverse pass, beyond that token by token.
-constexpr float kBwd2TcSpan = 20.f;
-enum : int { kChunkTc = 0, kChunkExact = 1, kChunkF32 = 2 };
 
 template <int DK>
 struct Bwd2Layout {
@@ -215,7 +210,7 @@ gdr2_bwd_simt_kernel(int T, int H, int dv, const Tio *__restrict__ q, const Tio 
                      float *__restrict__ dw_out, float *__restrict__ dS0, float *__restrict__ part_kb,
                      float *__restrict__ part_qe, float *__restrict__ part_ki, float *__restrict__ part_ec,
                      float *__restrict__ part_x, int *__restrict__ exact_flags, float *__restrict__ dAP,
-                     const float *__restrict__ TP, const float *__restrict__ D_chunks) {
+                     const float *__restrict__ TP, const float *__restrict__ D_chunks, int tc_took) {
     using L = Bwd2Layout<DK>;
     constexpr int NB = DK / 16;
     extern __shared__ float smem[];
@@ -240,6 +235,8 @@ gdr2_bwd_simt_kernel(int T, int H, int dv, const Tio *__restrict__ q, const Tio 
     // pass) the CTA reverses the one chunk blockIdx.y; otherwise it carries D
     // through all chunks, last to first.
     const bool chunk_par = D_chunks != nullptr;
+    // a chunk the tensor-core gradient kernel took (mode 0) is done
+    if (chunk_par && tc_took && exact_flags[(size_t)bh * nchunks + blockIdx.y] == kChunkTc) return;
     if (!chunk_par)
         for (int idx = tid; idx < kBwd2Dvs * DK; idx += blockDim.x) {
             const int r = idx / DK, c = idx % DK;
@@ -309,8 +306,11 @@ gdr2_bwd_simt_kernel(int T, int H, int dv, const Tio *__restrict__ q, const Tio 
         }
         __syncthreads();
         // s_flag: 0 moderate decay, 1 past the tensor-core span, 2 past e^80
-        const int mode = *s_flag == 2 ? kChunkExact : (*s_flag == 1 || !dAP) ? kChunkF32 : kChunkTc;
-        if (slice == 0 && tid == 0) exact_flags[(size_t)bh * nchunks + ch] = mode;
+        // after the tensor-core gradient kernel, its mode stands (the same
+        // thresholds, but the span summed in another order could round across one)
+        const int mode = tc_took ? exact_flags[(size_t)bh * nchunks + ch]
+                                 : *s_flag == 2 ? kChunkExact : (*s_flag == 1 || !dAP) ? kChunkF32 : kChunkTc;
+        if (slice == 0 && tid == 0 && !tc_took) exact_flags[(size_t)bh * nchunks + ch] = mode;
         if (mode == kChunkExact) {  // a channel decays past e^80 inside the chunk: token by token
             gdr2_chunk_reverse_exact<Tio, DK>(n, tok0, H, dv, vcol0, q, k, v, log_alpha, bgate, wgate, dO, smem,
                                               smem + L::odO, sS, sD, dv_out, dw_out, part_qe, part_kb, part_ki,
@@ -823,7 +823,14 @@ cudaError_t launch_bwd2_simt(int B, int T, int H, int dv, const void *q, const v
         err = launch_bwd2_ds(B, T, H, q, k, la, bg, dO, dS_T, dS0, w.Dch, stream);
         if (err != cudaSuccess) return err;
     }
-    // 3) reverse chunk pass per (b, h, slice), and per chunk with step 2
+    // 3) the chunks within the tensor-core span on the tensor cores (all value
+    //    rows at once); the others by the reverse pass per (b, h, slice), per
+    //    chunk with step 2
+    if (tc_fwd) {
+        err = launch_bwd2_grad_tc(B, T, H, k, v, dO, la, bg, wg, w.states, w.Dch, w.TP, dv_out, dw, w.part_kb,
+                                  w.part_qe, w.part_ki, w.part_ec, w.flags, w.dAP, stream);
+        if (err != cudaSuccess) return err;
+    }
     const bool tc = bwd2_uses_tc(DK, std::is_same<Tio, __nv_bfloat16>::value);
     using L = Bwd2Layout<DK>;
     auto kern = gdr2_bwd_simt_kernel<Tio, DK>;
@@ -835,7 +842,7 @@ cudaError_t launch_bwd2_simt(int B, int T, int H, int dv, const void *q, const v
         T, H, dv, static_cast<const Tio *>(q), static_cast<const Tio *>(k), static_cast<const Tio *>(v), la, bg,
         wg, static_cast<const Tio *>(dO), dS_T, w.states, static_cast<Tio *>(dv_out), dw, tc_fwd ? nullptr : dS0,
         w.part_kb, w.part_qe, w.part_ki, w.part_ec, w.part_x, w.flags, tc ? w.dAP : nullptr,
-        tc_fwd ? w.TP : nullptr, tc_fwd ? w.Dch : nullptr);
+        tc_fwd ? w.TP : nullptr, tc_fwd ? w.Dch : nullptr, tc_fwd ? 1 : 0);
     g_launches.fetch_add(1, std::memory_order_relaxed);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
@@ -849,7 +856,7 @@ cudaError_t launch_bwd2_simt(int B, int T, int H, int dv, const void *q, const v
         ck<<<(unsigned)(B * H * nch), kBwd2TcThreads, Bwd2TcSmem::kAlloc, stream>>>(
             T, H, static_cast<const Tio *>(q), static_cast<const Tio *>(k), la, bg, w.part_kb, w.part_qe,
             w.part_ki, w.part_ec, w.part_x, w.flags, w.dAP, static_cast<Tio *>(dq), static_cast<Tio *>(dk_out), dla,
-            db, (size_t)B * T * H);
+            db, (size_t)B * T * H, tc_fwd ? 1 : nslice);
         g_launches.fetch_add(1, std::memory_order_relaxed);
         return cudaGetLastError();
     }
