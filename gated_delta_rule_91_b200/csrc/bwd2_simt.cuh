@@ -823,12 +823,12 @@ cudaError_t launch_bwd2_simt(int B, int T, int H, int dv, const void *q, const v
         err = launch_bwd2_ds(B, T, H, q, k, la, bg, dO, dS_T, dS0, w.Dch, stream);
         if (err != cudaSuccess) return err;
     }
-    // 3) the chunks within the tensor-core span on the tensor cores (all value
-    //    rows at once); the others by the reverse pass per (b, h, slice), per
-    //    chunk with step 2
+    // 3) the chunks within the tensor-core span on the tensor cores, every
+    //    gradient at once; the others by the reverse pass per (b, h, slice),
+    //    per chunk with step 2, and the chunk kernel
     if (tc_fwd) {
-        err = launch_bwd2_grad_tc(B, T, H, k, v, dO, la, bg, wg, w.states, w.Dch, w.TP, dv_out, dw, w.part_kb,
-                                  w.part_qe, w.part_ki, w.part_ec, w.flags, w.dAP, stream);
+        err = launch_bwd2_grad_tc(B, T, H, q, k, v, dO, la, bg, wg, w.states, w.Dch, w.TP, dq, dk_out, dv_out, dla,
+                                  db, dw, w.flags, stream);
         if (err != cudaSuccess) return err;
     }
     const bool tc = bwd2_uses_tc(DK, std::is_same<Tio, __nv_bfloat16>::value);
@@ -856,7 +856,7 @@ cudaError_t launch_bwd2_simt(int B, int T, int H, int dv, const void *q, const v
         ck<<<(unsigned)(B * H * nch), kBwd2TcThreads, Bwd2TcSmem::kAlloc, stream>>>(
             T, H, static_cast<const Tio *>(q), static_cast<const Tio *>(k), la, bg, w.part_kb, w.part_qe,
             w.part_ki, w.part_ec, w.part_x, w.flags, w.dAP, static_cast<Tio *>(dq), static_cast<Tio *>(dk_out), dla,
-            db, (size_t)B * T * H, tc_fwd ? 1 : nslice);
+            db, (size_t)B * T * H, tc_fwd ? 1 : 0);
         g_launches.fetch_add(1, std::memory_order_relaxed);
         return cudaGetLastError();
     }

@@ -67,7 +67,7 @@ gdr2_bwd_chunk_tc_kernel(int T, int H, const Tio *__restrict__ q, const Tio *__r
                          const float *__restrict__ part_ki, const float *__restrict__ part_ec,
                          const float *__restrict__ part_x, const int *__restrict__ exact_flags,
                          const float *__restrict__ dAP, Tio *__restrict__ dq, Tio *__restrict__ dk,
-                         float *__restrict__ dlog_alpha, float *__restrict__ db, size_t BTH, int ns_tc) {
+                         float *__restrict__ dlog_alpha, float *__restrict__ db, size_t BTH, int tc_done) {
     using L = Bwd2TcSmem;
     using namespace sm100;
     constexpr int DK = 128, RQ = kChunk / 4;  // tokens per quarter
@@ -84,6 +84,7 @@ gdr2_bwd_chunk_tc_kernel(int T, int H, const Tio *__restrict__ q, const Tio *__r
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int j = (warp & 3) * 32 + lane, rq = warp >> 2, r0 = rq * RQ;
     const int mode = exact_flags[(size_t)bh * nchunks + ch];
+    if (mode == kChunkTc && tc_done) return;  // the tensor-core gradient kernel finished this chunk
 
     if (mode == 1) {
         // token-by-token partials: S_t^T do (part_qe), X = P^T gk (part_ki),
@@ -109,9 +110,6 @@ gdr2_bwd_chunk_tc_kernel(int T, int H, const Tio *__restrict__ q, const Tio *__r
         return;
     }
     const bool use_mma = mode == 0;  // 2: the reverse pass formed the products in fp32 (strong decay)
-    // slices holding this chunk's partials: ns_tc for a mode-0 chunk (1 when
-    // the tensor-core gradient kernel wrote the full sums into slice 0)
-    const int ns = use_mma ? ns_tc : NS;
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + L::oBar);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar + 1);
     float *scan = reinterpret_cast<float *>(sm + L::oScan);  // [4][DK]
@@ -165,7 +163,6 @@ gdr2_bwd_chunk_tc_kernel(int T, int H, const Tio *__restrict__ q, const Tio *__r
             float4 acc = *reinterpret_cast<const float4 *>(src + idx);
 #pragma unroll
             for (int s = 1; s < NS; ++s) {
-                if (s >= ns) break;
                 const float4 x = *reinterpret_cast<const float4 *>(src + (size_t)s * stride + idx);
                 acc.x += x.x; acc.y += x.y; acc.z += x.z; acc.w += x.w;
             }
@@ -231,7 +228,6 @@ gdr2_bwd_chunk_tc_kernel(int T, int H, const Tio *__restrict__ q, const Tio *__r
             g += log_alpha[off];
 #pragma unroll
             for (int s = 0; s < NS; ++s) {
-                if (s >= ns) break;
                 skb += part_kb[(size_t)s * BTH * DK + off];
                 sqe += part_qe[(size_t)s * BTH * DK + off];
                 ski += part_ki[(size_t)s * BTH * DK + off];
@@ -252,8 +248,7 @@ gdr2_bwd_chunk_tc_kernel(int T, int H, const Tio *__restrict__ q, const Tio *__r
         __syncthreads();
         float dec = 0.f;
 #pragma unroll
-        for (int s = 0; s < NS; ++s)
-            if (s < ns) dec += part_ec[(((size_t)s * nbh + bh) * nchunks + ch) * DK + j];
+        for (int s = 0; s < NS; ++s) dec += part_ec[(((size_t)s * nbh + bh) * nchunks + ch) * DK + j];
         float suffix = expf(gC) * dec;  // dG_C, carried by the chunk's last token
 #pragma unroll
         for (int u = 3; u > rq; --u) suffix += scan[u * DK + j];
