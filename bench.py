@@ -612,7 +612,7 @@ def secondary(pk):
         out["gdn2_bwd"] = {"workload": "B=4 T=4096 H=16 d=128 bf16", "ms": bms,
                            "mtok_per_s": w.B * w.T / (bms * 1e-3) / 1e6,
                            "tc_frac": bwd_flops(w.B, w.T, w.H, w.dk) / (bms * 1e-3) / (pk["bf16_tflops"] * 1e12),
-                           "kernels": "cluster recompute; tensor-core dS pass (dL/dS in TMEM); CUDA-core reverse per (slice of value rows, chunk); tensor-core chunk products and chain rule"}
+                           "kernels": "cluster recompute; tensor-core dS pass (dL/dS in TMEM); tensor-core per-chunk products, chain rule and dlog alpha suffix sums; CUDA-core paths only for chunks decaying past e^20"}
     except Exception as e:
         out["gdn2_fwd"] = {"unavailable": str(e).splitlines()[0][:200]}
     del d, x
