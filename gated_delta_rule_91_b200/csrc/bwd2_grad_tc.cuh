@@ -75,7 +75,7 @@ gdr2_bwd_grad_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
                         const float *__restrict__ TP, __nv_bfloat16 *__restrict__ dq_out,
                         __nv_bfloat16 *__restrict__ dk_out, __nv_bfloat16 *__restrict__ dv_out,
                         float *__restrict__ dla_out, float *__restrict__ db_out, float *__restrict__ dw_out,
-                        int *__restrict__ exact_flags) {
+                        int *__restrict__ exact_flags, int *__restrict__ todo, int *__restrict__ ntodo) {
     using L = G2gLayout;
     using namespace sm100;
     constexpr int DK = 128;
@@ -192,7 +192,10 @@ gdr2_bwd_grad_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
     }
     __syncthreads();
     const int mode = *code == 2 ? kChunkExact : *code == 1 ? kChunkF32 : kChunkTc;
-    if (tid == 0) exact_flags[tile] = mode;
+    if (tid == 0) {
+        exact_flags[tile] = mode;
+        if (mode != kChunkTc) todo[atomicAdd(ntodo, 1)] = (int)tile;  // left to the CUDA-core pass
+    }
     const bool work = mode == kChunkTc && !*abort_flag;
 
     if (work) {
@@ -467,13 +470,14 @@ gdr2_bwd_grad_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
 }
 
 // One CTA per (b, h, chunk): all gradients of the chunks it takes (mode 0);
-// the others get their mode in `flags` for the CUDA-core reverse pass and the
+// the others get their mode in `flags` and are appended to todo (*ntodo,
+// zeroed by the caller, counts them) for the CUDA-core reverse pass and the
 // chunk kernel.
 inline cudaError_t launch_bwd2_grad_tc(int B, int T, int H, const void *q, const void *k, const void *v,
                                        const void *dO, const float *la, const float *bgate, const float *wgate,
                                        const float *S_chunks, const float *D_chunks, const float *TP, void *dq,
                                        void *dk, void *dv, float *dla, float *db, float *dw, int *flags,
-                                       cudaStream_t stream) {
+                                       int *todo, int *ntodo, cudaStream_t stream) {
     CUtensorMap mk, mv, mdo, mla;
     if (!make_token_map(&mk, k, B, T, H, 128) || !make_token_map(&mv, v, B, T, H, 128) ||
         !make_token_map(&mdo, dO, B, T, H, 128) || !make_gate_map(&mla, la, B, T, H, 128))
@@ -485,7 +489,7 @@ inline cudaError_t launch_bwd2_grad_tc(int B, int T, int H, const void *q, const
     gdr2_bwd_grad_tc_kernel<<<(unsigned)(B * H * nch), kG2gThreads, G2gLayout::kAlloc, stream>>>(
         mk, mv, mdo, mla, T, H, static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
         bgate, wgate, S_chunks, D_chunks, TP, static_cast<__nv_bfloat16 *>(dq), static_cast<__nv_bfloat16 *>(dk),
-        static_cast<__nv_bfloat16 *>(dv), dla, db, dw, flags);
+        static_cast<__nv_bfloat16 *>(dv), dla, db, dw, flags, todo, ntodo);
     g_launches.fetch_add(1, std::memory_order_relaxed);
     return cudaGetLastError();
 }

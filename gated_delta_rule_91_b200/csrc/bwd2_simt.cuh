@@ -200,17 +200,19 @@ __device__ void gdr2_chunk_reverse_exact(int n, size_t tok0, int H, int dv, int 
     for (int jj = 0; jj < JW; ++jj) sD[row * LDK + j0 + jj] = d[jj];
 }
 
+// The reverse of one (b*H + h, slice of value rows) over its chunks, or over
+// the one chunk ch_sel when D_chunks (every chunk's exit-state gradient, from
+// the tensor-core dS pass) is given.
 template <typename Tio, int DK>
-__global__ void __launch_bounds__(kSimtThreads, 1)
-gdr2_bwd_simt_kernel(int T, int H, int dv, const Tio *__restrict__ q, const Tio *__restrict__ k,
-                     const Tio *__restrict__ v, const float *__restrict__ log_alpha,
-                     const float *__restrict__ bgate, const float *__restrict__ wgate,
-                     const Tio *__restrict__ dO, const float *__restrict__ dS_T,
-                     const float *__restrict__ S_chunks, Tio *__restrict__ dv_out,
-                     float *__restrict__ dw_out, float *__restrict__ dS0, float *__restrict__ part_kb,
-                     float *__restrict__ part_qe, float *__restrict__ part_ki, float *__restrict__ part_ec,
-                     float *__restrict__ part_x, int *__restrict__ exact_flags, float *__restrict__ dAP,
-                     const float *__restrict__ TP, const float *__restrict__ D_chunks, int tc_took) {
+__device__ __forceinline__ void gdr2_bwd_simt_body(
+    int T, int H, int dv, const Tio *__restrict__ q, const Tio *__restrict__ k, const Tio *__restrict__ v,
+    const float *__restrict__ log_alpha, const float *__restrict__ bgate, const float *__restrict__ wgate,
+    const Tio *__restrict__ dO, const float *__restrict__ dS_T, const float *__restrict__ S_chunks,
+    Tio *__restrict__ dv_out, float *__restrict__ dw_out, float *__restrict__ dS0, float *__restrict__ part_kb,
+    float *__restrict__ part_qe, float *__restrict__ part_ki, float *__restrict__ part_ec,
+    float *__restrict__ part_x, int *__restrict__ exact_flags, float *__restrict__ dAP,
+    const float *__restrict__ TP, const float *__restrict__ D_chunks, int tc_took, int bh, int slice, int ch_sel,
+    int BH) {
     using L = Bwd2Layout<DK>;
     constexpr int NB = DK / 16;
     extern __shared__ float smem[];
@@ -221,29 +223,21 @@ gdr2_bwd_simt_kernel(int T, int H, int dv, const Tio *__restrict__ q, const Tio 
     float *sEC = smem + L::oVec, *sOne = sEC + DK;
     int *s_flag = reinterpret_cast<int *>(sOne + kChunk);
 
-    const int nslice = dv / kBwd2Dvs;
-    const int slice = blockIdx.x % nslice;
-    const int bh = blockIdx.x / nslice;
     const int b = bh / H, h = bh % H;
     const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
     const int vcol0 = slice * kBwd2Dvs;
     const int nchunks = (T + kChunk - 1) / kChunk;
-    const size_t BTH = (size_t)gridDim.x / nslice * T;  // B*H*T token-heads
+    const size_t BTH = (size_t)BH * T;  // B*H*T token-heads
     const size_t pslice = (size_t)slice * BTH;
 
-    // With D_chunks (every chunk's exit-state gradient, from the tensor-core dS
-    // pass) the CTA reverses the one chunk blockIdx.y; otherwise it carries D
-    // through all chunks, last to first.
     const bool chunk_par = D_chunks != nullptr;
-    // a chunk the tensor-core gradient kernel took (mode 0) is done
-    if (chunk_par && tc_took && exact_flags[(size_t)bh * nchunks + blockIdx.y] == kChunkTc) return;
     if (!chunk_par)
         for (int idx = tid; idx < kBwd2Dvs * DK; idx += blockDim.x) {
             const int r = idx / DK, c = idx % DK;
             sD[r * L::LDK + c] = dS_T ? dS_T[((size_t)bh * dv + vcol0 + r) * DK + c] : 0.f;
         }
     if (tid < kChunk) sOne[tid] = 1.f;
-    const int ch_first = chunk_par ? (int)blockIdx.y : nchunks - 1, ch_last = chunk_par ? (int)blockIdx.y : 0;
+    const int ch_first = chunk_par ? ch_sel : nchunks - 1, ch_last = chunk_par ? ch_sel : 0;
 
 #pragma unroll 1
     for (int ch = ch_first; ch >= ch_last; --ch) {
@@ -680,6 +674,50 @@ gdr2_bwd_simt_kernel(int T, int H, int dv, const Tio *__restrict__ q, const Tio 
     }
 }
 
+// One CTA per (b*H + h, slice) walking all chunks, or per (b*H + h, slice,
+// chunk blockIdx.y) with D_chunks.
+template <typename Tio, int DK>
+__global__ void __launch_bounds__(kSimtThreads, 1)
+gdr2_bwd_simt_kernel(int T, int H, int dv, const Tio *__restrict__ q, const Tio *__restrict__ k,
+                     const Tio *__restrict__ v, const float *__restrict__ log_alpha,
+                     const float *__restrict__ bgate, const float *__restrict__ wgate,
+                     const Tio *__restrict__ dO, const float *__restrict__ dS_T,
+                     const float *__restrict__ S_chunks, Tio *__restrict__ dv_out,
+                     float *__restrict__ dw_out, float *__restrict__ dS0, float *__restrict__ part_kb,
+                     float *__restrict__ part_qe, float *__restrict__ part_ki, float *__restrict__ part_ec,
+                     float *__restrict__ part_x, int *__restrict__ exact_flags, float *__restrict__ dAP,
+                     const float *__restrict__ TP, const float *__restrict__ D_chunks) {
+    const int nslice = dv / kBwd2Dvs;
+    gdr2_bwd_simt_body<Tio, DK>(T, H, dv, q, k, v, log_alpha, bgate, wgate, dO, dS_T, S_chunks, dv_out, dw_out, dS0,
+                                part_kb, part_qe, part_ki, part_ec, part_x, exact_flags, dAP, TP, D_chunks, 0,
+                                (int)(blockIdx.x / nslice), (int)(blockIdx.x % nslice), (int)blockIdx.y,
+                                (int)(gridDim.x / nslice));
+}
+
+// The chunks the tensor-core gradient kernel left (todo[0 .. *ntodo), each
+// b*H*nchunks + chunk): CTA (slice, g) takes items g, g + gridDim.y, ...
+template <typename Tio, int DK>
+__global__ void __launch_bounds__(kSimtThreads, 1)
+gdr2_bwd_simt_list_kernel(int T, int H, int dv, const Tio *__restrict__ q, const Tio *__restrict__ k,
+                          const Tio *__restrict__ v, const float *__restrict__ log_alpha,
+                          const float *__restrict__ bgate, const float *__restrict__ wgate,
+                          const Tio *__restrict__ dO, const float *__restrict__ S_chunks,
+                          Tio *__restrict__ dv_out, float *__restrict__ dw_out, float *__restrict__ part_kb,
+                          float *__restrict__ part_qe, float *__restrict__ part_ki, float *__restrict__ part_ec,
+                          float *__restrict__ part_x, int *__restrict__ exact_flags, float *__restrict__ dAP,
+                          const float *__restrict__ D_chunks, const int *__restrict__ todo,
+                          const int *__restrict__ ntodo, int BH) {
+    const int nch = (T + kChunk - 1) / kChunk, n_items = *ntodo;
+#pragma unroll 1
+    for (int it = blockIdx.y; it < n_items; it += gridDim.y) {
+        __syncthreads();  // the previous item is done with shared memory
+        const int tile = todo[it];
+        gdr2_bwd_simt_body<Tio, DK>(T, H, dv, q, k, v, log_alpha, bgate, wgate, dO, nullptr, S_chunks, dv_out,
+                                    dw_out, nullptr, part_kb, part_qe, part_ki, part_ec, part_x, exact_flags, dAP,
+                                    nullptr, D_chunks, 1, tile / nch, (int)blockIdx.x, tile % nch, BH);
+    }
+}
+
 // Sum the per-slice partials in a fixed order and apply the per-element chain
 // rule; dlog alpha = the reverse prefix sum of dG per channel inside each
 // chunk.  One CTA per (b, h, chunk), one thread per key channel.
@@ -749,7 +787,7 @@ gdr2_bwd_reduce_kernel(int T, int H, int nslice, const Tio *__restrict__ q, cons
 
 struct Bwd2Workspace {
     float *states, *part_kb, *part_qe, *part_ki, *part_ec, *part_x, *dAP, *TP, *Dch;
-    int *flags;
+    int *flags, *todo, *ntodo;
 };
 
 // bf16 with dk = dv = 128 recomputes on the cluster forward and carries dL/dS
@@ -765,7 +803,7 @@ inline size_t bwd2_workspace_bytes(int B, int T, int H, int dk, int dv, bool bf1
     const size_t bth = (size_t)B * T * H;
     auto al = [](size_t x) { return (x + 255) / 256 * 256; };
     return al((size_t)B * H * nch * dv * dk * 4) + 4 * al(ns * bth * dk * 4) + al(ns * B * H * nch * dk * 4) +
-           al((size_t)B * H * nch * 4) +
+           al((2 * (size_t)B * H * nch + 1) * 4) +
            (bwd2_uses_tc(dk, bf16) ? al(ns * B * H * nch * 2 * kChunk * kChunk * 4) +
                                          al((size_t)B * H * nch * 2 * kChunk * kChunk * 4)
                                    : 0) +
@@ -791,8 +829,10 @@ inline Bwd2Workspace bwd2_carve(void *ws, int B, int T, int H, int dk, int dv) {
     p += al(ns * B * H * nch * dk * 4);
     w.part_x = reinterpret_cast<float *>(p);
     p += al(ns * bth * dk * 4);
-    w.flags = reinterpret_cast<int *>(p);
-    p += al((size_t)B * H * nch * 4);
+    w.flags = reinterpret_cast<int *>(p);  // then the list of chunks left to the CUDA cores and its length
+    w.todo = w.flags + (size_t)B * H * nch;
+    w.ntodo = w.todo + (size_t)B * H * nch;
+    p += al((2 * (size_t)B * H * nch + 1) * 4);
     w.dAP = reinterpret_cast<float *>(p);  // these two only on the tensor-core path
     p += al(ns * B * H * nch * 2 * kChunk * kChunk * 4);
     w.TP = reinterpret_cast<float *>(p);
@@ -823,32 +863,55 @@ cudaError_t launch_bwd2_simt(int B, int T, int H, int dv, const void *q, const v
         err = launch_bwd2_ds(B, T, H, q, k, la, bg, dO, dS_T, dS0, w.Dch, stream);
         if (err != cudaSuccess) return err;
     }
-    // 3) the chunks within the tensor-core span on the tensor cores, every
-    //    gradient at once; the others by the reverse pass per (b, h, slice),
-    //    per chunk with step 2, and the chunk kernel
-    if (tc_fwd) {
-        err = launch_bwd2_grad_tc(B, T, H, q, k, v, dO, la, bg, wg, w.states, w.Dch, w.TP, dq, dk_out, dv_out, dla,
-                                  db, dw, w.flags, stream);
-        if (err != cudaSuccess) return err;
-    }
     const bool tc = bwd2_uses_tc(DK, std::is_same<Tio, __nv_bfloat16>::value);
     using L = Bwd2Layout<DK>;
+    const int nslice = dv / kBwd2Dvs;
+    const int nch = (T + kChunk - 1) / kChunk;
+    if (tc_fwd) {
+        // 3) every chunk within the tensor-core span: all gradients on the
+        //    tensor cores; the others are listed for steps 4 and 5
+        err = cudaMemsetAsync(w.ntodo, 0, sizeof(int), stream);
+        if (err == cudaSuccess)
+            err = launch_bwd2_grad_tc(B, T, H, q, k, v, dO, la, bg, wg, w.states, w.Dch, w.TP, dq, dk_out, dv_out,
+                                      dla, db, dw, w.flags, w.todo, w.ntodo, stream);
+        if (err != cudaSuccess) return err;
+        // 4) the listed chunks: the reverse pass per (slice, chunk) from D_chunks
+        //    (a grid of one wave; with nothing listed every CTA exits at once)
+        auto lk = gdr2_bwd_simt_list_kernel<Tio, DK>;
+        err = cudaFuncSetAttribute(lk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kBytes);
+        if (err != cudaSuccess) return err;
+        const int gy = min(B * H * nch, 148);
+        lk<<<dim3((unsigned)nslice, (unsigned)gy), kSimtThreads, L::kBytes, stream>>>(
+            T, H, dv, static_cast<const Tio *>(q), static_cast<const Tio *>(k), static_cast<const Tio *>(v), la, bg,
+            wg, static_cast<const Tio *>(dO), w.states, static_cast<Tio *>(dv_out), dw, w.part_kb, w.part_qe,
+            w.part_ki, w.part_ec, w.part_x, w.flags, w.dAP, w.Dch, w.todo, w.ntodo, B * H);
+        g_launches.fetch_add(1, std::memory_order_relaxed);
+        err = cudaGetLastError();
+        if (err != cudaSuccess) return err;
+        // 5) their slices summed, chain rule, dlog alpha
+        auto ck = nslice == 4 ? gdr2_bwd_chunk_tc_list_kernel<Tio, 4> : gdr2_bwd_chunk_tc_list_kernel<Tio, 2>;
+        err = cudaFuncSetAttribute(ck, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Bwd2TcSmem::kAlloc);
+        if (err != cudaSuccess) return err;
+        ck<<<(unsigned)min(B * H * nch, 148), kBwd2TcThreads, Bwd2TcSmem::kAlloc, stream>>>(
+            T, H, static_cast<const Tio *>(q), static_cast<const Tio *>(k), la, bg, w.part_kb, w.part_qe,
+            w.part_ki, w.part_ec, w.part_x, w.flags, w.dAP, static_cast<Tio *>(dq), static_cast<Tio *>(dk_out), dla,
+            db, (size_t)B * T * H, w.todo, w.ntodo);
+        g_launches.fetch_add(1, std::memory_order_relaxed);
+        return cudaGetLastError();
+    }
+    // 3) reverse chunk pass per (b, h, slice)
     auto kern = gdr2_bwd_simt_kernel<Tio, DK>;
     err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kBytes);
     if (err != cudaSuccess) return err;
-    const int nslice = dv / kBwd2Dvs;
-    const int nch_grid = tc_fwd ? (T + kChunk - 1) / kChunk : 1;
-    kern<<<dim3((unsigned)(B * H * nslice), (unsigned)nch_grid), kSimtThreads, L::kBytes, stream>>>(
+    kern<<<dim3((unsigned)(B * H * nslice), 1u), kSimtThreads, L::kBytes, stream>>>(
         T, H, dv, static_cast<const Tio *>(q), static_cast<const Tio *>(k), static_cast<const Tio *>(v), la, bg,
-        wg, static_cast<const Tio *>(dO), dS_T, w.states, static_cast<Tio *>(dv_out), dw, tc_fwd ? nullptr : dS0,
-        w.part_kb, w.part_qe, w.part_ki, w.part_ec, w.part_x, w.flags, tc ? w.dAP : nullptr,
-        tc_fwd ? w.TP : nullptr, tc_fwd ? w.Dch : nullptr, tc_fwd ? 1 : 0);
+        wg, static_cast<const Tio *>(dO), dS_T, w.states, static_cast<Tio *>(dv_out), dw, dS0, w.part_kb,
+        w.part_qe, w.part_ki, w.part_ec, w.part_x, w.flags, tc ? w.dAP : nullptr, nullptr, nullptr);
     g_launches.fetch_add(1, std::memory_order_relaxed);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
     // 4) sum the slices (and, on the tensor cores, form the products with dA
     //    and dP), chain rule through the gates, dlog alpha by reverse prefix sums
-    const int nch = (T + kChunk - 1) / kChunk;
     if (tc) {
         auto ck = nslice == 4 ? gdr2_bwd_chunk_tc_kernel<Tio, 4> : gdr2_bwd_chunk_tc_kernel<Tio, 2>;
         err = cudaFuncSetAttribute(ck, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Bwd2TcSmem::kAlloc);
@@ -856,7 +919,7 @@ cudaError_t launch_bwd2_simt(int B, int T, int H, int dv, const void *q, const v
         ck<<<(unsigned)(B * H * nch), kBwd2TcThreads, Bwd2TcSmem::kAlloc, stream>>>(
             T, H, static_cast<const Tio *>(q), static_cast<const Tio *>(k), la, bg, w.part_kb, w.part_qe,
             w.part_ki, w.part_ec, w.part_x, w.flags, w.dAP, static_cast<Tio *>(dq), static_cast<Tio *>(dk_out), dla,
-            db, (size_t)B * T * H, tc_fwd ? 1 : 0);
+            db, (size_t)B * T * H);
         g_launches.fetch_add(1, std::memory_order_relaxed);
         return cudaGetLastError();
     }

@@ -59,15 +59,14 @@ struct Bwd2TcSmem {
 // tokens r = 16 (w / 4) .. of the chunk, which are its accumulator columns;
 // the prefix sum of the gates and the suffix sum of dG run as two-phase scans
 // over the four token quarters.
+// The chunk ch of (b*H + h) = bh.
 template <typename Tio, int NS>
-__global__ void __launch_bounds__(kBwd2TcThreads, 1)
-gdr2_bwd_chunk_tc_kernel(int T, int H, const Tio *__restrict__ q, const Tio *__restrict__ k,
-                         const float *__restrict__ log_alpha, const float *__restrict__ bgate,
-                         const float *__restrict__ part_kb, const float *__restrict__ part_qe,
-                         const float *__restrict__ part_ki, const float *__restrict__ part_ec,
-                         const float *__restrict__ part_x, const int *__restrict__ exact_flags,
-                         const float *__restrict__ dAP, Tio *__restrict__ dq, Tio *__restrict__ dk,
-                         float *__restrict__ dlog_alpha, float *__restrict__ db, size_t BTH, int tc_done) {
+__device__ __forceinline__ void gdr2_bwd_chunk_tc_body(
+    int T, int H, const Tio *__restrict__ q, const Tio *__restrict__ k, const float *__restrict__ log_alpha,
+    const float *__restrict__ bgate, const float *__restrict__ part_kb, const float *__restrict__ part_qe,
+    const float *__restrict__ part_ki, const float *__restrict__ part_ec, const float *__restrict__ part_x,
+    const int *__restrict__ exact_flags, const float *__restrict__ dAP, Tio *__restrict__ dq, Tio *__restrict__ dk,
+    float *__restrict__ dlog_alpha, float *__restrict__ db, size_t BTH, int bh, int ch) {
     using L = Bwd2TcSmem;
     using namespace sm100;
     constexpr int DK = 128, RQ = kChunk / 4;  // tokens per quarter
@@ -75,8 +74,6 @@ gdr2_bwd_chunk_tc_kernel(int T, int H, const Tio *__restrict__ q, const Tio *__r
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
     const int nchunks = (T + kChunk - 1) / kChunk;
-    const int ch = blockIdx.x % nchunks;
-    const int bh = blockIdx.x / nchunks;
     const int b = bh / H, h = bh % H;
     const int c0 = ch * kChunk, n = min(kChunk, T - c0);
     const size_t tok0 = ((size_t)b * T + c0) * H + h;
@@ -84,7 +81,6 @@ gdr2_bwd_chunk_tc_kernel(int T, int H, const Tio *__restrict__ q, const Tio *__r
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int j = (warp & 3) * 32 + lane, rq = warp >> 2, r0 = rq * RQ;
     const int mode = exact_flags[(size_t)bh * nchunks + ch];
-    if (mode == kChunkTc && tc_done) return;  // the tensor-core gradient kernel finished this chunk
 
     if (mode == 1) {
         // token-by-token partials: S_t^T do (part_qe), X = P^T gk (part_ki),
@@ -267,6 +263,45 @@ gdr2_bwd_chunk_tc_kernel(int T, int H, const Tio *__restrict__ q, const Tio *__r
     if (warp == 0) {
         tc_after_sync();
         tmem_dealloc(tmem, 256);
+    }
+}
+
+// One CTA per (b*H + h, chunk).
+template <typename Tio, int NS>
+__global__ void __launch_bounds__(kBwd2TcThreads, 1)
+gdr2_bwd_chunk_tc_kernel(int T, int H, const Tio *__restrict__ q, const Tio *__restrict__ k,
+                         const float *__restrict__ log_alpha, const float *__restrict__ bgate,
+                         const float *__restrict__ part_kb, const float *__restrict__ part_qe,
+                         const float *__restrict__ part_ki, const float *__restrict__ part_ec,
+                         const float *__restrict__ part_x, const int *__restrict__ exact_flags,
+                         const float *__restrict__ dAP, Tio *__restrict__ dq, Tio *__restrict__ dk,
+                         float *__restrict__ dlog_alpha, float *__restrict__ db, size_t BTH) {
+    const int nchunks = (T + kChunk - 1) / kChunk;
+    gdr2_bwd_chunk_tc_body<Tio, NS>(T, H, q, k, log_alpha, bgate, part_kb, part_qe, part_ki, part_ec, part_x,
+                                    exact_flags, dAP, dq, dk, dlog_alpha, db, BTH, (int)(blockIdx.x / nchunks),
+                                    (int)(blockIdx.x % nchunks));
+}
+
+// The chunks in todo[0 .. *ntodo) (each b*H*nchunks + chunk): CTA g takes
+// items g, g + gridDim.x, ...
+template <typename Tio, int NS>
+__global__ void __launch_bounds__(kBwd2TcThreads, 1)
+gdr2_bwd_chunk_tc_list_kernel(int T, int H, const Tio *__restrict__ q, const Tio *__restrict__ k,
+                              const float *__restrict__ log_alpha, const float *__restrict__ bgate,
+                              const float *__restrict__ part_kb, const float *__restrict__ part_qe,
+                              const float *__restrict__ part_ki, const float *__restrict__ part_ec,
+                              const float *__restrict__ part_x, const int *__restrict__ exact_flags,
+                              const float *__restrict__ dAP, Tio *__restrict__ dq, Tio *__restrict__ dk,
+                              float *__restrict__ dlog_alpha, float *__restrict__ db, size_t BTH,
+                              const int *__restrict__ todo, const int *__restrict__ ntodo) {
+    const int nchunks = (T + kChunk - 1) / kChunk, n_items = *ntodo;
+#pragma unroll 1
+    for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
+        __syncthreads();  // the previous item is done with shared memory and TMEM
+        const int tile = todo[it];
+        gdr2_bwd_chunk_tc_body<Tio, NS>(T, H, q, k, log_alpha, bgate, part_kb, part_qe, part_ki, part_ec, part_x,
+                                        exact_flags, dAP, dq, dk, dlog_alpha, db, BTH, tile / nchunks,
+                                        tile % nchunks);
     }
 }
 
