@@ -385,6 +385,8 @@ __global__ void __launch_bounds__(kBlkThreads)
 // second launch adds the G blocks of each pair in block order.
 constexpr int kProBwdRun = 64;
 constexpr int kProBwdStages = 2;
+constexpr int kProBwdRowsPerWarp = kProBwdRun / (kBlkThreads / 32);  // 8 consecutive rows per warp
+constexpr int kProBwdNB = 2;  // dz rows per step of phase 1
 constexpr int kProBwdMaxG = 32;  // blocks per (stream, head) pair: the workspace bound
 
 struct PrologueBwdArgs {
@@ -421,12 +423,15 @@ __device__ __forceinline__ void prologue_bwd_block(const PrologueBwdArgs &a, con
 
     const float *wsel = s == 0 ? a.w[0] : s == 1 ? a.w[1] : a.w[2];
     const float *bsel = s == 0 ? a.bias[0] : s == 1 ? a.bias[1] : a.bias[2];
+    // taps right-aligned as in the forward: wt[c][m] is tap m - (KW - K), and
+    // taps m < KW - K are zero; dwa[c][m] sums the gradient of the same tap
     float wt[CPL][KW], bias[CPL], dwa[CPL][KW], dba[CPL];
 #pragma unroll
     for (int c = 0; c < CPL; ++c) {
 #pragma unroll
         for (int m = 0; m < KW; ++m) {
-            wt[c][m] = m < K ? __ldg(wsel + (size_t)(c0 + c) * K + m) : 0.f;
+            const int j = m - (KW - K);
+            wt[c][m] = j >= 0 ? __ldg(wsel + (size_t)(c0 + c) * K + j) : 0.f;
             dwa[c][m] = 0.f;
         }
         bias[c] = bsel ? __ldg(bsel + c0 + c) : 0.f;
@@ -475,77 +480,122 @@ __device__ __forceinline__ void prologue_bwd_block(const PrologueBwdArgs &a, con
         const Tio *sx = reinterpret_cast<const Tio *>(stage) + lane * CPL;
         const Tio *sdy = reinterpret_cast<const Tio *>(stage + xalloc) + lane * CPL;
 
-        // phase 1: dz for tokens t0 .. t0+64+K-2 (row r = token t0 + r)
-        const int R1 = kProBwdRun + K - 1;
-#pragma unroll 1
-        for (int r = warp; r < R1; r += NW) {
-            float xv[KW][CPL], dyv[CPL], z[CPL], sg[CPL], u[CPL];
+        // phase 1: dz for tokens t0 .. t0+64+K-2 (row r = token t0 + r).  NB
+        // consecutive rows per step from a register window of x rows:
+        // win[m] = x row r + K - KW + m (stage row r + m' holds the x read by
+        // tap m' of row r), so row r + q reads win[q .. q + KW - 1].
+        constexpr int NBW = KW <= 4 ? kProBwdNB : 1, WR = KW + NBW - 1;  // one row per step at K > 4
+        // (rows r + nrows .. r + NB - 1 are computed from in-bounds stage
+        // memory and dropped)
+        auto dz_rows = [&](int r, int nrows, float(&win)[WR][CPL]) {
+            constexpr int NB = NBW;
+            float dyv[NB][CPL], z[NB][CPL], sg[NB][CPL], ss[NB], ud[NB];
 #pragma unroll
-            for (int m = 0; m < KW; ++m) {
-                if (m < K)
-                    ld_row<CPL>(sx + (r + m) * D, xv[m]);
-                else
-#pragma unroll
-                    for (int c = 0; c < CPL; ++c) xv[m][c] = 0.f;
-            }
-            ld_row<CPL>(sdy + r * D, dyv);
-            float ss = 0.f;
-#pragma unroll
-            for (int c = 0; c < CPL; ++c) {
-                float acc = bias[c];
-#pragma unroll
-                for (int m = 0; m < KW; ++m) acc = fmaf(wt[c][m], xv[m][c], acc);
-                z[c] = acc;
-                sg[c] = rcp_ftz(1.f + ex2_ftz(-kLog2e * acc));
-                u[c] = acc * sg[c];
-                ss = fmaf(u[c], u[c], ss);
-            }
-            float du[CPL];
-            if (l2) {
-                const float ninv = rsqrt_ftz(warp_sum(ss, 32) + a.eps);
-                float dot = 0.f;
-#pragma unroll
-                for (int c = 0; c < CPL; ++c) dot = fmaf(u[c] * ninv, dyv[c], dot);
-                dot = warp_sum(dot, 32);
-#pragma unroll
-                for (int c = 0; c < CPL; ++c) du[c] = fmaf(-u[c] * ninv, dot, dyv[c]) * ninv;
-            } else {
-#pragma unroll
-                for (int c = 0; c < CPL; ++c) du[c] = dyv[c];
-            }
-            const bool live = t0 + r < T;
-            float dz[CPL];
-#pragma unroll
-            for (int c = 0; c < CPL; ++c)
-                dz[c] = live ? du[c] * sg[c] * fmaf(z[c], 1.f - sg[c], 1.f) : 0.f;
-            st_row<CPL>(dzs + r * D + lane * CPL, dz);
-            if (r < kProBwdRun) {
+            for (int q = 0; q < NB; ++q) {
+                ld_row<CPL>(sdy + (r + q) * D, dyv[q]);
+                ss[q] = 0.f;
+                ud[q] = 0.f;
 #pragma unroll
                 for (int c = 0; c < CPL; ++c) {
+                    float acc = bias[c];
 #pragma unroll
-                    for (int m = 0; m < KW; ++m) dwa[c][m] = fmaf(dz[c], xv[m][c], dwa[c][m]);
-                    dba[c] += dz[c];
+                    for (int m = 0; m < KW; ++m) acc = fmaf(wt[c][m], win[q + m][c], acc);
+                    z[q][c] = acc;
+                    sg[q][c] = rcp_ftz(1.f + ex2_ftz(-kLog2e * acc));
+                    const float u = acc * sg[q][c];
+                    ss[q] = fmaf(u, u, ss[q]);
+                    ud[q] = fmaf(u, dyv[q][c], ud[q]);
                 }
             }
+            // L2 reverse: y = u/n, du = (dy - y (y . dy)) / n
+            //                        = (dy - u (u . dy) / n^2) / n;
+            // both row sums reduce together
+            float du[NB][CPL];
+            if (l2) {
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+                    for (int q = 0; q < NB; ++q) {
+                        ss[q] += __shfl_xor_sync(0xffffffffu, ss[q], off);
+                        ud[q] += __shfl_xor_sync(0xffffffffu, ud[q], off);
+                    }
+#pragma unroll
+                for (int q = 0; q < NB; ++q) {
+                    const float ninv = rsqrt_ftz(ss[q] + a.eps), f = -ud[q] * ninv * ninv;
+#pragma unroll
+                    for (int c = 0; c < CPL; ++c) du[q][c] = fmaf(z[q][c] * sg[q][c], f, dyv[q][c]) * ninv;
+                }
+            } else {
+#pragma unroll
+                for (int q = 0; q < NB; ++q)
+#pragma unroll
+                    for (int c = 0; c < CPL; ++c) du[q][c] = dyv[q][c];
+            }
+#pragma unroll
+            for (int q = 0; q < NB; ++q) {
+                if (q >= nrows) break;
+                const bool live = t0 + r + q < T;
+                float dz[CPL];
+#pragma unroll
+                for (int c = 0; c < CPL; ++c)
+                    dz[c] = live ? du[q][c] * sg[q][c] * fmaf(z[q][c], 1.f - sg[q][c], 1.f) : 0.f;
+                st_row<CPL>(dzs + (r + q) * D + lane * CPL, dz);
+                if (r + q < kProBwdRun) {  // the unit's own rows: dw and dbias
+#pragma unroll
+                    for (int c = 0; c < CPL; ++c) {
+#pragma unroll
+                        for (int m = 0; m < KW; ++m) dwa[c][m] = fmaf(dz[c], win[q + m][c], dwa[c][m]);
+                        dba[c] += dz[c];
+                    }
+                }
+            }
+        };
+        {  // the unit's 64 rows: warp w takes rows 8w .. 8w+7
+            const int r0 = warp * kProBwdRowsPerWarp;
+            float win[WR][CPL];
+#pragma unroll
+            for (int m = 0; m < KW - 1; ++m) {
+                const int row = r0 + K - KW + m;
+                if (row >= 0)
+                    ld_row<CPL>(sx + row * D, win[m]);
+                else
+#pragma unroll
+                    for (int c = 0; c < CPL; ++c) win[m][c] = 0.f;
+            }
+#pragma unroll
+            for (int p = 0; p < kProBwdRowsPerWarp; p += NBW) {
+                const int r = r0 + p;
+#pragma unroll
+                for (int m = KW - 1; m < WR; ++m) ld_row<CPL>(sx + (r + K - KW + m) * D, win[m]);
+                dz_rows(r, NBW, win);
+#pragma unroll
+                for (int m = 0; m < KW - 1; ++m)
+#pragma unroll
+                    for (int c = 0; c < CPL; ++c) win[m][c] = win[m + NBW][c];
+            }
+        }
+        if (warp < K - 1) {  // the K-1 rows after the unit, whose dz its last dx rows read
+            const int r = kProBwdRun + warp;
+            float win[WR][CPL];
+#pragma unroll
+            for (int m = 0; m < WR; ++m) ld_row<CPL>(sx + (r + K - KW + m) * D, win[m]);
+            dz_rows(r, 1, win);
         }
         __syncthreads();
 
-        // phase 2: dx for the unit's tokens (and the carried-in state's rows)
-        const int rlo = (t0 == 0 && dsi != nullptr) ? -(K - 1) : 0;
-#pragma unroll 1
-        for (int i = rlo + warp; i < len; i += NW) {
+        // phase 2: dx[i] = sum_j w[j] dz[i + K-1-j], from a window of dz rows
+        // dzw[n] = dz row i + n (n < KW), which tap K-1-n = wt[.][KW-1-n]
+        // multiplies (zero for n >= K; rows up to 64+KW-2 exist and rows past
+        // 64+K-2 hold zeros)
+        auto dx_row = [&](int i, const float (&dzw)[KW][CPL]) {
+            if (i >= len) return;  // past the end of a ragged last unit
             float acc[CPL];
 #pragma unroll
-            for (int c = 0; c < CPL; ++c) acc[c] = 0.f;
+            for (int c = 0; c < CPL; ++c) {
+                float v = 0.f;
 #pragma unroll
-            for (int m = 0; m < KW; ++m) {
-                const int r = i + K - 1 - m;  // dz row that read this x through tap m
-                if (m < K && r >= 0) {
-                    float dzv[CPL];
-                    ld_row<CPL>(dzs + r * D + lane * CPL, dzv);
-#pragma unroll
-                    for (int c = 0; c < CPL; ++c) acc[c] = fmaf(wt[c][m], dzv[c], acc[c]);
-                }
+                for (int n = 0; n < KW; ++n) v = fmaf(wt[c][KW - 1 - n], dzw[n][c], v);
+                acc[c] = v;
             }
             const int ms = t0 + i - (T - (K - 1));  // slot of this x in the returned state
             if (dso != nullptr && ms >= 0) {
@@ -554,10 +604,40 @@ __device__ __forceinline__ void prologue_bwd_block(const PrologueBwdArgs &a, con
 #pragma unroll
                 for (int c = 0; c < CPL; ++c) acc[c] += g[c];
             }
-            if (i >= 0)
+            if (i >= 0) {
                 st_row<CPL>(dxb + ((size_t)b * T + t0 + i) * H * D + c0, acc);
-            else
+            } else {
                 st_row<CPL>(dsi + ((size_t)b * (K - 1) + (K - 1 + i)) * Ctot + col + c0, acc);
+            }
+        };
+        const float *sdz = dzs + lane * CPL;
+        {
+            const int i0 = warp * kProBwdRowsPerWarp;
+            float dzw[KW][CPL];
+#pragma unroll
+            for (int n = 0; n < KW - 1; ++n) ld_row<CPL>(sdz + (i0 + n) * D, dzw[n]);
+#pragma unroll
+            for (int p = 0; p < kProBwdRowsPerWarp; ++p) {
+                ld_row<CPL>(sdz + (i0 + p + KW - 1) * D, dzw[KW - 1]);
+                dx_row(i0 + p, dzw);
+#pragma unroll
+                for (int n = 0; n < KW - 1; ++n)
+#pragma unroll
+                    for (int c = 0; c < CPL; ++c) dzw[n][c] = dzw[n + 1][c];
+            }
+        }
+        if (t0 == 0 && dsi != nullptr && warp < K - 1) {  // the carried-in state's rows
+            const int i = warp - (K - 1);
+            float dzw[KW][CPL];
+#pragma unroll
+            for (int n = 0; n < KW; ++n) {
+                if (i + n >= 0)
+                    ld_row<CPL>(sdz + (i + n) * D, dzw[n]);
+                else
+#pragma unroll
+                    for (int c = 0; c < CPL; ++c) dzw[n][c] = 0.f;
+            }
+            dx_row(i, dzw);
         }
         __syncthreads();
         st = st == kProBwdStages - 1 ? 0 : st + 1;
@@ -568,7 +648,8 @@ __device__ __forceinline__ void prologue_bwd_block(const PrologueBwdArgs &a, con
 #pragma unroll
     for (int c = 0; c < CPL; ++c) {
 #pragma unroll
-        for (int m = 0; m < KW; ++m) red[warp * E + (lane * CPL + c) * (KW + 1) + m] = dwa[c][m];
+        for (int m = 0; m < KW; ++m)
+            if (m >= KW - K) red[warp * E + (lane * CPL + c) * (KW + 1) + m - (KW - K)] = dwa[c][m];
         red[warp * E + (lane * CPL + c) * (KW + 1) + KW] = dba[c];
     }
     __syncthreads();
@@ -599,6 +680,8 @@ __global__ void __launch_bounds__(kBlkThreads)
         for (int i = 0; i < kProBwdStages; ++i) mbar_init(&bars[i], 1);
         fence_mbar_init();
     }
+    // dz rows past 64+K-2 are read (by taps that are zero) and never written
+    for (int i = threadIdx.x; i < (kProBwdRun + KW - 1) * DMAX; i += kBlkThreads) dzs[i] = 0.f;
     __syncthreads();
     if (s == 0)
         prologue_bwd_block<Tio, DQK, KW>(a, &tm_xq, &tm_dq, s, h, idx, G, smem, stage_bytes, xalloc, dzs, bars);
