@@ -375,14 +375,18 @@ __global__ void __launch_bounds__(kBlkThreads)
 //           s < 0: dstate_in)
 //   dw[c, j] = sum_t dz[t, c] x[t-K+1+j, c],   dbias[c] = sum_t dz[t, c].
 // Same (stream, head) pair ownership as the forward.  A unit is 64 tokens
-// [t0, t0+64); its stage holds x for tokens t0-(K-1) .. t0+64+K-2 and dy for
-// t0 .. t0+64+K-2 (one tiled TMA load each, zero past T), because dx of the
-// unit's last tokens needs dz of the K-1 tokens after it.  Phase 1 (a warp per
-// row, D/32 channels per lane) recomputes dz for those 64+K-1 tokens into a
-// fp32 shared buffer and adds the unit's own 64 rows into the lane's dw and
-// dbias registers; phase 2 reads K rows of dz per output row.  At the end the
-// block adds its warps' sums in warp order into one row of `partial`, and a
-// second launch adds the G blocks of each pair in block order.
+// [t0, t0+64); a block owns a contiguous range of the pair's (batch, run)
+// units and walks it from the last to the first.  The stage holds x for
+// tokens t0-(K-1) .. t0+63 and dy for t0 .. t0+63 (one tiled TMA load each,
+// zero past T).  dx of the unit's last tokens needs dz of the K-1 tokens
+// after it: those are the first rows of the unit walked just before, carried
+// in shared memory (zero at the end of a batch; computed from global memory
+// for the block's first unit).  Phase 1 (D/32 channels per lane, 8
+// consecutive rows per warp) recomputes dz into a fp32 shared buffer and adds
+// the rows into the lane's dw and dbias registers; phase 2 forms dx from a
+// sliding window of dz rows.  At the end the block adds its warps' sums in
+// warp order into one row of `partial`, and a second launch adds the G blocks
+// of each pair in block order.
 constexpr int kProBwdRun = 64;
 constexpr int kProBwdStages = 2;
 constexpr int kProBwdRowsPerWarp = kProBwdRun / (kBlkThreads / 32);  // 8 consecutive rows per warp
@@ -415,9 +419,12 @@ __device__ __forceinline__ void prologue_bwd_block(const PrologueBwdArgs &a, con
     const int K = a.K, T = a.T, H = a.H;
     const int runs = (T + kProBwdRun - 1) / kProBwdRun;
     const int units = a.B * runs;
+    // this block's units, walked from the last to the first
+    const int j_lo = (int)((long long)idx * units / G), j_hi = (int)((long long)(idx + 1) * units / G);
+    const int n_my = j_hi - j_lo;
     const int c0 = h * D + lane * CPL;  // this lane's first channel in the stream
-    const uint32_t xbox = (uint32_t)(kProBwdRun + 2 * (K - 1)) * D * (uint32_t)sizeof(Tio);
-    const uint32_t dybox = (uint32_t)(kProBwdRun + K - 1) * D * (uint32_t)sizeof(Tio);
+    const uint32_t xbox = (uint32_t)(kProBwdRun + K - 1) * D * (uint32_t)sizeof(Tio);
+    const uint32_t dybox = (uint32_t)kProBwdRun * D * (uint32_t)sizeof(Tio);
     const int Ctot = H * (2 * a.dk + a.dv);
     const int col = s == 0 ? 0 : s == 1 ? H * a.dk : 2 * H * a.dk;  // stream's columns in the state
 
@@ -438,7 +445,7 @@ __device__ __forceinline__ void prologue_bwd_block(const PrologueBwdArgs &a, con
         dba[c] = 0.f;
     }
     auto issue = [&](int k, int sidx) {  // one thread
-        const int j = idx + k * G, b = j / runs, t0 = (j % runs) * kProBwdRun;
+        const int j = j_hi - 1 - k, b = j / runs, t0 = (j % runs) * kProBwdRun;
         uint8_t *stg = smem + sidx * stage_bytes;
         mbar_expect_tx(&bars[sidx], xbox + dybox);
         tma_load_4d(stg, mx, &bars[sidx], 0, h, t0 - (K - 1), b);
@@ -446,24 +453,30 @@ __device__ __forceinline__ void prologue_bwd_block(const PrologueBwdArgs &a, con
     };
     if (threadIdx.x == 0)
         for (int k = 0; k < kProBwdStages - 1; ++k)
-            if (idx + k * G < units) issue(k, k);
+            if (k < n_my) issue(k, k);
     const bool l2 = s < 2;
+    const Tio *xg = static_cast<const Tio *>(s == 0 ? a.x[0] : s == 1 ? a.x[1] : a.x[2]);
+    const Tio *dyg = static_cast<const Tio *>(s == 0 ? a.dy[0] : s == 1 ? a.dy[1] : a.dy[2]);
     const Tio *dso = static_cast<const Tio *>(a.dstate_out);
     Tio *dxb = static_cast<Tio *>(s == 0 ? a.dx[0] : s == 1 ? a.dx[1] : a.dx[2]);
     Tio *dsi = static_cast<Tio *>(a.dstate_in);
+    // dz of the K-1 tokens after a unit (its last dx rows read them): the
+    // first rows of the unit walked just before it, kept in carry[k & 1]
+    // (rows K-1 .. KW-2 stay zero), or computed for the block's first unit
+    float *carry0 = dzs + kProBwdRun * D;
     int st = 0;
 #pragma unroll 1
-    for (int k = 0;; ++k) {
-        const int j = idx + k * G;
-        if (j >= units) break;
+    for (int k = 0; k < n_my; ++k) {
+        const int j = j_hi - 1 - k;
         const int b = j / runs, t0 = (j % runs) * kProBwdRun, len = min(kProBwdRun, T - t0);
-        if (threadIdx.x == 0 && j + (kProBwdStages - 1) * G < units) {
+        float *carry_in = carry0 + (k & 1) * (KW - 1) * D, *carry_out = carry0 + ((k + 1) & 1) * (KW - 1) * D;
+        if (threadIdx.x == 0 && k + kProBwdStages - 1 < n_my) {
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             issue(k + kProBwdStages - 1, st == 0 ? kProBwdStages - 1 : st - 1);
         }
         if (!mbar_wait(&bars[st], (uint32_t)(k / kProBwdStages) & 1u)) {
             record_status(GDR_ERR_TIMEOUT);
-            blk_drain<kProBwdStages>(bars, st, k, j, units, G);
+            blk_drain<kProBwdStages>(bars, st, k, k, n_my, 1);
             return;
         }
         uint8_t *stage = smem + st * stage_bytes;
@@ -480,29 +493,39 @@ __device__ __forceinline__ void prologue_bwd_block(const PrologueBwdArgs &a, con
         const Tio *sx = reinterpret_cast<const Tio *>(stage) + lane * CPL;
         const Tio *sdy = reinterpret_cast<const Tio *>(stage + xalloc) + lane * CPL;
 
-        // phase 1: dz for tokens t0 .. t0+64+K-2 (row r = token t0 + r).  NB
+        // phase 1: dz for tokens t0 .. t0+63 (row r = token t0 + r).  NB
         // consecutive rows per step from a register window of x rows:
         // win[m] = x row r + K - KW + m (stage row r + m' holds the x read by
-        // tap m' of row r), so row r + q reads win[q .. q + KW - 1].
+        // tap m' of row r), so row r + q reads win[q .. q + KW - 1].  dy of
+        // row r + q is at dyp + q * dys, its dz goes to dzp + q * D; rows
+        // r + nrows .. r + NB - 1 are computed on zeros and dropped.
         constexpr int NBW = KW <= 4 ? kProBwdNB : 1, WR = KW + NBW - 1;  // one row per step at K > 4
-        // (rows r + nrows .. r + NB - 1 are computed from in-bounds stage
-        // memory and dropped)
-        auto dz_rows = [&](int r, int nrows, float(&win)[WR][CPL]) {
+        auto dz_rows = [&](int r, int nrows, float(&win)[WR][CPL], const Tio *dyp, size_t dys, float *dzp) {
             constexpr int NB = NBW;
             float dyv[NB][CPL], z[NB][CPL], sg[NB][CPL], ss[NB], ud[NB];
 #pragma unroll
             for (int q = 0; q < NB; ++q) {
-                ld_row<CPL>(sdy + (r + q) * D, dyv[q]);
+                if (q < nrows)
+                    ld_row<CPL>(dyp + q * dys, dyv[q]);
+                else
+#pragma unroll
+                    for (int c = 0; c < CPL; ++c) dyv[q][c] = 0.f;
                 ss[q] = 0.f;
                 ud[q] = 0.f;
 #pragma unroll
-                for (int c = 0; c < CPL; ++c) {
-                    float acc = bias[c];
+                for (int c = 0; c < CPL; c += 2) {  // channel pairs on the packed FMA
+                    float2 acc = make_float2(bias[c], bias[c + 1]);
 #pragma unroll
-                    for (int m = 0; m < KW; ++m) acc = fmaf(wt[c][m], win[q + m][c], acc);
-                    z[q][c] = acc;
-                    sg[q][c] = rcp_ftz(1.f + ex2_ftz(-kLog2e * acc));
-                    const float u = acc * sg[q][c];
+                    for (int m = 0; m < KW; ++m)
+                        acc = ffma2(make_float2(wt[c][m], wt[c + 1][m]), make_float2(win[q + m][c], win[q + m][c + 1]),
+                                    acc);
+                    z[q][c] = acc.x;
+                    z[q][c + 1] = acc.y;
+                }
+#pragma unroll
+                for (int c = 0; c < CPL; ++c) {
+                    sg[q][c] = rcp_ftz(1.f + ex2_ftz(-kLog2e * z[q][c]));
+                    const float u = z[q][c] * sg[q][c];
                     ss[q] = fmaf(u, u, ss[q]);
                     ud[q] = fmaf(u, dyv[q][c], ud[q]);
                 }
@@ -539,14 +562,27 @@ __device__ __forceinline__ void prologue_bwd_block(const PrologueBwdArgs &a, con
 #pragma unroll
                 for (int c = 0; c < CPL; ++c)
                     dz[c] = live ? du[q][c] * sg[q][c] * fmaf(z[q][c], 1.f - sg[q][c], 1.f) : 0.f;
-                st_row<CPL>(dzs + (r + q) * D + lane * CPL, dz);
+                st_row<CPL>(dzp + q * D, dz);
                 if (r + q < kProBwdRun) {  // the unit's own rows: dw and dbias
 #pragma unroll
-                    for (int c = 0; c < CPL; ++c) {
+                    for (int c = 0; c < CPL; c += 2) {
 #pragma unroll
-                        for (int m = 0; m < KW; ++m) dwa[c][m] = fmaf(dz[c], win[q + m][c], dwa[c][m]);
+                        for (int m = 0; m < KW; ++m) {
+                            const float2 t = ffma2(make_float2(dz[c], dz[c + 1]),
+                                                   make_float2(win[q + m][c], win[q + m][c + 1]),
+                                                   make_float2(dwa[c][m], dwa[c + 1][m]));
+                            dwa[c][m] = t.x;
+                            dwa[c + 1][m] = t.y;
+                        }
                         dba[c] += dz[c];
+                        dba[c + 1] += dz[c + 1];
                     }
+                }
+                if (r + q < K - 1) {  // the next unit walked (tokens before t0) reads these
+                    if (t0 == 0)
+#pragma unroll
+                        for (int c = 0; c < CPL; ++c) dz[c] = 0.f;  // ... unless it is another batch's
+                    st_row<CPL>(carry_out + (r + q) * D + lane * CPL, dz);
                 }
             }
         };
@@ -567,35 +603,51 @@ __device__ __forceinline__ void prologue_bwd_block(const PrologueBwdArgs &a, con
                 const int r = r0 + p;
 #pragma unroll
                 for (int m = KW - 1; m < WR; ++m) ld_row<CPL>(sx + (r + K - KW + m) * D, win[m]);
-                dz_rows(r, NBW, win);
+                dz_rows(r, NBW, win, sdy + r * D, D, dzs + r * D + lane * CPL);
 #pragma unroll
                 for (int m = 0; m < KW - 1; ++m)
 #pragma unroll
                     for (int c = 0; c < CPL; ++c) win[m][c] = win[m + NBW][c];
             }
         }
-        if (warp < K - 1) {  // the K-1 rows after the unit, whose dz its last dx rows read
-            const int r = kProBwdRun + warp;
+        if (k == 0 && warp < K - 1) {
+            // the block's first unit: dz of token t0 + 64 + warp from global
+            // memory (zero past T; the x it reads are tokens t0 + 57 .. t)
+            const int r = kProBwdRun + warp, t = t0 + r;
             float win[WR][CPL];
 #pragma unroll
-            for (int m = 0; m < WR; ++m) ld_row<CPL>(sx + (r + K - KW + m) * D, win[m]);
-            dz_rows(r, 1, win);
+            for (int m = 0; m < WR; ++m) {
+                if (t < T && m < KW)
+                    ld_row<CPL>(xg + (((size_t)b * T + t + 1 - KW + m) * H) * D + c0, win[m]);
+                else
+#pragma unroll
+                    for (int c = 0; c < CPL; ++c) win[m][c] = 0.f;
+            }
+            dz_rows(r, t < T ? 1 : 0, win, dyg + (((size_t)b * T + t) * H) * D + c0, 0, carry_in + warp * D + lane * CPL);
+            if (t >= T) {
+                float zero[CPL];
+#pragma unroll
+                for (int c = 0; c < CPL; ++c) zero[c] = 0.f;
+                st_row<CPL>(carry_in + warp * D + lane * CPL, zero);
+            }
         }
         __syncthreads();
 
         // phase 2: dx[i] = sum_j w[j] dz[i + K-1-j], from a window of dz rows
         // dzw[n] = dz row i + n (n < KW), which tap K-1-n = wt[.][KW-1-n]
-        // multiplies (zero for n >= K; rows up to 64+KW-2 exist and rows past
-        // 64+K-2 hold zeros)
+        // multiplies (zero for n >= K); rows 64 .. 64+KW-2 are carry_in's
         auto dx_row = [&](int i, const float (&dzw)[KW][CPL]) {
             if (i >= len) return;  // past the end of a ragged last unit
             float acc[CPL];
 #pragma unroll
-            for (int c = 0; c < CPL; ++c) {
-                float v = 0.f;
+            for (int c = 0; c < CPL; c += 2) {
+                float2 v = make_float2(0.f, 0.f);
 #pragma unroll
-                for (int n = 0; n < KW; ++n) v = fmaf(wt[c][KW - 1 - n], dzw[n][c], v);
-                acc[c] = v;
+                for (int n = 0; n < KW; ++n)
+                    v = ffma2(make_float2(wt[c][KW - 1 - n], wt[c + 1][KW - 1 - n]), make_float2(dzw[n][c], dzw[n][c + 1]),
+                              v);
+                acc[c] = v.x;
+                acc[c + 1] = v.y;
             }
             const int ms = t0 + i - (T - (K - 1));  // slot of this x in the returned state
             if (dso != nullptr && ms >= 0) {
@@ -610,15 +662,17 @@ __device__ __forceinline__ void prologue_bwd_block(const PrologueBwdArgs &a, con
                 st_row<CPL>(dsi + ((size_t)b * (K - 1) + (K - 1 + i)) * Ctot + col + c0, acc);
             }
         };
-        const float *sdz = dzs + lane * CPL;
+        auto dz_row_ptr = [&](int row) {
+            return (row < kProBwdRun ? dzs + row * D : carry_in + (row - kProBwdRun) * D) + lane * CPL;
+        };
         {
             const int i0 = warp * kProBwdRowsPerWarp;
             float dzw[KW][CPL];
 #pragma unroll
-            for (int n = 0; n < KW - 1; ++n) ld_row<CPL>(sdz + (i0 + n) * D, dzw[n]);
+            for (int n = 0; n < KW - 1; ++n) ld_row<CPL>(dz_row_ptr(i0 + n), dzw[n]);
 #pragma unroll
             for (int p = 0; p < kProBwdRowsPerWarp; ++p) {
-                ld_row<CPL>(sdz + (i0 + p + KW - 1) * D, dzw[KW - 1]);
+                ld_row<CPL>(dz_row_ptr(i0 + p + KW - 1), dzw[KW - 1]);
                 dx_row(i0 + p, dzw);
 #pragma unroll
                 for (int n = 0; n < KW - 1; ++n)
@@ -632,7 +686,7 @@ __device__ __forceinline__ void prologue_bwd_block(const PrologueBwdArgs &a, con
 #pragma unroll
             for (int n = 0; n < KW; ++n) {
                 if (i + n >= 0)
-                    ld_row<CPL>(sdz + (i + n) * D, dzw[n]);
+                    ld_row<CPL>(dz_row_ptr(i + n), dzw[n]);
                 else
 #pragma unroll
                     for (int c = 0; c < CPL; ++c) dzw[n][c] = 0.f;
@@ -673,15 +727,15 @@ __global__ void __launch_bounds__(kBlkThreads)
     extern __shared__ __align__(128) uint8_t blk_smem[];
     uint8_t *smem = blk_smem;
     float *dzs = reinterpret_cast<float *>(smem + kProBwdStages * stage_bytes);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(dzs + (kProBwdRun + KW - 1) * DMAX);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(dzs + (kProBwdRun + 2 * (KW - 1)) * DMAX);
     const int P = 3 * a.H, pair = blockIdx.x % P, idx = blockIdx.x / P, G = gridDim.x / P;
     const int s = pair / a.H, h = pair % a.H;
     if (threadIdx.x == 0) {
         for (int i = 0; i < kProBwdStages; ++i) mbar_init(&bars[i], 1);
         fence_mbar_init();
     }
-    // dz rows past 64+K-2 are read (by taps that are zero) and never written
-    for (int i = threadIdx.x; i < (kProBwdRun + KW - 1) * DMAX; i += kBlkThreads) dzs[i] = 0.f;
+    // the carried dz rows past K-2 are read (by taps that are zero) and never written
+    for (int i = threadIdx.x; i < (kProBwdRun + 2 * (KW - 1)) * DMAX; i += kBlkThreads) dzs[i] = 0.f;
     __syncthreads();
     if (s == 0)
         prologue_bwd_block<Tio, DQK, KW>(a, &tm_xq, &tm_dq, s, h, idx, G, smem, stage_bytes, xalloc, dzs, bars);
@@ -1045,20 +1099,19 @@ inline cudaError_t launch_prologue_bwd_kw(PrologueBwdArgs a, float *const dw[3],
                                           cudaStream_t stream) {
     constexpr int DMAX = DQK > DV ? DQK : DV;
     auto kern = gdr_prologue_bwd_kernel<Tio, DQK, DV, KW>;
-    const int xalloc = (kProBwdRun + 2 * (KW - 1)) * DMAX * (int)sizeof(Tio);
-    const int stage_bytes = xalloc + (kProBwdRun + KW - 1) * DMAX * (int)sizeof(Tio);
-    static_assert((kBlkThreads / 32) * DMAX * (KW + 1) * 4 <=
-                      kProBwdStages * ((kProBwdRun + 2 * (KW - 1)) + (kProBwdRun + KW - 1)) * DMAX * 2,
+    const int xalloc = (kProBwdRun + KW - 1) * DMAX * (int)sizeof(Tio);
+    const int stage_bytes = xalloc + kProBwdRun * DMAX * (int)sizeof(Tio);
+    static_assert((kBlkThreads / 32) * DMAX * (KW + 1) * 4 <= kProBwdStages * (2 * kProBwdRun + KW - 1) * DMAX * 2,
                   "warp sums must fit in the stages");
-    const int smem = kProBwdStages * stage_bytes + (kProBwdRun + KW - 1) * DMAX * 4 + 8 * kProBwdStages;
+    const int smem = kProBwdStages * stage_bytes + (kProBwdRun + 2 * (KW - 1)) * DMAX * 4 + 8 * kProBwdStages;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     const int K = a.K;
     CUtensorMap mx[3], mdy[3];
     for (int s = 0; s < 3; ++s) {
         const int d = s < 2 ? a.dk : a.dv;
-        if (!make_prologue_map<Tio>(&mx[s], a.x[s], a.B, a.T, a.H, d, kProBwdRun + 2 * (K - 1)) ||
-            !make_prologue_map<Tio>(&mdy[s], a.dy[s], a.B, a.T, a.H, d, kProBwdRun + K - 1))
+        if (!make_prologue_map<Tio>(&mx[s], a.x[s], a.B, a.T, a.H, d, kProBwdRun + K - 1) ||
+            !make_prologue_map<Tio>(&mdy[s], a.dy[s], a.B, a.T, a.H, d, kProBwdRun))
             return cudaErrorInvalidValue;
     }
     const long long pairs = 3LL * a.H, units = (long long)a.B * ((a.T + kProBwdRun - 1) / kProBwdRun);
