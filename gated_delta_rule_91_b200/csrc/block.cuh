@@ -414,7 +414,9 @@ __device__ __forceinline__ void prologue_bwd_block(const PrologueBwdArgs &a, con
                                                    uint8_t *smem, int stage_bytes, int xalloc, float *dzs,
                                                    uint64_t *bars) {
     using namespace sm100;
-    constexpr int CPL = D / 32, NW = kBlkThreads / 32;
+    // a lane owns CPL = D/32 channels as NP pairs: every elementwise step runs
+    // on the packed fp32 pair instructions (each lane rounded as the scalar op)
+    constexpr int CPL = D / 32, NP = CPL / 2, NW = kBlkThreads / 32;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int K = a.K, T = a.T, H = a.H;
     const int runs = (T + kProBwdRun - 1) / kProBwdRun;
@@ -430,19 +432,22 @@ __device__ __forceinline__ void prologue_bwd_block(const PrologueBwdArgs &a, con
 
     const float *wsel = s == 0 ? a.w[0] : s == 1 ? a.w[1] : a.w[2];
     const float *bsel = s == 0 ? a.bias[0] : s == 1 ? a.bias[1] : a.bias[2];
-    // taps right-aligned as in the forward: wt[c][m] is tap m - (KW - K), and
-    // taps m < KW - K are zero; dwa[c][m] sums the gradient of the same tap
-    float wt[CPL][KW], bias[CPL], dwa[CPL][KW], dba[CPL];
+    // taps right-aligned as in the forward: wt[p][m] holds tap m - (KW - K) of
+    // the pair's two channels, and taps m < KW - K are zero; dwa[p][m] sums
+    // the gradient of the same tap
+    float2 wt[NP][KW], bias[NP], dwa[NP][KW], dba[NP];
 #pragma unroll
-    for (int c = 0; c < CPL; ++c) {
+    for (int p = 0; p < NP; ++p) {
 #pragma unroll
         for (int m = 0; m < KW; ++m) {
             const int j = m - (KW - K);
-            wt[c][m] = j >= 0 ? __ldg(wsel + (size_t)(c0 + c) * K + j) : 0.f;
-            dwa[c][m] = 0.f;
+            wt[p][m] = j >= 0 ? make_float2(__ldg(wsel + (size_t)(c0 + 2 * p) * K + j),
+                                            __ldg(wsel + (size_t)(c0 + 2 * p + 1) * K + j))
+                              : make_float2(0.f, 0.f);
+            dwa[p][m] = make_float2(0.f, 0.f);
         }
-        bias[c] = bsel ? __ldg(bsel + c0 + c) : 0.f;
-        dba[c] = 0.f;
+        bias[p] = bsel ? make_float2(__ldg(bsel + c0 + 2 * p), __ldg(bsel + c0 + 2 * p + 1)) : make_float2(0.f, 0.f);
+        dba[p] = make_float2(0.f, 0.f);
     }
     auto issue = [&](int k, int sidx) {  // one thread
         const int j = j_hi - 1 - k, b = j / runs, t0 = (j % runs) * kProBwdRun;
@@ -460,6 +465,12 @@ __device__ __forceinline__ void prologue_bwd_block(const PrologueBwdArgs &a, con
     const Tio *dso = static_cast<const Tio *>(a.dstate_out);
     Tio *dxb = static_cast<Tio *>(s == 0 ? a.dx[0] : s == 1 ? a.dx[1] : a.dx[2]);
     Tio *dsi = static_cast<Tio *>(a.dstate_in);
+    const float2 one2 = make_float2(1.f, 1.f), mone2 = make_float2(-1.f, -1.f);
+    const float2 ml2e2 = make_float2(-kLog2e, -kLog2e);
+    auto zero_row = [](float2 (&v)[NP]) {
+#pragma unroll
+        for (int p = 0; p < NP; ++p) v[p] = make_float2(0.f, 0.f);
+    };
     // dz of the K-1 tokens after a unit (its last dx rows read them): the
     // first rows of the unit walked just before it, kept in carry[k & 1]
     // (rows K-1 .. KW-2 stay zero), or computed for the block's first unit
@@ -498,42 +509,41 @@ __device__ __forceinline__ void prologue_bwd_block(const PrologueBwdArgs &a, con
         // win[m] = x row r + K - KW + m (stage row r + m' holds the x read by
         // tap m' of row r), so row r + q reads win[q .. q + KW - 1].  dy of
         // row r + q is at dyp + q * dys, its dz goes to dzp + q * D; rows
-        // r + nrows .. r + NB - 1 are computed on zeros and dropped.
+        // r + nrows .. r + NB - 1 are computed on zeros and dropped.  dy is
+        // zero past T (the TMA fill, or the caller), so dz is zero there.
+        //   u = SiLU(z) = z sg,  g = dSiLU/dz = sg (1 + z (1 - sg)) = sg + u (1 - sg)
         constexpr int NBW = KW <= 4 ? kProBwdNB : 1, WR = KW + NBW - 1;  // one row per step at K > 4
-        auto dz_rows = [&](int r, int nrows, float(&win)[WR][CPL], const Tio *dyp, size_t dys, float *dzp) {
+        auto dz_rows = [&](int r, int nrows, float2(&win)[WR][NP], const Tio *dyp, size_t dys, float *dzp) {
             constexpr int NB = NBW;
-            float dyv[NB][CPL], z[NB][CPL], sg[NB][CPL], ss[NB], ud[NB];
+            float2 dyv[NB][NP], u[NB][NP], g[NB][NP];
+            float ss[NB], ud[NB];
 #pragma unroll
             for (int q = 0; q < NB; ++q) {
                 if (q < nrows)
-                    ld_row<CPL>(dyp + q * dys, dyv[q]);
+                    ld_row<CPL>(dyp + q * dys, reinterpret_cast<float *>(dyv[q]));
                 else
+                    zero_row(dyv[q]);
+                float2 ss2 = make_float2(0.f, 0.f), ud2 = make_float2(0.f, 0.f);
 #pragma unroll
-                    for (int c = 0; c < CPL; ++c) dyv[q][c] = 0.f;
-                ss[q] = 0.f;
-                ud[q] = 0.f;
+                for (int p = 0; p < NP; ++p) {
+                    float2 z = bias[p];
 #pragma unroll
-                for (int c = 0; c < CPL; c += 2) {  // channel pairs on the packed FMA
-                    float2 acc = make_float2(bias[c], bias[c + 1]);
-#pragma unroll
-                    for (int m = 0; m < KW; ++m)
-                        acc = ffma2(make_float2(wt[c][m], wt[c + 1][m]), make_float2(win[q + m][c], win[q + m][c + 1]),
-                                    acc);
-                    z[q][c] = acc.x;
-                    z[q][c + 1] = acc.y;
+                    for (int m = 0; m < KW; ++m) z = ffma2(wt[p][m], win[q + m][p], z);
+                    const float2 e = fmul2(z, ml2e2);
+                    const float2 den = ffma2(make_float2(ex2_ftz(e.x), ex2_ftz(e.y)), one2, one2);
+                    const float2 sg = make_float2(rcp_ftz(den.x), rcp_ftz(den.y));
+                    u[q][p] = fmul2(z, sg);
+                    g[q][p] = ffma2(u[q][p], ffma2(sg, mone2, one2), sg);
+                    ss2 = ffma2(u[q][p], u[q][p], ss2);
+                    ud2 = ffma2(u[q][p], dyv[q][p], ud2);
                 }
-#pragma unroll
-                for (int c = 0; c < CPL; ++c) {
-                    sg[q][c] = rcp_ftz(1.f + ex2_ftz(-kLog2e * z[q][c]));
-                    const float u = z[q][c] * sg[q][c];
-                    ss[q] = fmaf(u, u, ss[q]);
-                    ud[q] = fmaf(u, dyv[q][c], ud[q]);
-                }
+                ss[q] = ss2.x + ss2.y;
+                ud[q] = ud2.x + ud2.y;
             }
             // L2 reverse: y = u/n, du = (dy - y (y . dy)) / n
             //                        = (dy - u (u . dy) / n^2) / n;
             // both row sums reduce together
-            float du[NB][CPL];
+            float2 dz[NB][NP];
             if (l2) {
 #pragma unroll
                 for (int off = 16; off > 0; off >>= 1)
@@ -544,91 +554,76 @@ __device__ __forceinline__ void prologue_bwd_block(const PrologueBwdArgs &a, con
                     }
 #pragma unroll
                 for (int q = 0; q < NB; ++q) {
-                    const float ninv = rsqrt_ftz(ss[q] + a.eps), f = -ud[q] * ninv * ninv;
+                    // zero past T, where u may be all zero (no 0 * inf with eps = 0)
+                    const float ninv = t0 + r + q < T ? rsqrt_ftz(ss[q] + a.eps) : 0.f, f = -ud[q] * ninv * ninv;
+                    const float2 f2 = make_float2(f, f), n2 = make_float2(ninv, ninv);
 #pragma unroll
-                    for (int c = 0; c < CPL; ++c) du[q][c] = fmaf(z[q][c] * sg[q][c], f, dyv[q][c]) * ninv;
+                    for (int p = 0; p < NP; ++p) dz[q][p] = fmul2(ffma2(u[q][p], f2, dyv[q][p]), fmul2(g[q][p], n2));
                 }
             } else {
 #pragma unroll
                 for (int q = 0; q < NB; ++q)
 #pragma unroll
-                    for (int c = 0; c < CPL; ++c) du[q][c] = dyv[q][c];
+                    for (int p = 0; p < NP; ++p) dz[q][p] = fmul2(dyv[q][p], g[q][p]);
             }
 #pragma unroll
             for (int q = 0; q < NB; ++q) {
                 if (q >= nrows) break;
-                const bool live = t0 + r + q < T;
-                float dz[CPL];
-#pragma unroll
-                for (int c = 0; c < CPL; ++c)
-                    dz[c] = live ? du[q][c] * sg[q][c] * fmaf(z[q][c], 1.f - sg[q][c], 1.f) : 0.f;
-                st_row<CPL>(dzp + q * D, dz);
+                st_row<CPL>(dzp + q * D, reinterpret_cast<const float *>(dz[q]));
                 if (r + q < kProBwdRun) {  // the unit's own rows: dw and dbias
 #pragma unroll
-                    for (int c = 0; c < CPL; c += 2) {
+                    for (int p = 0; p < NP; ++p) {
 #pragma unroll
-                        for (int m = 0; m < KW; ++m) {
-                            const float2 t = ffma2(make_float2(dz[c], dz[c + 1]),
-                                                   make_float2(win[q + m][c], win[q + m][c + 1]),
-                                                   make_float2(dwa[c][m], dwa[c + 1][m]));
-                            dwa[c][m] = t.x;
-                            dwa[c + 1][m] = t.y;
-                        }
-                        dba[c] += dz[c];
-                        dba[c + 1] += dz[c + 1];
+                        for (int m = 0; m < KW; ++m) dwa[p][m] = ffma2(dz[q][p], win[q + m][p], dwa[p][m]);
+                        dba[p] = ffma2(dz[q][p], one2, dba[p]);
                     }
                 }
                 if (r + q < K - 1) {  // the next unit walked (tokens before t0) reads these
-                    if (t0 == 0)
-#pragma unroll
-                        for (int c = 0; c < CPL; ++c) dz[c] = 0.f;  // ... unless it is another batch's
-                    st_row<CPL>(carry_out + (r + q) * D + lane * CPL, dz);
+                    if (t0 == 0) zero_row(dz[q]);  // ... unless it is another batch's
+                    st_row<CPL>(carry_out + (r + q) * D + lane * CPL, reinterpret_cast<const float *>(dz[q]));
                 }
             }
         };
         {  // the unit's 64 rows: warp w takes rows 8w .. 8w+7
             const int r0 = warp * kProBwdRowsPerWarp;
-            float win[WR][CPL];
+            float2 win[WR][NP];
 #pragma unroll
             for (int m = 0; m < KW - 1; ++m) {
                 const int row = r0 + K - KW + m;
                 if (row >= 0)
-                    ld_row<CPL>(sx + row * D, win[m]);
+                    ld_row<CPL>(sx + row * D, reinterpret_cast<float *>(win[m]));
                 else
-#pragma unroll
-                    for (int c = 0; c < CPL; ++c) win[m][c] = 0.f;
+                    zero_row(win[m]);
             }
 #pragma unroll
             for (int p = 0; p < kProBwdRowsPerWarp; p += NBW) {
                 const int r = r0 + p;
 #pragma unroll
-                for (int m = KW - 1; m < WR; ++m) ld_row<CPL>(sx + (r + K - KW + m) * D, win[m]);
+                for (int m = KW - 1; m < WR; ++m) ld_row<CPL>(sx + (r + K - KW + m) * D, reinterpret_cast<float *>(win[m]));
                 dz_rows(r, NBW, win, sdy + r * D, D, dzs + r * D + lane * CPL);
 #pragma unroll
                 for (int m = 0; m < KW - 1; ++m)
 #pragma unroll
-                    for (int c = 0; c < CPL; ++c) win[m][c] = win[m + NBW][c];
+                    for (int c = 0; c < NP; ++c) win[m][c] = win[m + NBW][c];
             }
         }
         if (k == 0 && warp < K - 1) {
             // the block's first unit: dz of token t0 + 64 + warp from global
             // memory (zero past T; the x it reads are tokens t0 + 57 .. t)
             const int r = kProBwdRun + warp, t = t0 + r;
-            float win[WR][CPL];
+            float2 win[WR][NP];
 #pragma unroll
             for (int m = 0; m < WR; ++m) {
                 if (t < T && m < KW)
-                    ld_row<CPL>(xg + (((size_t)b * T + t + 1 - KW + m) * H) * D + c0, win[m]);
+                    ld_row<CPL>(xg + (((size_t)b * T + t + 1 - KW + m) * H) * D + c0, reinterpret_cast<float *>(win[m]));
                 else
-#pragma unroll
-                    for (int c = 0; c < CPL; ++c) win[m][c] = 0.f;
+                    zero_row(win[m]);
             }
             dz_rows(r, t < T ? 1 : 0, win, dyg + (((size_t)b * T + t) * H) * D + c0, 0, carry_in + warp * D + lane * CPL);
             if (t >= T) {
-                float zero[CPL];
-#pragma unroll
-                for (int c = 0; c < CPL; ++c) zero[c] = 0.f;
-                st_row<CPL>(carry_in + warp * D + lane * CPL, zero);
+                float2 zero[NP];
+                zero_row(zero);
+                st_row<CPL>(carry_in + warp * D + lane * CPL, reinterpret_cast<const float *>(zero));
             }
         }
         __syncthreads();
@@ -636,30 +631,28 @@ __device__ __forceinline__ void prologue_bwd_block(const PrologueBwdArgs &a, con
         // phase 2: dx[i] = sum_j w[j] dz[i + K-1-j], from a window of dz rows
         // dzw[n] = dz row i + n (n < KW), which tap K-1-n = wt[.][KW-1-n]
         // multiplies (zero for n >= K); rows 64 .. 64+KW-2 are carry_in's
-        auto dx_row = [&](int i, const float (&dzw)[KW][CPL]) {
+        auto dx_row = [&](int i, const float2 (&dzw)[KW][NP]) {
             if (i >= len) return;  // past the end of a ragged last unit
-            float acc[CPL];
+            float2 acc[NP];
 #pragma unroll
-            for (int c = 0; c < CPL; c += 2) {
+            for (int p = 0; p < NP; ++p) {
                 float2 v = make_float2(0.f, 0.f);
 #pragma unroll
-                for (int n = 0; n < KW; ++n)
-                    v = ffma2(make_float2(wt[c][KW - 1 - n], wt[c + 1][KW - 1 - n]), make_float2(dzw[n][c], dzw[n][c + 1]),
-                              v);
-                acc[c] = v.x;
-                acc[c + 1] = v.y;
+                for (int n = 0; n < KW; ++n) v = ffma2(wt[p][KW - 1 - n], dzw[n][p], v);
+                acc[p] = v;
             }
             const int ms = t0 + i - (T - (K - 1));  // slot of this x in the returned state
             if (dso != nullptr && ms >= 0) {
-                float g[CPL];
-                ld_row<CPL>(dso + ((size_t)b * (K - 1) + ms) * Ctot + col + c0, g);
+                float2 gs[NP];
+                ld_row<CPL>(dso + ((size_t)b * (K - 1) + ms) * Ctot + col + c0, reinterpret_cast<float *>(gs));
 #pragma unroll
-                for (int c = 0; c < CPL; ++c) acc[c] += g[c];
+                for (int p = 0; p < NP; ++p) acc[p] = ffma2(gs[p], one2, acc[p]);
             }
             if (i >= 0) {
-                st_row<CPL>(dxb + ((size_t)b * T + t0 + i) * H * D + c0, acc);
+                st_row<CPL>(dxb + ((size_t)b * T + t0 + i) * H * D + c0, reinterpret_cast<const float *>(acc));
             } else {
-                st_row<CPL>(dsi + ((size_t)b * (K - 1) + (K - 1 + i)) * Ctot + col + c0, acc);
+                st_row<CPL>(dsi + ((size_t)b * (K - 1) + (K - 1 + i)) * Ctot + col + c0,
+                            reinterpret_cast<const float *>(acc));
             }
         };
         auto dz_row_ptr = [&](int row) {
@@ -667,29 +660,28 @@ __device__ __forceinline__ void prologue_bwd_block(const PrologueBwdArgs &a, con
         };
         {
             const int i0 = warp * kProBwdRowsPerWarp;
-            float dzw[KW][CPL];
+            float2 dzw[KW][NP];
 #pragma unroll
-            for (int n = 0; n < KW - 1; ++n) ld_row<CPL>(dz_row_ptr(i0 + n), dzw[n]);
+            for (int n = 0; n < KW - 1; ++n) ld_row<CPL>(dz_row_ptr(i0 + n), reinterpret_cast<float *>(dzw[n]));
 #pragma unroll
             for (int p = 0; p < kProBwdRowsPerWarp; ++p) {
-                ld_row<CPL>(dz_row_ptr(i0 + p + KW - 1), dzw[KW - 1]);
+                ld_row<CPL>(dz_row_ptr(i0 + p + KW - 1), reinterpret_cast<float *>(dzw[KW - 1]));
                 dx_row(i0 + p, dzw);
 #pragma unroll
                 for (int n = 0; n < KW - 1; ++n)
 #pragma unroll
-                    for (int c = 0; c < CPL; ++c) dzw[n][c] = dzw[n + 1][c];
+                    for (int c = 0; c < NP; ++c) dzw[n][c] = dzw[n + 1][c];
             }
         }
         if (t0 == 0 && dsi != nullptr && warp < K - 1) {  // the carried-in state's rows
             const int i = warp - (K - 1);
-            float dzw[KW][CPL];
+            float2 dzw[KW][NP];
 #pragma unroll
             for (int n = 0; n < KW; ++n) {
                 if (i + n >= 0)
-                    ld_row<CPL>(dz_row_ptr(i + n), dzw[n]);
+                    ld_row<CPL>(dz_row_ptr(i + n), reinterpret_cast<float *>(dzw[n]));
                 else
-#pragma unroll
-                    for (int c = 0; c < CPL; ++c) dzw[n][c] = 0.f;
+                    zero_row(dzw[n]);
             }
             dx_row(i, dzw);
         }
@@ -700,11 +692,16 @@ __device__ __forceinline__ void prologue_bwd_block(const PrologueBwdArgs &a, con
     float *red = reinterpret_cast<float *>(smem);
     constexpr int E = D * (KW + 1);
 #pragma unroll
-    for (int c = 0; c < CPL; ++c) {
+    for (int p = 0; p < NP; ++p) {
+        float *row0 = red + warp * E + (lane * CPL + 2 * p) * (KW + 1), *row1 = row0 + (KW + 1);
 #pragma unroll
         for (int m = 0; m < KW; ++m)
-            if (m >= KW - K) red[warp * E + (lane * CPL + c) * (KW + 1) + m - (KW - K)] = dwa[c][m];
-        red[warp * E + (lane * CPL + c) * (KW + 1) + KW] = dba[c];
+            if (m >= KW - K) {
+                row0[m - (KW - K)] = dwa[p][m].x;
+                row1[m - (KW - K)] = dwa[p][m].y;
+            }
+        row0[KW] = dba[p].x;
+        row1[KW] = dba[p].y;
     }
     __syncthreads();
     float *out = a.partial + (size_t)blockIdx.x * a.partial_stride;
