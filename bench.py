@@ -66,6 +66,9 @@ def parse_args():
     p.add_argument("--profile-step", action="store_true",
                    help="only run gdr_step three times on the decode workload (B256 H16 d128 bf16, "
                         "268 MB fp32 state) and exit")
+    p.add_argument("--profile-block-bwd", metavar="B,T,H", default=None,
+                   help="only run the block prologue backward (K=4) three times on seeded bf16 d=128 "
+                        "inputs of this shape and exit")
     p.add_argument("--profile-block", metavar="B,T,H", default=None,
                    help="only run the block prologue (K=4) and epilogue twice each on seeded bf16 "
                         "d=128 inputs of this shape and exit")
@@ -133,6 +136,26 @@ def profile_block(shape):
     torch.cuda.synchronize()
     gdr.check_status()
     print(json.dumps({"profile_block": shape, "status": "ok"}))
+
+
+def profile_block_bwd(shape):
+    """Three block prologue backward calls (ShortConv K=4, SiLU, q/k L2) on
+    the bench's seeded inputs (bf16, d = 128, dy ~ N(0, 1) seeded 25), then a
+    status check."""
+    import gated_delta_rule_91_b200 as gdr
+    B, T, H = (int(x) for x in shape.split(","))
+    d, K = 128, 4
+    px = {n: (t.cuda() if t is not None else None)
+          for n, t in synth.block_prologue_inputs(B, T, H, d, d, K, "bf16", seed=21, state=False).items()}
+    pg = torch.Generator().manual_seed(25)
+    dys = [torch.randn(B, T, H, d, generator=pg).to(torch.bfloat16).cuda() for _ in range(3)]
+    ws = torch.empty(gdr.lib().gdr_block_prologue_bwd_workspace_bytes(H, d, d, K), dtype=torch.uint8, device="cuda")
+    for _ in range(3):
+        gdr.gdr_block_prologue_bwd(px["xq"], px["xk"], px["xv"], px["wq"], px["wk"], px["wv"], *dys,
+                                   px["bq"], px["bk"], px["bv"], eps=1e-6, workspace=ws)
+    torch.cuda.synchronize()
+    gdr.check_status()
+    print(json.dumps({"profile_block_bwd": shape, "status": "ok"}))
 
 
 def profile_gdn2(shape):
@@ -736,6 +759,9 @@ def main():
         return
     if args.profile_block:
         profile_block(args.profile_block)
+        return
+    if args.profile_block_bwd:
+        profile_block_bwd(args.profile_block_bwd)
         return
     if args.profile_gdn2_bwd:
         profile_gdn2_bwd(args.profile_gdn2_bwd)
