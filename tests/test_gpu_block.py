@@ -315,6 +315,17 @@ def test_prologue_bwd_shorter_than_the_window(T, K, dtype, d):
     _check_pro_bwd(x, _pro_bwd_gpu(x, eps), _pro_bwd_ref(x, eps), dtype)
 
 
+@pytest.mark.parametrize("K", [3, 4, 8])
+def test_prologue_bwd_blocks_walk_several_runs(K):
+    # H16 gives 48 (stream, head) pairs and a few blocks per pair, so a block
+    # walks several 64-token runs from the last to the first, carrying the
+    # dz rows of each run's first tokens to the run before it.  At B4 T700
+    # (11 runs, the last of 60 tokens) some blocks' ranges cross a batch
+    # boundary, where the carried rows must be zero.
+    x = synth.block_prologue_bwd_inputs(4, 700, 16, 128, 128, K, "bf16", seed=40 + K, state=True, dstate=True)
+    _check_pro_bwd(x, _pro_bwd_gpu(x, 1e-6, want_dconv_state=True), _pro_bwd_ref(x, 1e-6), "bf16")
+
+
 def test_prologue_bwd_workload_full():
     # B4 T4096 H16 d128 K4 bf16: every element of dx and the full sums
     x = synth.block_prologue_bwd_inputs(4, 4096, 16, 128, 128, 4, "bf16", seed=31, state=False)
