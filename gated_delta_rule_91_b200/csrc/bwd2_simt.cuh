@@ -29,6 +29,14 @@
 // token instead, with the step's own reverse mode (gdr2_chunk_reverse_exact);
 // its per-token partials are summed by the same reduce kernel without the
 // E factors.
+//
+// For bf16 with dk = dv = 128, launch_bwd2_simt runs another sequence: the
+// cluster recompute (which also keeps every chunk's T and P), the
+// tensor-core dS pass (bwd2_ds.cuh, every chunk's D), and one tensor-core
+// CTA per chunk for all of its gradients (bwd2_grad_tc.cuh).  Only the
+// chunks that one lists (decay past e^20) come here: gdr2_bwd_simt_list_kernel
+// runs this reverse per (slice, listed chunk) from the stored D, and the
+// chunk kernel of bwd2_tc.cuh sums their slices.
 #pragma once
 #include "common.cuh"
 #include "bwd_simt.cuh"
