@@ -117,6 +117,89 @@ def test_chunkwise_gdr2_equals_recurrence(C, T):
     assert rel_err(STc, ST) < 1e-10
 
 
+def chunkwise_gdr_u_chain(q, k, v, la, be, S0, C):
+    """The chunkwise forward with U carried chunk to chunk instead of formed
+    from the freshly updated state.  With S_{n+1} = gamma_C S_n + U_n^T Kd_n
+    (Kd = diag(gamma_C/gamma) K), U_{n+1} = U^g_{n+1} - W_{n+1} S_{n+1}^T
+    expands to
+
+        U_{n+1} = U^g_{n+1} - gamma_C W_{n+1} S_n^T - (W_{n+1} Kd_n^T) U_n,
+
+    so U_{n+1} needs S_n (one step old) and U_n, and the state update leaves
+    the chain from U_n to U_{n+1}.  Algebraically the same map; a state-pass
+    kernel may take either form."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    o = np.zeros((B, T, H, dv))
+    ST = np.zeros((B, H, dv, dk))
+    for b in range(B):
+        for h in range(H):
+            S = np.zeros((dv, dk)) if S0 is None else S0[b, h].copy()
+            prev = None  # (S_n, gamma_C, Kd, U) of the chunk before
+            for c0 in range(0, T, C):
+                sl = slice(c0, min(c0 + C, T))
+                Q, K, V = q[b, sl, h], k[b, sl, h], v[b, sl, h]
+                beta = be[b, sl, h]
+                g = np.cumsum(la[b, sl, h])
+                n = len(g)
+                ratio = np.exp(g[:, None] - g[None, :])
+                A = np.tril(np.ones((n, n)), -1) * (beta[:, None] * ratio * (K @ K.T))
+                Tm = np.linalg.inv(np.eye(n) + A)
+                Ug = Tm @ (beta[:, None] * V)
+                W = Tm @ ((beta * np.exp(g))[:, None] * K)
+                if prev is None:
+                    U = Ug - W @ S.T
+                else:
+                    Sp, gCp, Kdp, Up = prev
+                    U = Ug - gCp * (W @ Sp.T) - (W @ Kdp.T) @ Up
+                o[b, sl, h] = np.exp(g)[:, None] * (Q @ S.T) + ((Q @ K.T) * ratio * np.tril(np.ones((n, n)))) @ U
+                Kd = np.exp(g[-1] - g)[:, None] * K
+                prev = (S, np.exp(g[-1]), Kd, U)
+                S = np.exp(g[-1]) * S + U.T @ Kd
+            ST[b, h] = S
+    return o, ST
+
+
+@pytest.mark.parametrize("C", [4, 64])
+@pytest.mark.parametrize("T", [64, 200, 256])
+def test_u_chain_form_equals_recurrence(C, T):
+    rng = np.random.default_rng(3 * C + T)
+    q, k, v, la, be, S0 = rand_inputs(rng, 1, T, 2, 8, 6)
+    o, ST = oracle.gdr_fwd(q, k, v, la, be, S0)
+    oc, STc = chunkwise_gdr_u_chain(q, k, v, la, be, S0, C)
+    assert rel_err(oc, o) < 1e-10
+    assert rel_err(STc, ST) < 1e-10
+
+
+def test_u_chain_form_needs_the_decay_on_the_old_state():
+    """Dropping gamma_C from the S_n term (a plausible slip when moving the
+    state update off the chain) is off by O(1)."""
+    rng = np.random.default_rng(5)
+    q, k, v, la, be, S0 = rand_inputs(rng, 1, 128, 1, 8, 6)
+    o, _ = oracle.gdr_fwd(q, k, v, la, be, S0)
+    Q, K, V = q[0, :, 0], k[0, :, 0], v[0, :, 0]
+    beta, g_all = be[0, :, 0], la[0, :, 0]
+    S = S0[0, 0]
+    parts = []
+    for c0 in (0, 64):
+        sl = slice(c0, c0 + 64)
+        g = np.cumsum(g_all[sl])
+        ratio = np.exp(g[:, None] - g[None, :])
+        A = np.tril(np.ones((64, 64)), -1) * (beta[sl][:, None] * ratio * (K[sl] @ K[sl].T))
+        Tm = np.linalg.inv(np.eye(64) + A)
+        Ug = Tm @ (beta[sl][:, None] * V[sl])
+        W = Tm @ ((beta[sl] * np.exp(g))[:, None] * K[sl])
+        parts.append((g, ratio, Ug, W))
+    g0, r0, Ug0, W0 = parts[0]
+    U0 = Ug0 - W0 @ S.T
+    Kd0 = np.exp(g0[-1] - g0)[:, None] * K[:64]
+    S1 = np.exp(g0[-1]) * S + U0.T @ Kd0
+    g1, r1, Ug1, W1 = parts[1]
+    U1_bad = Ug1 - W1 @ S.T - (W1 @ Kd0.T) @ U0
+    o1_bad = np.exp(g1)[:, None] * (Q[64:] @ S1.T) + ((Q[64:] @ K[64:].T) * r1 * np.tril(np.ones((64, 64)))) @ U1_bad
+    assert rel_err(o1_bad, o[0, 64:, 0]) > 1e-3
+
+
 def test_mask_without_decay_is_wrong():
     """The literal printed mask (no decay on the intra-chunk term) disagrees
     with the recurrence, which is why the decayed mask is the reading."""
