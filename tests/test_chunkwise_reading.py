@@ -304,3 +304,106 @@ def test_chunkwise_backward_equals_oracle_reverse_mode(T, C):
     got = chunkwise_gdr_bwd(q, k, v, la, be, S0, dO, dST, C)
     for name in ref:
         assert rel_err(got[name], ref[name]) < 1e-10, name
+
+
+def chunkwise_gdr2_bwd(q, k, v, la, bg, wg, S0, dO, dST, C=64, scaled_d=True):
+    """Per-chunk reverse mode of the Gated DeltaNet-2 chunk form (the formulas
+    the tensor-core GDN-2 backward evaluates), fp64.  Per chunk, with S the
+    entry state, D = dL/dS' the exit-state gradient and
+    KBE = K*B*E, QE = Q*E, KiE = K/E, Kt = K*exp(G_C - G) = KiE Diag(E_C):
+        dU = Kt D^T + P^T dO,   dR = T^T dU,
+        dA = -strictLower(dR U^T),   dP = inclLower(dO U^T),
+        dKBE = -dR S + dA KiE,   dQE = dO S + dP KiE,
+        dKiE = dA^T KBE + dP^T QE + (U D) Diag(E_C),
+        dE_C = colsum(S*D) + colsum((U D)*KiE),
+        D_prev = D Diag(E_C) + dO^T QE - dR^T KBE,
+    then dk = dKBE*B*E + dKiE/E, db = dKBE*K*E, dq = dQE*E, dv = W*dR,
+    dw = V*dR, dG = dKBE*KBE + dQE*QE - dKiE*KiE (+ E_C dE_C on the last
+    token) and dlog alpha = the in-chunk suffix sums of dG.  scaled_d uses
+    D' = D Diag(E_C) with KiE, the form the per-chunk kernel multiplies:
+    Kt D^T = KiE D'^T and (U D) Diag(E_C) = U D'."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    out = {n: np.zeros_like(x) for n, x in (("dq", q), ("dk", k), ("dv", v), ("dlog_alpha", la),
+                                            ("db", bg), ("dw", wg))}
+    out["dS0"] = np.zeros((B, H, dv, dk))
+    for b in range(B):
+        for h in range(H):
+            S = np.zeros((dv, dk)) if S0 is None else S0[b, h].copy()
+            starts = []
+            for c0 in range(0, T, C):
+                starts.append(S.copy())
+                sl = slice(c0, min(c0 + C, T))
+                Q, K, V = q[b, sl, h], k[b, sl, h], v[b, sl, h]
+                G = np.cumsum(la[b, sl, h], axis=0)
+                E = np.exp(G)
+                n = G.shape[0]
+                KBE = K * bg[b, sl, h] * E
+                A = np.tril(np.ones((n, n)), -1) * (KBE @ (K / E).T)
+                U = np.linalg.inv(np.eye(n) + A) @ (wg[b, sl, h] * V - KBE @ S.T)
+                S = S * E[-1][None, :] + U.T @ (K * np.exp(G[-1][None, :] - G))
+            D = dST[b, h].copy() if dST is not None else np.zeros((dv, dk))
+            for ci in reversed(range(len(starts))):
+                sl = slice(ci * C, min(ci * C + C, T))
+                Q, K, V, dOc = q[b, sl, h], k[b, sl, h], v[b, sl, h], dO[b, sl, h]
+                Bg, Wg = bg[b, sl, h], wg[b, sl, h]
+                S = starts[ci]
+                G = np.cumsum(la[b, sl, h], axis=0)
+                E = np.exp(G)
+                EC = E[-1]
+                n = G.shape[0]
+                strict = np.tril(np.ones((n, n)), -1)
+                incl = np.tril(np.ones((n, n)))
+                KBE, QE, KiE = K * Bg * E, Q * E, K / E
+                Kt = K * np.exp(G[-1][None, :] - G)
+                A = strict * (KBE @ KiE.T)
+                P = incl * (QE @ KiE.T)
+                Tm = np.linalg.inv(np.eye(n) + A)
+                R = Wg * V - KBE @ S.T
+                U = Tm @ R
+                if scaled_d:
+                    Dp = D * EC[None, :]
+                    dU = KiE @ Dp.T + P.T @ dOc
+                    UDs = U @ Dp
+                else:
+                    dU = Kt @ D.T + P.T @ dOc
+                    UDs = (U @ D) * EC[None, :]
+                dR = Tm.T @ dU
+                dA = -strict * (dR @ U.T)
+                dP = incl * (dOc @ U.T)
+                dKBE = -dR @ S + dA @ KiE
+                dQE = dOc @ S + dP @ KiE
+                dKiE = dA.T @ KBE + dP.T @ QE + UDs
+                dEC = np.sum(S * D, 0) + np.sum(UDs * KiE, 0) / EC
+                dG = dKBE * KBE + dQE * QE - dKiE * KiE
+                dG[-1] += EC * dEC
+                out["dq"][b, sl, h] = dQE * E
+                out["dk"][b, sl, h] = dKBE * Bg * E + dKiE / E
+                out["db"][b, sl, h] = dKBE * K * E
+                out["dv"][b, sl, h] = Wg * dR
+                out["dw"][b, sl, h] = V * dR
+                out["dlog_alpha"][b, sl, h] = np.cumsum(dG[::-1], axis=0)[::-1]
+                D = D * EC[None, :] + dOc.T @ QE - dR.T @ KBE
+            out["dS0"][b, h] = D
+    return out
+
+
+def _gdr2_bwd_inputs(rng, T):
+    q, k, v, _, _, S0 = rand_inputs(rng, 1, T, 2, 8, 6)
+    la = -np.log1p(np.exp(rng.normal(-2.0, 1.0, size=(1, T, 2, 8))))
+    bg = rng.uniform(0.0, 2.0, size=(1, T, 2, 8))
+    wg = rng.uniform(0.0, 1.0, size=(1, T, 2, 6))
+    dO = rng.normal(size=(1, T, 2, 6))
+    dST = rng.normal(size=(1, 2, 6, 8))
+    return q, k, v, la, bg, wg, S0, dO, dST
+
+
+@pytest.mark.parametrize("scaled_d", [False, True])
+@pytest.mark.parametrize("T,C", [(64, 64), (150, 64), (100, 16)])
+def test_chunkwise_gdr2_backward_equals_oracle_reverse_mode(T, C, scaled_d):
+    rng = np.random.default_rng(11 * T + C)
+    q, k, v, la, bg, wg, S0, dO, dST = _gdr2_bwd_inputs(rng, T)
+    ref = oracle.gdr2_bwd(q, k, v, la, bg, wg, S0, dO, dST)
+    got = chunkwise_gdr2_bwd(q, k, v, la, bg, wg, S0, dO, dST, C=C, scaled_d=scaled_d)
+    for name in ("dq", "dk", "dv", "dlog_alpha", "db", "dw", "dS0"):
+        assert rel_err(got[name], ref[name]) < 1e-9, name
